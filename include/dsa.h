@@ -1,0 +1,204 @@
+/*
+ * dsa.h -- C interface of the B200 (sm_100a) DeepSeek Sparse Attention hot path.
+ *
+ * The path has three stages, each a hand-written CUDA kernel, plus a split
+ * merge:
+ *   1. lightning-indexer scores   I[t,s] = sum_j w[t,j] * ReLU(q_I[t,j] . k_I[s])
+ *   2. per-query causal top-k     the min(k, n_t) highest scores of row t
+ *   3. sparse MLA attention       softmax over the selected latent rows only,
+ *                                 every query head sharing each row (MQA mode)
+ * Sources (page title, section):
+ *   - "DeepSeek Sparse Attention Explained" (kgptalkie): "How Does the Lightning
+ *     Indexer Score a Token?", "How Does the Selector Pick 1,024?", "What Does
+ *     the Whole Block Look Like?", "What Does the GPU Actually Run?".
+ *   - "DeepSeek Sparse Attention" (lizeman), section 2 (two stages) and
+ *     section 3 (the dsa_layer sketch whose arguments this interface follows).
+ *   - "DeepSeek V3.2-Exp Cuts Long-Context Costs" (kiadev), "How DSA works" and
+ *     "Training and implementation details" (FP8 indexer, top-k = 2048, MLA in
+ *     MQA mode).
+ *
+ * Conventions shared by every entry point:
+ *   - All pointers marked (device) are CUDA device pointers owned by the caller;
+ *     the library never allocates, frees or keeps them.  Every call is
+ *     asynchronous on `stream` (a cudaStream_t passed as void*, NULL = legacy
+ *     default stream) and returns once the kernels are queued.
+ *   - Arguments are checked on the host before any launch: NULL pointers,
+ *     16-byte alignment of every tensor base, supported sizes.  A failed check
+ *     returns an error status and launches nothing.
+ *   - Device-side errors (an index >= q_len, q_len > T_max, a bounded wait that
+ *     ran out) are recorded in a status word at the start of the workspace and
+ *     read back with dsa_get_device_status().  Kernels never trap.
+ *   - Query row t belongs to sequence q_seq[t] and sees the causal candidate
+ *     positions s in [0, q_len[t]).  Decode: q_len[t] is the cached length of
+ *     the sequence.  Prefill: q_len[t] = t + 1 (the token sees itself).
+ *
+ * Tensor layouts (row-major, contiguous, element counts):
+ *   q_I      [Nq, H_I, d_I]   FP8 e4m3 bytes (idx_dtype DSA_FP8_E4M3) or float
+ *   q_scale  [Nq, H_I]        float, > 0 (FP8 only; may be NULL for float)
+ *   w        [Nq, H_I]        bfloat16 (FP8 mode) or float (float mode)
+ *   k_I      [B, T_max, d_I]  FP8 e4m3 bytes or float
+ *   k_scale  [B, T_max]       float, > 0 (FP8 only; may be NULL for float)
+ *   q        [Nq, H, 576]     bfloat16 or float (absorbed MLA query: 512 latent + 64 rope)
+ *   kv       [B, T_max, 576]  bfloat16 or float (latent cache; value = first 512)
+ *   out      [Nq, H, 512]     same element type as kv
+ *   lse      [Nq, H]          float, natural-log sum of exp(scale * q.c) over the selection
+ *   scores   [Nq, ld_scores]  float, entries s >= q_len[t] are not written
+ *   idx      [Nq, k]          int32, ascending positions, -1 padded
+ *   q_seq, q_len [Nq]         int32
+ */
+#ifndef DSA_B200_H
+#define DSA_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    DSA_OK = 0,
+    DSA_ERR_INVALID_ARG = 1,   /* NULL, misaligned or inconsistent argument */
+    DSA_ERR_UNSUPPORTED = 2,   /* valid but not built: e.g. d_I not 64/128, H != 128 for bf16 */
+    DSA_ERR_WORKSPACE = 3,     /* workspace NULL or smaller than dsa_workspace_size() */
+    DSA_ERR_CUDA = 4,          /* a CUDA runtime call or launch failed (see dsa_last_cuda_error) */
+    DSA_ERR_TIMEOUT = 5,       /* device: a bounded wait inside a kernel ran out */
+    DSA_ERR_INDEX_OOB = 6,     /* device: an idx entry outside [-1, q_len[t]) (treated as -1) */
+    DSA_ERR_LENGTH = 7         /* device: q_len[t] > T_max or > ld_scores, or q_seq[t] outside [0, B) (row skipped) */
+} dsa_status_t;
+
+typedef enum { DSA_F32 = 0, DSA_BF16 = 1, DSA_FP8_E4M3 = 2 } dsa_dtype_t;
+
+typedef enum {
+    DSA_OP_INDEXER = 0,
+    DSA_OP_TOPK = 1,
+    DSA_OP_SPARSE_MLA = 2,
+    DSA_OP_DECODE = 3,
+    DSA_OP_PREFILL = 4
+} dsa_op_t;
+
+/* Problem sizes.  Supported builds:
+ *   idx_dtype DSA_FP8_E4M3: d_I in {64, 128}, H_I in {1..64}... exactly 64 for the tensor-core
+ *                           kernel (H_I is the MMA N dimension); w is bfloat16.
+ *   idx_dtype DSA_F32:      d_I in {64, 128}, 1 <= H_I <= 64; w is float.
+ *   kv_dtype  DSA_BF16:     H = 128 (MMA M dimension).
+ *   kv_dtype  DSA_F32:      1 <= H <= 128.
+ *   1 <= k <= 2048; 1 <= T_max; ld_scores >= 1 and a multiple of 4. */
+typedef struct {
+    int32_t B;          /* sequences held in the cache */
+    int32_t Nq;         /* query rows */
+    int32_t H_I;        /* indexer heads */
+    int32_t d_I;        /* indexer head width */
+    int32_t H;          /* MLA query heads */
+    int32_t k;          /* top-k budget */
+    int32_t T_max;      /* cache capacity per sequence, tokens (row stride of k_I/kv per sequence) */
+    int32_t idx_dtype;  /* dsa_dtype_t of q_I/k_I: DSA_FP8_E4M3 or DSA_F32 */
+    int32_t kv_dtype;   /* dsa_dtype_t of q/kv/out: DSA_BF16 or DSA_F32 */
+    int32_t reserved;   /* must be 0 */
+    int64_t ld_scores;  /* row stride of the scores matrix, elements */
+} dsa_dims;
+
+/* Optional per-stage timing: cudaEvent_t handles (as void*) recorded on the
+ * call's stream before the first stage and after each stage (indexer, top-k,
+ * attention, merge).  Any entry may be NULL. */
+typedef struct {
+    void* ev[5];
+} dsa_stage_events;
+
+/* Bytes of workspace the given operation needs for these sizes (0 when none
+ * beyond the 256-byte status block).  The plan depends on the current
+ * device's SM count.  Returns DSA_OK and writes *bytes, or DSA_ERR_INVALID_ARG /
+ * DSA_ERR_UNSUPPORTED. */
+dsa_status_t dsa_workspace_size(const dsa_dims* dims, int32_t op, size_t* bytes);
+
+/* Zero the workspace's status block (call once after allocating a workspace). */
+dsa_status_t dsa_workspace_init(void* workspace, size_t ws_bytes, void* stream);
+
+/* Stage 1 -- lightning-indexer scores (kgptalkie, "How Does the Lightning
+ * Indexer Score a Token?"; kiadev, "How DSA works": FP8, few small heads, ReLU).
+ * scores[t,s] = k_scale[b,s] * sum_j (w[t,j] q_scale[t,j]) * ReLU(sum_x q_I[t,j,x] k_I[b,s,x])
+ * for s < q_len[t], b = q_seq[t]; in float mode the scales are 1.  The per-head
+ * dot products are never written out.  Device errors go to workspace's status
+ * word (workspace may be NULL, then length errors are only skipped rows). */
+dsa_status_t dsa_indexer_scores(const dsa_dims* dims, const void* q_I, const float* q_scale,
+                                const void* w, const void* k_I, const float* k_scale,
+                                const int32_t* q_seq, const int32_t* q_len, float* scores,
+                                void* workspace, size_t ws_bytes, void* stream);
+
+/* Stage 2 -- per-row causal top-k (kgptalkie, "How Does the Selector Pick
+ * 1,024?": keep the highest index_topk scores, min(budget, tokens so far),
+ * redone for every query).  idx[t] holds the min(k, q_len[t]) positions of the
+ * largest scores[t, 0:q_len[t]] under the order (score descending, position
+ * ascending; -0.0 == +0.0), written in ascending position order, then -1.
+ * NaN scores are not supported.  Bit-exact and deterministic. */
+dsa_status_t dsa_topk(const dsa_dims* dims, const float* scores, const int32_t* q_len,
+                      int32_t* idx, void* workspace, size_t ws_bytes, void* stream);
+
+/* Stage 3 -- sparse MLA attention in MQA mode (kgptalkie, "What Does the
+ * Whole Block Look Like?": the softmax denominator runs over the selected
+ * tokens only; kiadev, "Training and implementation details": MQA mode, each
+ * latent row shared by all heads).  For each row t and head h:
+ *   out[t,h,:] = sum_{s in idx[t], s>=0} softmax_s(softmax_scale * q[t,h,:] . kv[b,s,:]) kv[b,s,0:512]
+ *   lse[t,h]   = ln sum_s exp(softmax_scale * q[t,h,:] . kv[b,s,:])
+ * An empty selection gives out = 0, lse = -inf.  lse may be NULL.
+ * Entries of idx outside [-1, q_len[t]) are treated as -1 and flagged
+ * DSA_ERR_INDEX_OOB in the status word.  Workspace (sized for
+ * DSA_OP_SPARSE_MLA) holds the split partial results. */
+dsa_status_t dsa_sparse_mla_attn(const dsa_dims* dims, const void* q, const void* kv,
+                                 const int32_t* idx, const int32_t* q_seq, const int32_t* q_len,
+                                 float softmax_scale, void* out, float* lse,
+                                 void* workspace, size_t ws_bytes, void* stream);
+
+/* The whole decode step: stages 1-3 back to back on `stream` (lizeman,
+ * section 3 sketch: indexer, top-K gather, attention over the K positions).
+ * scores_out / idx_out may be NULL (then the workspace holds them; size the
+ * workspace for DSA_OP_DECODE); when given they receive the intermediate
+ * results.  events may be NULL. */
+dsa_status_t dsa_decode_step(const dsa_dims* dims,
+                             const void* q_I, const float* q_scale, const void* w,
+                             const void* k_I, const float* k_scale,
+                             const void* q, const void* kv,
+                             const int32_t* q_seq, const int32_t* q_len, float softmax_scale,
+                             void* out, float* lse, float* scores_out, int32_t* idx_out,
+                             void* workspace, size_t ws_bytes, void* stream,
+                             const dsa_stage_events* events);
+
+/* Prefill: the same three stages for many query rows (every position of a
+ * prompt), processed in row chunks so the transient score rows fit the
+ * workspace (size it for DSA_OP_PREFILL).  Semantics per row are exactly those
+ * of dsa_decode_step; q_len[t] = t + 1 for a causal prompt.  idx_out may be
+ * NULL. */
+dsa_status_t dsa_prefill(const dsa_dims* dims,
+                         const void* q_I, const float* q_scale, const void* w,
+                         const void* k_I, const float* k_scale,
+                         const void* q, const void* kv,
+                         const int32_t* q_seq, const int32_t* q_len, float softmax_scale,
+                         void* out, float* lse, int32_t* idx_out,
+                         void* workspace, size_t ws_bytes, void* stream);
+
+/* Read and clear the device status word: synchronises `stream`, writes the
+ * first device-side error recorded since the last read into *status (DSA_OK if
+ * none) and resets it. */
+dsa_status_t dsa_get_device_status(void* workspace, void* stream, int32_t* status);
+
+/* Short text for a status code (static storage). */
+const char* dsa_status_string(int32_t status);
+
+/* The last CUDA runtime error seen by this thread inside the library (a
+ * cudaError_t value; 0 when none). */
+int32_t dsa_last_cuda_error(void);
+
+/* Self-test of the bounded wait used by every kernel: one CTA waits on a
+ * barrier that nothing arrives at, for about `timeout_us` microseconds, then
+ * records DSA_ERR_TIMEOUT in the status word and exits normally. */
+dsa_status_t dsa_selftest_wait_timeout(void* workspace, size_t ws_bytes, int32_t timeout_us,
+                                       void* stream);
+
+/* Library version string. */
+const char* dsa_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* DSA_B200_H */

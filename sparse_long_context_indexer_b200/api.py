@@ -1,0 +1,177 @@
+"""Python entry points with the names of the C interface (``include/dsa.h``).
+
+Marshalling only: each function checks the tensors' device, dtype and shape,
+passes their device pointers and torch's current CUDA stream to the C library
+and returns.  Every step of the hot path runs in the library's CUDA kernels;
+nothing here computes on the host or falls back to torch operations.
+"""
+from __future__ import annotations
+
+import ctypes
+from dataclasses import dataclass
+from typing import Optional, Sequence
+
+import torch
+
+from . import _lib
+
+D_K, D_V = 576, 512
+
+
+@dataclass
+class Dims:
+    B: int
+    Nq: int
+    H_I: int
+    d_I: int
+    H: int
+    k: int
+    T_max: int
+    idx_dtype: int
+    kv_dtype: int
+    ld_scores: int
+
+    def c(self) -> _lib.DsaDims:
+        return _lib.DsaDims(self.B, self.Nq, self.H_I, self.d_I, self.H, self.k, self.T_max, self.idx_dtype,
+                            self.kv_dtype, 0, self.ld_scores)
+
+
+def dims_of(inp, ld_scores: Optional[int] = None, Nq: Optional[int] = None) -> Dims:
+    """Dims for an ``inputs.DSAInputs`` workload (ld_scores defaults to T_max rounded up to 4)."""
+    ld = ld_scores if ld_scores is not None else (inp.T_max + 3) // 4 * 4
+    return Dims(inp.B, inp.Nq if Nq is None else Nq, inp.H_I, inp.d_I, inp.H, inp.k, inp.T_max, inp.idx_dtype,
+                inp.kv_dtype, ld)
+
+
+def _stream_ptr(stream=None) -> int:
+    s = torch.cuda.current_stream() if stream is None else stream
+    return s.cuda_stream
+
+
+def _ptr(t: Optional[torch.Tensor]) -> Optional[int]:
+    if t is None:
+        return None
+    if not t.is_cuda:
+        raise ValueError("tensor must live on a CUDA device")
+    if not t.is_contiguous():
+        raise ValueError("tensor must be contiguous")
+    return t.data_ptr()
+
+
+def workspace_size(dims: Dims, op: int) -> int:
+    lib = _lib.load()
+    n = ctypes.c_size_t(0)
+    d = dims.c()
+    _lib.check(lib, lib.dsa_workspace_size(ctypes.byref(d), op, ctypes.byref(n)), "dsa_workspace_size")
+    return int(n.value)
+
+
+def make_workspace(dims: Dims, op: int, device=None) -> torch.Tensor:
+    """A zero-initialised uint8 device buffer sized for `op` (torch allocates; the library never does)."""
+    lib = _lib.load()
+    nbytes = workspace_size(dims, op)
+    ws = torch.empty(max(nbytes, 256), dtype=torch.uint8, device=device or "cuda")
+    _lib.check(lib, lib.dsa_workspace_init(ws.data_ptr(), ws.numel(), _stream_ptr()), "dsa_workspace_init")
+    return ws
+
+
+def get_device_status(ws: torch.Tensor) -> int:
+    lib = _lib.load()
+    v = ctypes.c_int32(0)
+    _lib.check(lib, lib.dsa_get_device_status(ws.data_ptr(), _stream_ptr(), ctypes.byref(v)), "dsa_get_device_status")
+    return int(v.value)
+
+
+def status_string(code: int) -> str:
+    return _lib.load().dsa_status_string(code).decode()
+
+
+def indexer_scores(dims: Dims, q_I, q_scale, w, k_I, k_scale, q_seq, q_len, scores, ws=None):
+    lib = _lib.load()
+    d = dims.c()
+    rc = lib.dsa_indexer_scores(ctypes.byref(d), _ptr(q_I), _ptr(q_scale), _ptr(w), _ptr(k_I), _ptr(k_scale),
+                                _ptr(q_seq), _ptr(q_len), _ptr(scores), _ptr(ws),
+                                0 if ws is None else ws.numel(), _stream_ptr())
+    _lib.check(lib, rc, "dsa_indexer_scores")
+    return scores
+
+
+def topk(dims: Dims, scores, q_len, idx, ws=None):
+    lib = _lib.load()
+    d = dims.c()
+    rc = lib.dsa_topk(ctypes.byref(d), _ptr(scores), _ptr(q_len), _ptr(idx), _ptr(ws),
+                      0 if ws is None else ws.numel(), _stream_ptr())
+    _lib.check(lib, rc, "dsa_topk")
+    return idx
+
+
+def sparse_mla_attn(dims: Dims, q, kv, idx, q_seq, q_len, softmax_scale, out, lse, ws):
+    lib = _lib.load()
+    d = dims.c()
+    rc = lib.dsa_sparse_mla_attn(ctypes.byref(d), _ptr(q), _ptr(kv), _ptr(idx), _ptr(q_seq), _ptr(q_len),
+                                 ctypes.c_float(softmax_scale), _ptr(out), _ptr(lse), _ptr(ws), ws.numel(),
+                                 _stream_ptr())
+    _lib.check(lib, rc, "dsa_sparse_mla_attn")
+    return out, lse
+
+
+def decode_step(dims: Dims, q_I, q_scale, w, k_I, k_scale, q, kv, q_seq, q_len, softmax_scale, out, lse, ws,
+                scores_out=None, idx_out=None, events: Optional[Sequence] = None):
+    """One decode step (indexer -> top-k -> sparse MLA) on torch's current stream.
+
+    events: optional 5 ``torch.cuda.Event(enable_timing=True)`` recorded before
+    the first stage and after each stage (indexer, top-k, attention, merge).
+    """
+    lib = _lib.load()
+    d = dims.c()
+    evp = None
+    if events is not None:
+        evs = _lib.DsaStageEvents()
+        for i, e in enumerate(events):
+            if e is not None and not e.cuda_event:
+                e.record()  # torch creates the CUDA event lazily, on its first record
+            evs.ev[i] = None if e is None else e.cuda_event
+        evp = ctypes.byref(evs)
+    rc = lib.dsa_decode_step(ctypes.byref(d), _ptr(q_I), _ptr(q_scale), _ptr(w), _ptr(k_I), _ptr(k_scale), _ptr(q),
+                             _ptr(kv), _ptr(q_seq), _ptr(q_len), ctypes.c_float(softmax_scale), _ptr(out), _ptr(lse),
+                             _ptr(scores_out), _ptr(idx_out), _ptr(ws), ws.numel(), _stream_ptr(), evp)
+    _lib.check(lib, rc, "dsa_decode_step")
+    return out, lse
+
+
+def prefill(dims: Dims, q_I, q_scale, w, k_I, k_scale, q, kv, q_seq, q_len, softmax_scale, out, lse, ws,
+            idx_out=None):
+    lib = _lib.load()
+    d = dims.c()
+    rc = lib.dsa_prefill(ctypes.byref(d), _ptr(q_I), _ptr(q_scale), _ptr(w), _ptr(k_I), _ptr(k_scale), _ptr(q),
+                         _ptr(kv), _ptr(q_seq), _ptr(q_len), ctypes.c_float(softmax_scale), _ptr(out), _ptr(lse),
+                         _ptr(idx_out), _ptr(ws), ws.numel(), _stream_ptr())
+    _lib.check(lib, rc, "dsa_prefill")
+    return out, lse
+
+
+def selftest_wait_timeout(ws: torch.Tensor, timeout_us: int = 200000):
+    lib = _lib.load()
+    rc = lib.dsa_selftest_wait_timeout(ws.data_ptr(), ws.numel(), int(timeout_us), _stream_ptr())
+    _lib.check(lib, rc, "dsa_selftest_wait_timeout")
+
+
+# ---- conveniences over an inputs.DSAInputs workload --------------------------
+
+def alloc_outputs(inp, device=None):
+    dev = device or inp.device
+    odt = torch.bfloat16 if inp.kv_dtype == _lib.DSA_BF16 else torch.float32
+    out = torch.empty((inp.Nq, inp.H, D_V), dtype=odt, device=dev)
+    lse = torch.empty((inp.Nq, inp.H), dtype=torch.float32, device=dev)
+    return out, lse
+
+
+def run_decode(inp, ws=None, scores_out=None, idx_out=None, events=None, dims=None, out=None, lse=None):
+    """decode_step over a device-resident ``DSAInputs``; returns (out, lse)."""
+    dims = dims or dims_of(inp)
+    if ws is None:
+        ws = make_workspace(dims, _lib.DSA_OP_DECODE, inp.device)
+    if out is None:
+        out, lse = alloc_outputs(inp)
+    return decode_step(dims, inp.q_I, inp.q_scale, inp.w, inp.k_I, inp.k_scale, inp.q, inp.kv, inp.q_seq, inp.q_len,
+                       inp.softmax_scale, out, lse, ws, scores_out=scores_out, idx_out=idx_out, events=events)

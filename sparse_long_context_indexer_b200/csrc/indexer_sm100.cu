@@ -1,0 +1,335 @@
+// indexer_sm100.cu -- lightning-indexer scores on the sm_100a tensor cores.
+//
+// What it computes ("DeepSeek Sparse Attention Explained", section "How Does
+// the Lightning Indexer Score a Token?"; "DeepSeek V3.2-Exp Cuts Long-Context
+// Costs", "How DSA works": FP8, a few small heads, ReLU):
+//   I[t,s] = k_scale[s] * sum_j (w[t,j] * q_scale[t,j]) * ReLU(sum_x q8[t,j,x] k8[s,x])
+// which equals sum_j w[t,j] ReLU(q[t,j] . k[s]) with q = q8*q_scale, k = k8*k_scale
+// because both scales are positive and ReLU(c x) = c ReLU(x) for c > 0.
+//
+// Shape of the work: for one query row, [H_I x d_I] . [d_I x n] is a dense
+// FP8 contraction.  A tile is 128 cached tokens (MMA M = 128) against the 64
+// heads of one query (MMA N = 64), K = d_I, accumulated in fp32 in tensor
+// memory.  The epilogue reads one token row per thread from TMEM, applies
+// ReLU, the weighted head sum and the key scale, and writes one fp32 score:
+// per-head products never leave the chip.
+//
+// Roles (one persistent CTA per SM, each owning a contiguous range of the
+// flat list of (query row, key tile) pairs):
+//   warp 0       TMA producer: key tiles (8-stage ring) and the query's q8 block
+//   warp 1       TMEM allocator and single-thread tcgen05.mma issuer
+//   warps 2..5   epilogue group 0 (even tiles), warps 6..9 group 1 (odd tiles)
+// Every wait is bounded; a timeout records DSA_ERR_TIMEOUT and the CTA drains
+// and exits instead of hanging.
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include "kernels.h"
+#include "ptx.cuh"
+
+namespace dsa {
+namespace {
+
+template <int D_I>
+struct IdxCfg {
+    static constexpr int TILE = kIdxTile;
+    static constexpr int HEADS = kIdxHeads;
+    static constexpr int STAGES = 8;
+    static constexpr int KTILE_BYTES = TILE * D_I;
+    static constexpr int Q_BYTES = HEADS * D_I;
+    static constexpr uint32_t SWZ = D_I == 64 ? kSwizzle64B : kSwizzle128B;
+    static constexpr uint32_t SBO = 8 * D_I;  // 8-row swizzle atom
+    static constexpr int ACC = 4;             // TMEM accumulator buffers of HEADS columns
+    static constexpr int TMEM_COLS = 256;
+    static constexpr int THREADS = 320;
+    static constexpr int K_STEPS = D_I / 32;  // kind::f8f6f4 consumes 32 bytes of K per MMA
+    // shared memory map (offsets from a 1024-byte aligned base)
+    static constexpr int OFF_K = 0;
+    static constexpr int OFF_Q = OFF_K + STAGES * KTILE_BYTES;
+    static constexpr int OFF_BAR = OFF_Q + 2 * Q_BYTES;
+    static constexpr int NBAR = 2 * STAGES + 4 + 2 * ACC;
+    static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
+    static constexpr int SMEM_BYTES = OFF_MISC + 64 + 1024;  // + alignment slack
+    static constexpr uint32_t IDESC = make_idesc(TILE, HEADS, 0 /*e4m3*/, 0 /*e4m3*/, 0, 0);
+};
+
+struct IdxShared {
+    int row0, j0, count;
+    int tmem_base;
+    int abort_flag;
+};
+
+// Number of key tiles of query row r (0 for rows with invalid sizes).
+__device__ __forceinline__ int row_tiles(const IndexerArgs& a, int r) {
+    const int n = a.q_len[r];
+    const int b = a.q_seq[r];
+    if (n < 0 || n > a.T_max || (int64_t)n > a.ld || b < 0 || b >= a.B) return 0;
+    return (n + kIdxTile - 1) / kIdxTile;
+}
+
+// Walks the flat (row, tile) list.
+struct TileCursor {
+    int row, j, nt;
+    __device__ void start(const IndexerArgs& a, int r0, int j0) {
+        row = r0;
+        j = j0;
+        nt = row < a.Nq ? row_tiles(a, row) : 0;
+    }
+    __device__ void advance(const IndexerArgs& a) {
+        if (++j >= nt) {
+            j = 0;
+            do {
+                ++row;
+                nt = row < a.Nq ? row_tiles(a, row) : 1;
+            } while (nt == 0);
+        }
+    }
+};
+
+template <int D_I>
+__global__ void __launch_bounds__(IdxCfg<D_I>::THREADS, 1)
+    indexer_fp8_kernel(const IndexerArgs a, const __grid_constant__ CUtensorMap tmap_k,
+                       const __grid_constant__ CUtensorMap tmap_q) {
+    using C = IdxCfg<D_I>;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    const uint32_t sbase = smem_u32(smem);
+    const uint32_t sK = sbase + C::OFF_K;
+    const uint32_t sQ = sbase + C::OFF_Q;
+    const uint32_t bar0 = sbase + C::OFF_BAR;
+    auto bar_full = [&](int s) { return bar0 + 8u * s; };
+    auto bar_empty = [&](int s) { return bar0 + 8u * (C::STAGES + s); };
+    auto bar_qfull = [&](int q) { return bar0 + 8u * (2 * C::STAGES + q); };
+    auto bar_qempty = [&](int q) { return bar0 + 8u * (2 * C::STAGES + 2 + q); };
+    auto bar_tfull = [&](int c) { return bar0 + 8u * (2 * C::STAGES + 4 + c); };
+    auto bar_tempty = [&](int c) { return bar0 + 8u * (2 * C::STAGES + 4 + C::ACC + c); };
+    IdxShared* sh = reinterpret_cast<IdxShared*>(smem + C::OFF_MISC);
+    volatile int* abort_flag = &sh->abort_flag;
+
+    const int tid = threadIdx.x;
+    const int warp = tid >> 5;
+    const int lane = tid & 31;
+
+    if (tid == 0) {
+        for (int s = 0; s < C::STAGES; ++s) {
+            mbar_init(bar_full(s), 1);
+            mbar_init(bar_empty(s), 1);
+        }
+        for (int q = 0; q < 2; ++q) {
+            mbar_init(bar_qfull(q), 1);
+            mbar_init(bar_qempty(q), 1);
+        }
+        for (int c = 0; c < C::ACC; ++c) {
+            mbar_init(bar_tfull(c), 1);
+            mbar_init(bar_tempty(c), 4);
+        }
+        sh->abort_flag = 0;
+        fence_barrier_init();
+        tma_prefetch_desc(&tmap_k);
+        tma_prefetch_desc(&tmap_q);
+    }
+    if (warp == 1) {
+        tmem_alloc(smem_u32(&sh->tmem_base), C::TMEM_COLS);
+        tmem_relinquish();
+    }
+    // Work range: this CTA's slice of the flat tile list (warp 2 scans the rows).
+    if (warp == 2) {
+        long long total = 0;
+        for (int base = 0; base < a.Nq; base += 32) {
+            const int r = base + lane;
+            int v = r < a.Nq ? row_tiles(a, r) : 0;
+            if (r < a.Nq && v == 0 && a.q_len[r] != 0 && blockIdx.x == 0) record_status(a.status, DSA_STATUS_LENGTH);
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+            total += v;
+        }
+        const long long begin = total * blockIdx.x / gridDim.x;
+        const long long end = total * (blockIdx.x + 1) / gridDim.x;
+        int row0 = a.Nq, j0 = 0;
+        long long run = 0;
+        for (int base = 0; base < a.Nq && row0 == a.Nq; base += 32) {
+            const int r = base + lane;
+            const int v = r < a.Nq ? row_tiles(a, r) : 0;
+            int incl = v;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const int u = __shfl_up_sync(0xffffffffu, incl, o);
+                if (lane >= o) incl += u;
+            }
+            const long long excl = run + incl - v;
+            const bool hit = v > 0 && excl <= begin && begin < excl + v;
+            const unsigned m = __ballot_sync(0xffffffffu, hit);
+            if (m) {
+                const int src = __ffs(m) - 1;
+                row0 = base + src;
+                j0 = (int)(begin - __shfl_sync(0xffffffffu, excl, src));
+            }
+            run += __shfl_sync(0xffffffffu, incl, 31);
+        }
+        if (lane == 0) {
+            sh->row0 = row0;
+            sh->j0 = j0;
+            sh->count = (int)(end - begin);
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = (uint32_t)sh->tmem_base;
+    const int count = sh->count;
+
+    if (warp == 0) {
+        if (lane == 0 && count > 0) {
+            // ---------------- TMA producer
+            TileCursor cur;
+            cur.start(a, sh->row0, sh->j0);
+            int qi = -1;
+            int issued = 0;
+            for (int it = 0; it < count; ++it) {
+                if (it == 0 || cur.j == 0) {
+                    ++qi;
+                    const int qb = qi & 1;
+                    if (qi >= 2 && !mbar_wait(bar_qempty(qb), ((qi - 2) >> 1) & 1, abort_flag, a.status)) break;
+                    mbar_arrive_expect_tx(bar_qfull(qb), C::Q_BYTES);
+                    tma_load_2d(sQ + qb * C::Q_BYTES, &tmap_q, 0, cur.row * C::HEADS, bar_qfull(qb));
+                }
+                const int st = it % C::STAGES;
+                if (it >= C::STAGES &&
+                    !mbar_wait(bar_empty(st), ((it / C::STAGES) - 1) & 1, abort_flag, a.status))
+                    break;
+                mbar_arrive_expect_tx(bar_full(st), C::KTILE_BYTES);
+                const int b = a.q_seq[cur.row];
+                tma_load_2d(sK + st * C::KTILE_BYTES, &tmap_k, 0, b * a.T_max + cur.j * C::TILE, bar_full(st));
+                ++issued;
+                cur.advance(a);
+            }
+            if (*abort_flag) {
+                // drain loads still in flight before the CTA's shared memory is released
+                for (int it = issued - C::STAGES < 0 ? 0 : issued - C::STAGES; it < issued; ++it)
+                    mbar_wait(bar_full(it % C::STAGES), (it / C::STAGES) & 1, nullptr, nullptr, 50000000ull);
+            }
+        }
+    } else if (warp == 1) {
+        if (lane == 0 && count > 0) {
+            // ---------------- MMA issuer
+            TileCursor cur;
+            cur.start(a, sh->row0, sh->j0);
+            int qi = -1, qb = 0;
+            int last_acc = -1, last_it = -1;
+            for (int it = 0; it < count; ++it) {
+                if (it == 0 || cur.j == 0) {
+                    ++qi;
+                    qb = qi & 1;
+                    if (!mbar_wait(bar_qfull(qb), (qi >> 1) & 1, abort_flag, a.status)) break;
+                }
+                const int st = it % C::STAGES;
+                if (!mbar_wait(bar_full(st), (it / C::STAGES) & 1, abort_flag, a.status)) break;
+                const int acc = it % C::ACC;
+                if (it >= C::ACC && !mbar_wait(bar_tempty(acc), ((it / C::ACC) - 1) & 1, abort_flag, a.status))
+                    break;
+                tc_fence_after();
+                const uint32_t d = tmem + acc * C::HEADS;
+                const uint32_t a_addr = sK + st * C::KTILE_BYTES;
+                const uint32_t b_addr = sQ + qb * C::Q_BYTES;
+#pragma unroll
+                for (int ks = 0; ks < C::K_STEPS; ++ks) {
+                    const uint64_t ad = make_smem_desc(a_addr + ks * 32, 16, C::SBO, C::SWZ);
+                    const uint64_t bd = make_smem_desc(b_addr + ks * 32, 16, C::SBO, C::SWZ);
+                    mma_f8f6f4_ss(d, ad, bd, C::IDESC, ks > 0 ? 1u : 0u);
+                }
+                mma_commit(bar_empty(st));
+                mma_commit(bar_tfull(acc));
+                last_acc = acc;
+                last_it = it;
+                if (cur.j == cur.nt - 1 || it == count - 1) mma_commit(bar_qempty(qb));
+                cur.advance(a);
+            }
+            if (*abort_flag && last_it >= 0)
+                mbar_wait(bar_tfull(last_acc), (last_it / C::ACC) & 1, nullptr, nullptr, 50000000ull);
+        }
+    } else {
+        // ---------------- epilogue: one token row per thread
+        const int g = (warp - 2) >> 2;  // epilogue group
+        const int sub = warp & 3;       // TMEM sub-partition this warp may access
+        const int m = sub * 32 + lane;  // token row inside the tile
+        TileCursor cur;
+        if (count > 0) cur.start(a, sh->row0, sh->j0);
+        float wq[C::HEADS];
+        int cur_row = -1, b = 0, n = 0;
+        for (int it = 0; it < count; ++it, cur.advance(a)) {
+            if ((it & 1) != g) continue;
+            if (cur.row != cur_row) {
+                cur_row = cur.row;
+                b = a.q_seq[cur_row];
+                n = a.q_len[cur_row];
+                const __nv_bfloat16* wr = reinterpret_cast<const __nv_bfloat16*>(a.w) + (int64_t)cur_row * C::HEADS;
+                const float* qs = a.q_scale + (int64_t)cur_row * C::HEADS;
+#pragma unroll
+                for (int j = 0; j < C::HEADS; ++j) wq[j] = __bfloat162float(wr[j]) * qs[j];
+            }
+            const int s = cur.j * C::TILE + m;
+            const float ks = s < n ? a.k_scale[(int64_t)b * a.T_max + s] : 0.f;
+            const int acc = it % C::ACC;
+            if (!mbar_wait(bar_tfull(acc), (it / C::ACC) & 1, abort_flag, a.status)) break;
+            tc_fence_after();
+            uint32_t v0[32], v1[32];
+            const uint32_t taddr = tmem + ((uint32_t)(sub * 32) << 16) + acc * C::HEADS;
+            tmem_ld32(taddr, v0);
+            tmem_ld32(taddr + 32, v1);
+            tmem_wait_ld();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(bar_tempty(acc));
+            float p0 = 0.f, p1 = 0.f, p2 = 0.f, p3 = 0.f;
+#pragma unroll
+            for (int j = 0; j < 32; j += 4) {
+                p0 = fmaf(wq[j + 0], fmaxf(__uint_as_float(v0[j + 0]), 0.f), p0);
+                p1 = fmaf(wq[j + 1], fmaxf(__uint_as_float(v0[j + 1]), 0.f), p1);
+                p2 = fmaf(wq[j + 2], fmaxf(__uint_as_float(v0[j + 2]), 0.f), p2);
+                p3 = fmaf(wq[j + 3], fmaxf(__uint_as_float(v0[j + 3]), 0.f), p3);
+            }
+#pragma unroll
+            for (int j = 0; j < 32; j += 4) {
+                p0 = fmaf(wq[32 + j + 0], fmaxf(__uint_as_float(v1[j + 0]), 0.f), p0);
+                p1 = fmaf(wq[32 + j + 1], fmaxf(__uint_as_float(v1[j + 1]), 0.f), p1);
+                p2 = fmaf(wq[32 + j + 2], fmaxf(__uint_as_float(v1[j + 2]), 0.f), p2);
+                p3 = fmaf(wq[32 + j + 3], fmaxf(__uint_as_float(v1[j + 3]), 0.f), p3);
+            }
+            if (s < n) a.scores[(int64_t)cur_row * a.ld + s] = ks * ((p0 + p1) + (p2 + p3));
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem, C::TMEM_COLS);
+    }
+}
+
+template <int D_I>
+cudaError_t launch_fp8_impl(const IndexerArgs& a, int grid, cudaStream_t st) {
+    using C = IdxCfg<D_I>;
+    alignas(64) CUtensorMap tk, tq;
+    const int swz = D_I;  // 64-byte rows -> 64B swizzle, 128-byte rows -> 128B swizzle
+    if (!encode_tensor_map_2d(&tk, 1, a.k_I, D_I, (uint64_t)a.B * a.T_max, D_I, D_I, C::TILE, swz))
+        return cudaErrorInvalidValue;
+    if (!encode_tensor_map_2d(&tq, 1, a.q_I, D_I, (uint64_t)a.Nq * C::HEADS, D_I, D_I, C::HEADS, swz))
+        return cudaErrorInvalidValue;
+    auto kern = indexer_fp8_kernel<D_I>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
+    if (e != cudaSuccess) return e;
+    kern<<<grid, C::THREADS, C::SMEM_BYTES, st>>>(a, tk, tq);
+    return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_indexer_fp8(const IndexerArgs& a, int grid, cudaStream_t st) {
+    if (a.Nq == 0) return cudaSuccess;
+    if (a.d_I == 64) return launch_fp8_impl<64>(a, grid, st);
+    if (a.d_I == 128) return launch_fp8_impl<128>(a, grid, st);
+    return cudaErrorInvalidValue;
+}
+
+}  // namespace dsa

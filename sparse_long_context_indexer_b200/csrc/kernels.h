@@ -1,0 +1,71 @@
+// kernels.h -- host-side launch interface between the C ABI (dsa_api.cu) and
+// the kernel translation units.  Not installed; no torch types anywhere.
+#pragma once
+#include <cstddef>
+#include <cstdint>
+#include <cuda_runtime.h>
+
+namespace dsa {
+
+constexpr int kDK = 576;   // latent key width (512 latent + 64 rope)
+constexpr int kDV = 512;   // value width
+constexpr int kIdxTile = 128;  // indexer: cached tokens per tensor-core tile (MMA M)
+constexpr int kIdxHeads = 64;  // indexer: heads per query (MMA N) for the FP8 kernel
+constexpr int kMlaTile = 32;   // sparse MLA: gathered rows per tile (MMA N of Q K^T)
+constexpr int kMlaHeads = 128; // sparse MLA bf16 kernel: query heads (MMA M)
+
+struct IndexerArgs {
+    const void* q_I;
+    const float* q_scale;
+    const void* w;
+    const void* k_I;
+    const float* k_scale;
+    const int32_t* q_seq;
+    const int32_t* q_len;
+    float* scores;
+    int64_t ld;
+    int Nq, B, T_max, H_I, d_I;
+    int* status;
+};
+
+struct TopkArgs {
+    const float* scores;
+    int64_t ld;
+    const int32_t* q_len;
+    int32_t* idx;
+    int Nq, k, T_max;
+    int* status;
+};
+
+struct MlaArgs {
+    const void* q;
+    const void* kv;
+    const int32_t* idx;
+    const int32_t* q_seq;
+    const int32_t* q_len;
+    void* out;
+    float* lse;
+    float* part_o;    // [splits, Nq, H, 512] when splits > 1
+    float* part_lse;  // [splits, Nq, H]
+    int Nq, B, T_max, k, H;
+    int splits, rows_per_split;
+    float softmax_scale;
+    int* status;
+};
+
+cudaError_t launch_indexer_fp8(const IndexerArgs& a, int grid, cudaStream_t st);
+cudaError_t launch_indexer_f32(const IndexerArgs& a, cudaStream_t st);
+cudaError_t launch_topk(const TopkArgs& a, int cluster, cudaStream_t st);
+cudaError_t launch_sparse_mla_bf16(const MlaArgs& a, cudaStream_t st);
+cudaError_t launch_mla_combine(const MlaArgs& a, cudaStream_t st);
+cudaError_t launch_sparse_mla_f32(const MlaArgs& a, cudaStream_t st);
+cudaError_t launch_wait_timeout_selftest(int* status, int timeout_us, cudaStream_t st);
+
+// Largest row chunk kept in shared memory by one top-k CTA (elements).
+constexpr int kTopkSmemKeys = 49152;
+
+// cuTensorMapEncodeTiled through the runtime's driver entry point (no -lcuda).
+bool encode_tensor_map_2d(void* map, int dtype_bytes, const void* base, uint64_t inner, uint64_t outer,
+                          uint64_t row_stride_bytes, uint32_t box_inner, uint32_t box_outer, int swizzle_bytes);
+
+}  // namespace dsa

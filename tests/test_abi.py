@@ -1,0 +1,103 @@
+"""The C library: builds, loads, exports every symbol include/dsa.h declares,
+plans workspaces and rejects bad arguments on the host (no GPU needed)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from sparse_long_context_indexer_b200 import _lib, api, build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    build.build()
+    return _lib.load()
+
+
+def header_functions():
+    src = open(os.path.join(ROOT, "include", "dsa.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(dsa_[a-z_0-9]+)\s*\(", src)))
+
+
+def test_header_declares_the_boundary():
+    names = header_functions()
+    for required in ("dsa_indexer_scores", "dsa_topk", "dsa_sparse_mla_attn", "dsa_decode_step", "dsa_prefill"):
+        assert required in names
+    assert set(names) == set(_lib.EXPORTS)
+
+
+def test_library_exports_every_declared_symbol(lib):
+    for name in header_functions():
+        assert hasattr(lib, name), name
+        assert ctypes.cast(getattr(lib, name), ctypes.c_void_p).value
+
+
+def test_version_and_status_strings(lib):
+    assert b"sm_100a" in lib.dsa_version()
+    for code in range(8):
+        assert lib.dsa_status_string(code)
+
+
+def decode_dims(**kw):
+    d = dict(B=16, Nq=16, H_I=64, d_I=64, H=128, k=2048, T_max=131072, idx_dtype=_lib.DSA_FP8_E4M3,
+             kv_dtype=_lib.DSA_BF16, ld_scores=131072)
+    d.update(kw)
+    return api.Dims(**d)
+
+
+def test_workspace_sizes(lib):
+    d = decode_dims()
+    ws = api.workspace_size(d, _lib.DSA_OP_DECODE)
+    assert ws >= 16 * 131072 * 4 + 16 * 2048 * 4
+    assert api.workspace_size(d, _lib.DSA_OP_INDEXER) == 256
+    assert api.workspace_size(d, _lib.DSA_OP_TOPK) == 256
+    pre = api.workspace_size(decode_dims(B=1, Nq=65536, T_max=65536, ld_scores=65536), _lib.DSA_OP_PREFILL)
+    assert pre <= (64 << 20) + (16 << 20), "prefill works in L2-sized row chunks"
+
+
+@pytest.mark.parametrize("bad,code", [
+    (dict(d_I=96), _lib.DSA_ERR_UNSUPPORTED),
+    (dict(H_I=32), _lib.DSA_ERR_UNSUPPORTED),
+    (dict(H=64), _lib.DSA_ERR_UNSUPPORTED),
+    (dict(k=4096), _lib.DSA_ERR_UNSUPPORTED),
+    (dict(k=0), _lib.DSA_ERR_INVALID_ARG),
+    (dict(ld_scores=131071), _lib.DSA_ERR_INVALID_ARG),
+    (dict(idx_dtype=7), _lib.DSA_ERR_INVALID_ARG),
+])
+def test_bad_dims_rejected(lib, bad, code):
+    d = decode_dims(**bad).c()
+    n = ctypes.c_size_t(0)
+    assert lib.dsa_workspace_size(ctypes.byref(d), _lib.DSA_OP_DECODE, ctypes.byref(n)) == code
+
+
+def test_null_and_misaligned_pointers_rejected_before_launch(lib):
+    d = decode_dims().c()
+    P = 1 << 20
+    args = [P] * 9
+    # NULL q_I
+    rc = lib.dsa_decode_step(ctypes.byref(d), None, *args[1:], ctypes.c_float(0.07), P, P, None, None, P, 1 << 30,
+                             None, None)
+    assert rc == _lib.DSA_ERR_INVALID_ARG
+    # misaligned kv
+    bad = list(args)
+    bad[6] = P + 8  # kv
+    rc = lib.dsa_decode_step(ctypes.byref(d), *bad, ctypes.c_float(0.07), P, P, None, None, P, 1 << 30, None, None)
+    assert rc == _lib.DSA_ERR_INVALID_ARG
+    # workspace too small
+    rc = lib.dsa_decode_step(ctypes.byref(d), *args, ctypes.c_float(0.07), P, P, None, None, P, 1024, None, None)
+    assert rc == _lib.DSA_ERR_WORKSPACE
+    # non-finite softmax scale
+    rc = lib.dsa_decode_step(ctypes.byref(d), *args, ctypes.c_float(float("nan")), P, P, None, None, P, 1 << 30,
+                             None, None)
+    assert rc == _lib.DSA_ERR_INVALID_ARG
+
+
+def test_python_layer_has_no_compute_fallback():
+    """The binding marshals pointers only: no torch math on tensors in api.py."""
+    src = open(os.path.join(ROOT, "sparse_long_context_indexer_b200", "api.py")).read()
+    for forbidden in ("torch.topk", "torch.softmax", "torch.einsum", "torch.matmul", "@ ", "relu", "oracle"):
+        assert forbidden not in src, forbidden

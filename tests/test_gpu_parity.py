@@ -1,0 +1,260 @@
+"""CUDA path vs the CPU oracle, stage by stage and end to end (needs a B200).
+
+Inputs come from the seeded generator only; no oracle input is ever taken from
+the CUDA path.  Top-k is checked bit-exact on identical score buffers drawn by
+the generator; attention is checked on index lists chosen by the oracle.
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from sparse_long_context_indexer_b200 import _lib, api, inputs
+from tests.tolerances import check_attention, check_scores, check_sets
+
+pytestmark = pytest.mark.gpu
+
+SMALL_LENS = [4097, 2500, 777, 2048, 2049, 129, 1]
+
+
+@pytest.fixture(scope="module")
+def lib():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    return _lib.load()
+
+
+def small_decode(seed=11, lens=SMALL_LENS, k=2048, fp8=True, H_I=64, d_I=64, H=128):
+    return inputs.make_decode_inputs(f"small_{seed}", lens, H_I=H_I, d_I=d_I, H=H, k=k, fp8=fp8,
+                                     T_max=max(128, (max(lens) + 127) // 128 * 128), anchor_frac=0.01, seed=seed)
+
+
+def np_scores(t):
+    return t.detach().cpu().numpy()
+
+
+# ------------------------------------------------------------------ top-k
+
+def random_scores(rows, ld, seed, ties=True):
+    g = torch.Generator().manual_seed(seed)
+    sc = torch.randn((rows, ld), generator=g)
+    if ties:
+        sc = torch.round(sc * 16) / 16          # many exact ties
+        z = torch.rand((rows, ld), generator=g) < 0.05
+        sc[z] = 0.0
+        negz = torch.rand((rows, ld), generator=g) < 0.5
+        sc[z & negz] = -0.0
+    return sc.float()
+
+
+@pytest.mark.parametrize("lens,k", [
+    ([0, 1, 100, 2047, 2048, 2049, 5000, 40000, 131072], 2048),
+    ([131072] * 16, 2048),
+    ([60000] * 64, 2048),
+    ([30000] * 300, 2048),
+    ([4096], 256),
+    ([1048576, 300000], 2048),
+    ([9000, 9001, 9002, 9003], 1),
+    ([50000], 2000),
+])
+def test_topk_bit_exact_on_identical_scores(lib, lens, k):
+    ld = (max(lens) + 3) // 4 * 4
+    sc = random_scores(len(lens), ld, seed=len(lens) + k, ties=True)
+    q_len = torch.tensor(lens, dtype=torch.int32)
+    want = oracle.topk(sc.double().numpy(), q_len.numpy(), k)
+    dims = api.Dims(B=1, Nq=len(lens), H_I=64, d_I=64, H=128, k=k, T_max=ld, idx_dtype=2, kv_dtype=1, ld_scores=ld)
+    ws = api.make_workspace(dims, _lib.DSA_OP_TOPK)
+    idx = torch.full((len(lens), k), -7, dtype=torch.int32, device="cuda")
+    api.topk(dims, sc.cuda(), q_len.cuda(), idx, ws)
+    torch.cuda.synchronize()
+    assert api.get_device_status(ws) == 0
+    got = idx.cpu().numpy()
+    for t in range(len(lens)):
+        assert np.array_equal(got[t], want[t]), f"row {t} (n={lens[t]}): first diff at {np.argmax(got[t] != want[t])}"
+
+
+def test_topk_all_equal_scores_take_lowest_positions(lib):
+    n, k = 70000, 2048
+    sc = torch.full((2, n), 0.25)
+    sc[1, ::3] = -0.0
+    sc[1, 1::3] = 0.0
+    sc[1, 2::3] = -1.0
+    dims = api.Dims(B=1, Nq=2, H_I=64, d_I=64, H=128, k=k, T_max=n, idx_dtype=2, kv_dtype=1, ld_scores=n)
+    ws = api.make_workspace(dims, _lib.DSA_OP_TOPK)
+    idx = torch.empty((2, k), dtype=torch.int32, device="cuda")
+    api.topk(dims, sc.cuda(), torch.tensor([n, n], dtype=torch.int32, device="cuda"), idx, ws)
+    got = idx.cpu().numpy()
+    assert np.array_equal(got[0], np.arange(k))
+    want = oracle.topk(sc.double().numpy(), [n, n], k)
+    assert np.array_equal(got[1], want[1])
+
+
+# ------------------------------------------------------------------ indexer
+
+@pytest.mark.parametrize("d_I", [64, 128])
+def test_indexer_fp8_matches_oracle(lib, d_I):
+    inp = small_decode(seed=5 + d_I, d_I=d_I)
+    ora = oracle.indexer(inp, ld=inp.T_max)
+    g = inp.to("cuda")
+    dims = api.dims_of(g)
+    ws = api.make_workspace(dims, _lib.DSA_OP_INDEXER)
+    scores = torch.full((g.Nq, dims.ld_scores), float("nan"), device="cuda")
+    api.indexer_scores(dims, g.q_I, g.q_scale, g.w, g.k_I, g.k_scale, g.q_seq, g.q_len, scores, ws)
+    torch.cuda.synchronize()
+    assert api.get_device_status(ws) == 0
+    got = np_scores(scores)
+    check_scores(got, ora, inp.q_len.numpy())
+    for t, n in enumerate(inp.q_len.tolist()):   # entries past q_len untouched
+        assert np.all(np.isnan(got[t, n:]))
+
+
+def test_indexer_f32_tiny_matches_oracle(lib):
+    inp = inputs.tiny()
+    ora = oracle.indexer(inp, ld=inp.T_max)
+    g = inp.to("cuda")
+    dims = api.dims_of(g)
+    scores = torch.empty((1, dims.ld_scores), device="cuda")
+    api.indexer_scores(dims, g.q_I, None, g.w, g.k_I, None, g.q_seq, g.q_len, scores)
+    check_scores(np_scores(scores), ora, inp.q_len.numpy())
+
+
+# ------------------------------------------------------------------ sparse attention on oracle-chosen rows
+
+@pytest.mark.parametrize("lens", [SMALL_LENS, [4096] * 16, [3000] * 40, [2100] * 3])
+def test_sparse_mla_matches_oracle_on_same_indices(lib, lens):
+    inp = small_decode(seed=21 + len(lens), lens=lens)
+    sc = oracle.indexer(inp, ld=inp.T_max)
+    idx = oracle.topk(sc, inp.q_len.numpy(), inp.k)
+    o_out, o_lse = oracle.sparse_attn(inp, idx)
+    g = inp.to("cuda")
+    dims = api.dims_of(g)
+    ws = api.make_workspace(dims, _lib.DSA_OP_SPARSE_MLA)
+    out, lse = api.alloc_outputs(g)
+    api.sparse_mla_attn(dims, g.q, g.kv, torch.from_numpy(idx).cuda(), g.q_seq, g.q_len, g.softmax_scale, out, lse, ws)
+    torch.cuda.synchronize()
+    assert api.get_device_status(ws) == 0
+    check_attention(out.float().cpu().numpy(), o_out, lse.cpu().numpy(), o_lse)
+
+
+def test_sparse_mla_random_index_sets_and_padding(lib):
+    inp = small_decode(seed=31, lens=[5000, 5000, 300, 0], k=2048)
+    rng = np.random.default_rng(0)
+    idx = np.full((4, 2048), -1, np.int32)
+    idx[0] = np.sort(rng.choice(5000, 2048, replace=False))
+    idx[1, :1000] = np.sort(rng.choice(5000, 1000, replace=False))   # ragged tail of -1
+    idx[2, :300] = np.arange(300)
+    o_out, o_lse = oracle.sparse_attn(inp, idx)
+    g = inp.to("cuda")
+    dims = api.dims_of(g)
+    ws = api.make_workspace(dims, _lib.DSA_OP_SPARSE_MLA)
+    out, lse = api.alloc_outputs(g)
+    api.sparse_mla_attn(dims, g.q, g.kv, torch.from_numpy(idx).cuda(), g.q_seq, g.q_len, g.softmax_scale, out, lse, ws)
+    torch.cuda.synchronize()
+    check_attention(out.float().cpu().numpy(), o_out, lse.cpu().numpy(), o_lse)
+    assert torch.all(out[3] == 0) and torch.all(torch.isneginf(lse[3]))
+
+
+def test_sparse_mla_f32_tiny(lib):
+    inp = inputs.tiny()
+    sc = oracle.indexer(inp, ld=inp.T_max)
+    idx = oracle.topk(sc, inp.q_len.numpy(), inp.k)
+    o_out, o_lse = oracle.sparse_attn(inp, idx)
+    g = inp.to("cuda")
+    dims = api.dims_of(g)
+    ws = api.make_workspace(dims, _lib.DSA_OP_SPARSE_MLA)
+    out, lse = api.alloc_outputs(g)
+    api.sparse_mla_attn(dims, g.q, g.kv, torch.from_numpy(idx).cuda(), g.q_seq, g.q_len, g.softmax_scale, out, lse, ws)
+    torch.cuda.synchronize()
+    check_attention(out.cpu().numpy(), o_out, lse.cpu().numpy(), o_lse)
+
+
+# ------------------------------------------------------------------ end to end
+
+def run_decode_gpu(inp_gpu):
+    dims = api.dims_of(inp_gpu)
+    ws = api.make_workspace(dims, _lib.DSA_OP_DECODE)
+    scores = torch.empty((inp_gpu.Nq, dims.ld_scores), device="cuda")
+    idx = torch.empty((inp_gpu.Nq, inp_gpu.k), dtype=torch.int32, device="cuda")
+    out, lse = api.run_decode(inp_gpu, ws=ws, scores_out=scores, idx_out=idx, dims=dims)
+    torch.cuda.synchronize()
+    status = api.get_device_status(ws)
+    return scores, idx, out, lse, status
+
+
+@pytest.mark.parametrize("which", ["small", "tiny"])
+def test_decode_step_end_to_end(lib, which):
+    inp = small_decode(seed=41) if which == "small" else inputs.tiny()
+    sc_o, idx_o, out_o, lse_o = oracle.decode(inp)
+    scores, idx, out, lse, status = run_decode_gpu(inp.to("cuda"))
+    assert status == 0
+    check_scores(np_scores(scores), sc_o, inp.q_len.numpy())
+    same, total = check_sets(idx.cpu().numpy(), idx_o, sc_o, inp.q_len.numpy(), inp.k)
+    g_idx = idx.cpu().numpy()
+    rows = [t for t in range(inp.Nq) if np.array_equal(g_idx[t], idx_o[t])]
+    assert len(rows) >= max(1, total - 1), f"only {same}/{total} rows selected identical sets"
+    check_attention(out.float().cpu().numpy(), out_o, lse.cpu().numpy(), lse_o, rows=rows)
+
+
+def test_prefill_matches_oracle(lib):
+    L = 3000
+    inp = inputs.make_prefill_inputs("prefill_small", L, seed=7)
+    rows = np.r_[0:8, 1000:1004, 2040:2056, 2990:3000]
+    sub = inputs.make_prefill_inputs("prefill_small", L, seed=7, rows=rows.tolist())
+    sc_o, idx_o, out_o, lse_o = oracle.decode(sub)
+    g = inp.to("cuda")
+    dims = api.dims_of(g)
+    ws = api.make_workspace(dims, _lib.DSA_OP_PREFILL)
+    out, lse = api.alloc_outputs(g)
+    idx = torch.empty((L, g.k), dtype=torch.int32, device="cuda")
+    api.prefill(dims, g.q_I, g.q_scale, g.w, g.k_I, g.k_scale, g.q, g.kv, g.q_seq, g.q_len, g.softmax_scale,
+                out, lse, ws, idx_out=idx)
+    torch.cuda.synchronize()
+    assert api.get_device_status(ws) == 0
+    g_idx = idx.cpu().numpy()[rows]
+    check_sets(g_idx, idx_o, sc_o, sub.q_len.numpy(), sub.k)
+    same = [i for i in range(len(rows)) if np.array_equal(g_idx[i], idx_o[i])]
+    assert len(same) >= len(rows) - 2
+    check_attention(out.float().cpu().numpy()[rows], out_o, lse.cpu().numpy()[rows], lse_o, rows=same)
+    # rows t < k select every position <= t
+    for i, t in enumerate(rows):
+        if t + 1 <= g.k:
+            assert np.array_equal(g_idx[i][: t + 1], np.arange(t + 1)) and np.all(g_idx[i][t + 1:] == -1)
+
+
+# ------------------------------------------------------------------ device-side error reporting
+
+def test_out_of_range_index_is_reported_and_masked(lib):
+    inp = small_decode(seed=51, lens=[1000, 1000])
+    idx = np.full((2, 2048), -1, np.int32)
+    idx[0, :3] = [1, 5, 7]
+    idx[1, :3] = [2, 999, 1000]        # 1000 >= q_len
+    g = inp.to("cuda")
+    dims = api.dims_of(g)
+    ws = api.make_workspace(dims, _lib.DSA_OP_SPARSE_MLA)
+    out, lse = api.alloc_outputs(g)
+    api.sparse_mla_attn(dims, g.q, g.kv, torch.from_numpy(idx).cuda(), g.q_seq, g.q_len, g.softmax_scale, out, lse, ws)
+    assert api.get_device_status(ws) == _lib.DSA_ERR_INDEX_OOB
+    assert api.get_device_status(ws) == 0          # read clears it
+    idx_ok = idx.copy()
+    idx_ok[1, 2] = -1
+    o_out, o_lse = oracle.sparse_attn(inp, idx_ok)
+    check_attention(out.float().cpu().numpy(), o_out, lse.cpu().numpy(), o_lse)
+
+
+def test_length_beyond_cache_is_reported(lib):
+    inp = small_decode(seed=52, lens=[500, 600])
+    g = inp.to("cuda")
+    g.q_len = torch.tensor([500, g.T_max + 1], dtype=torch.int32, device="cuda")
+    scores, idx, out, lse, status = run_decode_gpu(g)
+    assert status == _lib.DSA_ERR_LENGTH
+
+
+def test_bounded_wait_times_out_with_status(lib):
+    dims = api.Dims(B=1, Nq=1, H_I=64, d_I=64, H=128, k=16, T_max=128, idx_dtype=2, kv_dtype=1, ld_scores=128)
+    ws = api.make_workspace(dims, _lib.DSA_OP_TOPK)
+    api.selftest_wait_timeout(ws, timeout_us=100000)
+    assert api.get_device_status(ws) == _lib.DSA_ERR_TIMEOUT
+    x = torch.ones(4, device="cuda") * 2       # the context is still usable
+    assert float(x.sum()) == 8.0

@@ -1,0 +1,73 @@
+"""Acceptance rules for CUDA-vs-oracle comparisons.
+
+Tolerances follow the stated targets for this path: indexer scores within 2e-2
+relative (given identical FP8 inputs), top-k indices bit-exact on identical
+score buffers, end-to-end selected sets differing only on entries whose oracle
+score lies within 1e-3 relative of the k-th threshold, and attention outputs
+within 2e-2 absolute / 1e-2 relative in bf16.
+"""
+import numpy as np
+
+SCORE_RTOL = 2e-2
+SCORE_FLOOR = 1e-2      # relative to the row's largest |score|, for scores that cancel to ~0
+SET_RTOL = 1e-3
+ATT_ATOL = 2e-2
+ATT_RTOL = 1e-2
+
+
+def check_scores(gpu, ora, q_len):
+    """gpu, ora: [Nq, ld]; only s < q_len[t] compared.  Returns worst normalised error."""
+    worst = 0.0
+    for t, n in enumerate(np.asarray(q_len)):
+        if n == 0:
+            continue
+        g = np.asarray(gpu[t, :n], np.float64)
+        o = np.asarray(ora[t, :n], np.float64)
+        tol = SCORE_RTOL * np.maximum(np.abs(o), SCORE_FLOOR * np.abs(o).max())
+        err = np.abs(g - o) / np.maximum(tol, 1e-300)
+        worst = max(worst, float(err.max()))
+        bad = np.where(err > 1.0)[0]
+        assert bad.size == 0, f"row {t}: {bad.size} scores off, first s={bad[0]} gpu={g[bad[0]]} oracle={o[bad[0]]}"
+    return worst
+
+
+def check_sets(gpu_idx, ora_idx, ora_scores, q_len, k):
+    """Selected sets may differ only on entries whose oracle score is within SET_RTOL of the k-th score.
+    Returns (rows with identical sets, total rows)."""
+    same = 0
+    for t, n in enumerate(np.asarray(q_len)):
+        g = np.asarray(gpu_idx[t])
+        o = np.asarray(ora_idx[t])
+        m = min(k, int(n))
+        assert np.all(g[m:] == -1), f"row {t}: padding wrong"
+        assert np.all(np.diff(g[:m]) > 0), f"row {t}: not strictly ascending"
+        assert g[:m].min(initial=0) >= 0 and g[:m].max(initial=-1) < n, f"row {t}: index out of range"
+        gs, os_ = set(g[:m].tolist()), set(o[:m].tolist())
+        if gs == os_:
+            same += 1
+            continue
+        sc = np.asarray(ora_scores[t, :n], np.float64)
+        tau = np.sort(sc)[::-1][m - 1]
+        lim = SET_RTOL * max(abs(tau), 1e-6 * np.abs(sc).max())
+        for s in gs ^ os_:
+            assert abs(sc[s] - tau) <= lim, f"row {t}: position {s} (score {sc[s]}) differs but tau={tau}"
+    return same, len(q_len)
+
+
+def check_attention(gpu_out, ora_out, gpu_lse=None, ora_lse=None, rows=None):
+    g = np.asarray(gpu_out, np.float64)
+    o = np.asarray(ora_out, np.float64)
+    if rows is not None:
+        g, o = g[rows], o[rows]
+    err = np.abs(g - o) - (ATT_ATOL + ATT_RTOL * np.abs(o))
+    worst = float(np.max(np.abs(g - o))) if g.size else 0.0
+    assert np.all(err <= 0), f"attention mismatch: max abs err {worst}"
+    if gpu_lse is not None:
+        gl = np.asarray(gpu_lse, np.float64)
+        ol = np.asarray(ora_lse, np.float64)
+        if rows is not None:
+            gl, ol = gl[rows], ol[rows]
+        both_inf = np.isneginf(gl) & np.isneginf(ol)
+        d = np.where(both_inf, 0.0, np.abs(gl - ol))
+        assert np.all(d <= 1e-2 + 1e-3 * np.abs(np.where(both_inf, 0, ol))), f"lse mismatch: {np.nanmax(d)}"
+    return worst
