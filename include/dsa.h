@@ -78,8 +78,8 @@ typedef enum {
 } dsa_op_t;
 
 /* Problem sizes.  Supported builds:
- *   idx_dtype DSA_FP8_E4M3: d_I in {64, 128}, H_I in {1..64}... exactly 64 for the tensor-core
- *                           kernel (H_I is the MMA N dimension); w is bfloat16.
+ *   idx_dtype DSA_FP8_E4M3: d_I in {64, 128}, H_I = 64 (the MMA N dimension of the
+ *                           tensor-core kernel), T_max a multiple of 4; w is bfloat16.
  *   idx_dtype DSA_F32:      d_I in {64, 128}, 1 <= H_I <= 64; w is float.
  *   kv_dtype  DSA_BF16:     H = 128 (MMA M dimension).
  *   kv_dtype  DSA_F32:      1 <= H <= 128.

@@ -44,6 +44,7 @@ dsa_status_t check_dims(const dsa_dims* d, bool need_indexer, bool need_mla, boo
         if (d->d_I != 64 && d->d_I != 128) return DSA_ERR_UNSUPPORTED;
         if (d->idx_dtype == DSA_FP8_E4M3) {
             if (d->H_I != dsa::kIdxHeads) return DSA_ERR_UNSUPPORTED;
+            if ((d->T_max & 3) != 0) return DSA_ERR_UNSUPPORTED;  // k_scale rows are fetched by TMA
         } else if (d->idx_dtype == DSA_F32) {
             if (d->H_I < 1 || d->H_I > 64) return DSA_ERR_UNSUPPORTED;
         } else {

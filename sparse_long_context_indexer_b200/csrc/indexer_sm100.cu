@@ -16,9 +16,14 @@
 //
 // Roles (one persistent CTA per SM, each owning a contiguous range of the
 // flat list of (query row, key tile) pairs):
-//   warp 0       TMA producer: key tiles (8-stage ring) and the query's q8 block
+//   warp 0       producer: lane 0 issues the TMA copies of each key tile and of
+//                its 128 fp32 scales into a deep stage ring; at a new query row
+//                the warp writes the folded weights w*q_scale to shared memory
+//                and lane 0 fetches the row's q8 block by TMA
 //   warp 1       TMEM allocator and single-thread tcgen05.mma issuer
-//   warps 2..5   epilogue group 0 (even tiles), warps 6..9 group 1 (odd tiles)
+//   warps 2..17  epilogue, four groups of four warps taking every fourth tile,
+//                with eight TMEM accumulators so the tensor core and the four
+//                groups each run several tiles ahead of the slowest hand-off
 // Every wait is bounded; a timeout records DSA_ERR_TIMEOUT and the CTA drains
 // and exits instead of hanging.
 #include <cuda.h>
@@ -35,19 +40,24 @@ template <int D_I>
 struct IdxCfg {
     static constexpr int TILE = kIdxTile;
     static constexpr int HEADS = kIdxHeads;
-    static constexpr int STAGES = 8;
+    static constexpr int STAGES = D_I == 64 ? 16 : 10;
     static constexpr int KTILE_BYTES = TILE * D_I;
     static constexpr int Q_BYTES = HEADS * D_I;
     static constexpr uint32_t SWZ = D_I == 64 ? kSwizzle64B : kSwizzle128B;
-    static constexpr uint32_t SBO = 8 * D_I;  // 8-row swizzle atom
-    static constexpr int ACC = 4;             // TMEM accumulator buffers of HEADS columns
-    static constexpr int TMEM_COLS = 256;
-    static constexpr int THREADS = 320;
-    static constexpr int K_STEPS = D_I / 32;  // kind::f8f6f4 consumes 32 bytes of K per MMA
+    static constexpr uint32_t SBO = 8 * D_I;      // 8-row swizzle atom
+    static constexpr int ACC = 8;                 // TMEM accumulator buffers of HEADS columns
+    static constexpr int TMEM_COLS = 512;
+    static constexpr int GROUPS = 4;              // epilogue groups of four warps
+    static constexpr int EPI_WARP0 = 2;
+    static constexpr int THREADS = (EPI_WARP0 + 4 * GROUPS) * 32;
+    static constexpr int K_STEPS = D_I / 32;      // kind::f8f6f4 consumes 32 bytes of K per MMA
     // shared memory map (offsets from a 1024-byte aligned base)
     static constexpr int OFF_K = 0;
     static constexpr int OFF_Q = OFF_K + STAGES * KTILE_BYTES;
-    static constexpr int OFF_BAR = OFF_Q + 2 * Q_BYTES;
+    static constexpr int OFF_SC = OFF_Q + 2 * Q_BYTES;     // per-stage key scales (TILE fp32)
+    static constexpr int SC_BYTES = TILE * 4;
+    static constexpr int OFF_WQ = OFF_SC + STAGES * SC_BYTES;  // 2 x HEADS folded weights
+    static constexpr int OFF_BAR = OFF_WQ + 2 * HEADS * 4;
     static constexpr int NBAR = 2 * STAGES + 4 + 2 * ACC;
     static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
     static constexpr int SMEM_BYTES = OFF_MISC + 64 + 1024;  // + alignment slack
@@ -60,28 +70,39 @@ struct IdxShared {
     int abort_flag;
 };
 
-// Number of key tiles of query row r (0 for rows with invalid sizes).
-__device__ __forceinline__ int row_tiles(const IndexerArgs& a, int r) {
-    const int n = a.q_len[r];
-    const int b = a.q_seq[r];
+// Number of key tiles of a query row with length n in sequence b (0 when the sizes are invalid).
+__device__ __forceinline__ int tiles_of(const IndexerArgs& a, int n, int b) {
     if (n < 0 || n > a.T_max || (int64_t)n > a.ld || b < 0 || b >= a.B) return 0;
     return (n + kIdxTile - 1) / kIdxTile;
 }
+__device__ __forceinline__ int row_tiles(const IndexerArgs& a, int r) { return tiles_of(a, a.q_len[r], a.q_seq[r]); }
 
-// Walks the flat (row, tile) list.
+// Walks the flat (row, tile) list.  The row's sequence and length are read
+// once per row, never per tile: every issuing loop depends on them.
 struct TileCursor {
-    int row, j, nt;
+    int row, j, nt, b, n;
+    __device__ void load_row(const IndexerArgs& a) {
+        if (row < a.Nq) {
+            n = a.q_len[row];
+            b = a.q_seq[row];
+            nt = tiles_of(a, n, b);
+        } else {
+            n = 0;
+            b = 0;
+            nt = 1;  // sentinel past the last row
+        }
+    }
     __device__ void start(const IndexerArgs& a, int r0, int j0) {
         row = r0;
         j = j0;
-        nt = row < a.Nq ? row_tiles(a, row) : 0;
+        load_row(a);
     }
     __device__ void advance(const IndexerArgs& a) {
         if (++j >= nt) {
             j = 0;
             do {
                 ++row;
-                nt = row < a.Nq ? row_tiles(a, row) : 1;
+                load_row(a);
             } while (nt == 0);
         }
     }
@@ -90,13 +111,16 @@ struct TileCursor {
 template <int D_I>
 __global__ void __launch_bounds__(IdxCfg<D_I>::THREADS, 1)
     indexer_fp8_kernel(const IndexerArgs a, const __grid_constant__ CUtensorMap tmap_k,
-                       const __grid_constant__ CUtensorMap tmap_q) {
+                       const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__ CUtensorMap tmap_s) {
     using C = IdxCfg<D_I>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const uint32_t sbase = smem_u32(smem);
     const uint32_t sK = sbase + C::OFF_K;
     const uint32_t sQ = sbase + C::OFF_Q;
+    const uint32_t sS = sbase + C::OFF_SC;
+    const float* scale_smem = reinterpret_cast<const float*>(smem + C::OFF_SC);
+    float* wq_smem = reinterpret_cast<float*>(smem + C::OFF_WQ);
     const uint32_t bar0 = sbase + C::OFF_BAR;
     auto bar_full = [&](int s) { return bar0 + 8u * s; };
     auto bar_empty = [&](int s) { return bar0 + 8u * (C::STAGES + s); };
@@ -114,11 +138,11 @@ __global__ void __launch_bounds__(IdxCfg<D_I>::THREADS, 1)
     if (tid == 0) {
         for (int s = 0; s < C::STAGES; ++s) {
             mbar_init(bar_full(s), 1);
-            mbar_init(bar_empty(s), 1);
+            mbar_init(bar_empty(s), 5);  // MMA commit + the 4 epilogue warps that read the stage's scales
         }
         for (int q = 0; q < 2; ++q) {
-            mbar_init(bar_qfull(q), 1);
-            mbar_init(bar_qempty(q), 1);
+            mbar_init(bar_qfull(q), 1);                   // producer arrival with the q8 block's tx bytes
+            mbar_init(bar_qempty(q), 1 + 4 * C::GROUPS);  // MMA commit + every epilogue warp
         }
         for (int c = 0; c < C::ACC; ++c) {
             mbar_init(bar_tfull(c), 1);
@@ -128,6 +152,7 @@ __global__ void __launch_bounds__(IdxCfg<D_I>::THREADS, 1)
         fence_barrier_init();
         tma_prefetch_desc(&tmap_k);
         tma_prefetch_desc(&tmap_q);
+        tma_prefetch_desc(&tmap_s);
     }
     if (warp == 1) {
         tmem_alloc(smem_u32(&sh->tmem_base), C::TMEM_COLS);
@@ -180,8 +205,8 @@ __global__ void __launch_bounds__(IdxCfg<D_I>::THREADS, 1)
     const int count = sh->count;
 
     if (warp == 0) {
-        if (lane == 0 && count > 0) {
-            // ---------------- TMA producer
+        // ---------------- producer
+        if (count > 0) {
             TileCursor cur;
             cur.start(a, sh->row0, sh->j0);
             int qi = -1;
@@ -190,22 +215,35 @@ __global__ void __launch_bounds__(IdxCfg<D_I>::THREADS, 1)
                 if (it == 0 || cur.j == 0) {
                     ++qi;
                     const int qb = qi & 1;
-                    if (qi >= 2 && !mbar_wait(bar_qempty(qb), ((qi - 2) >> 1) & 1, abort_flag, a.status)) break;
-                    mbar_arrive_expect_tx(bar_qfull(qb), C::Q_BYTES);
-                    tma_load_2d(sQ + qb * C::Q_BYTES, &tmap_q, 0, cur.row * C::HEADS, bar_qfull(qb));
+                    if (qi >= 2) {
+                        const bool okq = mbar_wait(bar_qempty(qb), ((qi - 2) >> 1) & 1, abort_flag, a.status);
+                        if (!__all_sync(0xffffffffu, okq)) break;
+                    }
+                    const int64_t o = (int64_t)cur.row * C::HEADS;
+                    const __nv_bfloat16* wr = reinterpret_cast<const __nv_bfloat16*>(a.w) + o;
+                    wq_smem[qb * C::HEADS + lane] = __bfloat162float(wr[lane]) * a.q_scale[o + lane];
+                    wq_smem[qb * C::HEADS + 32 + lane] = __bfloat162float(wr[32 + lane]) * a.q_scale[o + 32 + lane];
+                    __syncwarp();
+                    if (lane == 0) {
+                        mbar_arrive_expect_tx(bar_qfull(qb), C::Q_BYTES);
+                        tma_load_2d(sQ + qb * C::Q_BYTES, &tmap_q, 0, cur.row * C::HEADS, bar_qfull(qb));
+                    }
                 }
                 const int st = it % C::STAGES;
-                if (it >= C::STAGES &&
-                    !mbar_wait(bar_empty(st), ((it / C::STAGES) - 1) & 1, abort_flag, a.status))
-                    break;
-                mbar_arrive_expect_tx(bar_full(st), C::KTILE_BYTES);
-                const int b = a.q_seq[cur.row];
-                tma_load_2d(sK + st * C::KTILE_BYTES, &tmap_k, 0, b * a.T_max + cur.j * C::TILE, bar_full(st));
+                if (it >= C::STAGES) {
+                    const bool oke = mbar_wait(bar_empty(st), ((it / C::STAGES) - 1) & 1, abort_flag, a.status);
+                    if (!__all_sync(0xffffffffu, oke)) break;
+                }
+                if (lane == 0) {
+                    mbar_arrive_expect_tx(bar_full(st), C::KTILE_BYTES + C::SC_BYTES);
+                    tma_load_2d(sK + st * C::KTILE_BYTES, &tmap_k, 0, cur.b * a.T_max + cur.j * C::TILE, bar_full(st));
+                    tma_load_2d(sS + st * C::SC_BYTES, &tmap_s, cur.j * C::TILE, cur.b, bar_full(st));
+                }
                 ++issued;
                 cur.advance(a);
             }
-            if (*abort_flag) {
-                // drain loads still in flight before the CTA's shared memory is released
+            if (lane == 0 && *abort_flag) {
+                // drain copies still in flight before the CTA's shared memory is released
                 for (int it = issued - C::STAGES < 0 ? 0 : issued - C::STAGES; it < issued; ++it)
                     mbar_wait(bar_full(it % C::STAGES), (it / C::STAGES) & 1, nullptr, nullptr, 50000000ull);
             }
@@ -250,53 +288,73 @@ __global__ void __launch_bounds__(IdxCfg<D_I>::THREADS, 1)
         }
     } else {
         // ---------------- epilogue: one token row per thread
-        const int g = (warp - 2) >> 2;  // epilogue group
-        const int sub = warp & 3;       // TMEM sub-partition this warp may access
-        const int m = sub * 32 + lane;  // token row inside the tile
+        const int g = (warp - C::EPI_WARP0) >> 2;  // epilogue group: tiles it with it % GROUPS == g
+        const int sub = warp & 3;                  // TMEM sub-partition this warp may access
+        const int m = sub * 32 + lane;             // token row inside the tile
         TileCursor cur;
         if (count > 0) cur.start(a, sh->row0, sh->j0);
-        float wq[C::HEADS];
-        int cur_row = -1, b = 0, n = 0;
-        for (int it = 0; it < count; ++it, cur.advance(a)) {
-            if ((it & 1) != g) continue;
-            if (cur.row != cur_row) {
-                cur_row = cur.row;
-                b = a.q_seq[cur_row];
-                n = a.q_len[cur_row];
-                const __nv_bfloat16* wr = reinterpret_cast<const __nv_bfloat16*>(a.w) + (int64_t)cur_row * C::HEADS;
-                const float* qs = a.q_scale + (int64_t)cur_row * C::HEADS;
-#pragma unroll
-                for (int j = 0; j < C::HEADS; ++j) wq[j] = __bfloat162float(wr[j]) * qs[j];
+        int qi = -1, qb = 0, n = 0;
+        const float* wq = wq_smem;
+        for (int it = 0; it < count; ++it) {
+            const bool seg_start = it == 0 || cur.j == 0;
+            const bool seg_end = cur.j == cur.nt - 1 || it == count - 1;
+            if (seg_start) {
+                ++qi;
+                qb = qi & 1;
+                n = cur.n;
             }
-            const int s = cur.j * C::TILE + m;
-            const float ks = s < n ? a.k_scale[(int64_t)b * a.T_max + s] : 0.f;
-            const int acc = it % C::ACC;
-            if (!mbar_wait(bar_tfull(acc), (it / C::ACC) & 1, abort_flag, a.status)) break;
-            tc_fence_after();
-            uint32_t v0[32], v1[32];
-            const uint32_t taddr = tmem + ((uint32_t)(sub * 32) << 16) + acc * C::HEADS;
-            tmem_ld32(taddr, v0);
-            tmem_ld32(taddr + 32, v1);
-            tmem_wait_ld();
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(bar_tempty(acc));
-            float p0 = 0.f, p1 = 0.f, p2 = 0.f, p3 = 0.f;
+            if (it % C::GROUPS == g) {
+                {
+                    // folded weights of this row: published by the producer with the q8 block
+                    // (cannot move on before this warp releases the row at its end)
+                    const bool okq = mbar_wait(bar_qfull(qb), (qi >> 1) & 1, abort_flag, a.status);
+                    if (!__all_sync(0xffffffffu, okq)) break;
+                    wq = wq_smem + qb * C::HEADS;
+                }
+                const int s = cur.j * C::TILE + m;
+                const int st = it % C::STAGES;
+                const int acc = it % C::ACC;
+                bool ok = mbar_wait(bar_tfull(acc), (it / C::ACC) & 1, abort_flag, a.status);
+                ok = ok && mbar_wait(bar_full(st), (it / C::STAGES) & 1, abort_flag, a.status);
+                if (!__all_sync(0xffffffffu, ok)) break;
+                const float ks = scale_smem[st * C::TILE + m];
+                tc_fence_after();
+                uint32_t v0[32], v1[32];
+                const uint32_t taddr = tmem + ((uint32_t)(sub * 32) << 16) + acc * C::HEADS;
+                tmem_ld32(taddr, v0);
+                tmem_ld32(taddr + 32, v1);
+                tmem_wait_ld();
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) {
+                    mbar_arrive(bar_tempty(acc));
+                    mbar_arrive(bar_empty(st));
+                }
+                float p0 = 0.f, p1 = 0.f, p2 = 0.f, p3 = 0.f;
 #pragma unroll
-            for (int j = 0; j < 32; j += 4) {
-                p0 = fmaf(wq[j + 0], fmaxf(__uint_as_float(v0[j + 0]), 0.f), p0);
-                p1 = fmaf(wq[j + 1], fmaxf(__uint_as_float(v0[j + 1]), 0.f), p1);
-                p2 = fmaf(wq[j + 2], fmaxf(__uint_as_float(v0[j + 2]), 0.f), p2);
-                p3 = fmaf(wq[j + 3], fmaxf(__uint_as_float(v0[j + 3]), 0.f), p3);
-            }
+                for (int j = 0; j < 32; j += 4) {
+                    const float4 w4 = *reinterpret_cast<const float4*>(wq + j);
+                    p0 = fmaf(w4.x, fmaxf(__uint_as_float(v0[j + 0]), 0.f), p0);
+                    p1 = fmaf(w4.y, fmaxf(__uint_as_float(v0[j + 1]), 0.f), p1);
+                    p2 = fmaf(w4.z, fmaxf(__uint_as_float(v0[j + 2]), 0.f), p2);
+                    p3 = fmaf(w4.w, fmaxf(__uint_as_float(v0[j + 3]), 0.f), p3);
+                }
 #pragma unroll
-            for (int j = 0; j < 32; j += 4) {
-                p0 = fmaf(wq[32 + j + 0], fmaxf(__uint_as_float(v1[j + 0]), 0.f), p0);
-                p1 = fmaf(wq[32 + j + 1], fmaxf(__uint_as_float(v1[j + 1]), 0.f), p1);
-                p2 = fmaf(wq[32 + j + 2], fmaxf(__uint_as_float(v1[j + 2]), 0.f), p2);
-                p3 = fmaf(wq[32 + j + 3], fmaxf(__uint_as_float(v1[j + 3]), 0.f), p3);
+                for (int j = 0; j < 32; j += 4) {
+                    const float4 w4 = *reinterpret_cast<const float4*>(wq + 32 + j);
+                    p0 = fmaf(w4.x, fmaxf(__uint_as_float(v1[j + 0]), 0.f), p0);
+                    p1 = fmaf(w4.y, fmaxf(__uint_as_float(v1[j + 1]), 0.f), p1);
+                    p2 = fmaf(w4.z, fmaxf(__uint_as_float(v1[j + 2]), 0.f), p2);
+                    p3 = fmaf(w4.w, fmaxf(__uint_as_float(v1[j + 3]), 0.f), p3);
+                }
+                if (s < n) a.scores[(int64_t)cur.row * a.ld + s] = ks * ((p0 + p1) + (p2 + p3));
             }
-            if (s < n) a.scores[(int64_t)cur_row * a.ld + s] = ks * ((p0 + p1) + (p2 + p3));
+            if (seg_end) {
+                // this warp is done with the row's folded weights
+                __syncwarp();
+                if (lane == 0) mbar_arrive(bar_qempty(qb));
+            }
+            cur.advance(a);
         }
     }
     tc_fence_before();
@@ -310,16 +368,18 @@ __global__ void __launch_bounds__(IdxCfg<D_I>::THREADS, 1)
 template <int D_I>
 cudaError_t launch_fp8_impl(const IndexerArgs& a, int grid, cudaStream_t st) {
     using C = IdxCfg<D_I>;
-    alignas(64) CUtensorMap tk, tq;
+    alignas(64) CUtensorMap tk, tq, ts;
     const int swz = D_I;  // 64-byte rows -> 64B swizzle, 128-byte rows -> 128B swizzle
     if (!encode_tensor_map_2d(&tk, 1, a.k_I, D_I, (uint64_t)a.B * a.T_max, D_I, D_I, C::TILE, swz))
         return cudaErrorInvalidValue;
     if (!encode_tensor_map_2d(&tq, 1, a.q_I, D_I, (uint64_t)a.Nq * C::HEADS, D_I, D_I, C::HEADS, swz))
         return cudaErrorInvalidValue;
+    if (!encode_tensor_map_2d(&ts, 4, a.k_scale, a.T_max, (uint64_t)a.B, (uint64_t)a.T_max * 4, C::TILE, 1, 0))
+        return cudaErrorInvalidValue;
     auto kern = indexer_fp8_kernel<D_I>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
     if (e != cudaSuccess) return e;
-    kern<<<grid, C::THREADS, C::SMEM_BYTES, st>>>(a, tk, tq);
+    kern<<<grid, C::THREADS, C::SMEM_BYTES, st>>>(a, tk, tq, ts);
     return cudaGetLastError();
 }
 

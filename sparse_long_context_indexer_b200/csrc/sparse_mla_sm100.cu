@@ -55,11 +55,13 @@ constexpr int kOffKv = kOffQ + kQBytes;
 constexpr int kOffBar = kOffKv + kStages * kKvStageBytes;
 constexpr int kNumBar = 1 + 2 * kStages + 2 + 2 + 1;  // q_full, kv_full[2], kv_empty[2], s_full[2], p_full[2], o_done
 constexpr int kOffMisc = kOffBar + kNumBar * 8;
-constexpr int kSmemBytes = kOffMisc + 64 + 1024;
+constexpr int kOffIdx = kOffMisc + 64;                   // up to 2048 staged positions
+constexpr int kSmemBytes = kOffIdx + 2048 * 4 + 1024;
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kColO = 0;     // O half: columns [0, 256)
 constexpr uint32_t kColS = 256;   // S/P buffers: [256, 288), [288, 320)
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
+constexpr int kPrefetchTiles = 4;          // L2 prefetch distance of the gather, in tiles
 constexpr uint32_t kIdescQK = make_idesc(kHeads, kTileRows, 1 /*bf16*/, 1 /*bf16*/, 0, 0);
 constexpr uint32_t kIdescPV = make_idesc(kHeads, 256, 1 /*bf16*/, 1 /*bf16*/, 0 /*A K-major*/, 1 /*B MN-major*/);
 
@@ -94,6 +96,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     auto bar_p_full = [&](int s) { return bar0 + 8u * (3 + 2 * kStages + s); };
     const uint32_t bar_o = bar0 + 8u * (5 + 2 * kStages);
     MlaShared* sh = reinterpret_cast<MlaShared*>(smem + kOffMisc);
+    int32_t* sidx = reinterpret_cast<int32_t*>(smem + kOffIdx);  // this split's positions, -1 = skip
     volatile int* abort_flag = &sh->abort_flag;
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -102,7 +105,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     // rows of idx handled by this split
     const int j_lo = split * a.rows_per_split;
     const int j_hi = min(a.k, j_lo + a.rows_per_split);
-    const int ntiles = j_hi > j_lo ? (j_hi - j_lo + kTileRows - 1) / kTileRows : 0;
+    const int nrows = max(0, j_hi - j_lo);
+    const int ntiles = (nrows + kTileRows - 1) / kTileRows;
     int n_t = a.q_len[t];
     const int b = a.q_seq[t];
     const bool row_ok = n_t >= 0 && n_t <= a.T_max && b >= 0 && b < a.B;
@@ -110,7 +114,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (split == 0 && half == 0 && tid == 0) record_status(a.status, DSA_STATUS_LENGTH);
         n_t = 0;
     }
-    const int32_t* idx_row = a.idx + (int64_t)t * a.k;
+    const __nv_bfloat16* kv_seq = reinterpret_cast<const __nv_bfloat16*>(a.kv) + (int64_t)b * a.T_max * kDK;
 
     if (tid == 0) {
         mbar_init(bar_q, 1);
@@ -123,11 +127,29 @@ __global__ void __launch_bounds__(kThreads, 1)
         mbar_init(bar_o, 1);
         sh->abort_flag = 0;
         fence_barrier_init();
-        tma_prefetch_desc(&tmap_q);
+        if (ntiles > 0) {
+            // the query block is needed first and does not depend on the staging below
+            mbar_arrive_expect_tx(bar_q, kQBytes);
+#pragma unroll 1
+            for (int c = 0; c < kChunks; ++c) tma_load_2d(sQ + c * kQChunkBytes, &tmap_q, c * 64, t * kHeads, bar_q);
+        }
     }
     if (warp == 4) {
         tmem_alloc(smem_u32(&sh->tmem_base), kTmemCols);
         tmem_relinquish();
+    }
+    // Stage this split's positions (sanitised: anything outside [0, n_t) becomes -1)
+    // and start pulling the first tiles' rows into L2: each CTA of the value pair
+    // prefetches one half of the rows, so every row leaves HBM once, early.
+    for (int r = tid; r < ntiles * kTileRows; r += kThreads) {
+        int s = r < nrows ? a.idx[(int64_t)t * a.k + j_lo + r] : -1;
+        if (s < -1 || s >= n_t) {
+            if (half == 0 && row_ok) record_status(a.status, DSA_STATUS_INDEX_OOB);
+            s = -1;
+        }
+        sidx[r] = s;
+        if (s >= 0 && (r & 1) == half && r < kPrefetchTiles * kTileRows)
+            l2_prefetch_bulk(kv_seq + (int64_t)s * kDK, kDK * 2);
     }
     tc_fence_before();
     __syncthreads();
@@ -137,48 +159,57 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (warp == 4) {
         // ------------------------------------------------ Q load + MMA issue
         if (lane == 0 && ntiles > 0) {
-            mbar_arrive_expect_tx(bar_q, kQBytes);
-#pragma unroll 1
-            for (int c = 0; c < kChunks; ++c) tma_load_2d(sQ + c * kQChunkBytes, &tmap_q, c * 64, t * kHeads, bar_q);
             bool ok = mbar_wait(bar_q, 0, abort_flag, a.status);
-            int issued_pv = -1;
-            auto issue_pv = [&](int j) -> bool {
-                const int sb = j & 1;
-                if (!mbar_wait(bar_p_full(sb), (j >> 1) & 1, abort_flag, a.status)) return false;
-                tc_fence_after();
-                const uint32_t v_base = sKv + sb * kKvStageBytes + (4 * half) * kKvChunkBytes;
+            // Issue in dependency order, whichever is ready first: QK^T(q) needs its
+            // gathered tile and PV(q-2) already issued (S/P buffer reuse); PV(p) needs
+            // the softmax of tile p.  PV is preferred: it frees a gather stage.
+            int qk = 0, pv = 0;
+            uint64_t t_last = globaltimer_ns();
+            uint32_t spins = 0;
+            while (ok && pv < ntiles) {
+                if (pv < qk && mbar_test(bar_p_full(pv & 1), (pv >> 1) & 1)) {
+                    tc_fence_after();
+                    const int sb = pv & 1;
+                    const uint32_t v_base = sKv + sb * kKvStageBytes + (4 * half) * kKvChunkBytes;
 #pragma unroll
-                for (int ks = 0; ks < 2; ++ks) {
-                    const uint64_t bd = make_smem_desc(v_base + ks * 2048, kKvChunkBytes, 1024, kSwizzle128B);
-                    mma_f16_ts(tmem + kColO, tmem + kColS + 32 * sb + 8 * ks, bd, kIdescPV,
-                               (j > 0 || ks > 0) ? 1u : 0u);
-                }
-                mma_commit(bar_kv_empty(sb));
-                issued_pv = j;
-                return true;
-            };
-            for (int i = 0; ok && i < ntiles; ++i) {
-                const int st = i & 1;
-                if (!mbar_wait(bar_kv_full(st), (i >> 1) & 1, abort_flag, a.status)) { ok = false; break; }
-                tc_fence_after();
-                const uint32_t d = tmem + kColS + 32 * st;
-                const uint32_t k_base = sKv + st * kKvStageBytes;
+                    for (int ks = 0; ks < 2; ++ks) {
+                        const uint64_t bd = make_smem_desc(v_base + ks * 2048, kKvChunkBytes, 1024, kSwizzle128B);
+                        mma_f16_ts(tmem + kColO, tmem + kColS + 32 * sb + 8 * ks, bd, kIdescPV,
+                                   (pv > 0 || ks > 0) ? 1u : 0u);
+                    }
+                    mma_commit(bar_kv_empty(sb));
+                    ++pv;
+                    t_last = globaltimer_ns();
+                } else if (qk < ntiles && qk <= pv + 1 && mbar_test(bar_kv_full(qk & 1), (qk >> 1) & 1)) {
+                    tc_fence_after();
+                    const int st = qk & 1;
+                    const uint32_t d = tmem + kColS + 32 * st;
+                    const uint32_t k_base = sKv + st * kKvStageBytes;
 #pragma unroll 1
-                for (int c = 0; c < kChunks; ++c) {
+                    for (int c = 0; c < kChunks; ++c) {
 #pragma unroll
-                    for (int kk = 0; kk < 4; ++kk) {
-                        const uint64_t ad = make_smem_desc(sQ + c * kQChunkBytes + kk * 32, 16, 1024, kSwizzle128B);
-                        const uint64_t bd = make_smem_desc(k_base + c * kKvChunkBytes + kk * 32, 16, 1024, kSwizzle128B);
-                        mma_f16_ss(d, ad, bd, kIdescQK, (c | kk) ? 1u : 0u);
+                        for (int kk = 0; kk < 4; ++kk) {
+                            const uint64_t ad = make_smem_desc(sQ + c * kQChunkBytes + kk * 32, 16, 1024, kSwizzle128B);
+                            const uint64_t bd = make_smem_desc(k_base + c * kKvChunkBytes + kk * 32, 16, 1024, kSwizzle128B);
+                            mma_f16_ss(d, ad, bd, kIdescQK, (c | kk) ? 1u : 0u);
+                        }
+                    }
+                    mma_commit(bar_s_full(st));
+                    ++qk;
+                    t_last = globaltimer_ns();
+                } else if ((++spins & 255u) == 0) {
+                    if (*abort_flag) {
+                        ok = false;
+                    } else if (globaltimer_ns() - t_last > kWaitBudgetNs) {
+                        record_status(a.status, DSA_STATUS_TIMEOUT);
+                        *abort_flag = 1;
+                        ok = false;
                     }
                 }
-                mma_commit(bar_s_full(st));
-                if (i >= 1 && !issue_pv(i - 1)) { ok = false; break; }
             }
-            if (ok) ok = issue_pv(ntiles - 1);
             if (ok) mma_commit(bar_o);
-            if (!ok && issued_pv >= 0)
-                mbar_wait(bar_kv_empty(issued_pv & 1), (issued_pv >> 1) & 1, nullptr, nullptr, 50000000ull);
+            if (!ok && pv > 0)
+                mbar_wait(bar_kv_empty((pv - 1) & 1), ((pv - 1) >> 1) & 1, nullptr, nullptr, 50000000ull);
         }
     } else if (warp >= 5) {
         // ------------------------------------------------ gather producers
@@ -186,23 +217,22 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int i = 0; i < ntiles; ++i) {
             const int st = i & 1;
             if (i >= kStages && !mbar_wait(bar_kv_empty(st), ((i >> 1) - 1) & 1, abort_flag, a.status)) break;
+            // keep the L2 prefetch kPrefetchTiles tiles ahead of the gather (each CTA of
+            // the value pair takes every other row)
+            if (p < kTileRows && i + kPrefetchTiles < ntiles && (p & 1) == half) {
+                const int s = sidx[(i + kPrefetchTiles) * kTileRows + p];
+                if (s >= 0) l2_prefetch_bulk(kv_seq + (int64_t)s * kDK, kDK * 2);
+            }
             const uint32_t stage = sKv + st * kKvStageBytes;
-            const int j0 = j_lo + i * kTileRows;
+            const int32_t* tile_idx = sidx + i * kTileRows;
             uint4 v[kGranules / kGatherThreads];
 #pragma unroll
             for (int u = 0; u < kGranules / kGatherThreads; ++u) {
                 const int G = p + u * kGatherThreads;
                 const int r = G / 72, c = G % 72;
-                const int j = j0 + r;
-                int s = j < j_hi ? idx_row[j] : -1;
-                if (s < -1 || s >= n_t) {
-                    if (c == 0 && half == 0 && row_ok) record_status(a.status, DSA_STATUS_INDEX_OOB);
-                    s = -1;
-                }
+                const int s = tile_idx[r];
                 if (s >= 0) {
-                    const uint4* src = reinterpret_cast<const uint4*>(
-                        reinterpret_cast<const __nv_bfloat16*>(a.kv) + ((int64_t)b * a.T_max + s) * kDK);
-                    v[u] = __ldg(src + c);
+                    v[u] = __ldg(reinterpret_cast<const uint4*>(kv_seq + (int64_t)s * kDK) + c);
                 } else {
                     v[u] = make_uint4(0u, 0u, 0u, 0u);
                 }
@@ -230,10 +260,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         bool ok = true;
         for (int i = 0; i < ntiles; ++i) {
             const int sb = i & 1;
-            // validity of the tile's 32 rows (lane r checks row r), shared through a ballot
-            const int jr = j_lo + i * kTileRows + lane;
-            int sr = jr < j_hi ? idx_row[jr] : -1;
-            const unsigned valid = __ballot_sync(0xffffffffu, sr >= 0 && sr < n_t);
+            const unsigned valid = __ballot_sync(0xffffffffu, sidx[i * kTileRows + lane] >= 0);
             ok = mbar_wait(bar_s_full(sb), (i >> 1) & 1, abort_flag, a.status);
             ok = __all_sync(0xffffffffu, ok);
             if (!ok) break;
@@ -347,49 +374,41 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
 }
 
-// Merge of split partials: one CTA per query row, 256 threads, float4 lanes.
-__global__ void __launch_bounds__(256) mla_combine_kernel(const MlaArgs a) {
-    __shared__ float wgt[16][kHeads];
-    __shared__ float lse_s[kHeads];
-    const int t = blockIdx.x;
-    const int tid = threadIdx.x;
+// Merge of split partials: one CTA of 128 threads per (head, row); thread j
+// owns values [4j, 4j+4) of the 512-wide output row.
+__global__ void __launch_bounds__(128) mla_combine_kernel(const MlaArgs a) {
+    const int h = blockIdx.x, t = blockIdx.y, j = threadIdx.x;
     const int64_t plane = (int64_t)a.Nq * kHeads;
-    for (int h = tid; h < kHeads; h += blockDim.x) {
-        float L = -CUDART_INF_F;
-        for (int p = 0; p < a.splits; ++p) L = fmaxf(L, a.part_lse[p * plane + (int64_t)t * kHeads + h]);
-        float s = 0.f;
-        for (int p = 0; p < a.splits; ++p) {
-            const float lp = a.part_lse[p * plane + (int64_t)t * kHeads + h];
-            const float e = (L == -CUDART_INF_F) ? 0.f : __expf(lp - L);
-            wgt[p][h] = e;
+    const int64_t th = (int64_t)t * kHeads + h;
+    float lp[16];
+    float L = -CUDART_INF_F;
+#pragma unroll
+    for (int p = 0; p < 16; ++p) {
+        lp[p] = p < a.splits ? a.part_lse[p * plane + th] : -CUDART_INF_F;
+        L = fmaxf(L, lp[p]);
+    }
+    float s = 0.f;
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+    for (int p = 0; p < 16; ++p) {
+        if (p < a.splits) {
+            const float e = (L == -CUDART_INF_F) ? 0.f : __expf(lp[p] - L);
             s += e;
+            const float4 v = reinterpret_cast<const float4*>(a.part_o + (p * plane + th) * kDV)[j];
+            acc.x = fmaf(e, v.x, acc.x);
+            acc.y = fmaf(e, v.y, acc.y);
+            acc.z = fmaf(e, v.z, acc.z);
+            acc.w = fmaf(e, v.w, acc.w);
         }
-        const float inv = s > 0.f ? 1.f / s : 0.f;
-        for (int p = 0; p < a.splits; ++p) wgt[p][h] *= inv;
-        lse_s[h] = (s > 0.f) ? L + __logf(s) : -CUDART_INF_F;
     }
-    __syncthreads();
-    if (a.lse)
-        for (int h = tid; h < kHeads; h += blockDim.x) a.lse[(int64_t)t * kHeads + h] = lse_s[h];
-    __nv_bfloat16* out = reinterpret_cast<__nv_bfloat16*>(a.out) + (int64_t)t * kHeads * kDV;
-    for (int e = tid; e < kHeads * kDV / 4; e += blockDim.x) {
-        const int h = e / (kDV / 4);
-        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-        for (int p = 0; p < a.splits; ++p) {
-            const float wv = wgt[p][h];
-            const float4 v = reinterpret_cast<const float4*>(a.part_o + (p * plane + (int64_t)t * kHeads) * kDV)[e];
-            acc.x = fmaf(wv, v.x, acc.x);
-            acc.y = fmaf(wv, v.y, acc.y);
-            acc.z = fmaf(wv, v.z, acc.z);
-            acc.w = fmaf(wv, v.w, acc.w);
-        }
-        const __nv_bfloat162 lo = __floats2bfloat162_rn(acc.x, acc.y);
-        const __nv_bfloat162 hi = __floats2bfloat162_rn(acc.z, acc.w);
-        uint2 pk;
-        pk.x = *reinterpret_cast<const uint32_t*>(&lo);
-        pk.y = *reinterpret_cast<const uint32_t*>(&hi);
-        reinterpret_cast<uint2*>(out)[e] = pk;
-    }
+    const float inv = s > 0.f ? 1.f / s : 0.f;
+    const __nv_bfloat162 lo = __floats2bfloat162_rn(acc.x * inv, acc.y * inv);
+    const __nv_bfloat162 hi = __floats2bfloat162_rn(acc.z * inv, acc.w * inv);
+    uint2 pk;
+    pk.x = *reinterpret_cast<const uint32_t*>(&lo);
+    pk.y = *reinterpret_cast<const uint32_t*>(&hi);
+    reinterpret_cast<uint2*>(reinterpret_cast<__nv_bfloat16*>(a.out) + th * kDV)[j] = pk;
+    if (j == 0 && a.lse) a.lse[th] = s > 0.f ? L + __logf(s) : -CUDART_INF_F;
 }
 
 }  // namespace
@@ -409,7 +428,7 @@ cudaError_t launch_sparse_mla_bf16(const MlaArgs& a, cudaStream_t st) {
 cudaError_t launch_mla_combine(const MlaArgs& a, cudaStream_t st) {
     if (a.Nq == 0 || a.splits <= 1) return cudaSuccess;
     if (a.splits > 16) return cudaErrorInvalidValue;
-    mla_combine_kernel<<<a.Nq, 256, 0, st>>>(a);
+    mla_combine_kernel<<<dim3(kHeads, a.Nq), 128, 0, st>>>(a);
     return cudaGetLastError();
 }
 

@@ -6,33 +6,42 @@
 // Order: score descending, ties to the lower position, -0.0 == +0.0.  The
 // positions are written in ascending order and padded with -1.
 //
-// Method: each score becomes an order-preserving 32-bit key; a radix select
-// over three digits (11, 11, 10 bits, most significant first) finds the
-// k-th largest key tau and how many keys equal to tau must be taken.  A row is
-// split across a thread-block cluster of C CTAs (C <= 8): every CTA keeps its
-// slice of the row in shared memory, builds a digit histogram with warp-
-// aggregated shared atomics (match_any + ballot), and the C histograms are
-// merged through distributed shared memory.  A final pass compacts the
-// selected positions in order with block-wide scans; CTA r learns from the
-// lower-ranked CTAs how many ties and outputs precede it, which gives the
-// deterministic lower-index tie rule across the whole row.
+// Method: each score becomes an order-preserving 32-bit key; a most-
+// significant-digit-first radix select over four 8-bit digits finds the k-th
+// largest key tau and how many keys equal to tau are taken.  A row is split
+// across a thread-block cluster of C CTAs (C <= 8); every CTA keeps its slice
+// of the row in shared memory as keys.  Per digit: warp-private 256-bin
+// histograms (match_any aggregation inside a warp, no cross-warp atomic
+// contention), summed per CTA, then merged across the cluster through
+// distributed shared memory (256 bins x C loads).  The per-CTA counts of keys
+// above / equal to tau fall out of the histograms, so no extra counting pass
+// is needed.  A final pass compacts the selected positions in position order
+// with one block-wide vector scan per sweep; CTA r learns from the lower-
+// ranked CTAs how many ties and outputs precede it, which gives the lower-
+// index tie rule across the whole row.
 #include <cooperative_groups.h>
 #include <cuda_runtime.h>
 
 #include "kernels.h"
-#include "status.cuh"
+#include "ptx.cuh"
 
 namespace cg = cooperative_groups;
 
 namespace dsa {
 namespace {
 
-constexpr int kThreads = 1024;
-constexpr int kBins = 2048;
-constexpr int kOffHist = 0;              // 2 x kBins (ping-pong, read remotely)
-constexpr int kOffTot = 2 * kBins;       // kBins merged histogram
-constexpr int kOffMisc = 3 * kBins;      // 64 words: counts, scan scratch, results
-constexpr int kOffKeys = 3 * kBins + 64; // cached keys
+constexpr int kThreads = 512;
+constexpr int kWarps = kThreads / 32;
+constexpr int kBins = 256;
+constexpr int kRounds = 8;  // compaction: a thread owns 4 consecutive keys in each of kRounds rounds
+// shared memory map (32-bit words)
+constexpr int kOffPriv = 0;                          // kWarps x kBins warp-private histograms
+constexpr int kOffHist = kOffPriv + kWarps * kBins;  // 2 x kBins per-CTA histogram (ping-pong, read remotely)
+constexpr int kOffTot = kOffHist + 2 * kBins;        // kBins cluster-wide histogram
+constexpr int kOffMisc = kOffTot + kBins;            // 64 words: results, counts (read remotely), scan scratch
+constexpr int kOffScan = kOffMisc + 64;              // vector-scan scratch
+constexpr int kScanWords = kWarps * kRounds + kRounds + 16;
+constexpr int kOffKeys = (kOffScan + kScanWords + 3) & ~3;
 constexpr int kBaseWords = kOffKeys;
 
 __device__ __forceinline__ uint32_t score_key(float f) {
@@ -41,10 +50,8 @@ __device__ __forceinline__ uint32_t score_key(float f) {
     return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
 }
 
-// Block-wide exclusive scan of one int per thread (kThreads threads).
-// scratch: >= 33 ints of shared memory.  Returns the exclusive prefix; *total
-// receives the block sum.  Must be called by every thread of the block.
-__device__ __forceinline__ int block_exclusive_scan(int v, int* scratch, int* total) {
+// Block-wide exclusive scan of one int per thread.  scratch >= kWarps + 1 ints.
+__device__ __forceinline__ int block_scan1(int v, int* scratch, int* total) {
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     int incl = v;
 #pragma unroll
@@ -55,34 +62,75 @@ __device__ __forceinline__ int block_exclusive_scan(int v, int* scratch, int* to
     if (lane == 31) scratch[warp] = incl;
     __syncthreads();
     if (warp == 0) {
-        const int wv = scratch[lane];
+        const int wv = lane < kWarps ? scratch[lane] : 0;
         int wi = wv;
 #pragma unroll
         for (int o = 1; o < 32; o <<= 1) {
             const int u = __shfl_up_sync(0xffffffffu, wi, o);
             if (lane >= o) wi += u;
         }
-        scratch[lane] = wi - wv;
-        if (lane == 31) scratch[32] = wi;
+        if (lane < kWarps) scratch[lane] = wi - wv;
+        if (lane == 31) scratch[kWarps] = wi;
     }
     __syncthreads();
     const int r = scratch[warp] + incl - v;
-    *total = scratch[32];
+    *total = scratch[kWarps];
     __syncthreads();
     return r;
 }
 
-__global__ void __launch_bounds__(kThreads, 1) topk_radix_kernel(const TopkArgs a, int cached_cap) {
+// Block-wide exclusive scan of kRounds ints per thread, rounds in order:
+// element (rr, tid) is preceded by all of rounds < rr and by threads < tid of
+// round rr.  Returns exclusive prefixes in pre[] (offset by base) and the new base.
+__device__ __forceinline__ int block_scan_rounds(const int (&v)[kRounds], int (&pre)[kRounds], int base, int* scr) {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    int incl[kRounds];
+#pragma unroll
+    for (int rr = 0; rr < kRounds; ++rr) incl[rr] = v[rr];
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+#pragma unroll
+        for (int rr = 0; rr < kRounds; ++rr) {
+            const int u = __shfl_up_sync(0xffffffffu, incl[rr], o);
+            if (lane >= o) incl[rr] += u;
+        }
+    }
+    if (lane == 31) {
+#pragma unroll
+        for (int rr = 0; rr < kRounds; ++rr) scr[warp * kRounds + rr] = incl[rr];
+    }
+    __syncthreads();
+    if (threadIdx.x < kRounds) {
+        int run = 0;
+        for (int w = 0; w < kWarps; ++w) {
+            const int x = scr[w * kRounds + threadIdx.x];
+            scr[w * kRounds + threadIdx.x] = run;
+            run += x;
+        }
+        scr[kWarps * kRounds + threadIdx.x] = run;
+    }
+    __syncthreads();
+    int b = base;
+#pragma unroll
+    for (int rr = 0; rr < kRounds; ++rr) {
+        pre[rr] = b + scr[warp * kRounds + rr] + incl[rr] - v[rr];
+        b += scr[kWarps * kRounds + rr];
+    }
+    __syncthreads();
+    return b;
+}
+
+__global__ void __launch_bounds__(kThreads, 2) topk_radix_kernel(const TopkArgs a, int cached_cap) {
     cg::cluster_group cluster = cg::this_cluster();
     const int C = (int)cluster.num_blocks();
     const int rank = (int)cluster.block_rank();
     extern __shared__ uint32_t sm[];
+    uint32_t* priv = sm + kOffPriv;
     uint32_t* tot = sm + kOffTot;
     int* misc = reinterpret_cast<int*>(sm + kOffMisc);
-    int* scan_scratch = misc + 16;
+    int* scr = reinterpret_cast<int*>(sm + kOffScan);
     uint32_t* keys = sm + kOffKeys;
-    const int tid = threadIdx.x;
-    const int lane = tid & 31;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
 
     const int t = blockIdx.y;
     int n = a.q_len[t];
@@ -104,142 +152,207 @@ __global__ void __launch_bounds__(kThreads, 1) topk_radix_kernel(const TopkArgs 
     const int len = hi - lo;
     const bool cached = len <= cached_cap;
     if (cached) {
+        // 16-byte loads, four in flight per thread, keys written in place
         const int nv = len >> 2;
         const float4* r4 = reinterpret_cast<const float4*>(row + lo);
-        for (int i = tid; i < nv; i += kThreads) {
-            const float4 f = __ldg(r4 + i);
-            keys[4 * i + 0] = score_key(f.x);
-            keys[4 * i + 1] = score_key(f.y);
-            keys[4 * i + 2] = score_key(f.z);
-            keys[4 * i + 3] = score_key(f.w);
+        uint4* k4 = reinterpret_cast<uint4*>(keys);
+        for (int i0 = 0; i0 < nv; i0 += 4 * kThreads) {
+            float4 f[4];
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                const int i = i0 + u * kThreads + tid;
+                f[u] = i < nv ? __ldg(r4 + i) : make_float4(0.f, 0.f, 0.f, 0.f);
+            }
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                const int i = i0 + u * kThreads + tid;
+                if (i < nv)
+                    k4[i] = make_uint4(score_key(f[u].x), score_key(f[u].y), score_key(f[u].z), score_key(f[u].w));
+            }
         }
         for (int i = 4 * nv + tid; i < len; i += kThreads) keys[i] = score_key(__ldg(row + lo + i));
     }
     __syncthreads();
+    auto key_at = [&](int i) -> uint32_t { return cached ? keys[i] : score_key(__ldg(row + lo + i)); };
+    // the 4 consecutive keys starting at i (a multiple of 4); out-of-range keys read as 0 (never selected:
+    // the caller checks i < len)
+    auto keys4_at = [&](int i) -> uint4 {
+        if (cached && i + 3 < len) return reinterpret_cast<const uint4*>(keys)[i >> 2];
+        uint4 r;
+        r.x = i < len ? key_at(i) : 0u;
+        r.y = i + 1 < len ? key_at(i + 1) : 0u;
+        r.z = i + 2 < len ? key_at(i + 2) : 0u;
+        r.w = i + 3 < len ? key_at(i + 3) : 0u;
+        return r;
+    };
 
     uint32_t prefix = 0, pmask = 0;
     int remaining = a.k;
+    int local_gt = 0;  // keys of this CTA above tau
+    int local_eq = 0;  // keys of this CTA equal to tau
 #pragma unroll 1
-    for (int p = 0; p < 3; ++p) {
-        const int width = p == 2 ? 10 : 11;
-        const int sh = p == 0 ? 21 : (p == 1 ? 10 : 0);
-        uint32_t* h = sm + kOffHist + (p & 1) * kBins;
-        for (int i = tid; i < kBins; i += kThreads) h[i] = 0u;
+    for (int p = 0; p < 4; ++p) {
+        const int sh = 24 - 8 * p;
+        uint32_t* hist = sm + kOffHist + (p & 1) * kBins;
+        for (int i = tid; i < kWarps * kBins; i += kThreads) priv[i] = 0u;
         __syncthreads();
-        const uint32_t dmask = (1u << width) - 1u;
+        uint32_t* my = priv + warp * kBins;
         for (int i0 = 0; i0 < len; i0 += kThreads) {
             const int i = i0 + tid;
             uint32_t kk = 0;
             bool take = false;
             if (i < len) {
-                kk = cached ? keys[i] : score_key(__ldg(row + lo + i));
+                kk = key_at(i);
                 take = (kk & pmask) == prefix;
             }
             const unsigned act = __ballot_sync(0xffffffffu, take);
             if (take) {
-                const uint32_t bin = (kk >> sh) & dmask;
+                const uint32_t bin = (kk >> sh) & 0xFFu;
                 const unsigned peers = __match_any_sync(act, bin);
-                if (lane == __ffs(peers) - 1) atomicAdd(&h[bin], (uint32_t)__popc(peers));
+                if (lane == __ffs(peers) - 1) atomicAdd(&my[bin], (uint32_t)__popc(peers));
             }
         }
-        cluster.sync();
-        for (int i = tid; i < kBins; i += kThreads) {
+        __syncthreads();
+        if (tid < kBins) {
             uint32_t s = 0;
-            for (int r = 0; r < C; ++r) s += cluster.map_shared_rank(h, r)[i];
-            tot[i] = s;
+#pragma unroll
+            for (int w = 0; w < kWarps; ++w) s += priv[w * kBins + tid];
+            hist[tid] = s;
+        }
+        cluster.sync();
+        if (tid < kBins) {
+            uint32_t v[8];
+#pragma unroll
+            for (int r = 0; r < 8; ++r) v[r] = r < C ? cluster.map_shared_rank(hist, r)[tid] : 0u;
+            tot[tid] = ((v[0] + v[1]) + (v[2] + v[3])) + ((v[4] + v[5]) + (v[6] + v[7]));
         }
         __syncthreads();
-        // locate the digit holding the remaining-th largest key (scan from the top digit down)
-        const int nb = 1 << width;
-        const int d1 = nb - 1 - 2 * tid, d0 = nb - 2 - 2 * tid;
-        const int c1 = d1 >= 0 ? (int)tot[d1] : 0;
-        const int c0 = d0 >= 0 ? (int)tot[d0] : 0;
+        // digit holding the remaining-th largest key: scan from the top digit down
+        const int d = kBins - 1 - tid;
+        const int c = tid < kBins ? (int)tot[d] : 0;
         int tsum;
-        const int before = block_exclusive_scan(c1 + c0, scan_scratch, &tsum);
-        if (d1 >= 0 && before < remaining && remaining <= before + c1) {
-            misc[0] = d1;
+        const int before = block_scan1(c, scr, &tsum);
+        if (tid < kBins && before < remaining && remaining <= before + c) {
+            misc[0] = d;
             misc[1] = before;
-        } else if (d0 >= 0 && before + c1 < remaining && remaining <= before + c1 + c0) {
-            misc[0] = d0;
-            misc[1] = before + c1;
         }
         __syncthreads();
-        prefix |= (uint32_t)misc[0] << sh;
-        pmask |= dmask << sh;
-        remaining -= misc[1];
-        __syncthreads();
+        const int dsel = misc[0];
+        const int above = misc[1];
+        // this CTA's keys in digits above the chosen one (same prefix) are above tau
+        int atot;
+        block_scan1((tid < kBins && d > dsel) ? (int)hist[d] : 0, scr, &atot);
+        local_gt += atot;
+        if (p == 3) local_eq = (int)hist[dsel];
+        prefix |= (uint32_t)dsel << sh;
+        pmask |= 0xFFu << sh;
+        remaining -= above;
     }
     const uint32_t tau = prefix;
     const int take_eq_total = remaining;  // keys equal to tau that are selected, lowest positions first
 
-    // per-CTA counts of keys above / equal to tau
-    int my_gt = 0, my_eq = 0;
-    for (int i = tid; i < len; i += kThreads) {
-        const uint32_t kk = cached ? keys[i] : score_key(__ldg(row + lo + i));
-        my_gt += kk > tau;
-        my_eq += kk == tau;
-    }
-    int n_gt, n_eq;
-    block_exclusive_scan(my_gt, scan_scratch, &n_gt);
-    block_exclusive_scan(my_eq, scan_scratch, &n_eq);
     if (tid == 0) {
-        misc[2] = n_gt;
-        misc[3] = n_eq;
+        misc[2] = local_gt;
+        misc[3] = local_eq;
     }
     cluster.sync();
     int eq_before = 0, out_before = 0;
-    for (int r = 0; r < rank; ++r) {
-        const int* rm = cluster.map_shared_rank(misc, r);
-        const int g = rm[2], e = rm[3];
-        const int te = max(0, min(take_eq_total - eq_before, e));
-        out_before += g + te;
-        eq_before += e;
-    }
-    const int take_eq_local = max(0, min(take_eq_total - eq_before, n_eq));
-
-    // ordered compaction, 4 consecutive elements per thread per round
-    int eq_run = 0, sel_run = 0;
-    for (int r0 = 0; r0 < len; r0 += 4 * kThreads) {
-        const int e0 = r0 + 4 * tid;
-        uint32_t kk[4];
-        int ceq = 0;
+    {
+        int rg[8], re[8];
 #pragma unroll
-        for (int u = 0; u < 4; ++u) {
-            const int i = e0 + u;
-            kk[u] = i < len ? (cached ? keys[i] : score_key(__ldg(row + lo + i))) : 0u;
-            ceq += (i < len) && kk[u] == tau;
+        for (int r = 0; r < 8; ++r) {
+            const int* rm = cluster.map_shared_rank(misc, r < rank ? r : rank);
+            rg[r] = rm[2];
+            re[r] = rm[3];
         }
-        int eq_tot;
-        const int eqp = block_exclusive_scan(ceq, scan_scratch, &eq_tot);
-        int eq_seen = eq_run + eqp;
-        bool sel[4];
-        int csel = 0;
 #pragma unroll
-        for (int u = 0; u < 4; ++u) {
-            const int i = e0 + u;
-            bool s = false;
-            if (i < len) {
-                if (kk[u] > tau) {
-                    s = true;
-                } else if (kk[u] == tau) {
-                    s = eq_seen < take_eq_local;
-                    ++eq_seen;
+        for (int r = 0; r < 8; ++r) {
+            if (r < rank) {
+                const int te = max(0, min(take_eq_total - eq_before, re[r]));
+                out_before += rg[r] + te;
+                eq_before += re[r];
+            }
+        }
+    }
+    const int take_eq_local = max(0, min(take_eq_total - eq_before, local_eq));
+    const bool all_ties = take_eq_local == local_eq;  // selection is then a plain threshold
+    const uint64_t thr = take_eq_local > 0 ? (uint64_t)tau : (uint64_t)tau + 1u;
+
+    // ordered compaction in sweeps of kRounds x 4 x kThreads keys
+    const int sweep = kRounds * 4 * kThreads;
+    int out_run = out_before, eq_run = 0;
+    for (int s0 = 0; s0 < len; s0 += sweep) {
+        uint32_t sel = 0;  // bit 4*rr+u: key (rr, u) of this thread selected
+        int cnt[kRounds];
+        if (all_ties) {
+#pragma unroll
+            for (int rr = 0; rr < kRounds; ++rr) {
+                cnt[rr] = 0;
+                const int i0 = s0 + (rr * kThreads + tid) * 4;
+                const uint4 k4 = keys4_at(i0);
+                const uint32_t kv[4] = {k4.x, k4.y, k4.z, k4.w};
+#pragma unroll
+                for (int u = 0; u < 4; ++u) {
+                    if (i0 + u < len && (uint64_t)kv[u] >= thr) {
+                        sel |= 1u << (4 * rr + u);
+                        ++cnt[rr];
+                    }
                 }
             }
-            sel[u] = s;
-            csel += s;
-        }
-        int sel_tot;
-        const int selp = block_exclusive_scan(csel, scan_scratch, &sel_tot);
-        int o = out_before + sel_run + selp;
+        } else {
+            // rank of each tie among this CTA's ties decides it
+            int ceq[kRounds], pre[kRounds];
+            uint32_t eqm = 0;
 #pragma unroll
-        for (int u = 0; u < 4; ++u)
-            if (sel[u]) {
-                if (o < a.k) out[o] = lo + e0 + u;
-                ++o;
+            for (int rr = 0; rr < kRounds; ++rr) {
+                cnt[rr] = 0;
+                ceq[rr] = 0;
+                const int i0 = s0 + (rr * kThreads + tid) * 4;
+                const uint4 k4 = keys4_at(i0);
+                const uint32_t kv[4] = {k4.x, k4.y, k4.z, k4.w};
+#pragma unroll
+                for (int u = 0; u < 4; ++u) {
+                    if (i0 + u < len) {
+                        const uint32_t kk = kv[u];
+                        if (kk > tau) {
+                            sel |= 1u << (4 * rr + u);
+                            ++cnt[rr];
+                        } else if (kk == tau) {
+                            eqm |= 1u << (4 * rr + u);
+                            ++ceq[rr];
+                        }
+                    }
+                }
             }
-        eq_run += eq_tot;
-        sel_run += sel_tot;
+            eq_run = block_scan_rounds(ceq, pre, eq_run, scr);
+#pragma unroll
+            for (int rr = 0; rr < kRounds; ++rr) {
+                int e = pre[rr];
+#pragma unroll
+                for (int u = 0; u < 4; ++u) {
+                    if ((eqm >> (4 * rr + u)) & 1u) {
+                        if (e < take_eq_local) {
+                            sel |= 1u << (4 * rr + u);
+                            ++cnt[rr];
+                        }
+                        ++e;
+                    }
+                }
+            }
+        }
+        int pos[kRounds];
+        out_run = block_scan_rounds(cnt, pos, out_run, scr);
+#pragma unroll
+        for (int rr = 0; rr < kRounds; ++rr) {
+            int o = pos[rr];
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                if ((sel >> (4 * rr + u)) & 1u) {
+                    if (o < a.k) out[o] = lo + s0 + (rr * kThreads + tid) * 4 + u;
+                    ++o;
+                }
+            }
+        }
     }
     cluster.sync();  // keep this CTA's shared memory alive until every peer has read it
 }
