@@ -148,13 +148,8 @@ def dist_setup(n):
 
 
 def max_over_ranks(x: float, world: int) -> float:
-    if world <= 1:
-        return x
-    import torch
-    import torch.distributed as dist
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
-    dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    return float(t.item())
+    from sparse_long_context_indexer_b200 import dist as ddist
+    return ddist.max_over_ranks(x, device="cuda") if world > 1 else x
 
 
 def barrier(world):
