@@ -149,6 +149,31 @@ dsa_status_t dsa_sparse_mla_attn(const dsa_dims* dims, const void* q, const void
                                  float softmax_scale, void* out, float* lse,
                                  void* workspace, size_t ws_bytes, void* stream);
 
+/* Stage 3 for callers that cannot allocate device memory.  No counterpart in
+ * the paper: it exists for callers embedded in a host that owns all device
+ * memory -- plugin interfaces that hand a kernel only its input and output
+ * buffers, or serving loops whose device-memory budget is fixed at start-up --
+ * and so can neither call cudaMalloc nor size a workspace for
+ * dsa_sparse_mla_attn.  Same arguments and results as dsa_sparse_mla_attn with
+ * kv_dtype DSA_BF16, minus the workspace: the split partials live in a buffer
+ * the library holds statically on every GPU that loads it (about 16.1 MiB,
+ * kept until the process exits).
+ * Limit: (number of splits) x Nq <= 64 partial rows of 128 heads; the split
+ * count is the one dsa_sparse_mla_attn would use (it depends on Nq and the
+ * device's SM count; 1 split needs no scratch at all).  Larger requests return
+ * DSA_ERR_UNSUPPORTED before any launch.  kv_dtype DSA_F32 returns
+ * DSA_ERR_UNSUPPORTED.
+ * The first call on a device looks up the buffer's device address (once per
+ * device, with that device current); make that first call before any stream
+ * capture.  All calls share the buffer, so calls whose kernels overlap on the
+ * GPU (other streams, other host threads) race on it: serialise them.  No
+ * status word exists here: device-side index errors are not reported (entries
+ * outside [-1, q_len[t]) are still treated as -1).  Allocates nothing; calls no
+ * cudaMalloc or cudaFree. */
+dsa_status_t dsa_sparse_mla_attn_noalloc(const dsa_dims* dims, const void* q, const void* kv,
+                                         const int32_t* idx, const int32_t* q_seq, const int32_t* q_len,
+                                         float softmax_scale, void* out, float* lse, void* stream);
+
 /* The whole decode step: stages 1-3 back to back on `stream` (lizeman,
  * section 3 sketch: indexer, top-K gather, attention over the K positions).
  * scores_out / idx_out may be NULL (then the workspace holds them; size the

@@ -22,7 +22,7 @@ DSA_OP_INDEXER, DSA_OP_TOPK, DSA_OP_SPARSE_MLA, DSA_OP_DECODE, DSA_OP_PREFILL = 
 EXPORTS = (
     "dsa_workspace_size", "dsa_workspace_init", "dsa_indexer_scores", "dsa_topk", "dsa_sparse_mla_attn",
     "dsa_decode_step", "dsa_prefill", "dsa_get_device_status", "dsa_status_string", "dsa_last_cuda_error",
-    "dsa_selftest_wait_timeout", "dsa_version",
+    "dsa_selftest_wait_timeout", "dsa_version", "dsa_sparse_mla_attn_noalloc",
 )
 
 
@@ -64,6 +64,7 @@ def _declare(lib):
     lib.dsa_indexer_scores.argtypes = [D, P, P, P, P, P, P, P, P, P, S, P]
     lib.dsa_topk.argtypes = [D, P, P, P, P, S, P]
     lib.dsa_sparse_mla_attn.argtypes = [D, P, P, P, P, P, F, P, P, P, S, P]
+    lib.dsa_sparse_mla_attn_noalloc.argtypes = [D, P, P, P, P, P, F, P, P, P]
     lib.dsa_decode_step.argtypes = [D, P, P, P, P, P, P, P, P, P, F, P, P, P, P, P, S, P,
                                     ctypes.POINTER(DsaStageEvents)]
     lib.dsa_prefill.argtypes = [D, P, P, P, P, P, P, P, P, P, F, P, P, P, P, S, P]
@@ -71,7 +72,7 @@ def _declare(lib):
     lib.dsa_selftest_wait_timeout.argtypes = [P, S, I32, P]
     for name in ("dsa_workspace_size", "dsa_workspace_init", "dsa_indexer_scores", "dsa_topk",
                  "dsa_sparse_mla_attn", "dsa_decode_step", "dsa_prefill", "dsa_get_device_status",
-                 "dsa_selftest_wait_timeout"):
+                 "dsa_selftest_wait_timeout", "dsa_sparse_mla_attn_noalloc"):
         getattr(lib, name).restype = st
     lib.dsa_status_string.argtypes = [I32]
     lib.dsa_status_string.restype = ctypes.c_char_p

@@ -294,6 +294,45 @@ dsa_status_t dsa_sparse_mla_attn(const dsa_dims* dims, const void* q, const void
                    reinterpret_cast<cudaStream_t>(stream));
 }
 
+dsa_status_t dsa_sparse_mla_attn_noalloc(const dsa_dims* dims, const void* q, const void* kv, const int32_t* idx,
+                                         const int32_t* q_seq, const int32_t* q_len, float softmax_scale, void* out,
+                                         float* lse, void* stream) {
+    dsa_status_t s = check_dims(dims, false, true);
+    if (s != DSA_OK) return s;
+    if (dims->kv_dtype != DSA_BF16) return DSA_ERR_UNSUPPORTED;
+    if (dims->Nq == 0) return DSA_OK;
+    if (!q || !kv || !idx || !q_seq || !q_len || !out || !std::isfinite(softmax_scale)) return DSA_ERR_INVALID_ARG;
+    if (!aligned16(q) || !aligned16(kv) || !aligned16(out)) return DSA_ERR_INVALID_ARG;
+    const MlaPlan p = plan_mla(dims, dims->Nq);
+    if (p.splits > 1 && (size_t)p.splits * dims->Nq > dsa::kStaticScratchPartials) return DSA_ERR_UNSUPPORTED;
+    void* scratch = nullptr;
+    cudaError_t e = dsa::static_mla_scratch(&scratch);
+    if (e != cudaSuccess) return cuda_fail(e);
+    dsa::MlaArgs a{};
+    a.q = q;
+    a.kv = kv;
+    a.idx = idx;
+    a.q_seq = q_seq;
+    a.q_len = q_len;
+    a.out = out;
+    a.lse = lse;
+    a.part_o = reinterpret_cast<float*>(scratch);
+    a.part_lse = reinterpret_cast<float*>(static_cast<char*>(scratch) + dsa::kStaticScratchOBytes);
+    a.Nq = dims->Nq;
+    a.B = dims->B;
+    a.T_max = dims->T_max;
+    a.k = dims->k;
+    a.H = dims->H;
+    a.splits = p.splits;
+    a.rows_per_split = p.rows_per_split;
+    a.softmax_scale = softmax_scale;
+    a.status = nullptr;  // no caller memory to report device-side errors into
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    e = dsa::launch_sparse_mla_bf16(a, st);
+    if (e == cudaSuccess) e = dsa::launch_mla_combine(a, st);
+    return e == cudaSuccess ? DSA_OK : cuda_fail(e);
+}
+
 dsa_status_t dsa_decode_step(const dsa_dims* dims, const void* q_I, const float* q_scale, const void* w,
                              const void* k_I, const float* k_scale, const void* q, const void* kv,
                              const int32_t* q_seq, const int32_t* q_len, float softmax_scale, void* out, float* lse,

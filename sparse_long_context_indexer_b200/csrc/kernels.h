@@ -61,6 +61,16 @@ cudaError_t launch_mla_combine(const MlaArgs& a, cudaStream_t st);
 cudaError_t launch_sparse_mla_f32(const MlaArgs& a, cudaStream_t st);
 cudaError_t launch_wait_timeout_selftest(int* status, int timeout_us, cudaStream_t st);
 
+// Statically allocated split scratch of the attention kernel (no-allocation entry point):
+// fp32 partial outputs for up to kStaticScratchPartials (split, row) pairs of 128 heads x 512,
+// then their lse values.
+constexpr int kMaxDevices = 64;
+constexpr size_t kStaticScratchPartials = 64;
+constexpr size_t kStaticScratchOBytes = kStaticScratchPartials * kMlaHeads * kDV * sizeof(float);  // 16 MiB
+constexpr size_t kStaticScratchBytes = kStaticScratchOBytes + kStaticScratchPartials * kMlaHeads * sizeof(float);
+// Device address of this device's static scratch (looked up on first use per device).
+cudaError_t static_mla_scratch(void** ptr);
+
 // Largest row chunk kept in shared memory by one top-k CTA (elements).
 constexpr int kTopkSmemKeys = 49152;
 

@@ -33,6 +33,8 @@
 #include <cuda_runtime.h>
 #include <math_constants.h>
 
+#include <mutex>
+
 #include "kernels.h"
 #include "ptx.cuh"
 
@@ -423,6 +425,37 @@ cudaError_t launch_sparse_mla_bf16(const MlaArgs& a, cudaStream_t st) {
     dim3 grid(a.splits, 2, a.Nq);
     sparse_mla_bf16_kernel<<<grid, kThreads, kSmemBytes, st>>>(a, tq);
     return cudaGetLastError();
+}
+
+// ---------------------------------------------------------------------------
+// Library-owned scratch for callers that cannot allocate device memory.
+// One statically sized buffer per device holds the split partials of the
+// attention kernel (normalised fp32 O and lse of every split).  Every call
+// shares it: calls whose kernels overlap on the GPU race on it.  Nothing in
+// it needs to start at zero (each call overwrites every partial it reads).
+static __device__ __align__(256) unsigned char g_mla_static_scratch[kStaticScratchBytes];
+
+namespace {
+std::mutex g_scratch_mu;
+void* g_scratch_ptr[kMaxDevices] = {};
+}  // namespace
+
+cudaError_t static_mla_scratch(void** ptr) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+    std::lock_guard<std::mutex> lock(g_scratch_mu);
+    if (g_scratch_ptr[dev] == nullptr) {
+        // host code only sees a stand-in for the array: ask the runtime for the
+        // device address, once per device, with that device current
+        void* p = nullptr;
+        e = cudaGetSymbolAddress(&p, g_mla_static_scratch);
+        if (e != cudaSuccess) return e;
+        g_scratch_ptr[dev] = p;
+    }
+    *ptr = g_scratch_ptr[dev];
+    return cudaSuccess;
 }
 
 cudaError_t launch_mla_combine(const MlaArgs& a, cudaStream_t st) {
