@@ -11,8 +11,8 @@ constexpr int kDK = 576;   // latent key width (512 latent + 64 rope)
 constexpr int kDV = 512;   // value width
 constexpr int kIdxTile = 128;  // indexer: cached tokens per tensor-core tile (MMA M)
 constexpr int kIdxHeads = 64;  // indexer: heads per query (MMA N) for the FP8 kernel
-constexpr int kMlaTile = 32;   // sparse MLA: gathered rows per tile (MMA N of Q K^T)
-constexpr int kMlaHeads = 128; // sparse MLA bf16 kernel: query heads (MMA M)
+constexpr int kMlaTile = 64;   // sparse MLA: gathered rows per tile (MMA N of Q K^T, K of P V)
+constexpr int kMlaHeads = 128; // sparse MLA bf16 kernel: query heads (two CTAs of MMA M = 64)
 
 struct IndexerArgs {
     const void* q_I;

@@ -9,23 +9,36 @@
 //   out[t,h,:] = sum_{s in idx[t]} softmax_s(scale * q[t,h,:] . c[s,:]) c[s,0:512]
 //   lse[t,h]   = ln sum_s exp(scale * q[t,h,:] . c[s,:])
 //
-// Design (one CTA per SM):
-//   grid = (splits, 2 value halves, Nq).  TMEM holds 128 lanes x 512 fp32
-//   columns; the 128-head x 512 output alone would fill it, so each CTA of a
-//   pair owns one 256-wide half of the value dimension (256 columns) and both
-//   recompute S = Q K^T (M = 128 heads, N = 32 rows, K = 576).  The second CTA's
-//   gather of the same rows is served by L2.
-//   warps 0..3  softmax: thread h owns head h (TMEM lane h); online softmax in
+// Design (one CTA per SM, no cluster):
+//   grid = (splits, 2 head halves, Nq).  Each CTA owns 64 of the 128 heads, so
+//   its query block (64 x 576 bf16, 72 KB) and two 64-row gather stages (72 KB
+//   each) fit in shared memory together, and every MMA is M = 64:
+//     S = Q K^T   M = 64 heads, N = 64 rows, K = 576   (36 MMAs of K = 16)
+//     O += P V    M = 64 heads, N = 2 x 256 values, K = 64 rows
+//   The two CTAs of a (split, row) pair read the same rows; the second read is
+//   an L2 hit.  TMEM (M = 64 layout: rows in lanes 0..15 of each 32-lane
+//   subpartition, a second accumulator at lane offset 16):
+//     O[:, 0:256]   lanes +0,  columns [0, 256)
+//     O[:, 256:512] lanes +16, columns [0, 256)
+//     S buffers     lanes +0,  columns [256, 320) and [320, 384)
+//   warps 0..3  softmax: two threads per head (lanes r and r+16 of warp w own
+//               head 16w+r, columns [0,32) and [32,64) of S); online softmax in
 //               the exp2 domain with lazy rescaling of O (only when the running
-//               maximum grows by more than 8, i.e. a factor 256); P is written
-//               back into TMEM as bf16 over the S columns it came from.
-//   warp 4      TMEM allocator, Q TMA (9 boxes of 128 x 64, 128B swizzle) and
-//               the single-thread tcgen05.mma issuer: QK^T(i+1) is issued
-//               before PV(i) so the softmax of tile i overlaps the tensor core.
-//   warps 5..8  gather: each selected 1152-byte row is read with 16-byte vector
-//               loads (consecutive lanes -> consecutive bytes of one row) and
-//               stored into the 128B-swizzled K-major tile the MMA reads; the
-//               same tile serves as the MN-major V operand of P V.
+//               maximum grows by more than 8, i.e. a factor 256); P goes to a
+//               128B-swizzled K-major shared tile, the A operand of P V.
+//   warp 4      TMEM allocator and the single-thread tcgen05.mma issuer:
+//               QK^T(i+1) is issued before PV(i) so the softmax of tile i
+//               overlaps the tensor core.
+//   warps 5..12 row gather: 16-byte cp.async copies, eight threads per
+//               128-byte piece of a row (a full line per eight lanes), straight
+//               into the 128B-swizzled K-major tile the MMA reads; the same tile
+//               serves as the MN-major V operand of P V.  Completion is tracked
+//               by the stage's mbarrier (cp.async.mbarrier.arrive.noinc), so the
+//               copiers never block on their own loads.  Skipped rows are
+//               zero-filled without a read.  Rows a few tiles ahead are
+//               prefetched to L2.  (Measured on B200: per-thread 16-byte copies
+//               from 256 threads gather random 128-byte pieces at ~3.3 TB/s,
+//               TMA tile::gather4 at ~1.4 TB/s.)
 // Splits > 1 write normalised fp32 partials and their lse; mla_combine_kernel
 // merges them: O = sum_p exp(lse_p - L) O_p with L = logsumexp_p lse_p.
 #include <cuda.h>
@@ -41,31 +54,32 @@
 namespace dsa {
 namespace {
 
-constexpr int kTileRows = kMlaTile;          // 32 gathered rows per tile
-constexpr int kHeads = kMlaHeads;            // 128 (MMA M)
-constexpr int kChunks = kDK / 64;            // 9 swizzle chunks of 64 bf16 (128 B)
-constexpr int kQBytes = kHeads * kDK * 2;    // 147456
-constexpr int kQChunkBytes = kHeads * 128;   // 16384
-constexpr int kKvChunkBytes = kTileRows * 128;  // 4096
-constexpr int kKvStageBytes = kChunks * kKvChunkBytes;  // 36864
+constexpr int kTileRows = kMlaTile;             // 64 gathered rows per tile
+constexpr int kCtaHeads = kMlaHeads / 2;        // 64 heads per CTA (MMA M)
+constexpr int kChunks = kDK / 64;               // 9 swizzle chunks of 64 bf16 (128 B)
+constexpr int kChunkBytes = 64 * 128;           // one chunk of 64 rows (Q block or KV tile)
+constexpr int kQBytes = kChunks * kChunkBytes;  // 73728
+constexpr int kKvStageBytes = kChunks * kChunkBytes;  // 73728
+constexpr int kPBytes = kCtaHeads * kTileRows * 2;    // 8192
 constexpr int kStages = 2;
-constexpr int kThreads = 288;
-constexpr int kGatherThreads = 128;
-constexpr int kGranules = kTileRows * (kDK * 2 / 16);  // 2304 16-byte granules per tile
+constexpr int kGatherWarp0 = 5;
+constexpr int kGatherThreads = 256;
+constexpr int kThreads = 32 * kGatherWarp0 + kGatherThreads;  // 416
 constexpr int kOffQ = 0;
 constexpr int kOffKv = kOffQ + kQBytes;
-constexpr int kOffBar = kOffKv + kStages * kKvStageBytes;
-constexpr int kNumBar = 1 + 2 * kStages + 2 + 2 + 1;  // q_full, kv_full[2], kv_empty[2], s_full[2], p_full[2], o_done
+constexpr int kOffP = kOffKv + kStages * kKvStageBytes;
+constexpr int kOffBar = kOffP + kPBytes;
+constexpr int kNumBar = 1 + 2 * kStages + 2 + 1 + 1;  // q_full, kv_full[2], kv_empty[2], s_full[2], p_full, o_done
 constexpr int kOffMisc = kOffBar + kNumBar * 8;
-constexpr int kOffIdx = kOffMisc + 64;                   // up to 2048 staged positions
-constexpr int kSmemBytes = kOffIdx + 2048 * 4 + 1024;
+constexpr int kSmemBytes = kOffMisc + 16 + 1024;
+static_assert(kSmemBytes <= 232448, "shared memory budget of one CTA");
 constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kColO = 0;     // O half: columns [0, 256)
-constexpr uint32_t kColS = 256;   // S/P buffers: [256, 288), [288, 320)
+constexpr uint32_t kLaneHi = 16u << 16;  // TMEM lane offset of the second M = 64 accumulator
+constexpr uint32_t kColS = 256;          // S buffers at columns [256, 320), [320, 384)
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
-constexpr int kPrefetchTiles = 4;          // L2 prefetch distance of the gather, in tiles
-constexpr uint32_t kIdescQK = make_idesc(kHeads, kTileRows, 1 /*bf16*/, 1 /*bf16*/, 0, 0);
-constexpr uint32_t kIdescPV = make_idesc(kHeads, 256, 1 /*bf16*/, 1 /*bf16*/, 0 /*A K-major*/, 1 /*B MN-major*/);
+constexpr int kPrefetchTiles = 3;          // L2 prefetch distance of the gather, in tiles
+constexpr uint32_t kIdescQK = make_idesc(kCtaHeads, kTileRows, 1 /*bf16*/, 1 /*bf16*/, 0, 0);
+constexpr uint32_t kIdescPV = make_idesc(kCtaHeads, 256, 1 /*bf16*/, 1 /*bf16*/, 0 /*A K-major*/, 1 /*B MN-major*/);
 
 struct MlaShared {
     int tmem_base;
@@ -84,21 +98,22 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
 }
 
 __global__ void __launch_bounds__(kThreads, 1)
-    sparse_mla_bf16_kernel(const MlaArgs a, const __grid_constant__ CUtensorMap tmap_q) {
+    sparse_mla_bf16_kernel(const MlaArgs a, const __grid_constant__ CUtensorMap tmap_q,
+                           const __grid_constant__ CUtensorMap tmap_o) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const uint32_t sbase = smem_u32(smem);
     const uint32_t sQ = sbase + kOffQ;
     const uint32_t sKv = sbase + kOffKv;
+    const uint32_t sP = sbase + kOffP;
     const uint32_t bar0 = sbase + kOffBar;
     const uint32_t bar_q = bar0;
     auto bar_kv_full = [&](int s) { return bar0 + 8u * (1 + s); };
     auto bar_kv_empty = [&](int s) { return bar0 + 8u * (1 + kStages + s); };
     auto bar_s_full = [&](int s) { return bar0 + 8u * (1 + 2 * kStages + s); };
-    auto bar_p_full = [&](int s) { return bar0 + 8u * (3 + 2 * kStages + s); };
-    const uint32_t bar_o = bar0 + 8u * (5 + 2 * kStages);
+    const uint32_t bar_p_full = bar0 + 8u * (3 + 2 * kStages);
+    const uint32_t bar_o = bar0 + 8u * (4 + 2 * kStages);
     MlaShared* sh = reinterpret_cast<MlaShared*>(smem + kOffMisc);
-    int32_t* sidx = reinterpret_cast<int32_t*>(smem + kOffIdx);  // this split's positions, -1 = skip
     volatile int* abort_flag = &sh->abort_flag;
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -116,7 +131,32 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (split == 0 && half == 0 && tid == 0) record_status(a.status, DSA_STATUS_LENGTH);
         n_t = 0;
     }
+    const int32_t* idx_row = a.idx + (int64_t)t * a.k;
     const __nv_bfloat16* kv_seq = reinterpret_cast<const __nv_bfloat16*>(a.kv) + (int64_t)b * a.T_max * kDK;
+    // position r of tile i -> selected token, -1 past the end of the split
+    auto load_pos = [&](int i, int r) -> int {
+        const int j = j_lo + i * kTileRows + r;
+        return j < j_hi ? __ldg(idx_row + j) : -1;
+    };
+    auto valid = [&](int s) { return s >= 0 && s < n_t; };
+
+    // the first index loads of each role go out before the setup barrier
+    const int p = tid - 32 * kGatherWarp0;  // gather thread (warps >= kGatherWarp0)
+    const int rr = (p >> 3) & 31, gl = p & 7;
+    const bool pf_lane = warp >= kGatherWarp0 && gl == 0;  // 32 threads issue the L2 prefetches
+    int cur0 = -1, cur1 = -1, pf = -1, pf_first = -1, v0 = -1, v1 = -1;
+    if (ntiles > 0) {
+        if (warp >= kGatherWarp0) {
+            cur0 = load_pos(0, rr);
+            cur1 = load_pos(0, rr + 32);
+            // each CTA of the head pair prefetches one half of the rows
+            if (pf_lane && kStages < ntiles) pf_first = load_pos(kStages, rr + 32 * half);
+            if (pf_lane && kPrefetchTiles < ntiles) pf = load_pos(kPrefetchTiles, rr + 32 * half);
+        } else if (warp < 4) {
+            v0 = load_pos(0, lane);
+            v1 = load_pos(0, lane + 32);
+        }
+    }
 
     if (tid == 0) {
         mbar_init(bar_q, 1);
@@ -124,175 +164,197 @@ __global__ void __launch_bounds__(kThreads, 1)
             mbar_init(bar_kv_full(s), kGatherThreads);
             mbar_init(bar_kv_empty(s), 1);
             mbar_init(bar_s_full(s), 1);
-            mbar_init(bar_p_full(s), 128);
         }
+        mbar_init(bar_p_full, 128);
         mbar_init(bar_o, 1);
         sh->abort_flag = 0;
         fence_barrier_init();
         if (ntiles > 0) {
-            // the query block is needed first and does not depend on the staging below
             mbar_arrive_expect_tx(bar_q, kQBytes);
 #pragma unroll 1
-            for (int c = 0; c < kChunks; ++c) tma_load_2d(sQ + c * kQChunkBytes, &tmap_q, c * 64, t * kHeads, bar_q);
+            for (int c = 0; c < kChunks; ++c)
+                tma_load_2d(sQ + c * kChunkBytes, &tmap_q, c * 64, t * kMlaHeads + half * kCtaHeads, bar_q);
         }
     }
     if (warp == 4) {
         tmem_alloc(smem_u32(&sh->tmem_base), kTmemCols);
         tmem_relinquish();
     }
-    // Stage this split's positions (sanitised: anything outside [0, n_t) becomes -1)
-    // and start pulling the first tiles' rows into L2: each CTA of the value pair
-    // prefetches one half of the rows, so every row leaves HBM once, early.
-    for (int r = tid; r < ntiles * kTileRows; r += kThreads) {
-        int s = r < nrows ? a.idx[(int64_t)t * a.k + j_lo + r] : -1;
-        if (s < -1 || s >= n_t) {
-            if (half == 0 && row_ok) record_status(a.status, DSA_STATUS_INDEX_OOB);
-            s = -1;
-        }
-        sidx[r] = s;
-        if (s >= 0 && (r & 1) == half && r < kPrefetchTiles * kTileRows)
-            l2_prefetch_bulk(kv_seq + (int64_t)s * kDK, kDK * 2);
-    }
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = (uint32_t)sh->tmem_base;
 
-    if (warp == 4) {
-        // ------------------------------------------------ Q load + MMA issue
-        if (lane == 0 && ntiles > 0) {
+    if (warp >= kGatherWarp0) {
+        // ------------------------------------------------ row gather (8 warps)
+        // thread p copies 16-byte granule (p & 7) of every 128-byte piece of rows
+        // (p >> 3) and (p >> 3) + 32 of each tile.
+        auto prefetch_row = [&](int s) {
+            if (valid(s)) l2_prefetch_bulk(kv_seq + (int64_t)s * kDK, kDK * 2);
+        };
+        if (pf_lane) prefetch_row(pf_first);
+        for (int i = 0; i < ntiles; ++i) {
+            const int st = i & 1;
+            if (gl == 0 && row_ok && half == 0 &&
+                ((cur0 < -1 || cur0 >= n_t) || (cur1 < -1 || cur1 >= n_t)))
+                record_status(a.status, DSA_STATUS_INDEX_OOB);
+            const uint32_t stage = sKv + st * kKvStageBytes;
+#pragma unroll
+            for (int h2 = 0; h2 < 2; ++h2) {
+                const int s = h2 ? cur1 : cur0;
+                const int r = rr + 32 * h2;
+                const bool ok_row = valid(s);
+                const __nv_bfloat16* src = ok_row ? kv_seq + (int64_t)s * kDK + gl * 8 : reinterpret_cast<const __nv_bfloat16*>(a.kv);
+                const uint32_t dst = stage + r * 128 + ((gl ^ (r & 7)) << 4);
+#pragma unroll
+                for (int c = 0; c < kChunks; ++c) cp_async16_zfill(dst + c * kChunkBytes, src + c * 64, ok_row ? 16u : 0u);
+            }
+            cp_async_arrive_noinc(bar_kv_full(st));
+            if (pf_lane && i + kPrefetchTiles < ntiles) prefetch_row(pf);
+            if (i + 1 < ntiles) {
+                cur0 = load_pos(i + 1, rr);
+                cur1 = load_pos(i + 1, rr + 32);
+                if (pf_lane && i + 1 + kPrefetchTiles < ntiles) pf = load_pos(i + 1 + kPrefetchTiles, rr + 32 * half);
+                // the next tile's stage is free once PV(i - 1) has completed
+                if (i + 1 >= kStages) {
+                    bool ok = true;
+                    if (lane == 0)
+                        ok = mbar_wait_spin(bar_kv_empty((i + 1) & 1), (((i + 1) >> 1) - 1) & 1, abort_flag, a.status);
+                    ok = __shfl_sync(0xffffffffu, ok, 0);
+                    if (!ok) break;
+                }
+            }
+        }
+        // copies still in flight on an early exit land before the CTA's shared memory goes away
+        cp_async_wait_all();
+    } else if (warp == 4) {
+        // ------------------------------------------------ MMA issue (converged warp, one elected lane)
+        if (ntiles > 0) {
+            // warp-uniform copies of the bases keep the per-MMA operands in uniform registers
+            const uint32_t tm = __shfl_sync(0xffffffffu, tmem, 0);
+            const uint32_t sb0 = __shfl_sync(0xffffffffu, sbase, 0);
             bool ok = mbar_wait(bar_q, 0, abort_flag, a.status);
+            ok = __shfl_sync(0xffffffffu, ok, 0);
+            const uint64_t dq = make_smem_desc(sb0 + kOffQ, 16, 1024, kSwizzle128B);
+            const uint64_t dk = make_smem_desc(sb0 + kOffKv, 16, 1024, kSwizzle128B);
+            const uint64_t dp = make_smem_desc(sb0 + kOffP, 16, 1024, kSwizzle128B);
+            const uint64_t dv = make_smem_desc(sb0 + kOffKv, kChunkBytes, 1024, kSwizzle128B);
             // Issue in dependency order, whichever is ready first: QK^T(q) needs its
-            // gathered tile and PV(q-2) already issued (S/P buffer reuse); PV(p) needs
+            // gathered tile and PV(q-2) already issued (S buffer reuse); PV(p) needs
             // the softmax of tile p.  PV is preferred: it frees a gather stage.
             int qk = 0, pv = 0;
             uint64_t t_last = globaltimer_ns();
             uint32_t spins = 0;
             while (ok && pv < ntiles) {
-                if (pv < qk && mbar_test(bar_p_full(pv & 1), (pv >> 1) & 1)) {
+                const bool pv_ready = pv < qk && __shfl_sync(0xffffffffu, mbar_test(bar_p_full, pv & 1), 0);
+                const bool qk_ready = !pv_ready && qk < ntiles && qk <= pv + 1 &&
+                                      __shfl_sync(0xffffffffu, mbar_test(bar_kv_full(qk & 1), (qk >> 1) & 1), 0);
+                if (pv_ready) {
                     tc_fence_after();
-                    const int sb = pv & 1;
-                    const uint32_t v_base = sKv + sb * kKvStageBytes + (4 * half) * kKvChunkBytes;
+                    const uint32_t soff = (pv & 1) * kKvStageBytes;
 #pragma unroll
-                    for (int ks = 0; ks < 2; ++ks) {
-                        const uint64_t bd = make_smem_desc(v_base + ks * 2048, kKvChunkBytes, 1024, kSwizzle128B);
-                        mma_f16_ts(tmem + kColO, tmem + kColS + 32 * sb + 8 * ks, bd, kIdescPV,
-                                   (pv > 0 || ks > 0) ? 1u : 0u);
+                    for (int vh = 0; vh < 2; ++vh) {
+#pragma unroll
+                        for (int ks = 0; ks < 4; ++ks) {
+                            const uint64_t ad = dp + ((ks * 32) >> 4);
+                            const uint64_t bd = dv + ((soff + vh * 4 * kChunkBytes + ks * 2048) >> 4);
+                            if (elect_one())
+                                mma_f16_ss(tm + (vh ? kLaneHi : 0u), ad, bd, kIdescPV, (pv > 0 || ks > 0) ? 1u : 0u);
+                        }
                     }
-                    mma_commit(bar_kv_empty(sb));
+                    if (elect_one()) mma_commit(bar_kv_empty(pv & 1));
+                    __syncwarp();
                     ++pv;
                     t_last = globaltimer_ns();
-                } else if (qk < ntiles && qk <= pv + 1 && mbar_test(bar_kv_full(qk & 1), (qk >> 1) & 1)) {
+                } else if (qk_ready) {
                     tc_fence_after();
-                    const int st = qk & 1;
-                    const uint32_t d = tmem + kColS + 32 * st;
-                    const uint32_t k_base = sKv + st * kKvStageBytes;
-#pragma unroll 1
+                    const uint32_t d = tm + kColS + 64 * (qk & 1);
+                    const uint32_t soff = (qk & 1) * kKvStageBytes;
+#pragma unroll
                     for (int c = 0; c < kChunks; ++c) {
 #pragma unroll
                         for (int kk = 0; kk < 4; ++kk) {
-                            const uint64_t ad = make_smem_desc(sQ + c * kQChunkBytes + kk * 32, 16, 1024, kSwizzle128B);
-                            const uint64_t bd = make_smem_desc(k_base + c * kKvChunkBytes + kk * 32, 16, 1024, kSwizzle128B);
-                            mma_f16_ss(d, ad, bd, kIdescQK, (c | kk) ? 1u : 0u);
+                            const uint32_t off = c * kChunkBytes + kk * 32;
+                            if (elect_one())
+                                mma_f16_ss(d, dq + (off >> 4), dk + ((soff + off) >> 4), kIdescQK, (c | kk) ? 1u : 0u);
                         }
                     }
-                    mma_commit(bar_s_full(st));
+                    if (elect_one()) mma_commit(bar_s_full(qk & 1));
+                    __syncwarp();
                     ++qk;
                     t_last = globaltimer_ns();
                 } else if ((++spins & 255u) == 0) {
+                    bool stop = false;
                     if (*abort_flag) {
-                        ok = false;
+                        stop = true;
                     } else if (globaltimer_ns() - t_last > kWaitBudgetNs) {
-                        record_status(a.status, DSA_STATUS_TIMEOUT);
-                        *abort_flag = 1;
-                        ok = false;
+                        if (lane == 0) {
+                            record_status(a.status, DSA_STATUS_TIMEOUT);
+                            *abort_flag = 1;
+                        }
+                        stop = true;
                     }
+                    ok = !__shfl_sync(0xffffffffu, stop, 0);
                 }
             }
-            if (ok) mma_commit(bar_o);
-            if (!ok && pv > 0)
+            if (ok && elect_one()) mma_commit(bar_o);
+            __syncwarp();
+            if (!ok && pv > 0 && lane == 0)
                 mbar_wait(bar_kv_empty((pv - 1) & 1), ((pv - 1) >> 1) & 1, nullptr, nullptr, 50000000ull);
         }
-    } else if (warp >= 5) {
-        // ------------------------------------------------ gather producers
-        const int p = tid - 5 * 32;  // 0..127
-        for (int i = 0; i < ntiles; ++i) {
-            const int st = i & 1;
-            if (i >= kStages && !mbar_wait(bar_kv_empty(st), ((i >> 1) - 1) & 1, abort_flag, a.status)) break;
-            // keep the L2 prefetch kPrefetchTiles tiles ahead of the gather (each CTA of
-            // the value pair takes every other row)
-            if (p < kTileRows && i + kPrefetchTiles < ntiles && (p & 1) == half) {
-                const int s = sidx[(i + kPrefetchTiles) * kTileRows + p];
-                if (s >= 0) l2_prefetch_bulk(kv_seq + (int64_t)s * kDK, kDK * 2);
-            }
-            const uint32_t stage = sKv + st * kKvStageBytes;
-            const int32_t* tile_idx = sidx + i * kTileRows;
-            uint4 v[kGranules / kGatherThreads];
-#pragma unroll
-            for (int u = 0; u < kGranules / kGatherThreads; ++u) {
-                const int G = p + u * kGatherThreads;
-                const int r = G / 72, c = G % 72;
-                const int s = tile_idx[r];
-                if (s >= 0) {
-                    v[u] = __ldg(reinterpret_cast<const uint4*>(kv_seq + (int64_t)s * kDK) + c);
-                } else {
-                    v[u] = make_uint4(0u, 0u, 0u, 0u);
-                }
-            }
-#pragma unroll
-            for (int u = 0; u < kGranules / kGatherThreads; ++u) {
-                const int G = p + u * kGatherThreads;
-                const int r = G / 72, c = G % 72;
-                const int chunk = c >> 3, g = c & 7;
-                const uint32_t dst = stage + chunk * kKvChunkBytes + (r >> 3) * 1024 + (r & 7) * 128 + ((g ^ (r & 7)) << 4);
-                asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(dst), "r"(v[u].x), "r"(v[u].y),
-                             "r"(v[u].z), "r"(v[u].w)
-                             : "memory");
-            }
-            fence_proxy_async_smem();
-            mbar_arrive(bar_kv_full(st));
-        }
     } else {
-        // ------------------------------------------------ softmax, one head per thread
-        const int h = tid;  // warps 0..3 -> TMEM lanes 0..127
-        const uint32_t lane_addr = tmem + ((uint32_t)(warp * 32) << 16);
+        // ------------------------------------------------ softmax, two threads per head
+        const int r = lane & 15, hh = lane >> 4;
+        const uint32_t lane_base = tmem + ((uint32_t)(warp * 32) << 16);
         const float scale_log2 = a.softmax_scale * 1.4426950408889634f;
+        const int prow = warp * 16 + r;  // head within this CTA = row of P
+        const uint32_t prow_addr = sP + (prow >> 3) * 1024 + (prow & 7) * 128;
         float m_used = -CUDART_INF_F;
         float l = 0.f;
         bool ok = true;
         for (int i = 0; i < ntiles; ++i) {
             const int sb = i & 1;
-            const unsigned valid = __ballot_sync(0xffffffffu, sidx[i * kTileRows + lane] >= 0);
-            ok = mbar_wait(bar_s_full(sb), (i >> 1) & 1, abort_flag, a.status);
+            const unsigned b0 = __ballot_sync(0xffffffffu, valid(v0));
+            const unsigned b1 = __ballot_sync(0xffffffffu, valid(v1));
+            const unsigned vbits = hh ? b1 : b0;
+            if (i + 1 < ntiles) {
+                v0 = load_pos(i + 1, lane);
+                v1 = load_pos(i + 1, lane + 32);
+            }
+            ok = mbar_wait_spin(bar_s_full(sb), (i >> 1) & 1, abort_flag, a.status);
             ok = __all_sync(0xffffffffu, ok);
             if (!ok) break;
             tc_fence_after();
             uint32_t sv[32];
-            tmem_ld32(lane_addr + kColS + 32 * sb, sv);
+            tmem_ld16x2_32(lane_base + kColS + 64 * sb, sv);
             tmem_wait_ld();
             float x[32];
             float mx = -CUDART_INF_F;
 #pragma unroll
             for (int c = 0; c < 32; ++c) {
-                x[c] = ((valid >> c) & 1u) ? __uint_as_float(sv[c]) * scale_log2 : -CUDART_INF_F;
+                x[c] = ((vbits >> c) & 1u) ? __uint_as_float(sv[c]) * scale_log2 : -CUDART_INF_F;
                 mx = fmaxf(mx, x[c]);
+            }
+            mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
+            // P's buffer and O are free once PV(i-1) has completed
+            if (i > 0) {
+                ok = mbar_wait_spin(bar_kv_empty((i - 1) & 1), ((i - 1) >> 1) & 1, abort_flag, a.status);
+                ok = __all_sync(0xffffffffu, ok);
+                if (!ok) break;
+                tc_fence_after();
             }
             if (mx > m_used + kRescaleThreshold) {
                 if (m_used != -CUDART_INF_F) {
-                    // O holds data scaled by 2^-m_used: wait until PV(i-1) landed, then rescale it
+                    // this thread's TMEM lane holds one 256-wide half of its head's O row
                     const float alpha = fast_exp2(m_used - mx);
-                    ok = mbar_wait(bar_kv_empty((i - 1) & 1), ((i - 1) >> 1) & 1, abort_flag, a.status);
-                    ok = __all_sync(0xffffffffu, ok);
-                    if (!ok) break;
-                    tc_fence_after();
 #pragma unroll 1
                     for (int c0 = 0; c0 < 256; c0 += 32) {
                         uint32_t ov[32];
-                        tmem_ld32(lane_addr + kColO + c0, ov);
+                        tmem_ld32(lane_base + c0, ov);
                         tmem_wait_ld();
 #pragma unroll
                         for (int c = 0; c < 32; ++c) ov[c] = __float_as_uint(__uint_as_float(ov[c]) * alpha);
-                        tmem_st32(lane_addr + kColO + c0, ov);
+                        tmem_st32(lane_base + c0, ov);
                     }
                     tmem_wait_st();
                     l *= alpha;
@@ -310,62 +372,88 @@ __global__ void __launch_bounds__(kThreads, 1)
                 pk[c] = pack_bf16x2(p0, p1);
             }
             l += rs;
-            tmem_st16(lane_addr + kColS + 32 * sb, pk);
-            tmem_wait_st();
+#pragma unroll
+            for (int q4 = 0; q4 < 4; ++q4) {
+                const int g = 4 * hh + q4;  // 16-byte granule = 8 positions of the tile
+                asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(prow_addr + ((g ^ (prow & 7)) << 4)),
+                             "r"(pk[4 * q4]), "r"(pk[4 * q4 + 1]), "r"(pk[4 * q4 + 2]), "r"(pk[4 * q4 + 3])
+                             : "memory");
+            }
+            fence_proxy_async_smem();
             tc_fence_before();
-            mbar_arrive(bar_p_full(sb));
+            mbar_arrive(bar_p_full);
         }
-        // ---- epilogue
-        const float inv_l = l > 0.f ? 1.f / l : 0.f;
-        const float lse_v = l > 0.f ? (m_used + __log2f(l)) * 0.6931471805599453f : -CUDART_INF_F;
+        // ---- epilogue: lane r owns O[head, 0:256], lane r + 16 owns O[head, 256:512].
+        // The normalised tile is staged in the (now idle) gather stages as 128B-swizzled
+        // boxes of 64 heads x 128 bytes and written by TMA tensor stores, so the global
+        // writes are whole lines instead of one 16-byte piece per head row.
+        const float l_row = l + __shfl_xor_sync(0xffffffffu, l, 16);
+        const float inv_l = l_row > 0.f ? 1.f / l_row : 0.f;
+        const float lse_v = l_row > 0.f ? (m_used + __log2f(l_row)) * 0.6931471805599453f : -CUDART_INF_F;
         const bool have_o = ok && ntiles > 0;
         if (have_o) {
-            ok = mbar_wait(bar_o, 0, abort_flag, a.status);
+            ok = mbar_wait_spin(bar_o, 0, abort_flag, a.status);
             ok = __all_sync(0xffffffffu, ok);
         }
-        const int64_t th = (int64_t)t * kHeads + h;
-        if (a.splits == 1) {
-            __nv_bfloat16* o = reinterpret_cast<__nv_bfloat16*>(a.out) + th * kDV + half * 256;
-            if (half == 0 && a.lse) a.lse[th] = lse_v;
-            if (have_o && ok) tc_fence_after();
-#pragma unroll 1
-            for (int c0 = 0; c0 < 256; c0 += 32) {
-                uint32_t ov[32];
-                if (have_o && ok) {
-                    tmem_ld32(lane_addr + kColO + c0, ov);
-                    tmem_wait_ld();
-                } else {
-#pragma unroll
-                    for (int c = 0; c < 32; ++c) ov[c] = 0u;
-                }
-                uint32_t pk[16];
-#pragma unroll
-                for (int c = 0; c < 16; ++c)
-                    pk[c] = pack_bf16x2(__uint_as_float(ov[2 * c]) * inv_l, __uint_as_float(ov[2 * c + 1]) * inv_l);
-                uint4* dst = reinterpret_cast<uint4*>(o + c0);
-#pragma unroll
-                for (int q4 = 0; q4 < 4; ++q4) dst[q4] = make_uint4(pk[4 * q4], pk[4 * q4 + 1], pk[4 * q4 + 2], pk[4 * q4 + 3]);
+        const bool read_o = have_o && ok;
+        if (read_o) tc_fence_after();
+        const int64_t th = (int64_t)t * kMlaHeads + half * kCtaHeads + prow;
+        const bool final_out = a.splits == 1;
+        if (hh == 0) {
+            if (final_out) {
+                if (a.lse) a.lse[th] = lse_v;
+            } else {
+                a.part_lse[(int64_t)split * a.Nq * kMlaHeads + th] = lse_v;
             }
-        } else {
-            float* o = a.part_o + ((int64_t)split * a.Nq * kHeads + th) * kDV + half * 256;
-            if (half == 0) a.part_lse[(int64_t)split * a.Nq * kHeads + th] = lse_v;
-            if (have_o && ok) tc_fence_after();
+        }
+        const uint32_t row_addr = sKv + prow * 128;
 #pragma unroll 1
-            for (int c0 = 0; c0 < 256; c0 += 32) {
-                uint32_t ov[32];
-                if (have_o && ok) {
-                    tmem_ld32(lane_addr + kColO + c0, ov);
-                    tmem_wait_ld();
-                } else {
+        for (int c0 = 0; c0 < 256; c0 += 32) {
+            uint32_t ov[32];
+            if (read_o) {
+                tmem_ld32(lane_base + c0, ov);
+                tmem_wait_ld();
+            } else {
 #pragma unroll
-                    for (int c = 0; c < 32; ++c) ov[c] = 0u;
-                }
-                float4* dst = reinterpret_cast<float4*>(o + c0);
-#pragma unroll
-                for (int q4 = 0; q4 < 8; ++q4)
-                    dst[q4] = make_float4(__uint_as_float(ov[4 * q4]) * inv_l, __uint_as_float(ov[4 * q4 + 1]) * inv_l,
-                                          __uint_as_float(ov[4 * q4 + 2]) * inv_l, __uint_as_float(ov[4 * q4 + 3]) * inv_l);
+                for (int c = 0; c < 32; ++c) ov[c] = 0u;
             }
+            const int col = hh * 256 + c0;  // first output column of this piece
+            if (final_out) {
+                // bf16: box k holds columns [64k, 64k + 64); this piece is 4 granules of it
+                const uint32_t box = row_addr + (col >> 6) * kChunkBytes;
+                const int g0 = (col & 63) >> 3;
+#pragma unroll
+                for (int q4 = 0; q4 < 4; ++q4) {
+                    uint32_t w[4];
+#pragma unroll
+                    for (int e = 0; e < 4; ++e)
+                        w[e] = pack_bf16x2(__uint_as_float(ov[8 * q4 + 2 * e]) * inv_l,
+                                           __uint_as_float(ov[8 * q4 + 2 * e + 1]) * inv_l);
+                    asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(box + (((g0 + q4) ^ (prow & 7)) << 4)),
+                                 "r"(w[0]), "r"(w[1]), "r"(w[2]), "r"(w[3])
+                                 : "memory");
+                }
+            } else {
+                // fp32: box k holds columns [32k, 32k + 32); this piece is the whole box row
+                const uint32_t box = row_addr + (col >> 5) * kChunkBytes;
+#pragma unroll
+                for (int g = 0; g < 8; ++g)
+                    asm volatile("st.shared.v4.f32 [%0], {%1, %2, %3, %4};" ::"r"(box + ((g ^ (prow & 7)) << 4)),
+                                 "f"(__uint_as_float(ov[4 * g]) * inv_l), "f"(__uint_as_float(ov[4 * g + 1]) * inv_l),
+                                 "f"(__uint_as_float(ov[4 * g + 2]) * inv_l), "f"(__uint_as_float(ov[4 * g + 3]) * inv_l)
+                                 : "memory");
+            }
+        }
+        fence_proxy_async_smem();
+        named_barrier_sync(1, 128);
+        if (tid == 0) {
+            const int nbox = final_out ? kDV / 64 : kDV / 32;
+            const int y = final_out ? t * kMlaHeads + half * kCtaHeads
+                                    : (split * a.Nq + t) * kMlaHeads + half * kCtaHeads;
+            for (int k = 0; k < nbox; ++k)
+                tma_store_2d(&tmap_o, k * (final_out ? 64 : 32), y, sKv + k * kChunkBytes);
+            bulk_commit_group();
+            bulk_wait_group_read0();
         }
     }
     tc_fence_before();
@@ -380,8 +468,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 // owns values [4j, 4j+4) of the 512-wide output row.
 __global__ void __launch_bounds__(128) mla_combine_kernel(const MlaArgs a) {
     const int h = blockIdx.x, t = blockIdx.y, j = threadIdx.x;
-    const int64_t plane = (int64_t)a.Nq * kHeads;
-    const int64_t th = (int64_t)t * kHeads + h;
+    const int64_t plane = (int64_t)a.Nq * kMlaHeads;
+    const int64_t th = (int64_t)t * kMlaHeads + h;
     float lp[16];
     float L = -CUDART_INF_F;
 #pragma unroll
@@ -417,13 +505,22 @@ __global__ void __launch_bounds__(128) mla_combine_kernel(const MlaArgs a) {
 
 cudaError_t launch_sparse_mla_bf16(const MlaArgs& a, cudaStream_t st) {
     if (a.Nq == 0) return cudaSuccess;
+    // q: [Nq * 128 heads, 576] bf16, 64 x 64 boxes, 128B-swizzled
     alignas(64) CUtensorMap tq;
-    if (!encode_tensor_map_2d(&tq, 2, a.q, kDK, (uint64_t)a.Nq * kHeads, kDK * 2, 64, kHeads, 128))
+    if (!encode_tensor_map_2d(&tq, 2, a.q, kDK, (uint64_t)a.Nq * kMlaHeads, kDK * 2, 64, kCtaHeads, 128))
+        return cudaErrorInvalidValue;
+    // output: bf16 [Nq * 128, 512] (one split) or fp32 partials [splits * Nq * 128, 512];
+    // boxes of 128 bytes x 64 heads, 128B-swizzled
+    alignas(64) CUtensorMap to;
+    const bool final_out = a.splits == 1;
+    const uint64_t out_rows = (uint64_t)(final_out ? 1 : a.splits) * a.Nq * kMlaHeads;
+    if (!encode_tensor_map_2d(&to, final_out ? 2 : 4, final_out ? a.out : static_cast<void*>(a.part_o), kDV, out_rows,
+                              kDV * (final_out ? 2 : 4), final_out ? 64 : 32, kCtaHeads, 128))
         return cudaErrorInvalidValue;
     cudaError_t e = cudaFuncSetAttribute(sparse_mla_bf16_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
     if (e != cudaSuccess) return e;
     dim3 grid(a.splits, 2, a.Nq);
-    sparse_mla_bf16_kernel<<<grid, kThreads, kSmemBytes, st>>>(a, tq);
+    sparse_mla_bf16_kernel<<<grid, kThreads, kSmemBytes, st>>>(a, tq, to);
     return cudaGetLastError();
 }
 
@@ -461,7 +558,7 @@ cudaError_t static_mla_scratch(void** ptr) {
 cudaError_t launch_mla_combine(const MlaArgs& a, cudaStream_t st) {
     if (a.Nq == 0 || a.splits <= 1) return cudaSuccess;
     if (a.splits > 16) return cudaErrorInvalidValue;
-    mla_combine_kernel<<<dim3(kHeads, a.Nq), 128, 0, st>>>(a);
+    mla_combine_kernel<<<dim3(kMlaHeads, a.Nq), 128, 0, st>>>(a);
     return cudaGetLastError();
 }
 

@@ -66,8 +66,15 @@ def test_noalloc_matches_workspace_entry_on_two_calls(lib):
 
 def test_noalloc_refuses_requests_beyond_its_scratch(lib):
     sms = torch.cuda.get_device_properties(0).multi_processor_count
-    # the split count the library plans: sms // (2 nq), clamped to [1, 16]
-    nq = next(q for q in range(1, 75) if max(1, min(16, sms // (2 * q))) * q > 64)
+
+    def planned_splits(q, k=2048, tile=64):
+        # the library's plan: sms // (2 nq) splits clamped to [1, 16], rows per
+        # split rounded up to whole 64-row tiles, then the splits those rows need
+        s = max(1, min(16, sms // (2 * q)))
+        rows = -(-(-(-k // s)) // tile) * tile
+        return -(-k // rows)
+
+    nq = next(q for q in range(1, 75) if planned_splits(q) * q > 64)
     g = inputs.make_decode_inputs("noalloc_big", [2048] * nq, T_max=2048, seed=7).to("cuda")
     idx = random_index_lists(nq, 2048, g.k, 7).cuda()
     out, lse = api.alloc_outputs(g)

@@ -68,6 +68,6 @@ def check_attention(gpu_out, ora_out, gpu_lse=None, ora_lse=None, rows=None):
         if rows is not None:
             gl, ol = gl[rows], ol[rows]
         both_inf = np.isneginf(gl) & np.isneginf(ol)
-        d = np.where(both_inf, 0.0, np.abs(gl - ol))
+        d = np.abs(np.where(both_inf, 0.0, gl) - np.where(both_inf, 0.0, ol))
         assert np.all(d <= 1e-2 + 1e-3 * np.abs(np.where(both_inf, 0, ol))), f"lse mismatch: {np.nanmax(d)}"
     return worst
