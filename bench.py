@@ -235,7 +235,10 @@ def run_ours(args):
     if status != 0:
         raise SystemExit(f"device status {status}: {api.status_string(status)}")
 
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(K)]
+    # Headline pass: one start and one end event per step.  Events recorded between the
+    # stages cost ~2 us of GPU time each, so the per-stage breakdown (and the indexer
+    # duration the roofline uses) comes from a second pass right after this one.
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(K)]
     vis = os.environ.get("CUDA_VISIBLE_DEVICES", "")
     ids = [x for x in vis.split(",") if x.strip()]
     li = local if world > 1 else 0
@@ -247,17 +250,27 @@ def run_ours(args):
     wall0 = time.perf_counter()
     for i in range(K):
         flush.zero_()   # L2 flush outside the timed events
-        api.run_decode(inp, ws=ws, out=out, lse=lse, dims=dims, events=evs[i])
+        evs[i][0].record()
+        api.run_decode(inp, ws=ws, out=out, lse=lse, dims=dims)
+        evs[i][1].record()
     torch.cuda.synchronize()
     wall1 = time.perf_counter()
     wall = wall1 - wall0
     barrier(world)
     clocks = sampler.stop(window=(wall0, wall1))
-    stage = [[evs[i][j].elapsed_time(evs[i][j + 1]) for j in range(4)] for i in range(K)]
-    step_ms = [sum(s) for s in stage]
+    step_ms = [evs[i][0].elapsed_time(evs[i][1]) for i in range(K)]
     mean_ms = sum(step_ms) / K
     mean_ms = max_over_ranks(mean_ms, world)
-    stage_us = [1000 * sum(s[j] for s in stage) / K for j in range(4)]
+
+    # Stage pass: the same steps with an event before the indexer and after every stage.
+    KS = min(K, 1000)
+    sev = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(KS)]
+    for i in range(KS):
+        flush.zero_()
+        api.run_decode(inp, ws=ws, out=out, lse=lse, dims=dims, events=sev[i])
+    torch.cuda.synchronize()
+    stage = [[sev[i][j].elapsed_time(sev[i][j + 1]) for j in range(4)] for i in range(KS)]
+    stage_us = [1000 * sum(s[j] for s in stage) / KS for j in range(4)]
     status = api.get_device_status(ws)
 
     # ---- end to end through the C interface with host buffers
@@ -306,7 +319,9 @@ def run_ours(args):
                       "merge": stage_us[3]},
         "e2e": {"value": BATCH * world / (e2e_ms * 1e-3), "unit": UNIT, "h2d_bytes_per_step": e2e["h2d"],
                 "d2h_bytes_per_step": e2e["d2h"], "ms_per_step": e2e_ms},
-        "gpu_launches": 4 * K,
+        "gpu_launches": launches_per_step() * K,
+        "timing": {"step": "one start and one end event per step on the launching stream",
+                   "stages_us": f"separate pass of {KS} steps with an event between stages (each adds ~2 us)"},
         "clocks": {"sm_mhz": clocks["sm_mhz"], "sm_max_mhz": clocks["sm_max_mhz"], "reasons": clocks["reasons"],
                    "samples": clocks["samples"]},
         "device_status": status,
@@ -316,6 +331,17 @@ def run_ours(args):
         line["cpu_baseline"] = cpu
     print(json.dumps(line), flush=True)
     return 0
+
+
+def launches_per_step():
+    """Kernels one decode step launches: indexer, top-k, attention, plus the split
+    merge when the attention's split count is above the cluster limit (8)."""
+    import torch
+    sms = torch.cuda.get_device_properties(0).multi_processor_count
+    s = max(1, min(16, sms // (2 * BATCH)))
+    rows = -(-(-(-2048 // s)) // 64) * 64
+    splits = -(-2048 // rows)
+    return 4 if splits > 8 else 3
 
 
 def measure_e2e(inp, dims, ws, dev, steps, warmup):

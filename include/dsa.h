@@ -142,8 +142,10 @@ dsa_status_t dsa_topk(const dsa_dims* dims, const float* scores, const int32_t* 
  *   lse[t,h]   = ln sum_s exp(softmax_scale * q[t,h,:] . kv[b,s,:])
  * An empty selection gives out = 0, lse = -inf.  lse may be NULL.
  * Entries of idx outside [-1, q_len[t]) are treated as -1 and flagged
- * DSA_ERR_INDEX_OOB in the status word.  Workspace (sized for
- * DSA_OP_SPARSE_MLA) holds the split partial results. */
+ * DSA_ERR_INDEX_OOB in the status word.  The k positions of a row are split
+ * across CTAs; up to 8 splits of a row run as one thread-block cluster and
+ * merge on chip, more (small Nq) write fp32 partial results into the
+ * workspace (sized for DSA_OP_SPARSE_MLA) for a merge pass. */
 dsa_status_t dsa_sparse_mla_attn(const dsa_dims* dims, const void* q, const void* kv,
                                  const int32_t* idx, const int32_t* q_seq, const int32_t* q_len,
                                  float softmax_scale, void* out, float* lse,
@@ -158,11 +160,12 @@ dsa_status_t dsa_sparse_mla_attn(const dsa_dims* dims, const void* q, const void
  * kv_dtype DSA_BF16, minus the workspace: the split partials live in a buffer
  * the library holds statically on every GPU that loads it (about 16.1 MiB,
  * kept until the process exits).
- * Limit: (number of splits) x Nq <= 64 partial rows of 128 heads; the split
- * count is the one dsa_sparse_mla_attn would use (it depends on Nq and the
- * device's SM count; 1 split needs no scratch at all).  Larger requests return
- * DSA_ERR_UNSUPPORTED before any launch.  kv_dtype DSA_F32 returns
- * DSA_ERR_UNSUPPORTED.
+ * Limit: when the split count is above 8 (the partials path of
+ * dsa_sparse_mla_attn), (number of splits) x Nq <= 64 partial rows of 128
+ * heads; the split count is the one dsa_sparse_mla_attn would use (it depends
+ * on Nq and the device's SM count).  1 to 8 splits need no scratch at all.
+ * Larger requests return DSA_ERR_UNSUPPORTED before any launch.  kv_dtype
+ * DSA_F32 returns DSA_ERR_UNSUPPORTED.
  * The first call on a device looks up the buffer's device address (once per
  * device, with that device current); make that first call before any stream
  * capture.  All calls share the buffer, so calls whose kernels overlap on the

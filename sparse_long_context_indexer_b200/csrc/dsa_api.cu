@@ -304,7 +304,9 @@ dsa_status_t dsa_sparse_mla_attn_noalloc(const dsa_dims* dims, const void* q, co
     if (!q || !kv || !idx || !q_seq || !q_len || !out || !std::isfinite(softmax_scale)) return DSA_ERR_INVALID_ARG;
     if (!aligned16(q) || !aligned16(kv) || !aligned16(out)) return DSA_ERR_INVALID_ARG;
     const MlaPlan p = plan_mla(dims, dims->Nq);
-    if (p.splits > 1 && (size_t)p.splits * dims->Nq > dsa::kStaticScratchPartials) return DSA_ERR_UNSUPPORTED;
+    // clustered splits merge on chip; only the partials path needs the static scratch
+    if (p.splits > 1 && !dsa::mla_cluster_merge(p.splits) && (size_t)p.splits * dims->Nq > dsa::kStaticScratchPartials)
+        return DSA_ERR_UNSUPPORTED;
     void* scratch = nullptr;
     cudaError_t e = dsa::static_mla_scratch(&scratch);
     if (e != cudaSuccess) return cuda_fail(e);

@@ -57,6 +57,11 @@ cudaError_t launch_indexer_fp8(const IndexerArgs& a, int grid, cudaStream_t st);
 cudaError_t launch_indexer_f32(const IndexerArgs& a, cudaStream_t st);
 cudaError_t launch_topk(const TopkArgs& a, int cluster, cudaStream_t st);
 cudaError_t launch_sparse_mla_bf16(const MlaArgs& a, cudaStream_t st);
+// Splits of one (row, head half) up to this count run as one thread-block cluster and
+// merge through distributed shared memory inside the attention kernel; beyond it they
+// write fp32 partials that launch_mla_combine merges (a no-op in the cluster case).
+constexpr int kMlaClusterMaxSplits = 8;
+inline bool mla_cluster_merge(int splits) { return splits >= 2 && splits <= kMlaClusterMaxSplits; }
 cudaError_t launch_mla_combine(const MlaArgs& a, cudaStream_t st);
 cudaError_t launch_sparse_mla_f32(const MlaArgs& a, cudaStream_t st);
 cudaError_t launch_wait_timeout_selftest(int* status, int timeout_us, cudaStream_t st);

@@ -97,6 +97,11 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
     return *reinterpret_cast<const uint32_t*>(&v);
 }
 
+// Output modes: the final bf16 rows (one split), fp32 partials for the merge kernel,
+// or a cluster of the splits that merges through distributed shared memory.
+enum : int { kOutFinal = 0, kOutPartials = 1, kOutCluster = 2 };
+
+template <int kOut>
 __global__ void __launch_bounds__(kThreads, 1)
     sparse_mla_bf16_kernel(const MlaArgs a, const __grid_constant__ CUtensorMap tmap_q,
                            const __grid_constant__ CUtensorMap tmap_o) {
@@ -398,63 +403,143 @@ __global__ void __launch_bounds__(kThreads, 1)
         const bool read_o = have_o && ok;
         if (read_o) tc_fence_after();
         const int64_t th = (int64_t)t * kMlaHeads + half * kCtaHeads + prow;
-        const bool final_out = a.splits == 1;
-        if (hh == 0) {
-            if (final_out) {
-                if (a.lse) a.lse[th] = lse_v;
-            } else {
-                a.part_lse[(int64_t)split * a.Nq * kMlaHeads + th] = lse_v;
-            }
-        }
-        const uint32_t row_addr = sKv + prow * 128;
+        if (kOut == kOutCluster) {
+            // normalised fp32 rows for the peers: row h at h * 2048 bytes, 16-byte granule j
+            // stored at (j & ~7) | ((j ^ h) & 7); the row's lse beside P's (now idle) tile
+            if (hh == 0) reinterpret_cast<float*>(smem + kOffP)[prow] = lse_v;
+            const uint32_t row_addr = sKv + prow * (kDV * 4);
 #pragma unroll 1
-        for (int c0 = 0; c0 < 256; c0 += 32) {
-            uint32_t ov[32];
-            if (read_o) {
-                tmem_ld32(lane_base + c0, ov);
-                tmem_wait_ld();
-            } else {
+            for (int c0 = 0; c0 < 256; c0 += 32) {
+                uint32_t ov[32];
+                if (read_o) {
+                    tmem_ld32(lane_base + c0, ov);
+                    tmem_wait_ld();
+                } else {
 #pragma unroll
-                for (int c = 0; c < 32; ++c) ov[c] = 0u;
-            }
-            const int col = hh * 256 + c0;  // first output column of this piece
-            if (final_out) {
-                // bf16: box k holds columns [64k, 64k + 64); this piece is 4 granules of it
-                const uint32_t box = row_addr + (col >> 6) * kChunkBytes;
-                const int g0 = (col & 63) >> 3;
-#pragma unroll
-                for (int q4 = 0; q4 < 4; ++q4) {
-                    uint32_t w[4];
-#pragma unroll
-                    for (int e = 0; e < 4; ++e)
-                        w[e] = pack_bf16x2(__uint_as_float(ov[8 * q4 + 2 * e]) * inv_l,
-                                           __uint_as_float(ov[8 * q4 + 2 * e + 1]) * inv_l);
-                    asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(box + (((g0 + q4) ^ (prow & 7)) << 4)),
-                                 "r"(w[0]), "r"(w[1]), "r"(w[2]), "r"(w[3])
-                                 : "memory");
+                    for (int c = 0; c < 32; ++c) ov[c] = 0u;
                 }
-            } else {
-                // fp32: box k holds columns [32k, 32k + 32); this piece is the whole box row
-                const uint32_t box = row_addr + (col >> 5) * kChunkBytes;
+                const int jb = (hh * 256 + c0) >> 2;  // first granule of this piece (a multiple of 8)
 #pragma unroll
                 for (int g = 0; g < 8; ++g)
-                    asm volatile("st.shared.v4.f32 [%0], {%1, %2, %3, %4};" ::"r"(box + ((g ^ (prow & 7)) << 4)),
+                    asm volatile("st.shared.v4.f32 [%0], {%1, %2, %3, %4};" ::"r"(row_addr + ((jb | (g ^ (prow & 7))) << 4)),
                                  "f"(__uint_as_float(ov[4 * g]) * inv_l), "f"(__uint_as_float(ov[4 * g + 1]) * inv_l),
                                  "f"(__uint_as_float(ov[4 * g + 2]) * inv_l), "f"(__uint_as_float(ov[4 * g + 3]) * inv_l)
                                  : "memory");
             }
+        } else {
+            constexpr bool final_out = kOut == kOutFinal;
+            if (hh == 0) {
+                if (final_out) {
+                    if (a.lse) a.lse[th] = lse_v;
+                } else {
+                    a.part_lse[(int64_t)split * a.Nq * kMlaHeads + th] = lse_v;
+                }
+            }
+            const uint32_t row_addr = sKv + prow * 128;
+#pragma unroll 1
+            for (int c0 = 0; c0 < 256; c0 += 32) {
+                uint32_t ov[32];
+                if (read_o) {
+                    tmem_ld32(lane_base + c0, ov);
+                    tmem_wait_ld();
+                } else {
+#pragma unroll
+                    for (int c = 0; c < 32; ++c) ov[c] = 0u;
+                }
+                const int col = hh * 256 + c0;  // first output column of this piece
+                if (final_out) {
+                    // bf16: box k holds columns [64k, 64k + 64); this piece is 4 granules of it
+                    const uint32_t box = row_addr + (col >> 6) * kChunkBytes;
+                    const int g0 = (col & 63) >> 3;
+#pragma unroll
+                    for (int q4 = 0; q4 < 4; ++q4) {
+                        uint32_t w[4];
+#pragma unroll
+                        for (int e = 0; e < 4; ++e)
+                            w[e] = pack_bf16x2(__uint_as_float(ov[8 * q4 + 2 * e]) * inv_l,
+                                               __uint_as_float(ov[8 * q4 + 2 * e + 1]) * inv_l);
+                        asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(box + (((g0 + q4) ^ (prow & 7)) << 4)),
+                                     "r"(w[0]), "r"(w[1]), "r"(w[2]), "r"(w[3])
+                                     : "memory");
+                    }
+                } else {
+                    // fp32: box k holds columns [32k, 32k + 32); this piece is the whole box row
+                    const uint32_t box = row_addr + (col >> 5) * kChunkBytes;
+#pragma unroll
+                    for (int g = 0; g < 8; ++g)
+                        asm volatile("st.shared.v4.f32 [%0], {%1, %2, %3, %4};" ::"r"(box + ((g ^ (prow & 7)) << 4)),
+                                     "f"(__uint_as_float(ov[4 * g]) * inv_l), "f"(__uint_as_float(ov[4 * g + 1]) * inv_l),
+                                     "f"(__uint_as_float(ov[4 * g + 2]) * inv_l), "f"(__uint_as_float(ov[4 * g + 3]) * inv_l)
+                                     : "memory");
+                }
+            }
+            fence_proxy_async_smem();
+            named_barrier_sync(1, 128);
+            if (tid == 0) {
+                const int nbox = final_out ? kDV / 64 : kDV / 32;
+                const int y = final_out ? t * kMlaHeads + half * kCtaHeads
+                                        : (split * a.Nq + t) * kMlaHeads + half * kCtaHeads;
+                for (int k = 0; k < nbox; ++k)
+                    tma_store_2d(&tmap_o, k * (final_out ? 64 : 32), y, sKv + k * kChunkBytes);
+                bulk_commit_group();
+                bulk_wait_group_read0();
+            }
         }
-        fence_proxy_async_smem();
-        named_barrier_sync(1, 128);
-        if (tid == 0) {
-            const int nbox = final_out ? kDV / 64 : kDV / 32;
-            const int y = final_out ? t * kMlaHeads + half * kCtaHeads
-                                    : (split * a.Nq + t) * kMlaHeads + half * kCtaHeads;
-            for (int k = 0; k < nbox; ++k)
-                tma_store_2d(&tmap_o, k * (final_out ? 64 : 32), y, sKv + k * kChunkBytes);
-            bulk_commit_group();
-            bulk_wait_group_read0();
+    }
+    if (kOut == kOutCluster) {
+        // ---- merge of the splits: CTA `rank` of the cluster owns heads [rank * hp, rank * hp + hp)
+        // O = sum_s exp(lse_s - L) O_s / sum_s exp(lse_s - L),  lse = L + ln sum_s exp(lse_s - L)
+        __syncthreads();
+        cluster_sync_all();
+        const int S = a.splits;
+        const int rank = (int)cluster_ctarank();
+        const int hp = (kCtaHeads + S - 1) / S;
+        const int h0 = rank * hp;
+        const int nunits = 2 * max(0, min(kCtaHeads, h0 + hp) - h0);  // (head, half row) units
+        // every unit: lane j owns granules {j, j + 32} of its half row, i.e. two 16-byte pieces
+        // from each split, all loaded before any is used (the reads cross the cluster network)
+        for (int u = warp; u < nunits; u += kThreads / 32) {
+            const int h = h0 + (u >> 1);
+            const int jh = (u & 1) * 64;  // first granule of the half row
+            const float ls = lane < S ? ld_shared_cluster_f32(mapa_shared(sP + h * 4, lane)) : -CUDART_INF_F;
+            float x[kMlaClusterMaxSplits][8];
+            const uint32_t g0 = ((jh + lane) & ~7) | (((jh + lane) ^ h) & 7);
+            const uint32_t g1 = ((jh + lane + 32) & ~7) | (((jh + lane + 32) ^ h) & 7);
+#pragma unroll
+            for (int sp = 0; sp < kMlaClusterMaxSplits; ++sp) {
+                if (sp < S) {
+                    const uint32_t rbase = mapa_shared(sKv + h * (kDV * 4), (uint32_t)sp);
+                    const float4 v0 = ld_shared_cluster_v4_f32(rbase + (g0 << 4));
+                    const float4 v1 = ld_shared_cluster_v4_f32(rbase + (g1 << 4));
+                    x[sp][0] = v0.x; x[sp][1] = v0.y; x[sp][2] = v0.z; x[sp][3] = v0.w;
+                    x[sp][4] = v1.x; x[sp][5] = v1.y; x[sp][6] = v1.z; x[sp][7] = v1.w;
+                }
+            }
+            float L = ls;
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) L = fmaxf(L, __shfl_xor_sync(0xffffffffu, L, o));
+            const float e = (lane < S && L != -CUDART_INF_F) ? __expf(ls - L) : 0.f;
+            float esum = e;
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) esum += __shfl_xor_sync(0xffffffffu, esum, o);
+            float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+            for (int sp = 0; sp < kMlaClusterMaxSplits; ++sp) {
+                const float es = __shfl_sync(0xffffffffu, e, sp);  // 0 for absent or empty splits
+                if (sp < S) {
+#pragma unroll
+                    for (int c = 0; c < 8; ++c) acc[c] = fmaf(es, x[sp][c], acc[c]);
+                }
+            }
+            const float inv = esum > 0.f ? 1.f / esum : 0.f;
+            const int64_t trow = (int64_t)t * kMlaHeads + half * kCtaHeads + h;
+            uint2* o = reinterpret_cast<uint2*>(reinterpret_cast<__nv_bfloat16*>(a.out) + trow * kDV);
+            o[jh + lane] = make_uint2(pack_bf16x2(acc[0] * inv, acc[1] * inv), pack_bf16x2(acc[2] * inv, acc[3] * inv));
+            o[jh + lane + 32] = make_uint2(pack_bf16x2(acc[4] * inv, acc[5] * inv), pack_bf16x2(acc[6] * inv, acc[7] * inv));
+            if (lane == 0 && (u & 1) == 0 && a.lse) a.lse[trow] = esum > 0.f ? L + __logf(esum) : -CUDART_INF_F;
         }
+        // peers keep reading this CTA's rows until every CTA of the cluster is done
+        cluster_sync_all();
     }
     tc_fence_before();
     __syncthreads();
@@ -509,6 +594,27 @@ cudaError_t launch_sparse_mla_bf16(const MlaArgs& a, cudaStream_t st) {
     alignas(64) CUtensorMap tq;
     if (!encode_tensor_map_2d(&tq, 2, a.q, kDK, (uint64_t)a.Nq * kMlaHeads, kDK * 2, 64, kCtaHeads, 128))
         return cudaErrorInvalidValue;
+    dim3 grid(a.splits, 2, a.Nq);
+    if (mla_cluster_merge(a.splits)) {
+        auto kern = sparse_mla_bf16_kernel<kOutCluster>;
+        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+        if (e != cudaSuccess) return e;
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = grid;
+        cfg.blockDim = dim3(kThreads, 1, 1);
+        cfg.dynamicSmemBytes = kSmemBytes;
+        cfg.stream = st;
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeClusterDimension;
+        attr[0].val.clusterDim.x = (unsigned)a.splits;
+        attr[0].val.clusterDim.y = 1;
+        attr[0].val.clusterDim.z = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        e = cudaLaunchKernelEx(&cfg, kern, a, tq, tq);  // the output map is unused in this mode
+        if (e != cudaSuccess) return e;
+        return cudaGetLastError();
+    }
     // output: bf16 [Nq * 128, 512] (one split) or fp32 partials [splits * Nq * 128, 512];
     // boxes of 128 bytes x 64 heads, 128B-swizzled
     alignas(64) CUtensorMap to;
@@ -517,10 +623,10 @@ cudaError_t launch_sparse_mla_bf16(const MlaArgs& a, cudaStream_t st) {
     if (!encode_tensor_map_2d(&to, final_out ? 2 : 4, final_out ? a.out : static_cast<void*>(a.part_o), kDV, out_rows,
                               kDV * (final_out ? 2 : 4), final_out ? 64 : 32, kCtaHeads, 128))
         return cudaErrorInvalidValue;
-    cudaError_t e = cudaFuncSetAttribute(sparse_mla_bf16_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+    auto kern = final_out ? sparse_mla_bf16_kernel<kOutFinal> : sparse_mla_bf16_kernel<kOutPartials>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
     if (e != cudaSuccess) return e;
-    dim3 grid(a.splits, 2, a.Nq);
-    sparse_mla_bf16_kernel<<<grid, kThreads, kSmemBytes, st>>>(a, tq, to);
+    kern<<<grid, kThreads, kSmemBytes, st>>>(a, tq, to);
     return cudaGetLastError();
 }
 
@@ -556,7 +662,7 @@ cudaError_t static_mla_scratch(void** ptr) {
 }
 
 cudaError_t launch_mla_combine(const MlaArgs& a, cudaStream_t st) {
-    if (a.Nq == 0 || a.splits <= 1) return cudaSuccess;
+    if (a.Nq == 0 || a.splits <= 1 || mla_cluster_merge(a.splits)) return cudaSuccess;
     if (a.splits > 16) return cudaErrorInvalidValue;
     mla_combine_kernel<<<dim3(kMlaHeads, a.Nq), 128, 0, st>>>(a);
     return cudaGetLastError();
