@@ -9,25 +9,26 @@
 //   out[t,h,:] = sum_{s in idx[t]} softmax_s(scale * q[t,h,:] . c[s,:]) c[s,0:512]
 //   lse[t,h]   = ln sum_s exp(scale * q[t,h,:] . c[s,:])
 //
-// Design (one CTA per SM, no cluster):
+// Design (one CTA per SM):
 //   grid = (splits, 2 head halves, Nq).  Each CTA owns 64 of the 128 heads, so
-//   its query block (64 x 576 bf16, 72 KB) and two 64-row gather stages (72 KB
-//   each) fit in shared memory together, and every MMA is M = 64:
-//     S = Q K^T   M = 64 heads, N = 64 rows, K = 576   (36 MMAs of K = 16)
-//     O += P V    M = 64 heads, N = 2 x 256 values, K = 64 rows
-//   The two CTAs of a (split, row) pair read the same rows; the second read is
-//   an L2 hit.  TMEM (M = 64 layout: rows in lanes 0..15 of each 32-lane
-//   subpartition, a second accumulator at lane offset 16):
-//     O[:, 0:256]   lanes +0,  columns [0, 256)
-//     O[:, 256:512] lanes +16, columns [0, 256)
-//     S buffers     lanes +0,  columns [256, 320) and [320, 384)
-//   warps 0..3  softmax: two threads per head (lanes r and r+16 of warp w own
-//               head 16w+r, columns [0,32) and [32,64) of S); online softmax in
-//               the exp2 domain with lazy rescaling of O (only when the running
-//               maximum grows by more than 8, i.e. a factor 256); P goes to a
-//               128B-swizzled K-major shared tile, the A operand of P V.
-//   warp 4      TMEM allocator and the single-thread tcgen05.mma issuer:
-//               QK^T(i+1) is issued before PV(i) so the softmax of tile i
+//   every MMA is M = 64:
+//     S = Q K^T   M = 64 heads, N = 64 rows, K = 576   (36 MMAs of K = 16, Q from TMEM)
+//     O += P V    M = 64 heads, N = 2 x 256 values, K = 64 rows (P and V from shared memory)
+//   The query block lives in tensor memory, which leaves shared memory to three
+//   64-row gather stages (72 KB each).  The two CTAs of a (split, row) pair read
+//   the same rows; the second read is an L2 hit.  TMEM (M = 64 layout: rows in
+//   lanes 0..15 of each 32-lane subpartition, "low"; a second set at lane offset
+//   16, "high"):
+//     low   Q (two bf16 per column) at columns [0, 288); S buffers at [384, 448), [448, 512)
+//     high  O[:, 0:256] at columns [0, 256), O[:, 256:512] at [256, 512)
+//   warps 0..3  Q into TMEM at start; softmax with two threads per head (lanes r
+//               and r+16 of warp w own head 16w+r: columns [0,32) and [32,64) of
+//               S, alternate 32-column blocks of O); online softmax in the exp2
+//               domain with lazy rescaling of O (only when the running maximum
+//               grows by more than 8, i.e. a factor 256); P goes to a 128B-swizzled
+//               K-major shared tile, the A operand of P V.
+//   warp 4      TMEM allocator and the MMA issuer (converged warp, one elected
+//               lane): QK^T(i+1) is issued before PV(i) so the softmax of tile i
 //               overlaps the tensor core.
 //   warps 5..12 row gather: 16-byte cp.async copies, eight threads per
 //               128-byte piece of a row (a full line per eight lanes), straight
@@ -39,8 +40,11 @@
 //               prefetched to L2.  (Measured on B200: per-thread 16-byte copies
 //               from 256 threads gather random 128-byte pieces at ~3.3 TB/s,
 //               TMA tile::gather4 at ~1.4 TB/s.)
-// Splits > 1 write normalised fp32 partials and their lse; mla_combine_kernel
-// merges them: O = sum_p exp(lse_p - L) O_p with L = logsumexp_p lse_p.
+// Splits of a (row, head half) up to 8 run as one cluster: each CTA stages its
+// normalised fp32 output and lse in shared memory and, after a cluster barrier,
+// merges a slice of heads from all of them through distributed shared memory:
+// O = sum_p exp(lse_p - L) O_p / sum_p exp(lse_p - L) with L = max_p lse_p.
+// More splits write fp32 partials that mla_combine_kernel merges the same way.
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
@@ -61,23 +65,26 @@ constexpr int kChunkBytes = 64 * 128;           // one chunk of 64 rows (Q block
 constexpr int kQBytes = kChunks * kChunkBytes;  // 73728
 constexpr int kKvStageBytes = kChunks * kChunkBytes;  // 73728
 constexpr int kPBytes = kCtaHeads * kTileRows * 2;    // 8192
-constexpr int kStages = 2;
+constexpr int kStages = 3;
 constexpr int kGatherWarp0 = 5;
 constexpr int kGatherThreads = 256;
 constexpr int kThreads = 32 * kGatherWarp0 + kGatherThreads;  // 416
-constexpr int kOffQ = 0;
-constexpr int kOffKv = kOffQ + kQBytes;
+constexpr int kOffKv = 0;
 constexpr int kOffP = kOffKv + kStages * kKvStageBytes;
 constexpr int kOffBar = kOffP + kPBytes;
-constexpr int kNumBar = 1 + 2 * kStages + 2 + 1 + 1;  // q_full, kv_full[2], kv_empty[2], s_full[2], p_full, o_done
+// q_tma, q_full, kv_full[3], kv_empty[3], s_full[2], p_full, o_done
+constexpr int kNumBar = 2 + 2 * kStages + 2 + 1 + 1;
 constexpr int kOffMisc = kOffBar + kNumBar * 8;
 constexpr int kSmemBytes = kOffMisc + 16 + 1024;
 static_assert(kSmemBytes <= 232448, "shared memory budget of one CTA");
+static_assert(kQBytes <= kKvStageBytes, "the query block is staged through the last gather stage");
+constexpr int kQStage = kStages - 1;     // stage that holds the query block until it is in TMEM
 constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kLaneHi = 16u << 16;  // TMEM lane offset of the second M = 64 accumulator
-constexpr uint32_t kColS = 256;          // S buffers at columns [256, 320), [320, 384)
+constexpr uint32_t kLaneHi = 16u << 16;  // TMEM lane offset of the high M = 64 set
+constexpr uint32_t kColQ = 0;            // Q: 288 columns (576 bf16), low lanes
+constexpr uint32_t kColS = 384;          // S buffers: [384, 448), [448, 512), low lanes
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
-constexpr int kPrefetchTiles = 3;          // L2 prefetch distance of the gather, in tiles
+constexpr int kPrefetchTiles = kStages + 1;  // L2 prefetch distance of the gather, in tiles
 constexpr uint32_t kIdescQK = make_idesc(kCtaHeads, kTileRows, 1 /*bf16*/, 1 /*bf16*/, 0, 0);
 constexpr uint32_t kIdescPV = make_idesc(kCtaHeads, 256, 1 /*bf16*/, 1 /*bf16*/, 0 /*A K-major*/, 1 /*B MN-major*/);
 
@@ -108,16 +115,17 @@ __global__ void __launch_bounds__(kThreads, 1)
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const uint32_t sbase = smem_u32(smem);
-    const uint32_t sQ = sbase + kOffQ;
     const uint32_t sKv = sbase + kOffKv;
+    const uint32_t sQs = sKv + kQStage * kKvStageBytes;  // query block staging (TMA -> TMEM)
     const uint32_t sP = sbase + kOffP;
     const uint32_t bar0 = sbase + kOffBar;
-    const uint32_t bar_q = bar0;
-    auto bar_kv_full = [&](int s) { return bar0 + 8u * (1 + s); };
-    auto bar_kv_empty = [&](int s) { return bar0 + 8u * (1 + kStages + s); };
-    auto bar_s_full = [&](int s) { return bar0 + 8u * (1 + 2 * kStages + s); };
-    const uint32_t bar_p_full = bar0 + 8u * (3 + 2 * kStages);
-    const uint32_t bar_o = bar0 + 8u * (4 + 2 * kStages);
+    const uint32_t bar_q_tma = bar0;
+    const uint32_t bar_q = bar0 + 8u;
+    auto bar_kv_full = [&](int s) { return bar0 + 8u * (2 + s); };
+    auto bar_kv_empty = [&](int s) { return bar0 + 8u * (2 + kStages + s); };
+    auto bar_s_full = [&](int s) { return bar0 + 8u * (2 + 2 * kStages + s); };
+    const uint32_t bar_p_full = bar0 + 8u * (4 + 2 * kStages);
+    const uint32_t bar_o = bar0 + 8u * (5 + 2 * kStages);
     MlaShared* sh = reinterpret_cast<MlaShared*>(smem + kOffMisc);
     volatile int* abort_flag = &sh->abort_flag;
 
@@ -164,21 +172,23 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
 
     if (tid == 0) {
-        mbar_init(bar_q, 1);
+        mbar_init(bar_q_tma, 1);
+        mbar_init(bar_q, 128);
         for (int s = 0; s < kStages; ++s) {
             mbar_init(bar_kv_full(s), kGatherThreads);
             mbar_init(bar_kv_empty(s), 1);
-            mbar_init(bar_s_full(s), 1);
         }
+        for (int s = 0; s < 2; ++s) mbar_init(bar_s_full(s), 1);
         mbar_init(bar_p_full, 128);
         mbar_init(bar_o, 1);
         sh->abort_flag = 0;
         fence_barrier_init();
         if (ntiles > 0) {
-            mbar_arrive_expect_tx(bar_q, kQBytes);
+            // the query block lands in the last gather stage and moves to TMEM from there
+            mbar_arrive_expect_tx(bar_q_tma, kQBytes);
 #pragma unroll 1
             for (int c = 0; c < kChunks; ++c)
-                tma_load_2d(sQ + c * kChunkBytes, &tmap_q, c * 64, t * kMlaHeads + half * kCtaHeads, bar_q);
+                tma_load_2d(sQs + c * kChunkBytes, &tmap_q, c * 64, t * kMlaHeads + half * kCtaHeads, bar_q_tma);
         }
     }
     if (warp == 4) {
@@ -199,7 +209,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         };
         if (pf_lane) prefetch_row(pf_first);
         for (int i = 0; i < ntiles; ++i) {
-            const int st = i & 1;
+            const int st = i % kStages;
             if (gl == 0 && row_ok && half == 0 &&
                 ((cur0 < -1 || cur0 >= n_t) || (cur1 < -1 || cur1 >= n_t)))
                 record_status(a.status, DSA_STATUS_INDEX_OOB);
@@ -209,7 +219,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const int s = h2 ? cur1 : cur0;
                 const int r = rr + 32 * h2;
                 const bool ok_row = valid(s);
-                const __nv_bfloat16* src = ok_row ? kv_seq + (int64_t)s * kDK + gl * 8 : reinterpret_cast<const __nv_bfloat16*>(a.kv);
+                const __nv_bfloat16* src =
+                    ok_row ? kv_seq + (int64_t)s * kDK + gl * 8 : reinterpret_cast<const __nv_bfloat16*>(a.kv);
                 const uint32_t dst = stage + r * 128 + ((gl ^ (r & 7)) << 4);
 #pragma unroll
                 for (int c = 0; c < kChunks; ++c) cp_async16_zfill(dst + c * kChunkBytes, src + c * 64, ok_row ? 16u : 0u);
@@ -220,14 +231,19 @@ __global__ void __launch_bounds__(kThreads, 1)
                 cur0 = load_pos(i + 1, rr);
                 cur1 = load_pos(i + 1, rr + 32);
                 if (pf_lane && i + 1 + kPrefetchTiles < ntiles) pf = load_pos(i + 1 + kPrefetchTiles, rr + 32 * half);
-                // the next tile's stage is free once PV(i - 1) has completed
-                if (i + 1 >= kStages) {
-                    bool ok = true;
-                    if (lane == 0)
-                        ok = mbar_wait_spin(bar_kv_empty((i + 1) & 1), (((i + 1) >> 1) - 1) & 1, abort_flag, a.status);
-                    ok = __shfl_sync(0xffffffffu, ok, 0);
-                    if (!ok) break;
+                const int nx = i + 1;
+                bool ok = true;
+                if (lane == 0) {
+                    if (nx == kQStage) {
+                        // the query block's staging must have moved to TMEM first
+                        ok = mbar_wait_spin(bar_q, 0, abort_flag, a.status);
+                    } else if (nx >= kStages) {
+                        // the stage is free once PV(nx - kStages) has completed
+                        ok = mbar_wait_spin(bar_kv_empty(nx % kStages), ((nx / kStages) - 1) & 1, abort_flag, a.status);
+                    }
                 }
+                ok = __shfl_sync(0xffffffffu, ok, 0);
+                if (!ok) break;
             }
         }
         // copies still in flight on an early exit land before the CTA's shared memory goes away
@@ -240,7 +256,6 @@ __global__ void __launch_bounds__(kThreads, 1)
             const uint32_t sb0 = __shfl_sync(0xffffffffu, sbase, 0);
             bool ok = mbar_wait(bar_q, 0, abort_flag, a.status);
             ok = __shfl_sync(0xffffffffu, ok, 0);
-            const uint64_t dq = make_smem_desc(sb0 + kOffQ, 16, 1024, kSwizzle128B);
             const uint64_t dk = make_smem_desc(sb0 + kOffKv, 16, 1024, kSwizzle128B);
             const uint64_t dp = make_smem_desc(sb0 + kOffP, 16, 1024, kSwizzle128B);
             const uint64_t dv = make_smem_desc(sb0 + kOffKv, kChunkBytes, 1024, kSwizzle128B);
@@ -252,39 +267,46 @@ __global__ void __launch_bounds__(kThreads, 1)
             uint32_t spins = 0;
             while (ok && pv < ntiles) {
                 const bool pv_ready = pv < qk && __shfl_sync(0xffffffffu, mbar_test(bar_p_full, pv & 1), 0);
-                const bool qk_ready = !pv_ready && qk < ntiles && qk <= pv + 1 &&
-                                      __shfl_sync(0xffffffffu, mbar_test(bar_kv_full(qk & 1), (qk >> 1) & 1), 0);
+                const bool qk_ready =
+                    !pv_ready && qk < ntiles && qk <= pv + 1 &&
+                    __shfl_sync(0xffffffffu, mbar_test(bar_kv_full(qk % kStages), (qk / kStages) & 1), 0);
                 if (pv_ready) {
                     tc_fence_after();
-                    const uint32_t soff = (pv & 1) * kKvStageBytes;
+                    const uint32_t soff = (pv % kStages) * kKvStageBytes;
+                    if (elect_one()) {
 #pragma unroll
-                    for (int vh = 0; vh < 2; ++vh) {
+                        for (int vh = 0; vh < 2; ++vh) {
 #pragma unroll
-                        for (int ks = 0; ks < 4; ++ks) {
-                            const uint64_t ad = dp + ((ks * 32) >> 4);
-                            const uint64_t bd = dv + ((soff + vh * 4 * kChunkBytes + ks * 2048) >> 4);
-                            if (elect_one())
-                                mma_f16_ss(tm + (vh ? kLaneHi : 0u), ad, bd, kIdescPV, (pv > 0 || ks > 0) ? 1u : 0u);
+                            for (int ks = 0; ks < 4; ++ks) {
+                                const uint64_t ad = dp + ((ks * 32) >> 4);
+                                const uint64_t bd = dv + ((soff + vh * 4 * kChunkBytes + ks * 2048) >> 4);
+                                mma_f16_ss(tm + kLaneHi + 256u * vh, ad, bd, kIdescPV, (pv > 0 || ks > 0) ? 1u : 0u);
+                            }
                         }
+                        mma_commit(bar_kv_empty(pv % kStages));
                     }
-                    if (elect_one()) mma_commit(bar_kv_empty(pv & 1));
                     __syncwarp();
                     ++pv;
                     t_last = globaltimer_ns();
                 } else if (qk_ready) {
                     tc_fence_after();
                     const uint32_t d = tm + kColS + 64 * (qk & 1);
-                    const uint32_t soff = (qk & 1) * kKvStageBytes;
+                    const uint32_t soff = (qk % kStages) * kKvStageBytes;
+                    // one elected lane issues the whole pass (operands computed by the
+                    // converged warp beforehand stay in uniform registers)
+                    if (elect_one()) {
 #pragma unroll
-                    for (int c = 0; c < kChunks; ++c) {
+                        for (int c = 0; c < kChunks; ++c) {
 #pragma unroll
-                        for (int kk = 0; kk < 4; ++kk) {
-                            const uint32_t off = c * kChunkBytes + kk * 32;
-                            if (elect_one())
-                                mma_f16_ss(d, dq + (off >> 4), dk + ((soff + off) >> 4), kIdescQK, (c | kk) ? 1u : 0u);
+                            for (int kk = 0; kk < 4; ++kk) {
+                                const uint32_t off = c * kChunkBytes + kk * 32;
+                                // K step 4c + kk: 16 bf16 of Q = 8 TMEM columns
+                                mma_f16_ts(d, tm + kColQ + 8u * (4 * c + kk), dk + ((soff + off) >> 4), kIdescQK,
+                                           (c | kk) ? 1u : 0u);
+                            }
                         }
+                        mma_commit(bar_s_full(qk & 1));
                     }
-                    if (elect_one()) mma_commit(bar_s_full(qk & 1));
                     __syncwarp();
                     ++qk;
                     t_last = globaltimer_ns();
@@ -305,19 +327,42 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (ok && elect_one()) mma_commit(bar_o);
             __syncwarp();
             if (!ok && pv > 0 && lane == 0)
-                mbar_wait(bar_kv_empty((pv - 1) & 1), ((pv - 1) >> 1) & 1, nullptr, nullptr, 50000000ull);
+                mbar_wait(bar_kv_empty((pv - 1) % kStages), ((pv - 1) / kStages) & 1, nullptr, nullptr, 50000000ull);
         }
     } else {
         // ------------------------------------------------ softmax, two threads per head
         const int r = lane & 15, hh = lane >> 4;
-        const uint32_t lane_base = tmem + ((uint32_t)(warp * 32) << 16);
+        const uint32_t lane_base = tmem + ((uint32_t)(warp * 32) << 16);  // low lanes of this subpartition
+        const uint32_t o_base = lane_base + kLaneHi;                       // high lanes: O
         const float scale_log2 = a.softmax_scale * 1.4426950408889634f;
         const int prow = warp * 16 + r;  // head within this CTA = row of P
         const uint32_t prow_addr = sP + (prow >> 3) * 1024 + (prow & 7) * 128;
         float m_used = -CUDART_INF_F;
         float l = 0.f;
         bool ok = true;
-        for (int i = 0; i < ntiles; ++i) {
+        if (ntiles > 0) {
+            // ---- the query block into TMEM: 32-column step c of row prow takes 16 columns
+            // (32 bf16, four 16-byte granules of chunk c) per thread
+            ok = mbar_wait(bar_q_tma, 0, abort_flag, a.status);
+            ok = __all_sync(0xffffffffu, ok);
+            if (ok) {
+#pragma unroll 1
+                for (int c = 0; c < kChunks; ++c) {
+                    const uint32_t src = sQs + c * kChunkBytes + prow * 128;
+                    uint32_t w[16];
+#pragma unroll
+                    for (int q4 = 0; q4 < 4; ++q4)
+                        asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
+                                     : "=r"(w[4 * q4]), "=r"(w[4 * q4 + 1]), "=r"(w[4 * q4 + 2]), "=r"(w[4 * q4 + 3])
+                                     : "r"(src + (((4 * hh + q4) ^ (prow & 7)) << 4)));
+                    tmem_st16x2_16(lane_base + kColQ + 32 * c, w);
+                }
+                tmem_wait_st();
+            }
+            tc_fence_before();
+            mbar_arrive(bar_q);
+        }
+        for (int i = 0; i < ntiles && ok; ++i) {
             const int sb = i & 1;
             const unsigned b0 = __ballot_sync(0xffffffffu, valid(v0));
             const unsigned b1 = __ballot_sync(0xffffffffu, valid(v1));
@@ -343,23 +388,23 @@ __global__ void __launch_bounds__(kThreads, 1)
             mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
             // P's buffer and O are free once PV(i-1) has completed
             if (i > 0) {
-                ok = mbar_wait_spin(bar_kv_empty((i - 1) & 1), ((i - 1) >> 1) & 1, abort_flag, a.status);
+                ok = mbar_wait_spin(bar_kv_empty((i - 1) % kStages), ((i - 1) / kStages) & 1, abort_flag, a.status);
                 ok = __all_sync(0xffffffffu, ok);
                 if (!ok) break;
                 tc_fence_after();
             }
             if (mx > m_used + kRescaleThreshold) {
                 if (m_used != -CUDART_INF_F) {
-                    // this thread's TMEM lane holds one 256-wide half of its head's O row
+                    // this thread owns the 32-column blocks [c0 + 32 hh, c0 + 32 hh + 32) of its O row
                     const float alpha = fast_exp2(m_used - mx);
 #pragma unroll 1
-                    for (int c0 = 0; c0 < 256; c0 += 32) {
+                    for (int c0 = 0; c0 < kDV; c0 += 64) {
                         uint32_t ov[32];
-                        tmem_ld32(lane_base + c0, ov);
+                        tmem_ld16x2_32(o_base + c0, ov);
                         tmem_wait_ld();
 #pragma unroll
                         for (int c = 0; c < 32; ++c) ov[c] = __float_as_uint(__uint_as_float(ov[c]) * alpha);
-                        tmem_st32(lane_base + c0, ov);
+                        tmem_st16x2_32(o_base + c0, ov);
                     }
                     tmem_wait_st();
                     l *= alpha;
@@ -388,10 +433,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             tc_fence_before();
             mbar_arrive(bar_p_full);
         }
-        // ---- epilogue: lane r owns O[head, 0:256], lane r + 16 owns O[head, 256:512].
-        // The normalised tile is staged in the (now idle) gather stages as 128B-swizzled
-        // boxes of 64 heads x 128 bytes and written by TMA tensor stores, so the global
-        // writes are whole lines instead of one 16-byte piece per head row.
+        // ---- epilogue: the normalised row goes to shared memory (the gather stages are idle
+        // now), 32 columns per step: this thread's blocks start at col = c0 + 32 hh
         const float l_row = l + __shfl_xor_sync(0xffffffffu, l, 16);
         const float inv_l = l_row > 0.f ? 1.f / l_row : 0.f;
         const float lse_v = l_row > 0.f ? (m_used + __log2f(l_row)) * 0.6931471805599453f : -CUDART_INF_F;
@@ -403,76 +446,65 @@ __global__ void __launch_bounds__(kThreads, 1)
         const bool read_o = have_o && ok;
         if (read_o) tc_fence_after();
         const int64_t th = (int64_t)t * kMlaHeads + half * kCtaHeads + prow;
-        if (kOut == kOutCluster) {
-            // normalised fp32 rows for the peers: row h at h * 2048 bytes, 16-byte granule j
-            // stored at (j & ~7) | ((j ^ h) & 7); the row's lse beside P's (now idle) tile
-            if (hh == 0) reinterpret_cast<float*>(smem + kOffP)[prow] = lse_v;
-            const uint32_t row_addr = sKv + prow * (kDV * 4);
+        if (hh == 0) {
+            if (kOut == kOutCluster) {
+                reinterpret_cast<float*>(smem + kOffP)[prow] = lse_v;  // beside P's (now idle) tile
+            } else if (kOut == kOutFinal) {
+                if (a.lse) a.lse[th] = lse_v;
+            } else {
+                a.part_lse[(int64_t)split * a.Nq * kMlaHeads + th] = lse_v;
+            }
+        }
 #pragma unroll 1
-            for (int c0 = 0; c0 < 256; c0 += 32) {
-                uint32_t ov[32];
-                if (read_o) {
-                    tmem_ld32(lane_base + c0, ov);
-                    tmem_wait_ld();
-                } else {
+        for (int c0 = 0; c0 < kDV; c0 += 64) {
+            uint32_t ov[32];
+            if (read_o) {
+                tmem_ld16x2_32(o_base + c0, ov);
+                tmem_wait_ld();
+            } else {
 #pragma unroll
-                    for (int c = 0; c < 32; ++c) ov[c] = 0u;
-                }
-                const int jb = (hh * 256 + c0) >> 2;  // first granule of this piece (a multiple of 8)
+                for (int c = 0; c < 32; ++c) ov[c] = 0u;
+            }
+            const int col = c0 + 32 * hh;  // first output column of this piece
+            if (kOut == kOutCluster) {
+                // fp32 rows for the peers: row h at h * 2048 bytes, 16-byte granule j at
+                // (j & ~7) | ((j ^ h) & 7)
+                const uint32_t row_addr = sKv + prow * (kDV * 4);
+                const int jb = col >> 2;  // a multiple of 8
 #pragma unroll
                 for (int g = 0; g < 8; ++g)
                     asm volatile("st.shared.v4.f32 [%0], {%1, %2, %3, %4};" ::"r"(row_addr + ((jb | (g ^ (prow & 7))) << 4)),
                                  "f"(__uint_as_float(ov[4 * g]) * inv_l), "f"(__uint_as_float(ov[4 * g + 1]) * inv_l),
                                  "f"(__uint_as_float(ov[4 * g + 2]) * inv_l), "f"(__uint_as_float(ov[4 * g + 3]) * inv_l)
                                  : "memory");
+            } else if (kOut == kOutFinal) {
+                // bf16 TMA-store boxes of 64 heads x 64 columns: box k holds columns [64k, 64k + 64)
+                const uint32_t box = sKv + prow * 128 + (col >> 6) * kChunkBytes;
+                const int g0 = (col & 63) >> 3;
+#pragma unroll
+                for (int q4 = 0; q4 < 4; ++q4) {
+                    uint32_t w[4];
+#pragma unroll
+                    for (int e = 0; e < 4; ++e)
+                        w[e] = pack_bf16x2(__uint_as_float(ov[8 * q4 + 2 * e]) * inv_l,
+                                           __uint_as_float(ov[8 * q4 + 2 * e + 1]) * inv_l);
+                    asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(box + (((g0 + q4) ^ (prow & 7)) << 4)),
+                                 "r"(w[0]), "r"(w[1]), "r"(w[2]), "r"(w[3])
+                                 : "memory");
+                }
+            } else {
+                // fp32 TMA-store boxes of 64 heads x 32 columns: box k holds columns [32k, 32k + 32)
+                const uint32_t box = sKv + prow * 128 + (col >> 5) * kChunkBytes;
+#pragma unroll
+                for (int g = 0; g < 8; ++g)
+                    asm volatile("st.shared.v4.f32 [%0], {%1, %2, %3, %4};" ::"r"(box + ((g ^ (prow & 7)) << 4)),
+                                 "f"(__uint_as_float(ov[4 * g]) * inv_l), "f"(__uint_as_float(ov[4 * g + 1]) * inv_l),
+                                 "f"(__uint_as_float(ov[4 * g + 2]) * inv_l), "f"(__uint_as_float(ov[4 * g + 3]) * inv_l)
+                                 : "memory");
             }
-        } else {
+        }
+        if (kOut != kOutCluster) {
             constexpr bool final_out = kOut == kOutFinal;
-            if (hh == 0) {
-                if (final_out) {
-                    if (a.lse) a.lse[th] = lse_v;
-                } else {
-                    a.part_lse[(int64_t)split * a.Nq * kMlaHeads + th] = lse_v;
-                }
-            }
-            const uint32_t row_addr = sKv + prow * 128;
-#pragma unroll 1
-            for (int c0 = 0; c0 < 256; c0 += 32) {
-                uint32_t ov[32];
-                if (read_o) {
-                    tmem_ld32(lane_base + c0, ov);
-                    tmem_wait_ld();
-                } else {
-#pragma unroll
-                    for (int c = 0; c < 32; ++c) ov[c] = 0u;
-                }
-                const int col = hh * 256 + c0;  // first output column of this piece
-                if (final_out) {
-                    // bf16: box k holds columns [64k, 64k + 64); this piece is 4 granules of it
-                    const uint32_t box = row_addr + (col >> 6) * kChunkBytes;
-                    const int g0 = (col & 63) >> 3;
-#pragma unroll
-                    for (int q4 = 0; q4 < 4; ++q4) {
-                        uint32_t w[4];
-#pragma unroll
-                        for (int e = 0; e < 4; ++e)
-                            w[e] = pack_bf16x2(__uint_as_float(ov[8 * q4 + 2 * e]) * inv_l,
-                                               __uint_as_float(ov[8 * q4 + 2 * e + 1]) * inv_l);
-                        asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(box + (((g0 + q4) ^ (prow & 7)) << 4)),
-                                     "r"(w[0]), "r"(w[1]), "r"(w[2]), "r"(w[3])
-                                     : "memory");
-                    }
-                } else {
-                    // fp32: box k holds columns [32k, 32k + 32); this piece is the whole box row
-                    const uint32_t box = row_addr + (col >> 5) * kChunkBytes;
-#pragma unroll
-                    for (int g = 0; g < 8; ++g)
-                        asm volatile("st.shared.v4.f32 [%0], {%1, %2, %3, %4};" ::"r"(box + ((g ^ (prow & 7)) << 4)),
-                                     "f"(__uint_as_float(ov[4 * g]) * inv_l), "f"(__uint_as_float(ov[4 * g + 1]) * inv_l),
-                                     "f"(__uint_as_float(ov[4 * g + 2]) * inv_l), "f"(__uint_as_float(ov[4 * g + 3]) * inv_l)
-                                     : "memory");
-                }
-            }
             fence_proxy_async_smem();
             named_barrier_sync(1, 128);
             if (tid == 0) {
