@@ -77,7 +77,7 @@ constexpr size_t kStaticScratchBytes = kStaticScratchOBytes + kStaticScratchPart
 cudaError_t static_mla_scratch(void** ptr);
 
 // Largest row chunk kept in shared memory by one top-k CTA (elements).
-constexpr int kTopkSmemKeys = 49152;
+constexpr int kTopkSmemKeys = 45056;
 
 // cuTensorMapEncodeTiled through the runtime's driver entry point (no -lcuda).
 bool encode_tensor_map_2d(void* map, int dtype_bytes, const void* base, uint64_t inner, uint64_t outer,

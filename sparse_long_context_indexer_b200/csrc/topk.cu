@@ -6,19 +6,27 @@
 // Order: score descending, ties to the lower position, -0.0 == +0.0.  The
 // positions are written in ascending order and padded with -1.
 //
-// Method: each score becomes an order-preserving 32-bit key; a most-
-// significant-digit-first radix select over four 8-bit digits finds the k-th
-// largest key tau and how many keys equal to tau are taken.  A row is split
-// across a thread-block cluster of C CTAs (C <= 8); every CTA keeps its slice
-// of the row in shared memory as keys.  Per digit: warp-private 256-bin
-// histograms (match_any aggregation inside a warp, no cross-warp atomic
-// contention), summed per CTA, then merged across the cluster through
-// distributed shared memory (256 bins x C loads).  The per-CTA counts of keys
-// above / equal to tau fall out of the histograms, so no extra counting pass
-// is needed.  A final pass compacts the selected positions in position order
-// with one block-wide vector scan per sweep; CTA r learns from the lower-
-// ranked CTAs how many ties and outputs precede it, which gives the lower-
-// index tie rule across the whole row.
+// Method: each score becomes an order-preserving 32-bit key; the selection is
+// the k-th largest key tau plus how many keys equal to tau are taken.  A row is
+// split across a thread-block cluster of C CTAs (C <= 8); every CTA keeps its
+// slice of the row in shared memory as keys and tracks their min and max.
+//  1. One histogram of 2048 bins over (key - min) >> shift, the shift chosen
+//     so that the row's key range fills the bins (the top digits of a float
+//     key -- sign and exponent -- put most scores of a row in a handful of
+//     bins, so fixed digits would need several full passes).  CTA r of the
+//     cluster sums one range of bins over all CTAs (distributed shared
+//     memory); the owner of the threshold bin b* broadcasts it.
+//  2. The keys of bin b* are collected (usually a few dozen); CTA 0 gathers
+//     them from the cluster and finds tau among them with a radix select over
+//     four 8-bit digits.  If bin b* holds more than kCandMax keys (extremely
+//     concentrated scores) the kernel falls back to a radix select over four
+//     8-bit digits of all keys (warp-private histograms with match_any
+//     aggregation, merged across the cluster).  Rows whose keys are all equal
+//     take the first k positions directly.
+//  3. A final pass compacts the selected positions in position order with one
+//     block-wide vector scan per sweep; CTA r learns from the lower-ranked CTAs
+//     how many ties and outputs precede it, which gives the lower-index tie
+//     rule across the whole row.
 #include <cooperative_groups.h>
 #include <cuda_runtime.h>
 
@@ -41,7 +49,16 @@ constexpr int kOffTot = kOffHist + 2 * kBins;        // kBins cluster-wide histo
 constexpr int kOffMisc = kOffTot + kBins;            // 64 words: results, counts (read remotely), scan scratch
 constexpr int kOffScan = kOffMisc + 64;              // vector-scan scratch
 constexpr int kScanWords = kWarps * kRounds + kRounds + 16;
-constexpr int kOffKeys = (kOffScan + kScanWords + 3) & ~3;
+constexpr int kFineBits = 11;
+constexpr int kFineBins = 1 << kFineBits;  // adaptive histogram bins
+constexpr int kCandMax = 2048;             // threshold-bin keys resolved on chip by CTA 0
+// Keep a CTA small enough for two per SM at the long-decode chunk (16K keys): with one per
+// SM, 16 clusters of 8 no longer fit the GPCs in one wave.
+constexpr int kOffFine = (kOffScan + kScanWords + 3) & ~3;  // kFineBins counts (read remotely)
+constexpr int kOffRange = kOffFine + kFineBins;            // this CTA's range of cluster-wide bin totals
+constexpr int kOffGather = kOffRange + kFineBins;          // all candidates of the row
+constexpr int kOffKeys = (kOffGather + kCandMax + 3) & ~3;
+static_assert(kWarps * kBins >= kCandMax, "the local candidate list lives in the warp-private histograms");
 constexpr int kBaseWords = kOffKeys;
 
 __device__ __forceinline__ uint32_t score_key(float f) {
@@ -151,6 +168,14 @@ __global__ void __launch_bounds__(kThreads, 2) topk_radix_kernel(const TopkArgs 
     const int hi = min(n, lo + chunk);
     const int len = hi - lo;
     const bool cached = len <= cached_cap;
+    if (tid == 0) {
+        misc[4] = -1;  // key min (as uint32), max
+        misc[5] = 0;
+        misc[6] = 0;   // this CTA's range total
+        misc[13] = 0;  // local candidate count
+    }
+    __syncthreads();
+    uint32_t kmn = 0xFFFFFFFFu, kmx = 0u;
     if (cached) {
         // 16-byte loads, four in flight per thread, keys written in place
         const int nv = len >> 2;
@@ -166,11 +191,35 @@ __global__ void __launch_bounds__(kThreads, 2) topk_radix_kernel(const TopkArgs 
 #pragma unroll
             for (int u = 0; u < 4; ++u) {
                 const int i = i0 + u * kThreads + tid;
-                if (i < nv)
-                    k4[i] = make_uint4(score_key(f[u].x), score_key(f[u].y), score_key(f[u].z), score_key(f[u].w));
+                if (i < nv) {
+                    const uint4 kk = make_uint4(score_key(f[u].x), score_key(f[u].y), score_key(f[u].z), score_key(f[u].w));
+                    k4[i] = kk;
+                    kmn = min(kmn, min(min(kk.x, kk.y), min(kk.z, kk.w)));
+                    kmx = max(kmx, max(max(kk.x, kk.y), max(kk.z, kk.w)));
+                }
             }
         }
-        for (int i = 4 * nv + tid; i < len; i += kThreads) keys[i] = score_key(__ldg(row + lo + i));
+        for (int i = 4 * nv + tid; i < len; i += kThreads) {
+            const uint32_t kk = score_key(__ldg(row + lo + i));
+            keys[i] = kk;
+            kmn = min(kmn, kk);
+            kmx = max(kmx, kk);
+        }
+    } else {
+        for (int i = tid; i < len; i += kThreads) {
+            const uint32_t kk = score_key(__ldg(row + lo + i));
+            kmn = min(kmn, kk);
+            kmx = max(kmx, kk);
+        }
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+        kmn = min(kmn, __shfl_xor_sync(0xffffffffu, kmn, o));
+        kmx = max(kmx, __shfl_xor_sync(0xffffffffu, kmx, o));
+    }
+    if (lane == 0) {
+        atomicMin(reinterpret_cast<unsigned*>(misc + 4), kmn);
+        atomicMax(reinterpret_cast<unsigned*>(misc + 5), kmx);
     }
     __syncthreads();
     auto key_at = [&](int i) -> uint32_t { return cached ? keys[i] : score_key(__ldg(row + lo + i)); };
@@ -185,71 +234,267 @@ __global__ void __launch_bounds__(kThreads, 2) topk_radix_kernel(const TopkArgs 
         r.w = i + 3 < len ? key_at(i + 3) : 0u;
         return r;
     };
-
-    uint32_t prefix = 0, pmask = 0;
-    int remaining = a.k;
-    int local_gt = 0;  // keys of this CTA above tau
-    int local_eq = 0;  // keys of this CTA equal to tau
-#pragma unroll 1
-    for (int p = 0; p < 4; ++p) {
-        const int sh = 24 - 8 * p;
-        uint32_t* hist = sm + kOffHist + (p & 1) * kBins;
-        for (int i = tid; i < kWarps * kBins; i += kThreads) priv[i] = 0u;
-        __syncthreads();
-        uint32_t* my = priv + warp * kBins;
-        for (int i0 = 0; i0 < len; i0 += kThreads) {
-            const int i = i0 + tid;
-            uint32_t kk = 0;
-            bool take = false;
-            if (i < len) {
-                kk = key_at(i);
-                take = (kk & pmask) == prefix;
-            }
-            const unsigned act = __ballot_sync(0xffffffffu, take);
-            if (take) {
-                const uint32_t bin = (kk >> sh) & 0xFFu;
-                const unsigned peers = __match_any_sync(act, bin);
-                if (lane == __ffs(peers) - 1) atomicAdd(&my[bin], (uint32_t)__popc(peers));
-            }
-        }
-        __syncthreads();
-        if (tid < kBins) {
-            uint32_t s = 0;
+    cluster.sync();
+    uint32_t kmin = 0xFFFFFFFFu, kmax = 0u;
 #pragma unroll
-            for (int w = 0; w < kWarps; ++w) s += priv[w * kBins + tid];
-            hist[tid] = s;
+    for (int r = 0; r < 8; ++r) {
+        if (r < C) {
+            const int* rm = cluster.map_shared_rank(misc, r);
+            kmin = min(kmin, (uint32_t)rm[4]);
+            kmax = max(kmax, (uint32_t)rm[5]);
         }
+    }
+
+    uint32_t tau;
+    int take_eq_total;  // keys equal to tau that are selected, lowest positions first
+    int local_gt = 0;   // keys of this CTA above tau
+    int local_eq = 0;   // keys of this CTA equal to tau
+    if (kmin == kmax) {
+        // every key of the row is equal: the first k positions
+        tau = kmin;
+        take_eq_total = a.k;
+        local_eq = len;
+    } else {
+        // ---- 1. adaptive histogram over the row's key range, cluster totals per range of
+        // bins, threshold bin b*
+        const uint32_t span = kmax - kmin;
+        const int shift = max(0, 32 - __clz((int)span) - kFineBits);
+        uint32_t* fine = sm + kOffFine;
+        uint32_t* rng = sm + kOffRange;
+        for (int i = tid; i < kFineBins; i += kThreads) fine[i] = 0u;
+        __syncthreads();
+        for (int i0 = 4 * tid; i0 < len; i0 += 4 * kThreads) {
+            const uint4 k4 = keys4_at(i0);
+            const uint32_t kv[4] = {k4.x, k4.y, k4.z, k4.w};
+#pragma unroll
+            for (int u = 0; u < 4; ++u)
+                if (i0 + u < len) atomicAdd(&fine[(kv[u] - kmin) >> shift], 1u);
+        }
+        __syncthreads();
         cluster.sync();
-        if (tid < kBins) {
+        // CTA rank owns bins [b_lo, b_hi): their totals over the cluster
+        const int per = (kFineBins + C - 1) / C;
+        const int b_lo = min(kFineBins, rank * per), b_hi = min(kFineBins, b_lo + per);
+        int part = 0;
+        for (int bb = b_lo + tid; bb < b_hi; bb += kThreads) {
             uint32_t v[8];
 #pragma unroll
-            for (int r = 0; r < 8; ++r) v[r] = r < C ? cluster.map_shared_rank(hist, r)[tid] : 0u;
-            tot[tid] = ((v[0] + v[1]) + (v[2] + v[3])) + ((v[4] + v[5]) + (v[6] + v[7]));
+            for (int r = 0; r < 8; ++r) v[r] = r < C ? cluster.map_shared_rank(fine, r)[bb] : 0u;
+            const uint32_t tot_b = ((v[0] + v[1]) + (v[2] + v[3])) + ((v[4] + v[5]) + (v[6] + v[7]));
+            rng[bb - b_lo] = tot_b;
+            part += (int)tot_b;
         }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) part += __shfl_xor_sync(0xffffffffu, part, o);
+        if (lane == 0) atomicAdd(misc + 6, part);
         __syncthreads();
-        // digit holding the remaining-th largest key: scan from the top digit down
-        const int d = kBins - 1 - tid;
-        const int c = tid < kBins ? (int)tot[d] : 0;
-        int tsum;
-        const int before = block_scan1(c, scr, &tsum);
-        if (tid < kBins && before < remaining && remaining <= before + c) {
-            misc[0] = d;
-            misc[1] = before;
+        cluster.sync();
+        // every CTA finds b* itself: the range holding the k-th largest key (ranges of higher
+        // ranks hold larger keys), then that range's bins read from its owner, top down
+        int above_r = 0, owner = 0;
+        {
+            int rs[8];
+#pragma unroll
+            for (int r = 0; r < 8; ++r) rs[r] = r < C ? cluster.map_shared_rank(misc, r)[6] : 0;
+            int acc = 0;
+            bool found = false;
+#pragma unroll
+            for (int r = 7; r >= 0; --r) {
+                if (r < C && !found) {
+                    if (acc < a.k && a.k <= acc + rs[r]) {
+                        owner = r;
+                        above_r = acc;
+                        found = true;
+                    }
+                    acc += rs[r];
+                }
+            }
         }
-        __syncthreads();
-        const int dsel = misc[0];
-        const int above = misc[1];
-        // this CTA's keys in digits above the chosen one (same prefix) are above tau
-        int atot;
-        block_scan1((tid < kBins && d > dsel) ? (int)hist[d] : 0, scr, &atot);
-        local_gt += atot;
-        if (p == 3) local_eq = (int)hist[dsel];
-        prefix |= (uint32_t)dsel << sh;
-        pmask |= 0xFFu << sh;
-        remaining -= above;
+        {
+            const int o_lo = min(kFineBins, owner * per), o_hi = min(kFineBins, o_lo + per);
+            const uint32_t* orng = cluster.map_shared_rank(rng, owner);
+            const int need = a.k - above_r;
+            int cb[4], c4 = 0;
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                const int bb = o_hi - 1 - 4 * tid - u;
+                cb[u] = bb >= o_lo ? (int)orng[bb - o_lo] : 0;
+                c4 += cb[u];
+            }
+            int tsum;
+            const int before = block_scan1(c4, scr, &tsum);
+            if (before < need && need <= before + c4) {
+                int run = before;
+#pragma unroll
+                for (int u = 0; u < 4; ++u) {
+                    if (run < need && need <= run + cb[u]) {
+                        misc[8] = o_hi - 1 - 4 * tid - u;
+                        misc[9] = above_r + run;
+                        misc[10] = cb[u];
+                    }
+                    run += cb[u];
+                }
+            }
+            __syncthreads();
+        }
+        const int bstar = misc[8];
+        const int above_total = misc[9];
+        const int Tc = misc[10];
+        // this CTA's keys in bins above b*
+        int la = 0;
+        for (int bb = bstar + 1 + tid; bb < kFineBins; bb += kThreads) la += (int)fine[bb];
+        int latot;
+        block_scan1(la, scr, &latot);
+        if (Tc <= kCandMax) {
+            // ---- 2. the keys of bin b*: every CTA gathers them all and finds tau itself
+            uint32_t* cand = priv;
+            for (int i0 = 4 * tid; i0 < len; i0 += 4 * kThreads) {
+                const uint4 k4 = keys4_at(i0);
+                const uint32_t kv[4] = {k4.x, k4.y, k4.z, k4.w};
+#pragma unroll
+                for (int u = 0; u < 4; ++u)
+                    if (i0 + u < len && (int)((kv[u] - kmin) >> shift) == bstar) cand[atomicAdd(misc + 13, 1)] = kv[u];
+            }
+            __syncthreads();
+            cluster.sync();
+            uint32_t* gbuf = sm + kOffGather;
+            int off = 0;
+            for (int r = 0; r < C; ++r) {
+                const int cnt = cluster.map_shared_rank(misc, r)[13];
+                const uint32_t* rc = cluster.map_shared_rank(cand, r);
+                for (int i = tid; i < cnt; i += kThreads) gbuf[off + i] = rc[i];
+                off += cnt;
+            }
+            __syncthreads();
+            {
+                // tau among the candidates (keys in [base, base + 2^shift)): refine by 2048-bin
+                // histograms of the bits below the bin base, at most two levels for shift <= 22;
+                // this CTA's own fine histogram is free now (peers read it only before the range merge)
+                int rem = a.k - above_total;
+                uint64_t base = (uint64_t)kmin + ((uint64_t)bstar << shift);
+                int sh = shift;
+#pragma unroll 1
+                while (sh > 0) {
+                    const int sh2 = max(0, sh - kFineBits);
+                    const int nb = 1 << (sh - sh2);  // <= kFineBins
+                    for (int i = tid; i < nb; i += kThreads) fine[i] = 0u;
+                    __syncthreads();
+                    for (int i = tid; i < off; i += kThreads) {
+                        const uint64_t kk = gbuf[i];
+                        if (kk >= base && kk < base + (1ull << sh)) atomicAdd(&fine[(uint32_t)((kk - base) >> sh2)], 1u);
+                    }
+                    __syncthreads();
+                    int cb[4], c4 = 0;
+#pragma unroll
+                    for (int u = 0; u < 4; ++u) {
+                        const int bb = nb - 1 - 4 * tid - u;
+                        cb[u] = bb >= 0 ? (int)fine[bb] : 0;
+                        c4 += cb[u];
+                    }
+                    int tsum;
+                    const int before = block_scan1(c4, scr, &tsum);
+                    if (before < rem && rem <= before + c4) {
+                        int run = before;
+#pragma unroll
+                        for (int u = 0; u < 4; ++u) {
+                            if (run < rem && rem <= run + cb[u]) {
+                                misc[14] = nb - 1 - 4 * tid - u;
+                                misc[15] = run;
+                            }
+                            run += cb[u];
+                        }
+                    }
+                    __syncthreads();
+                    base += (uint64_t)misc[14] << sh2;
+                    rem -= misc[15];
+                    sh = sh2;
+                    __syncthreads();
+                }
+                if (tid == 0) {
+                    misc[11] = (int)(uint32_t)base;
+                    misc[12] = rem;  // candidates equal to tau that are taken
+                }
+                __syncthreads();
+            }
+            tau = (uint32_t)misc[11];
+            take_eq_total = misc[12];
+            const int nc = misc[13];
+            int g = 0, e = 0;
+            for (int i = tid; i < nc; i += kThreads) {
+                g += cand[i] > tau;
+                e += cand[i] == tau;
+            }
+            int gtot, etot;
+            block_scan1(g, scr, &gtot);
+            block_scan1(e, scr, &etot);
+            local_gt = latot + gtot;
+            local_eq = etot;
+        } else {
+            // ---- fallback: radix select over four 8-bit digits of all keys
+            uint32_t prefix = 0, pmask = 0;
+            int remaining = a.k;
+#pragma unroll 1
+            for (int p = 0; p < 4; ++p) {
+                const int sh = 24 - 8 * p;
+                uint32_t* hist = sm + kOffHist + (p & 1) * kBins;
+                for (int i = tid; i < kWarps * kBins; i += kThreads) priv[i] = 0u;
+                __syncthreads();
+                uint32_t* my = priv + warp * kBins;
+                for (int i0 = 0; i0 < len; i0 += kThreads) {
+                    const int i = i0 + tid;
+                    uint32_t kk = 0;
+                    bool take = false;
+                    if (i < len) {
+                        kk = key_at(i);
+                        take = (kk & pmask) == prefix;
+                    }
+                    const unsigned act = __ballot_sync(0xffffffffu, take);
+                    if (take) {
+                        const uint32_t bin = (kk >> sh) & 0xFFu;
+                        const unsigned peers = __match_any_sync(act, bin);
+                        if (lane == __ffs(peers) - 1) atomicAdd(&my[bin], (uint32_t)__popc(peers));
+                    }
+                }
+                __syncthreads();
+                if (tid < kBins) {
+                    uint32_t sum = 0;
+#pragma unroll
+                    for (int w = 0; w < kWarps; ++w) sum += priv[w * kBins + tid];
+                    hist[tid] = sum;
+                }
+                cluster.sync();
+                if (tid < kBins) {
+                    uint32_t v[8];
+#pragma unroll
+                    for (int r = 0; r < 8; ++r) v[r] = r < C ? cluster.map_shared_rank(hist, r)[tid] : 0u;
+                    tot[tid] = ((v[0] + v[1]) + (v[2] + v[3])) + ((v[4] + v[5]) + (v[6] + v[7]));
+                }
+                __syncthreads();
+                // digit holding the remaining-th largest key: scan from the top digit down
+                const int d = kBins - 1 - tid;
+                const int c = tid < kBins ? (int)tot[d] : 0;
+                int tsum;
+                const int before = block_scan1(c, scr, &tsum);
+                if (tid < kBins && before < remaining && remaining <= before + c) {
+                    misc[0] = d;
+                    misc[1] = before;
+                }
+                __syncthreads();
+                const int dsel = misc[0];
+                const int above = misc[1];
+                // this CTA's keys in digits above the chosen one (same prefix) are above tau
+                int atot;
+                block_scan1((tid < kBins && d > dsel) ? (int)hist[d] : 0, scr, &atot);
+                local_gt += atot;
+                if (p == 3) local_eq = (int)hist[dsel];
+                prefix |= (uint32_t)dsel << sh;
+                pmask |= 0xFFu << sh;
+                remaining -= above;
+            }
+            tau = prefix;
+            take_eq_total = remaining;
+        }
     }
-    const uint32_t tau = prefix;
-    const int take_eq_total = remaining;  // keys equal to tau that are selected, lowest positions first
 
     if (tid == 0) {
         misc[2] = local_gt;
