@@ -8,22 +8,29 @@
 // because both scales are positive and ReLU(c x) = c ReLU(x) for c > 0.
 //
 // Shape of the work: for one query row, [H_I x d_I] . [d_I x n] is a dense
-// FP8 contraction.  A tile is 128 cached tokens (MMA M = 128) against the 64
-// heads of one query (MMA N = 64), K = d_I, accumulated in fp32 in tensor
-// memory.  The epilogue reads one token row per thread from TMEM, applies
-// ReLU, the weighted head sum and the key scale, and writes one fp32 score:
-// per-head products never leave the chip.
+// FP8 contraction.  A stage is 256 cached tokens: two MMA tiles of 128 tokens
+// (MMA M = 128) against the 64 heads of one query (MMA N = 64), K = d_I,
+// accumulated in fp32 in tensor memory.  The epilogue reads one token row per
+// thread and tile from TMEM, applies ReLU, the weighted head sum and the key
+// scale, and writes one fp32 score: per-head products never leave the chip.
+//
+// Every asynchronous hand-off (a TMA copy, an MMA, a commit) costs the
+// per-SM pipeline time of its own (measured on B200: ~60 cycles per MMA and
+// ~100 per commit on the critical path of a 128-token tile, which held the
+// kernel at ~2.1 TB/s with 128-token stages), so a stage carries 256 tokens
+// with one key copy, one scale copy and one commit, and the key stage is
+// released by the epilogue warps (which have seen the MMA complete) rather
+// than by a second commit.
 //
 // Roles (one persistent CTA per SM, each owning a contiguous range of the
-// flat list of (query row, key tile) pairs):
-//   warp 0       producer: lane 0 issues the TMA copies of each key tile and of
-//                its 128 fp32 scales into a deep stage ring; at a new query row
-//                the warp writes the folded weights w*q_scale to shared memory
-//                and lane 0 fetches the row's q8 block by TMA
+// flat list of (query row, 256-token stage) pairs):
+//   warp 0       producer: lane 0 issues the TMA copies of each 256-token key
+//                block and of its 256 fp32 scales into a stage ring; at a new
+//                query row the warp writes the folded weights w*q_scale to
+//                shared memory and lane 0 fetches the row's q8 block by TMA
 //   warp 1       TMEM allocator and single-thread tcgen05.mma issuer
-//   warps 2..17  epilogue, four groups of four warps taking every fourth tile,
-//                with eight TMEM accumulators so the tensor core and the four
-//                groups each run several tiles ahead of the slowest hand-off
+//   warps 2..17  epilogue, four groups of four warps taking every fourth stage,
+//                each with its own 128-column TMEM accumulator pair
 // Every wait is bounded; a timeout records DSA_ERR_TIMEOUT and the CTA drains
 // and exits instead of hanging.
 #include <cuda.h>
@@ -38,24 +45,29 @@ namespace {
 
 template <int D_I>
 struct IdxCfg {
-    static constexpr int TILE = kIdxTile;
+    static constexpr int TILE = kIdxTile;         // MMA M: tokens per MMA tile
+    static constexpr int SUB = D_I == 64 ? 4 : 2; // MMA tiles per stage
+    static constexpr int STOK = SUB * TILE;       // tokens per stage
+    static constexpr int BOX = 256;               // tokens per TMA box (the box limit)
+    static constexpr int NBOX = STOK / BOX;       // key and scale boxes per stage
     static constexpr int HEADS = kIdxHeads;
-    static constexpr int STAGES = D_I == 64 ? 16 : 10;
-    static constexpr int KTILE_BYTES = TILE * D_I;
+    static constexpr int STAGES = D_I == 64 ? 4 : 5;
+    static constexpr int KTILE_BYTES = STOK * D_I;
     static constexpr int Q_BYTES = HEADS * D_I;
     static constexpr uint32_t SWZ = D_I == 64 ? kSwizzle64B : kSwizzle128B;
     static constexpr uint32_t SBO = 8 * D_I;      // 8-row swizzle atom
-    static constexpr int ACC = 8;                 // TMEM accumulator buffers of HEADS columns
     static constexpr int TMEM_COLS = 512;
-    static constexpr int GROUPS = 4;              // epilogue groups of four warps
+    static constexpr int ACC = TMEM_COLS / (SUB * HEADS);  // TMEM accumulators of SUB x HEADS columns
+    static constexpr int GROUPS = ACC;            // epilogue groups of four warps, one accumulator each
+    static_assert(ACC * SUB * HEADS <= TMEM_COLS, "accumulators must fit TMEM");
     static constexpr int EPI_WARP0 = 2;
     static constexpr int THREADS = (EPI_WARP0 + 4 * GROUPS) * 32;
     static constexpr int K_STEPS = D_I / 32;      // kind::f8f6f4 consumes 32 bytes of K per MMA
     // shared memory map (offsets from a 1024-byte aligned base)
     static constexpr int OFF_K = 0;
     static constexpr int OFF_Q = OFF_K + STAGES * KTILE_BYTES;
-    static constexpr int OFF_SC = OFF_Q + 2 * Q_BYTES;     // per-stage key scales (TILE fp32)
-    static constexpr int SC_BYTES = TILE * 4;
+    static constexpr int OFF_SC = OFF_Q + 2 * Q_BYTES;     // per-stage key scales (STOK fp32)
+    static constexpr int SC_BYTES = STOK * 4;
     static constexpr int OFF_WQ = OFF_SC + STAGES * SC_BYTES;  // 2 x HEADS folded weights
     static constexpr int OFF_BAR = OFF_WQ + 2 * HEADS * 4;
     static constexpr int NBAR = 2 * STAGES + 4 + 2 * ACC;
@@ -70,29 +82,34 @@ struct IdxShared {
     int abort_flag;
 };
 
-// Number of key tiles of a query row with length n in sequence b (0 when the sizes are invalid).
-__device__ __forceinline__ int tiles_of(const IndexerArgs& a, int n, int b) {
+// Number of key stages (stok tokens each) of a query row with length n in sequence b (0 when the
+// sizes are invalid).
+__device__ __forceinline__ int tiles_of(const IndexerArgs& a, int n, int b, int stok) {
     if (n < 0 || n > a.T_max || (int64_t)n > a.ld || b < 0 || b >= a.B) return 0;
-    return (n + kIdxTile - 1) / kIdxTile;
+    return (n + stok - 1) / stok;
 }
-__device__ __forceinline__ int row_tiles(const IndexerArgs& a, int r) { return tiles_of(a, a.q_len[r], a.q_seq[r]); }
+__device__ __forceinline__ int row_tiles(const IndexerArgs& a, int r, int stok) {
+    return tiles_of(a, a.q_len[r], a.q_seq[r], stok);
+}
 
 // Walks the flat (row, tile) list.  The row's sequence and length are read
 // once per row, never per tile: every issuing loop depends on them.
 struct TileCursor {
     int row, j, nt, b, n;
+    int stok;  // tokens per stage
     __device__ void load_row(const IndexerArgs& a) {
         if (row < a.Nq) {
             n = a.q_len[row];
             b = a.q_seq[row];
-            nt = tiles_of(a, n, b);
+            nt = tiles_of(a, n, b, stok);
         } else {
             n = 0;
             b = 0;
             nt = 1;  // sentinel past the last row
         }
     }
-    __device__ void start(const IndexerArgs& a, int r0, int j0) {
+    __device__ void start(const IndexerArgs& a, int r0, int j0, int stok_) {
+        stok = stok_;
         row = r0;
         j = j0;
         load_row(a);
@@ -138,7 +155,7 @@ __global__ void __launch_bounds__(IdxCfg<D_I>::THREADS, 1)
     if (tid == 0) {
         for (int s = 0; s < C::STAGES; ++s) {
             mbar_init(bar_full(s), 1);
-            mbar_init(bar_empty(s), 5);  // MMA commit + the 4 epilogue warps that read the stage's scales
+            mbar_init(bar_empty(s), 4);  // the 4 epilogue warps of the stage (they have seen the MMA complete)
         }
         for (int q = 0; q < 2; ++q) {
             mbar_init(bar_qfull(q), 1);                   // producer arrival with the q8 block's tx bytes
@@ -163,7 +180,7 @@ __global__ void __launch_bounds__(IdxCfg<D_I>::THREADS, 1)
         long long total = 0;
         for (int base = 0; base < a.Nq; base += 32) {
             const int r = base + lane;
-            int v = r < a.Nq ? row_tiles(a, r) : 0;
+            int v = r < a.Nq ? row_tiles(a, r, C::STOK) : 0;
             if (r < a.Nq && v == 0 && a.q_len[r] != 0 && blockIdx.x == 0) record_status(a.status, DSA_STATUS_LENGTH);
 #pragma unroll
             for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
@@ -175,7 +192,7 @@ __global__ void __launch_bounds__(IdxCfg<D_I>::THREADS, 1)
         long long run = 0;
         for (int base = 0; base < a.Nq && row0 == a.Nq; base += 32) {
             const int r = base + lane;
-            const int v = r < a.Nq ? row_tiles(a, r) : 0;
+            const int v = r < a.Nq ? row_tiles(a, r, C::STOK) : 0;
             int incl = v;
 #pragma unroll
             for (int o = 1; o < 32; o <<= 1) {
@@ -208,7 +225,7 @@ __global__ void __launch_bounds__(IdxCfg<D_I>::THREADS, 1)
         // ---------------- producer
         if (count > 0) {
             TileCursor cur;
-            cur.start(a, sh->row0, sh->j0);
+            cur.start(a, sh->row0, sh->j0, C::STOK);
             int qi = -1;
             int issued = 0;
             for (int it = 0; it < count; ++it) {
@@ -236,8 +253,13 @@ __global__ void __launch_bounds__(IdxCfg<D_I>::THREADS, 1)
                 }
                 if (lane == 0) {
                     mbar_arrive_expect_tx(bar_full(st), C::KTILE_BYTES + C::SC_BYTES);
-                    tma_load_2d(sK + st * C::KTILE_BYTES, &tmap_k, 0, cur.b * a.T_max + cur.j * C::TILE, bar_full(st));
-                    tma_load_2d(sS + st * C::SC_BYTES, &tmap_s, cur.j * C::TILE, cur.b, bar_full(st));
+#pragma unroll
+                    for (int q = 0; q < C::NBOX; ++q) {
+                        const int tok = cur.j * C::STOK + q * C::BOX;
+                        tma_load_2d(sK + st * C::KTILE_BYTES + q * (C::BOX * D_I), &tmap_k, 0, cur.b * a.T_max + tok,
+                                    bar_full(st));
+                        tma_load_2d(sS + st * C::SC_BYTES + q * (C::BOX * 4), &tmap_s, tok, cur.b, bar_full(st));
+                    }
                 }
                 ++issued;
                 cur.advance(a);
@@ -252,7 +274,7 @@ __global__ void __launch_bounds__(IdxCfg<D_I>::THREADS, 1)
         if (lane == 0 && count > 0) {
             // ---------------- MMA issuer
             TileCursor cur;
-            cur.start(a, sh->row0, sh->j0);
+            cur.start(a, sh->row0, sh->j0, C::STOK);
             int qi = -1, qb = 0;
             int last_acc = -1, last_it = -1;
             for (int it = 0; it < count; ++it) {
@@ -267,16 +289,18 @@ __global__ void __launch_bounds__(IdxCfg<D_I>::THREADS, 1)
                 if (it >= C::ACC && !mbar_wait(bar_tempty(acc), ((it / C::ACC) - 1) & 1, abort_flag, a.status))
                     break;
                 tc_fence_after();
-                const uint32_t d = tmem + acc * C::HEADS;
-                const uint32_t a_addr = sK + st * C::KTILE_BYTES;
                 const uint32_t b_addr = sQ + qb * C::Q_BYTES;
 #pragma unroll
-                for (int ks = 0; ks < C::K_STEPS; ++ks) {
-                    const uint64_t ad = make_smem_desc(a_addr + ks * 32, 16, C::SBO, C::SWZ);
-                    const uint64_t bd = make_smem_desc(b_addr + ks * 32, 16, C::SBO, C::SWZ);
-                    mma_f8f6f4_ss(d, ad, bd, C::IDESC, ks > 0 ? 1u : 0u);
+                for (int h = 0; h < C::SUB; ++h) {
+                    const uint32_t d = tmem + acc * (C::SUB * C::HEADS) + h * C::HEADS;
+                    const uint32_t a_addr = sK + st * C::KTILE_BYTES + h * (C::TILE * D_I);
+#pragma unroll
+                    for (int ks = 0; ks < C::K_STEPS; ++ks) {
+                        const uint64_t ad = make_smem_desc(a_addr + ks * 32, 16, C::SBO, C::SWZ);
+                        const uint64_t bd = make_smem_desc(b_addr + ks * 32, 16, C::SBO, C::SWZ);
+                        mma_f8f6f4_ss(d, ad, bd, C::IDESC, ks > 0 ? 1u : 0u);
+                    }
                 }
-                mma_commit(bar_empty(st));
                 mma_commit(bar_tfull(acc));
                 last_acc = acc;
                 last_it = it;
@@ -292,7 +316,7 @@ __global__ void __launch_bounds__(IdxCfg<D_I>::THREADS, 1)
         const int sub = warp & 3;                  // TMEM sub-partition this warp may access
         const int m = sub * 32 + lane;             // token row inside the tile
         TileCursor cur;
-        if (count > 0) cur.start(a, sh->row0, sh->j0);
+        if (count > 0) cur.start(a, sh->row0, sh->j0, C::STOK);
         int qi = -1, qb = 0, n = 0;
         const float* wq = wq_smem;
         for (int it = 0; it < count; ++it) {
@@ -311,43 +335,49 @@ __global__ void __launch_bounds__(IdxCfg<D_I>::THREADS, 1)
                     if (!__all_sync(0xffffffffu, okq)) break;
                     wq = wq_smem + qb * C::HEADS;
                 }
-                const int s = cur.j * C::TILE + m;
                 const int st = it % C::STAGES;
                 const int acc = it % C::ACC;
                 bool ok = mbar_wait(bar_tfull(acc), (it / C::ACC) & 1, abort_flag, a.status);
                 ok = ok && mbar_wait(bar_full(st), (it / C::STAGES) & 1, abort_flag, a.status);
                 if (!__all_sync(0xffffffffu, ok)) break;
-                const float ks = scale_smem[st * C::TILE + m];
                 tc_fence_after();
-                uint32_t v0[32], v1[32];
-                const uint32_t taddr = tmem + ((uint32_t)(sub * 32) << 16) + acc * C::HEADS;
-                tmem_ld32(taddr, v0);
-                tmem_ld32(taddr + 32, v1);
-                tmem_wait_ld();
+#pragma unroll
+                for (int h = 0; h < C::SUB; ++h) {
+                    // token h * TILE + m of the stage: TMEM lane m of accumulator half h
+                    uint32_t v0[32], v1[32];
+                    const uint32_t taddr =
+                        tmem + ((uint32_t)(sub * 32) << 16) + acc * (C::SUB * C::HEADS) + h * C::HEADS;
+                    tmem_ld32(taddr, v0);
+                    tmem_ld32(taddr + 32, v1);
+                    tmem_wait_ld();
+                    float p0 = 0.f, p1 = 0.f, p2 = 0.f, p3 = 0.f;
+#pragma unroll
+                    for (int j = 0; j < 32; j += 4) {
+                        const float4 w4 = *reinterpret_cast<const float4*>(wq + j);
+                        p0 = fmaf(w4.x, fmaxf(__uint_as_float(v0[j + 0]), 0.f), p0);
+                        p1 = fmaf(w4.y, fmaxf(__uint_as_float(v0[j + 1]), 0.f), p1);
+                        p2 = fmaf(w4.z, fmaxf(__uint_as_float(v0[j + 2]), 0.f), p2);
+                        p3 = fmaf(w4.w, fmaxf(__uint_as_float(v0[j + 3]), 0.f), p3);
+                    }
+#pragma unroll
+                    for (int j = 0; j < 32; j += 4) {
+                        const float4 w4 = *reinterpret_cast<const float4*>(wq + 32 + j);
+                        p0 = fmaf(w4.x, fmaxf(__uint_as_float(v1[j + 0]), 0.f), p0);
+                        p1 = fmaf(w4.y, fmaxf(__uint_as_float(v1[j + 1]), 0.f), p1);
+                        p2 = fmaf(w4.z, fmaxf(__uint_as_float(v1[j + 2]), 0.f), p2);
+                        p3 = fmaf(w4.w, fmaxf(__uint_as_float(v1[j + 3]), 0.f), p3);
+                    }
+                    const int s = cur.j * C::STOK + h * C::TILE + m;
+                    const float sc = scale_smem[st * C::STOK + h * C::TILE + m] * ((p0 + p1) + (p2 + p3));
+                    if (s < n) a.scores[(int64_t)cur.row * a.ld + s] = sc;
+                }
+                // TMEM and the key stage (its scales included) are free: the MMA has completed
                 tc_fence_before();
                 __syncwarp();
                 if (lane == 0) {
                     mbar_arrive(bar_tempty(acc));
                     mbar_arrive(bar_empty(st));
                 }
-                float p0 = 0.f, p1 = 0.f, p2 = 0.f, p3 = 0.f;
-#pragma unroll
-                for (int j = 0; j < 32; j += 4) {
-                    const float4 w4 = *reinterpret_cast<const float4*>(wq + j);
-                    p0 = fmaf(w4.x, fmaxf(__uint_as_float(v0[j + 0]), 0.f), p0);
-                    p1 = fmaf(w4.y, fmaxf(__uint_as_float(v0[j + 1]), 0.f), p1);
-                    p2 = fmaf(w4.z, fmaxf(__uint_as_float(v0[j + 2]), 0.f), p2);
-                    p3 = fmaf(w4.w, fmaxf(__uint_as_float(v0[j + 3]), 0.f), p3);
-                }
-#pragma unroll
-                for (int j = 0; j < 32; j += 4) {
-                    const float4 w4 = *reinterpret_cast<const float4*>(wq + 32 + j);
-                    p0 = fmaf(w4.x, fmaxf(__uint_as_float(v1[j + 0]), 0.f), p0);
-                    p1 = fmaf(w4.y, fmaxf(__uint_as_float(v1[j + 1]), 0.f), p1);
-                    p2 = fmaf(w4.z, fmaxf(__uint_as_float(v1[j + 2]), 0.f), p2);
-                    p3 = fmaf(w4.w, fmaxf(__uint_as_float(v1[j + 3]), 0.f), p3);
-                }
-                if (s < n) a.scores[(int64_t)cur.row * a.ld + s] = ks * ((p0 + p1) + (p2 + p3));
             }
             if (seg_end) {
                 // this warp is done with the row's folded weights
@@ -370,11 +400,11 @@ cudaError_t launch_fp8_impl(const IndexerArgs& a, int grid, cudaStream_t st) {
     using C = IdxCfg<D_I>;
     alignas(64) CUtensorMap tk, tq, ts;
     const int swz = D_I;  // 64-byte rows -> 64B swizzle, 128-byte rows -> 128B swizzle
-    if (!encode_tensor_map_2d(&tk, 1, a.k_I, D_I, (uint64_t)a.B * a.T_max, D_I, D_I, C::TILE, swz))
+    if (!encode_tensor_map_2d(&tk, 1, a.k_I, D_I, (uint64_t)a.B * a.T_max, D_I, D_I, C::BOX, swz))
         return cudaErrorInvalidValue;
     if (!encode_tensor_map_2d(&tq, 1, a.q_I, D_I, (uint64_t)a.Nq * C::HEADS, D_I, D_I, C::HEADS, swz))
         return cudaErrorInvalidValue;
-    if (!encode_tensor_map_2d(&ts, 4, a.k_scale, a.T_max, (uint64_t)a.B, (uint64_t)a.T_max * 4, C::TILE, 1, 0))
+    if (!encode_tensor_map_2d(&ts, 4, a.k_scale, a.T_max, (uint64_t)a.B, (uint64_t)a.T_max * 4, C::BOX, 1, 0))
         return cudaErrorInvalidValue;
     auto kern = indexer_fp8_kernel<D_I>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
