@@ -275,6 +275,8 @@ def run_ours(args):
 
     # ---- end to end through the C interface with host buffers
     e2e = measure_e2e(inp, dims, ws, dev, steps=min(K, 200), warmup=min(W, 10))
+    if not e2e["readback_ok"]:
+        raise SystemExit("end-to-end loop: the host copy of the last step's output differs from the device's")
     e2e_ms = max_over_ranks(e2e["ms"], world)
 
     hbm, peak_kind = peaks()
@@ -318,7 +320,9 @@ def run_ours(args):
         "stages_us": {"indexer": stage_us[0], "topk": stage_us[1], "sparse_mla": stage_us[2],
                       "merge": stage_us[3]},
         "e2e": {"value": BATCH * world / (e2e_ms * 1e-3), "unit": UNIT, "h2d_bytes_per_step": e2e["h2d"],
-                "d2h_bytes_per_step": e2e["d2h"], "ms_per_step": e2e_ms},
+                "d2h_bytes_per_step": e2e["d2h"], "ms_per_step": e2e_ms,
+                "pipeline": "one packed H2D copy per step; copy-in, compute and copy-out streams with two "
+                            "buffer slots (copies of neighbouring steps overlap a step's compute)"},
         "gpu_launches": launches_per_step() * K,
         "timing": {"step": "one start and one end event per step on the launching stream",
                    "stages_us": f"separate pass of {KS} steps with an event between stages (each adds ~2 us)"},
@@ -345,48 +349,85 @@ def launches_per_step():
 
 
 def measure_e2e(inp, dims, ws, dev, steps, warmup):
-    """Per step: H2D of the step's query-side inputs and the new token's cache
-    entries from pinned host memory, the decode step, D2H of out and lse."""
+    """End to end through the public API, as a serving loop would run it.  Per step:
+    one H2D copy of all of the step's inputs (query-side tensors and the new token's
+    cache entries, packed in one pinned buffer), the cache append, the decode step,
+    and the D2H copy of out and lse.  Two buffer slots on separate copy-in, compute and
+    copy-out streams: the copies of step i+1 and step i-1 overlap the compute of step
+    i; each step's append and decode stay in order on the compute stream."""
     import torch
     from sparse_long_context_indexer_b200 import api
     B = inp.B
     pos = (inp.q_len - 1).long()
-    host = {
-        "q": inp.q.cpu().pin_memory(), "q_I": inp.q_I.cpu().pin_memory(), "q_scale": inp.q_scale.cpu().pin_memory(),
-        "w": inp.w.cpu().pin_memory(), "q_len": inp.q_len.cpu().pin_memory(),
-        "kv_new": inp.kv[torch.arange(B, device=dev), pos].cpu().pin_memory(),
-        "k_new": inp.k_I[torch.arange(B, device=dev), pos].cpu().pin_memory(),
-        "ks_new": inp.k_scale[torch.arange(B, device=dev), pos].cpu().pin_memory(),
+    fields = {
+        "q": inp.q, "q_I": inp.q_I, "q_scale": inp.q_scale, "w": inp.w, "q_len": inp.q_len,
+        "kv_new": inp.kv[torch.arange(B, device=dev), pos], "k_new": inp.k_I[torch.arange(B, device=dev), pos],
+        "ks_new": inp.k_scale[torch.arange(B, device=dev), pos],
     }
-    dv = {k: torch.empty_like(v, device=dev) for k, v in host.items()}
-    out_h = torch.empty((inp.Nq, inp.H, 512), dtype=torch.bfloat16).pin_memory()
-    lse_h = torch.empty((inp.Nq, inp.H), dtype=torch.float32).pin_memory()
-    out, lse = api.alloc_outputs(inp)
+    offs, off = {}, 0
+    for k, v in fields.items():
+        offs[k] = off
+        off += (v.numel() * v.element_size() + 255) // 256 * 256
+    total = off
+    h2d = sum(v.numel() * v.element_size() for v in fields.values())
+    host_pack = torch.empty(total, dtype=torch.uint8).pin_memory()
+    for k, v in fields.items():
+        nb = v.numel() * v.element_size()
+        host_pack[offs[k]:offs[k] + nb].copy_(v.contiguous().cpu().view(-1).view(torch.uint8))
+    slots = []
+    for _ in range(2):
+        dbuf = torch.empty(total, dtype=torch.uint8, device=dev)
+        views = {k: dbuf[offs[k]:offs[k] + v.numel() * v.element_size()].view(v.dtype).view(v.shape)
+                 for k, v in fields.items()}
+        o, l = api.alloc_outputs(inp)
+        slots.append({"dbuf": dbuf, "v": views, "out": o, "lse": l,
+                      "out_h": torch.empty(o.shape, dtype=o.dtype).pin_memory(),
+                      "lse_h": torch.empty(l.shape, dtype=l.dtype).pin_memory(),
+                      "in_done": torch.cuda.Event(), "comp_done": torch.cuda.Event(), "out_done": torch.cuda.Event()})
+    d2h = slots[0]["out_h"].numel() * slots[0]["out_h"].element_size() + \
+        slots[0]["lse_h"].numel() * slots[0]["lse_h"].element_size()
+    s_in, s_out = torch.cuda.Stream(device=dev), torch.cuda.Stream(device=dev)
+    s_c = torch.cuda.current_stream(dev)
     bidx = torch.arange(B, device=dev)
-    h2d = sum(v.numel() * v.element_size() for v in host.values())
-    d2h = out_h.numel() * out_h.element_size() + lse_h.numel() * lse_h.element_size()
+    first = [True, True]
 
-    def step():
-        for k in host:
-            dv[k].copy_(host[k], non_blocking=True)
-        inp.kv[bidx, pos] = dv["kv_new"]
-        inp.k_I[bidx, pos] = dv["k_new"]
-        inp.k_scale[bidx, pos] = dv["ks_new"]
-        api.decode_step(dims, dv["q_I"], dv["q_scale"], dv["w"], inp.k_I, inp.k_scale, dv["q"], inp.kv, inp.q_seq,
-                        dv["q_len"], inp.softmax_scale, out, lse, ws)
-        out_h.copy_(out, non_blocking=True)
-        lse_h.copy_(lse, non_blocking=True)
+    def step(i):
+        sl = slots[i % 2]
+        with torch.cuda.stream(s_in):
+            if not first[i % 2]:
+                s_in.wait_event(sl["comp_done"])       # the slot's previous decode has read its inputs
+            sl["dbuf"].copy_(host_pack, non_blocking=True)
+            sl["in_done"].record(s_in)
+        s_c.wait_event(sl["in_done"])
+        if not first[i % 2]:
+            s_c.wait_event(sl["out_done"])             # the slot's previous outputs have been read back
+        v = sl["v"]
+        inp.kv[bidx, pos] = v["kv_new"]
+        inp.k_I[bidx, pos] = v["k_new"]
+        inp.k_scale[bidx, pos] = v["ks_new"]
+        api.decode_step(dims, v["q_I"], v["q_scale"], v["w"], inp.k_I, inp.k_scale, v["q"], inp.kv, inp.q_seq,
+                        v["q_len"], inp.softmax_scale, sl["out"], sl["lse"], ws)
+        sl["comp_done"].record(s_c)
+        with torch.cuda.stream(s_out):
+            s_out.wait_event(sl["comp_done"])
+            sl["out_h"].copy_(sl["out"], non_blocking=True)
+            sl["lse_h"].copy_(sl["lse"], non_blocking=True)
+            sl["out_done"].record(s_out)
+        first[i % 2] = False
 
-    for _ in range(warmup):
-        step()
-    torch.cuda.synchronize()
+    for i in range(warmup):
+        step(i)
+    torch.cuda.synchronize(dev)
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record()
-    for _ in range(steps):
-        step()
-    e1.record()
-    torch.cuda.synchronize()
-    return {"ms": e0.elapsed_time(e1) / steps, "h2d": h2d, "d2h": d2h}
+    e0.record(s_in)
+    for i in range(steps):
+        step(i)
+    # the last step's read-back ends the timed region
+    s_in.wait_stream(s_out)
+    e1.record(s_in)
+    torch.cuda.synchronize(dev)
+    ok = torch.equal(slots[(steps - 1) % 2]["out_h"], slots[(steps - 1) % 2]["out"].cpu())
+    return {"ms": e0.elapsed_time(e1) / steps, "h2d": h2d, "d2h": d2h, "readback_ok": ok}
 
 
 def main():

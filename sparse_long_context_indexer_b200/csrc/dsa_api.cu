@@ -165,7 +165,7 @@ dsa_status_t run_indexer(const dsa_dims* d, int nq, const void* q_I, const float
 }
 
 dsa_status_t run_topk(const dsa_dims* d, int nq, const float* scores, const int32_t* q_len, int32_t* idx, int* status,
-                      cudaStream_t st) {
+                      cudaStream_t st, bool pdl = false) {
     dsa::TopkArgs a{};
     a.scores = scores;
     a.ld = d->ld_scores;
@@ -175,13 +175,14 @@ dsa_status_t run_topk(const dsa_dims* d, int nq, const float* scores, const int3
     a.k = d->k;
     a.T_max = d->T_max;
     a.status = status;
+    a.pdl = pdl ? 1 : 0;
     cudaError_t e = dsa::launch_topk(a, plan_topk_cluster(d, nq), st);
     return e == cudaSuccess ? DSA_OK : cuda_fail(e);
 }
 
 dsa_status_t run_mla(const dsa_dims* d, int nq, const void* q, const void* kv, const int32_t* idx, const int32_t* q_seq,
                      const int32_t* q_len, float scale, void* out, float* lse, void* ws, const Layout& L,
-                     const dsa_stage_events* ev, cudaStream_t st) {
+                     const dsa_stage_events* ev, cudaStream_t st, bool pdl = false) {
     const MlaPlan p = plan_mla(d, nq);
     dsa::MlaArgs a{};
     a.q = q;
@@ -202,6 +203,7 @@ dsa_status_t run_mla(const dsa_dims* d, int nq, const void* q, const void* kv, c
     a.rows_per_split = p.rows_per_split;
     a.softmax_scale = scale;
     a.status = ws ? status_word(ws) : nullptr;
+    a.pdl = pdl ? 1 : 0;
     cudaError_t e;
     if (d->kv_dtype == DSA_BF16) {
         e = dsa::launch_sparse_mla_bf16(a, st);
@@ -361,10 +363,12 @@ dsa_status_t dsa_decode_step(const dsa_dims* dims, const void* q_I, const float*
     s = run_indexer(dims, dims->Nq, q_I, q_scale, w, k_I, k_scale, q_seq, q_len, scores, status, st);
     if (s != DSA_OK) return s;
     record_event(events, 1, st);
-    s = run_topk(dims, dims->Nq, scores, q_len, idx, status, st);
+    // top-k and attention follow their producer as programmatic dependents: their setup
+    // overlaps the previous kernel's tail and they wait on the device for its output
+    s = run_topk(dims, dims->Nq, scores, q_len, idx, status, st, true);
     if (s != DSA_OK) return s;
     record_event(events, 2, st);
-    s = run_mla(dims, dims->Nq, q, kv, idx, q_seq, q_len, softmax_scale, out, lse, workspace, L, events, st);
+    s = run_mla(dims, dims->Nq, q, kv, idx, q_seq, q_len, softmax_scale, out, lse, workspace, L, events, st, true);
     if (s != DSA_OK) return s;
     record_event(events, 4, st);
     return DSA_OK;
@@ -404,11 +408,11 @@ dsa_status_t dsa_prefill(const dsa_dims* dims, const void* q_I, const float* q_s
         const char* wr = static_cast<const char*>(w) + r0 * w_row;
         s = run_indexer(dims, nq, qi, qs, wr, k_I, k_scale, q_seq + r0, q_len + r0, scores, status, st);
         if (s != DSA_OK) return s;
-        s = run_topk(dims, nq, scores, q_len + r0, idx, status, st);
+        s = run_topk(dims, nq, scores, q_len + r0, idx, status, st, true);
         if (s != DSA_OK) return s;
         s = run_mla(dims, nq, static_cast<const char*>(q) + r0 * q_row, kv, idx, q_seq + r0, q_len + r0,
                     softmax_scale, static_cast<char*>(out) + r0 * o_row, lse ? lse + (size_t)r0 * dims->H : nullptr,
-                    workspace, L, nullptr, st);
+                    workspace, L, nullptr, st, true);
         if (s != DSA_OK) return s;
     }
     return DSA_OK;

@@ -220,6 +220,7 @@ __global__ void __launch_bounds__(IdxCfg<D_I>::THREADS, 1)
     tc_fence_after();
     const uint32_t tmem = (uint32_t)sh->tmem_base;
     const int count = sh->count;
+    griddep_launch_dependents();  // the top-k may start its setup on SMs this grid leaves free
 
     if (warp == 0) {
         // ---------------- producer

@@ -35,6 +35,7 @@ struct TopkArgs {
     int32_t* idx;
     int Nq, k, T_max;
     int* status;
+    int pdl;  // launch as a programmatic dependent of the previous kernel (the library's own pipelines)
 };
 
 struct MlaArgs {
@@ -51,6 +52,7 @@ struct MlaArgs {
     int splits, rows_per_split;
     float softmax_scale;
     int* status;
+    int pdl;  // launch as a programmatic dependent of the previous kernel (the library's own pipelines)
 };
 
 cudaError_t launch_indexer_fp8(const IndexerArgs& a, int grid, cudaStream_t st);

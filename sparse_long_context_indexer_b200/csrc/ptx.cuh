@@ -110,6 +110,17 @@ __device__ __forceinline__ bool mbar_wait_spin(uint32_t bar, uint32_t parity, vo
     }
 }
 
+// ---------------------------------------------------------------- programmatic dependent launch
+
+// Wait until the grid this one depends on (the previous kernel of the stream, when
+// launched with programmatic stream serialization) has completed and its memory
+// is visible; returns at once otherwise.  Reads of that grid's output go after it.
+__device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+// Let the dependent grid be scheduled once every CTA of this grid has executed
+// this (or exited).  Issued after a CTA has started, so a dependent never takes
+// an SM that this grid's own CTAs still need.
+__device__ __forceinline__ void griddep_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
 // ---------------------------------------------------------------- clusters (distributed shared memory)
 
 __device__ __forceinline__ uint32_t cluster_ctarank() {

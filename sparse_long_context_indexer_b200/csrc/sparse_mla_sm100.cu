@@ -153,24 +153,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     };
     auto valid = [&](int s) { return s >= 0 && s < n_t; };
 
-    // the first index loads of each role go out before the setup barrier
-    const int p = tid - 32 * kGatherWarp0;  // gather thread (warps >= kGatherWarp0)
-    const int rr = (p >> 3) & 31, gl = p & 7;
-    const bool pf_lane = warp >= kGatherWarp0 && gl == 0;  // 32 threads issue the L2 prefetches
-    int cur0 = -1, cur1 = -1, pf = -1, pf_first = -1, v0 = -1, v1 = -1;
-    if (ntiles > 0) {
-        if (warp >= kGatherWarp0) {
-            cur0 = load_pos(0, rr);
-            cur1 = load_pos(0, rr + 32);
-            // each CTA of the head pair prefetches one half of the rows
-            if (pf_lane && kStages < ntiles) pf_first = load_pos(kStages, rr + 32 * half);
-            if (pf_lane && kPrefetchTiles < ntiles) pf = load_pos(kPrefetchTiles, rr + 32 * half);
-        } else if (warp < 4) {
-            v0 = load_pos(0, lane);
-            v1 = load_pos(0, lane + 32);
-        }
-    }
-
     if (tid == 0) {
         mbar_init(bar_q_tma, 1);
         mbar_init(bar_q, 128);
@@ -195,6 +177,28 @@ __global__ void __launch_bounds__(kThreads, 1)
         tmem_alloc(smem_u32(&sh->tmem_base), kTmemCols);
         tmem_relinquish();
     }
+    // Everything above (barriers, TMEM, the query block) may overlap the previous kernel;
+    // the index lists come from it (programmatic dependent launch).  The first index
+    // loads of each role go out before the setup barrier.
+    griddep_wait();
+    griddep_launch_dependents();
+    const int p = tid - 32 * kGatherWarp0;  // gather thread (warps >= kGatherWarp0)
+    const int rr = (p >> 3) & 31, gl = p & 7;
+    const bool pf_lane = warp >= kGatherWarp0 && gl == 0;  // 32 threads issue the L2 prefetches
+    int cur0 = -1, cur1 = -1, pf = -1, pf_first = -1, v0 = -1, v1 = -1;
+    if (ntiles > 0) {
+        if (warp >= kGatherWarp0) {
+            cur0 = load_pos(0, rr);
+            cur1 = load_pos(0, rr + 32);
+            // each CTA of the head pair prefetches one half of the rows
+            if (pf_lane && kStages < ntiles) pf_first = load_pos(kStages, rr + 32 * half);
+            if (pf_lane && kPrefetchTiles < ntiles) pf = load_pos(kPrefetchTiles, rr + 32 * half);
+        } else if (warp < 4) {
+            v0 = load_pos(0, lane);
+            v1 = load_pos(0, lane + 32);
+        }
+    }
+
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
@@ -636,13 +640,15 @@ cudaError_t launch_sparse_mla_bf16(const MlaArgs& a, cudaStream_t st) {
         cfg.blockDim = dim3(kThreads, 1, 1);
         cfg.dynamicSmemBytes = kSmemBytes;
         cfg.stream = st;
-        cudaLaunchAttribute attr[1];
+        cudaLaunchAttribute attr[2];
         attr[0].id = cudaLaunchAttributeClusterDimension;
         attr[0].val.clusterDim.x = (unsigned)a.splits;
         attr[0].val.clusterDim.y = 1;
         attr[0].val.clusterDim.z = 1;
+        attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        attr[1].val.programmaticStreamSerializationAllowed = 1;
         cfg.attrs = attr;
-        cfg.numAttrs = 1;
+        cfg.numAttrs = a.pdl ? 2 : 1;
         e = cudaLaunchKernelEx(&cfg, kern, a, tq, tq);  // the output map is unused in this mode
         if (e != cudaSuccess) return e;
         return cudaGetLastError();
@@ -658,7 +664,18 @@ cudaError_t launch_sparse_mla_bf16(const MlaArgs& a, cudaStream_t st) {
     auto kern = final_out ? sparse_mla_bf16_kernel<kOutFinal> : sparse_mla_bf16_kernel<kOutPartials>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
     if (e != cudaSuccess) return e;
-    kern<<<grid, kThreads, kSmemBytes, st>>>(a, tq, to);
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = dim3(kThreads, 1, 1);
+    cfg.dynamicSmemBytes = kSmemBytes;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = a.pdl ? 1 : 0;
+    e = cudaLaunchKernelEx(&cfg, kern, a, tq, to);
+    if (e != cudaSuccess) return e;
     return cudaGetLastError();
 }
 

@@ -148,6 +148,7 @@ __global__ void __launch_bounds__(kThreads, 2) topk_radix_kernel(const TopkArgs 
     int* scr = reinterpret_cast<int*>(sm + kOffScan);
     uint32_t* keys = sm + kOffKeys;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    griddep_launch_dependents();  // the attention kernel may start its setup on free SMs
 
     const int t = blockIdx.y;
     int n = a.q_len[t];
@@ -157,11 +158,15 @@ __global__ void __launch_bounds__(kThreads, 2) topk_radix_kernel(const TopkArgs 
     }
     int32_t* out = a.idx + (int64_t)t * a.k;
     if (n <= a.k) {
-        // short prompt: everything is selected (same branch for the whole cluster)
+        // short prompt: everything is selected (same branch for the whole cluster); the
+        // previous kernel may still be writing the workspace this output may live in
+        griddep_wait();
         for (int i = rank * kThreads + tid; i < a.k; i += C * kThreads) out[i] = i < n ? i : -1;
         return;
     }
 
+    // the score rows come from the previous kernel (programmatic dependent launch)
+    griddep_wait();
     const float* row = a.scores + (int64_t)t * a.ld;
     const int chunk = (((n + C - 1) / C) + 3) & ~3;
     const int lo = min(n, rank * chunk);
@@ -619,13 +624,15 @@ cudaError_t launch_topk(const TopkArgs& a, int cluster, cudaStream_t st) {
     cfg.blockDim = dim3(kThreads, 1, 1);
     cfg.dynamicSmemBytes = smem;
     cfg.stream = st;
-    cudaLaunchAttribute attr[1];
+    cudaLaunchAttribute attr[2];
     attr[0].id = cudaLaunchAttributeClusterDimension;
     attr[0].val.clusterDim.x = cluster;
     attr[0].val.clusterDim.y = 1;
     attr[0].val.clusterDim.z = 1;
+    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[1].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
-    cfg.numAttrs = 1;
+    cfg.numAttrs = a.pdl ? 2 : 1;
     e = cudaLaunchKernelEx(&cfg, topk_radix_kernel, a, cap);
     if (e != cudaSuccess) return e;
     return cudaGetLastError();
