@@ -191,11 +191,14 @@ dsa_status_t dsa_decode_step(const dsa_dims* dims,
                              void* workspace, size_t ws_bytes, void* stream,
                              const dsa_stage_events* events);
 
-/* Prefill: the same three stages for many query rows (every position of a
- * prompt), processed in row chunks so the transient score rows fit the
- * workspace (size it for DSA_OP_PREFILL).  Semantics per row are exactly those
- * of dsa_decode_step; q_len[t] = t + 1 for a causal prompt.  idx_out may be
- * NULL. */
+/* Prefill: the same three stages for many query rows of ONE sequence (every
+ * position of a prompt), processed in row chunks so the transient score rows
+ * fit the workspace (size it for DSA_OP_PREFILL).  Semantics per row are
+ * exactly those of dsa_decode_step; q_len[t] = t + 1 for a causal prompt.
+ * The indexer serves four consecutive rows per tensor-core pass, so every
+ * q_seq[t] must name the same sequence: groups of four rows that do not are
+ * skipped and DSA_ERR_INVALID_ARG is recorded in the device status word.
+ * idx_out may be NULL. */
 dsa_status_t dsa_prefill(const dsa_dims* dims,
                          const void* q_I, const float* q_scale, const void* w,
                          const void* k_I, const float* k_scale,

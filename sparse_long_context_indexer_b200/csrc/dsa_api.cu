@@ -142,7 +142,7 @@ void record_event(const dsa_stage_events* ev, int i, cudaStream_t st) {
 
 dsa_status_t run_indexer(const dsa_dims* d, int nq, const void* q_I, const float* q_scale, const void* w,
                          const void* k_I, const float* k_scale, const int32_t* q_seq, const int32_t* q_len,
-                         float* scores, int* status, cudaStream_t st) {
+                         float* scores, int* status, cudaStream_t st, bool rows_of_one_sequence = false) {
     dsa::IndexerArgs a{};
     a.q_I = q_I;
     a.q_scale = q_scale;
@@ -159,8 +159,9 @@ dsa_status_t run_indexer(const dsa_dims* d, int nq, const void* q_I, const float
     a.H_I = d->H_I;
     a.d_I = d->d_I;
     a.status = status;
-    cudaError_t e = d->idx_dtype == DSA_FP8_E4M3 ? dsa::launch_indexer_fp8(a, device_sms(), st)
-                                                 : dsa::launch_indexer_f32(a, st);
+    cudaError_t e = d->idx_dtype != DSA_FP8_E4M3 ? dsa::launch_indexer_f32(a, st)
+                    : rows_of_one_sequence      ? dsa::launch_indexer_fp8_units4(a, device_sms(), st)
+                                                : dsa::launch_indexer_fp8(a, device_sms(), st);
     return e == cudaSuccess ? DSA_OK : cuda_fail(e);
 }
 
@@ -406,7 +407,7 @@ dsa_status_t dsa_prefill(const dsa_dims* dims, const void* q_I, const float* q_s
         const char* qi = static_cast<const char*>(q_I) + r0 * qi_row;
         const float* qs = fp8 ? q_scale + (size_t)r0 * dims->H_I : nullptr;
         const char* wr = static_cast<const char*>(w) + r0 * w_row;
-        s = run_indexer(dims, nq, qi, qs, wr, k_I, k_scale, q_seq + r0, q_len + r0, scores, status, st);
+        s = run_indexer(dims, nq, qi, qs, wr, k_I, k_scale, q_seq + r0, q_len + r0, scores, status, st, true);
         if (s != DSA_OK) return s;
         s = run_topk(dims, nq, scores, q_len + r0, idx, status, st, true);
         if (s != DSA_OK) return s;

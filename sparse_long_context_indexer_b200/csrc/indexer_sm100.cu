@@ -43,23 +43,27 @@
 namespace dsa {
 namespace {
 
-template <int D_I>
+// R = query rows per MMA: 1 for decode (rows of different sequences), 4 for prefill
+// (consecutive rows of one sequence share every key tile, so one MMA of N = 4 x 64
+// covers four rows and a key tile is read once per four rows).
+template <int D_I, int R>
 struct IdxCfg {
     static constexpr int TILE = kIdxTile;         // MMA M: tokens per MMA tile
-    static constexpr int SUB = D_I == 64 ? 4 : 2; // MMA tiles per stage
+    static constexpr int HEADS = kIdxHeads;       // heads per query row
+    static constexpr int NCOL = R * HEADS;        // MMA N: R rows x HEADS heads
+    static constexpr int SUB = R > 1 ? 1 : (D_I == 64 ? 4 : 2);  // MMA tiles per stage
     static constexpr int STOK = SUB * TILE;       // tokens per stage
-    static constexpr int BOX = 256;               // tokens per TMA box (the box limit)
+    static constexpr int BOX = STOK < 256 ? STOK : 256;  // tokens per TMA box (the box limit is 256)
     static constexpr int NBOX = STOK / BOX;       // key and scale boxes per stage
-    static constexpr int HEADS = kIdxHeads;
-    static constexpr int STAGES = D_I == 64 ? 4 : 5;
+    static constexpr int STAGES = R > 1 ? (D_I == 64 ? 12 : 6) : (D_I == 64 ? 4 : 5);
     static constexpr int KTILE_BYTES = STOK * D_I;
-    static constexpr int Q_BYTES = HEADS * D_I;
+    static constexpr int Q_BYTES = NCOL * D_I;
     static constexpr uint32_t SWZ = D_I == 64 ? kSwizzle64B : kSwizzle128B;
     static constexpr uint32_t SBO = 8 * D_I;      // 8-row swizzle atom
     static constexpr int TMEM_COLS = 512;
-    static constexpr int ACC = TMEM_COLS / (SUB * HEADS);  // TMEM accumulators of SUB x HEADS columns
+    static constexpr int ACC = TMEM_COLS / (SUB * NCOL);  // TMEM accumulators of SUB x NCOL columns
     static constexpr int GROUPS = ACC;            // epilogue groups of four warps, one accumulator each
-    static_assert(ACC * SUB * HEADS <= TMEM_COLS, "accumulators must fit TMEM");
+    static_assert(ACC >= 2 && ACC * SUB * NCOL <= TMEM_COLS, "accumulators must fit TMEM twice");
     static constexpr int EPI_WARP0 = 2;
     static constexpr int THREADS = (EPI_WARP0 + 4 * GROUPS) * 32;
     static constexpr int K_STEPS = D_I / 32;      // kind::f8f6f4 consumes 32 bytes of K per MMA
@@ -68,12 +72,12 @@ struct IdxCfg {
     static constexpr int OFF_Q = OFF_K + STAGES * KTILE_BYTES;
     static constexpr int OFF_SC = OFF_Q + 2 * Q_BYTES;     // per-stage key scales (STOK fp32)
     static constexpr int SC_BYTES = STOK * 4;
-    static constexpr int OFF_WQ = OFF_SC + STAGES * SC_BYTES;  // 2 x HEADS folded weights
-    static constexpr int OFF_BAR = OFF_WQ + 2 * HEADS * 4;
+    static constexpr int OFF_WQ = OFF_SC + STAGES * SC_BYTES;  // 2 x NCOL folded weights
+    static constexpr int OFF_BAR = OFF_WQ + 2 * NCOL * 4;
     static constexpr int NBAR = 2 * STAGES + 4 + 2 * ACC;
     static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
     static constexpr int SMEM_BYTES = OFF_MISC + 64 + 1024;  // + alignment slack
-    static constexpr uint32_t IDESC = make_idesc(TILE, HEADS, 0 /*e4m3*/, 0 /*e4m3*/, 0, 0);
+    static constexpr uint32_t IDESC = make_idesc(TILE, NCOL, 0 /*e4m3*/, 0 /*e4m3*/, 0, 0);
 };
 
 struct IdxShared {
@@ -91,25 +95,44 @@ __device__ __forceinline__ int tiles_of(const IndexerArgs& a, int n, int b, int 
 __device__ __forceinline__ int row_tiles(const IndexerArgs& a, int r, int stok) {
     return tiles_of(a, a.q_len[r], a.q_seq[r], stok);
 }
+// A unit is R consecutive query rows of one sequence; its key range is the longest of
+// its rows.  -1 (unit skipped) for an invalid length or rows of different sequences.
+__device__ __forceinline__ int unit_len(const IndexerArgs& a, int u, int R) {
+    int n = 0;
+    const int b = a.q_seq[u * R];
+    for (int r = u * R; r < min(a.Nq, u * R + R); ++r) {
+        const int nr = a.q_len[r];
+        if (nr < 0 || nr > a.T_max || (int64_t)nr > a.ld || a.q_seq[r] != b) return -1;
+        n = max(n, nr);
+    }
+    return n;
+}
+__device__ __forceinline__ int unit_tiles(const IndexerArgs& a, int u, int R, int stok) {
+    if (R == 1) return row_tiles(a, u, stok);
+    const int n = unit_len(a, u, R);
+    return n < 0 ? 0 : tiles_of(a, n, a.q_seq[u * R], stok);
+}
 
 // Walks the flat (row, tile) list.  The row's sequence and length are read
 // once per row, never per tile: every issuing loop depends on them.
 struct TileCursor {
-    int row, j, nt, b, n;
+    int row, j, nt, b, n;  // row = unit (R query rows), n = the unit's longest row
     int stok;  // tokens per stage
+    int R;     // query rows per unit
     __device__ void load_row(const IndexerArgs& a) {
-        if (row < a.Nq) {
-            n = a.q_len[row];
-            b = a.q_seq[row];
-            nt = tiles_of(a, n, b, stok);
+        if (row * R < a.Nq) {
+            n = R == 1 ? a.q_len[row] : max(0, unit_len(a, row, R));
+            b = a.q_seq[row * R];
+            nt = unit_tiles(a, row, R, stok);
         } else {
             n = 0;
             b = 0;
             nt = 1;  // sentinel past the last row
         }
     }
-    __device__ void start(const IndexerArgs& a, int r0, int j0, int stok_) {
+    __device__ void start(const IndexerArgs& a, int r0, int j0, int stok_, int R_) {
         stok = stok_;
+        R = R_;
         row = r0;
         j = j0;
         load_row(a);
@@ -125,11 +148,11 @@ struct TileCursor {
     }
 };
 
-template <int D_I>
-__global__ void __launch_bounds__(IdxCfg<D_I>::THREADS, 1)
+template <int D_I, int R>
+__global__ void __launch_bounds__(IdxCfg<D_I, R>::THREADS, 1)
     indexer_fp8_kernel(const IndexerArgs a, const __grid_constant__ CUtensorMap tmap_k,
                        const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__ CUtensorMap tmap_s) {
-    using C = IdxCfg<D_I>;
+    using C = IdxCfg<D_I, R>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const uint32_t sbase = smem_u32(smem);
@@ -175,24 +198,30 @@ __global__ void __launch_bounds__(IdxCfg<D_I>::THREADS, 1)
         tmem_alloc(smem_u32(&sh->tmem_base), C::TMEM_COLS);
         tmem_relinquish();
     }
-    // Work range: this CTA's slice of the flat tile list (warp 2 scans the rows).
+    // Work range: this CTA's slice of the flat (unit, stage) list (warp 2 scans the units).
+    const int nunits = (a.Nq + R - 1) / R;
     if (warp == 2) {
+        if (blockIdx.x == 0) {
+            for (int r = lane; r < a.Nq; r += 32) {
+                if (a.q_len[r] != 0 && row_tiles(a, r, C::STOK) == 0) record_status(a.status, DSA_STATUS_LENGTH);
+                if (R > 1 && a.q_seq[r] != a.q_seq[r - r % R]) record_status(a.status, DSA_STATUS_INVALID_ARG);
+            }
+        }
         long long total = 0;
-        for (int base = 0; base < a.Nq; base += 32) {
+        for (int base = 0; base < nunits; base += 32) {
             const int r = base + lane;
-            int v = r < a.Nq ? row_tiles(a, r, C::STOK) : 0;
-            if (r < a.Nq && v == 0 && a.q_len[r] != 0 && blockIdx.x == 0) record_status(a.status, DSA_STATUS_LENGTH);
+            int v = r < nunits ? unit_tiles(a, r, R, C::STOK) : 0;
 #pragma unroll
             for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
             total += v;
         }
         const long long begin = total * blockIdx.x / gridDim.x;
         const long long end = total * (blockIdx.x + 1) / gridDim.x;
-        int row0 = a.Nq, j0 = 0;
+        int row0 = nunits, j0 = 0;
         long long run = 0;
-        for (int base = 0; base < a.Nq && row0 == a.Nq; base += 32) {
+        for (int base = 0; base < nunits && row0 == nunits; base += 32) {
             const int r = base + lane;
-            const int v = r < a.Nq ? row_tiles(a, r, C::STOK) : 0;
+            const int v = r < nunits ? unit_tiles(a, r, R, C::STOK) : 0;
             int incl = v;
 #pragma unroll
             for (int o = 1; o < 32; o <<= 1) {
@@ -226,7 +255,7 @@ __global__ void __launch_bounds__(IdxCfg<D_I>::THREADS, 1)
         // ---------------- producer
         if (count > 0) {
             TileCursor cur;
-            cur.start(a, sh->row0, sh->j0, C::STOK);
+            cur.start(a, sh->row0, sh->j0, C::STOK, R);
             int qi = -1;
             int issued = 0;
             for (int it = 0; it < count; ++it) {
@@ -237,14 +266,16 @@ __global__ void __launch_bounds__(IdxCfg<D_I>::THREADS, 1)
                         const bool okq = mbar_wait(bar_qempty(qb), ((qi - 2) >> 1) & 1, abort_flag, a.status);
                         if (!__all_sync(0xffffffffu, okq)) break;
                     }
-                    const int64_t o = (int64_t)cur.row * C::HEADS;
+                    // folded weights w * q_scale of the unit's rows (0 past the last row)
+                    const int64_t o = (int64_t)cur.row * C::NCOL;
                     const __nv_bfloat16* wr = reinterpret_cast<const __nv_bfloat16*>(a.w) + o;
-                    wq_smem[qb * C::HEADS + lane] = __bfloat162float(wr[lane]) * a.q_scale[o + lane];
-                    wq_smem[qb * C::HEADS + 32 + lane] = __bfloat162float(wr[32 + lane]) * a.q_scale[o + 32 + lane];
+                    const int64_t lim = (int64_t)a.Nq * C::HEADS - o;
+                    for (int i = lane; i < C::NCOL; i += 32)
+                        wq_smem[qb * C::NCOL + i] = i < lim ? __bfloat162float(wr[i]) * a.q_scale[o + i] : 0.f;
                     __syncwarp();
                     if (lane == 0) {
                         mbar_arrive_expect_tx(bar_qfull(qb), C::Q_BYTES);
-                        tma_load_2d(sQ + qb * C::Q_BYTES, &tmap_q, 0, cur.row * C::HEADS, bar_qfull(qb));
+                        tma_load_2d(sQ + qb * C::Q_BYTES, &tmap_q, 0, cur.row * C::NCOL, bar_qfull(qb));
                     }
                 }
                 const int st = it % C::STAGES;
@@ -275,7 +306,7 @@ __global__ void __launch_bounds__(IdxCfg<D_I>::THREADS, 1)
         if (lane == 0 && count > 0) {
             // ---------------- MMA issuer
             TileCursor cur;
-            cur.start(a, sh->row0, sh->j0, C::STOK);
+            cur.start(a, sh->row0, sh->j0, C::STOK, R);
             int qi = -1, qb = 0;
             int last_acc = -1, last_it = -1;
             for (int it = 0; it < count; ++it) {
@@ -293,7 +324,7 @@ __global__ void __launch_bounds__(IdxCfg<D_I>::THREADS, 1)
                 const uint32_t b_addr = sQ + qb * C::Q_BYTES;
 #pragma unroll
                 for (int h = 0; h < C::SUB; ++h) {
-                    const uint32_t d = tmem + acc * (C::SUB * C::HEADS) + h * C::HEADS;
+                    const uint32_t d = tmem + acc * (C::SUB * C::NCOL) + h * C::NCOL;
                     const uint32_t a_addr = sK + st * C::KTILE_BYTES + h * (C::TILE * D_I);
 #pragma unroll
                     for (int ks = 0; ks < C::K_STEPS; ++ks) {
@@ -317,8 +348,11 @@ __global__ void __launch_bounds__(IdxCfg<D_I>::THREADS, 1)
         const int sub = warp & 3;                  // TMEM sub-partition this warp may access
         const int m = sub * 32 + lane;             // token row inside the tile
         TileCursor cur;
-        if (count > 0) cur.start(a, sh->row0, sh->j0, C::STOK);
-        int qi = -1, qb = 0, n = 0;
+        if (count > 0) cur.start(a, sh->row0, sh->j0, C::STOK, R);
+        int qi = -1, qb = 0;
+        int nr[R];  // lengths of the unit's rows (0 past the last row)
+#pragma unroll
+        for (int r = 0; r < R; ++r) nr[r] = 0;
         const float* wq = wq_smem;
         for (int it = 0; it < count; ++it) {
             const bool seg_start = it == 0 || cur.j == 0;
@@ -326,7 +360,11 @@ __global__ void __launch_bounds__(IdxCfg<D_I>::THREADS, 1)
             if (seg_start) {
                 ++qi;
                 qb = qi & 1;
-                n = cur.n;
+#pragma unroll
+                for (int r = 0; r < R; ++r) {
+                    const int row = cur.row * R + r;
+                    nr[r] = R == 1 ? cur.n : (row < a.Nq ? max(0, min(a.q_len[row], cur.n)) : 0);
+                }
             }
             if (it % C::GROUPS == g) {
                 {
@@ -334,7 +372,7 @@ __global__ void __launch_bounds__(IdxCfg<D_I>::THREADS, 1)
                     // (cannot move on before this warp releases the row at its end)
                     const bool okq = mbar_wait(bar_qfull(qb), (qi >> 1) & 1, abort_flag, a.status);
                     if (!__all_sync(0xffffffffu, okq)) break;
-                    wq = wq_smem + qb * C::HEADS;
+                    wq = wq_smem + qb * C::NCOL;
                 }
                 const int st = it % C::STAGES;
                 const int acc = it % C::ACC;
@@ -344,33 +382,38 @@ __global__ void __launch_bounds__(IdxCfg<D_I>::THREADS, 1)
                 tc_fence_after();
 #pragma unroll
                 for (int h = 0; h < C::SUB; ++h) {
-                    // token h * TILE + m of the stage: TMEM lane m of accumulator half h
-                    uint32_t v0[32], v1[32];
-                    const uint32_t taddr =
-                        tmem + ((uint32_t)(sub * 32) << 16) + acc * (C::SUB * C::HEADS) + h * C::HEADS;
-                    tmem_ld32(taddr, v0);
-                    tmem_ld32(taddr + 32, v1);
-                    tmem_wait_ld();
-                    float p0 = 0.f, p1 = 0.f, p2 = 0.f, p3 = 0.f;
-#pragma unroll
-                    for (int j = 0; j < 32; j += 4) {
-                        const float4 w4 = *reinterpret_cast<const float4*>(wq + j);
-                        p0 = fmaf(w4.x, fmaxf(__uint_as_float(v0[j + 0]), 0.f), p0);
-                        p1 = fmaf(w4.y, fmaxf(__uint_as_float(v0[j + 1]), 0.f), p1);
-                        p2 = fmaf(w4.z, fmaxf(__uint_as_float(v0[j + 2]), 0.f), p2);
-                        p3 = fmaf(w4.w, fmaxf(__uint_as_float(v0[j + 3]), 0.f), p3);
-                    }
-#pragma unroll
-                    for (int j = 0; j < 32; j += 4) {
-                        const float4 w4 = *reinterpret_cast<const float4*>(wq + 32 + j);
-                        p0 = fmaf(w4.x, fmaxf(__uint_as_float(v1[j + 0]), 0.f), p0);
-                        p1 = fmaf(w4.y, fmaxf(__uint_as_float(v1[j + 1]), 0.f), p1);
-                        p2 = fmaf(w4.z, fmaxf(__uint_as_float(v1[j + 2]), 0.f), p2);
-                        p3 = fmaf(w4.w, fmaxf(__uint_as_float(v1[j + 3]), 0.f), p3);
-                    }
+                    // token h * TILE + m of the stage: TMEM lane m of accumulator h; the unit's
+                    // row r holds columns [r * HEADS, r * HEADS + HEADS)
                     const int s = cur.j * C::STOK + h * C::TILE + m;
-                    const float sc = scale_smem[st * C::STOK + h * C::TILE + m] * ((p0 + p1) + (p2 + p3));
-                    if (s < n) a.scores[(int64_t)cur.row * a.ld + s] = sc;
+                    const float ks = scale_smem[st * C::STOK + h * C::TILE + m];
+#pragma unroll 1
+                    for (int r = 0; r < R; ++r) {
+                        uint32_t v0[32], v1[32];
+                        const uint32_t taddr = tmem + ((uint32_t)(sub * 32) << 16) + acc * (C::SUB * C::NCOL) +
+                                               h * C::NCOL + r * C::HEADS;
+                        tmem_ld32(taddr, v0);
+                        tmem_ld32(taddr + 32, v1);
+                        tmem_wait_ld();
+                        const float* wr = wq + r * C::HEADS;
+                        float p0 = 0.f, p1 = 0.f, p2 = 0.f, p3 = 0.f;
+#pragma unroll
+                        for (int j = 0; j < 32; j += 4) {
+                            const float4 w4 = *reinterpret_cast<const float4*>(wr + j);
+                            p0 = fmaf(w4.x, fmaxf(__uint_as_float(v0[j + 0]), 0.f), p0);
+                            p1 = fmaf(w4.y, fmaxf(__uint_as_float(v0[j + 1]), 0.f), p1);
+                            p2 = fmaf(w4.z, fmaxf(__uint_as_float(v0[j + 2]), 0.f), p2);
+                            p3 = fmaf(w4.w, fmaxf(__uint_as_float(v0[j + 3]), 0.f), p3);
+                        }
+#pragma unroll
+                        for (int j = 0; j < 32; j += 4) {
+                            const float4 w4 = *reinterpret_cast<const float4*>(wr + 32 + j);
+                            p0 = fmaf(w4.x, fmaxf(__uint_as_float(v1[j + 0]), 0.f), p0);
+                            p1 = fmaf(w4.y, fmaxf(__uint_as_float(v1[j + 1]), 0.f), p1);
+                            p2 = fmaf(w4.z, fmaxf(__uint_as_float(v1[j + 2]), 0.f), p2);
+                            p3 = fmaf(w4.w, fmaxf(__uint_as_float(v1[j + 3]), 0.f), p3);
+                        }
+                        if (s < nr[r]) a.scores[(int64_t)(cur.row * R + r) * a.ld + s] = ks * ((p0 + p1) + (p2 + p3));
+                    }
                 }
                 // TMEM and the key stage (its scales included) are free: the MMA has completed
                 tc_fence_before();
@@ -396,18 +439,19 @@ __global__ void __launch_bounds__(IdxCfg<D_I>::THREADS, 1)
     }
 }
 
-template <int D_I>
+template <int D_I, int R>
 cudaError_t launch_fp8_impl(const IndexerArgs& a, int grid, cudaStream_t st) {
-    using C = IdxCfg<D_I>;
+    using C = IdxCfg<D_I, R>;
     alignas(64) CUtensorMap tk, tq, ts;
     const int swz = D_I;  // 64-byte rows -> 64B swizzle, 128-byte rows -> 128B swizzle
     if (!encode_tensor_map_2d(&tk, 1, a.k_I, D_I, (uint64_t)a.B * a.T_max, D_I, D_I, C::BOX, swz))
         return cudaErrorInvalidValue;
-    if (!encode_tensor_map_2d(&tq, 1, a.q_I, D_I, (uint64_t)a.Nq * C::HEADS, D_I, D_I, C::HEADS, swz))
+    // q8 rows of a unit are consecutive: [Nq * HEADS, d_I], boxes of NCOL rows
+    if (!encode_tensor_map_2d(&tq, 1, a.q_I, D_I, (uint64_t)a.Nq * C::HEADS, D_I, D_I, C::NCOL, swz))
         return cudaErrorInvalidValue;
     if (!encode_tensor_map_2d(&ts, 4, a.k_scale, a.T_max, (uint64_t)a.B, (uint64_t)a.T_max * 4, C::BOX, 1, 0))
         return cudaErrorInvalidValue;
-    auto kern = indexer_fp8_kernel<D_I>;
+    auto kern = indexer_fp8_kernel<D_I, R>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
     if (e != cudaSuccess) return e;
     kern<<<grid, C::THREADS, C::SMEM_BYTES, st>>>(a, tk, tq, ts);
@@ -418,8 +462,15 @@ cudaError_t launch_fp8_impl(const IndexerArgs& a, int grid, cudaStream_t st) {
 
 cudaError_t launch_indexer_fp8(const IndexerArgs& a, int grid, cudaStream_t st) {
     if (a.Nq == 0) return cudaSuccess;
-    if (a.d_I == 64) return launch_fp8_impl<64>(a, grid, st);
-    if (a.d_I == 128) return launch_fp8_impl<128>(a, grid, st);
+    if (a.d_I == 64) return launch_fp8_impl<64, 1>(a, grid, st);
+    if (a.d_I == 128) return launch_fp8_impl<128, 1>(a, grid, st);
+    return cudaErrorInvalidValue;
+}
+
+cudaError_t launch_indexer_fp8_units4(const IndexerArgs& a, int grid, cudaStream_t st) {
+    if (a.Nq == 0) return cudaSuccess;
+    if (a.d_I == 64) return launch_fp8_impl<64, 4>(a, grid, st);
+    if (a.d_I == 128) return launch_fp8_impl<128, 4>(a, grid, st);
     return cudaErrorInvalidValue;
 }
 

@@ -56,6 +56,9 @@ struct MlaArgs {
 };
 
 cudaError_t launch_indexer_fp8(const IndexerArgs& a, int grid, cudaStream_t st);
+// Same scores, four consecutive query rows per tensor-core pass: every group of four
+// rows (row 4u .. 4u+3) must belong to one sequence (prefill).
+cudaError_t launch_indexer_fp8_units4(const IndexerArgs& a, int grid, cudaStream_t st);
 cudaError_t launch_indexer_f32(const IndexerArgs& a, cudaStream_t st);
 cudaError_t launch_topk(const TopkArgs& a, int cluster, cudaStream_t st);
 cudaError_t launch_sparse_mla_bf16(const MlaArgs& a, cudaStream_t st);

@@ -9,6 +9,7 @@ namespace dsa {
 
 enum : int {
     DSA_STATUS_OK = 0,
+    DSA_STATUS_INVALID_ARG = 1,  // an argument only the device can check (dsa_prefill: rows of different sequences)
     DSA_STATUS_TIMEOUT = 5,
     DSA_STATUS_INDEX_OOB = 6,
     DSA_STATUS_LENGTH = 7,
