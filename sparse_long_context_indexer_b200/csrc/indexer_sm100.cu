@@ -8,29 +8,41 @@
 // because both scales are positive and ReLU(c x) = c ReLU(x) for c > 0.
 //
 // Shape of the work: for one query row, [H_I x d_I] . [d_I x n] is a dense
-// FP8 contraction.  A stage is 256 cached tokens: two MMA tiles of 128 tokens
-// (MMA M = 128) against the 64 heads of one query (MMA N = 64), K = d_I,
-// accumulated in fp32 in tensor memory.  The epilogue reads one token row per
-// thread and tile from TMEM, applies ReLU, the weighted head sum and the key
-// scale, and writes one fp32 score: per-head products never leave the chip.
+// FP8 contraction.  Decode (rows of different sequences): a stage is 512
+// cached tokens, four MMA tiles of 128 tokens (MMA M = 128) against the 64
+// heads of one query (MMA N = 64), K = d_I, accumulated in fp32 in tensor
+// memory.  Prefill (consecutive rows of one sequence): a stage is one tile of
+// 128 tokens against four query rows at once (MMA N = 4 x 64 = 256), so a key
+// tile is read once per four rows.  Either way an accumulator is four blocks of
+// 64 columns.  The epilogue reads one token row per thread from TMEM, applies
+// ReLU, the weighted head sum and the key scale, and writes one fp32 score:
+// per-head products never leave the chip.
 //
 // Every asynchronous hand-off (a TMA copy, an MMA, a commit) costs the
 // per-SM pipeline time of its own (measured on B200: ~60 cycles per MMA and
 // ~100 per commit on the critical path of a 128-token tile, which held the
-// kernel at ~2.1 TB/s with 128-token stages), so a stage carries 256 tokens
-// with one key copy, one scale copy and one commit, and the key stage is
-// released by the epilogue warps (which have seen the MMA complete) rather
-// than by a second commit.
+// kernel at ~2.1 TB/s with 128-token stages), so a decode stage carries 512
+// tokens with one commit, and the key stage and the accumulator are released
+// by the epilogue warps (which have seen the MMA complete and hold its result
+// in registers) rather than by a second commit.
+//
+// The epilogue is ALU bound in prefill: per (token, head) one ReLU (FMNMX, on
+// the half-rate ALU pipe) and half a packed fp32 FMA, with the weights
+// broadcast from shared memory.  Sixteen epilogue warps, four per TMEM
+// sub-partition, each own one 64-column block of every accumulator, and give
+// the accumulator back as soon as their loads have landed, so the tensor pipe
+// never waits for the arithmetic.
 //
 // Roles (one persistent CTA per SM, each owning a contiguous range of the
-// flat list of (query row, 256-token stage) pairs):
-//   warp 0       producer: lane 0 issues the TMA copies of each 256-token key
-//                block and of its 256 fp32 scales into a stage ring; at a new
-//                query row the warp writes the folded weights w*q_scale to
-//                shared memory and lane 0 fetches the row's q8 block by TMA
+// flat list of (unit, stage) pairs; a unit is one query row in decode, four
+// in prefill):
+//   warp 0       producer: lane 0 issues the TMA copies of each key stage and
+//                of its fp32 scales into a stage ring; at a new unit the warp
+//                writes the folded weights w*q_scale to shared memory and lane
+//                0 fetches the unit's q8 block by TMA
 //   warp 1       TMEM allocator and single-thread tcgen05.mma issuer
-//   warps 2..17  epilogue, four groups of four warps taking every fourth stage,
-//                each with its own 128-column TMEM accumulator pair
+//   warps 2..    epilogue, quad q (one warp per TMEM sub-partition) reading
+//                block q of every accumulator
 // Every wait is bounded; a timeout records DSA_ERR_TIMEOUT and the CTA drains
 // and exits instead of hanging.
 #include <cuda.h>
@@ -39,6 +51,10 @@
 
 #include "kernels.h"
 #include "ptx.cuh"
+
+#ifndef PREFILL_ROWS
+#define PREFILL_ROWS 4
+#endif
 
 namespace dsa {
 namespace {
@@ -62,10 +78,15 @@ struct IdxCfg {
     static constexpr uint32_t SBO = 8 * D_I;      // 8-row swizzle atom
     static constexpr int TMEM_COLS = 512;
     static constexpr int ACC = TMEM_COLS / (SUB * NCOL);  // TMEM accumulators of SUB x NCOL columns
-    static constexpr int GROUPS = ACC;            // epilogue groups of four warps, one accumulator each
     static_assert(ACC >= 2 && ACC * SUB * NCOL <= TMEM_COLS, "accumulators must fit TMEM twice");
+    // 64-column blocks of one accumulator (one query row of one 128-token tile each).  An
+    // epilogue quad (four warps, one per TMEM sub-partition) reads one block; a group of NB
+    // quads covers an accumulator, and with QP groups group g takes the stages it % QP == g.
+    static constexpr int NB = SUB * R;
+    static constexpr int QP = R == 2 ? 2 : 1;
     static constexpr int EPI_WARP0 = 2;
-    static constexpr int THREADS = (EPI_WARP0 + 4 * GROUPS) * 32;
+    static constexpr int EPI_WARPS = 4 * NB * QP;
+    static constexpr int THREADS = (EPI_WARP0 + EPI_WARPS) * 32;
     static constexpr int K_STEPS = D_I / 32;      // kind::f8f6f4 consumes 32 bytes of K per MMA
     // shared memory map (offsets from a 1024-byte aligned base)
     static constexpr int OFF_K = 0;
@@ -113,26 +134,23 @@ __device__ __forceinline__ int unit_tiles(const IndexerArgs& a, int u, int R, in
     return n < 0 ? 0 : tiles_of(a, n, a.q_seq[u * R], stok);
 }
 
-// Walks the flat (row, tile) list.  The row's sequence and length are read
-// once per row, never per tile: every issuing loop depends on them.
+// Walks the flat (unit, stage) list.  The unit's sequence and length are read
+// once per unit, never per stage: every issuing loop depends on them.
+template <int STOK, int R>
 struct TileCursor {
     int row, j, nt, b, n;  // row = unit (R query rows), n = the unit's longest row
-    int stok;  // tokens per stage
-    int R;     // query rows per unit
     __device__ void load_row(const IndexerArgs& a) {
         if (row * R < a.Nq) {
             n = R == 1 ? a.q_len[row] : max(0, unit_len(a, row, R));
             b = a.q_seq[row * R];
-            nt = unit_tiles(a, row, R, stok);
+            nt = unit_tiles(a, row, R, STOK);
         } else {
             n = 0;
             b = 0;
             nt = 1;  // sentinel past the last row
         }
     }
-    __device__ void start(const IndexerArgs& a, int r0, int j0, int stok_, int R_) {
-        stok = stok_;
-        R = R_;
+    __device__ void start(const IndexerArgs& a, int r0, int j0) {
         row = r0;
         j = j0;
         load_row(a);
@@ -178,15 +196,17 @@ __global__ void __launch_bounds__(IdxCfg<D_I, R>::THREADS, 1)
     if (tid == 0) {
         for (int s = 0; s < C::STAGES; ++s) {
             mbar_init(bar_full(s), 1);
-            mbar_init(bar_empty(s), 4);  // the 4 epilogue warps of the stage (they have seen the MMA complete)
+            mbar_init(bar_empty(s), 4 * C::NB);  // every warp of the stage's epilogue group, once it
+                                                 // has its scales (the MMA that read the keys has
+                                                 // completed before)
         }
         for (int q = 0; q < 2; ++q) {
-            mbar_init(bar_qfull(q), 1);                   // producer arrival with the q8 block's tx bytes
-            mbar_init(bar_qempty(q), 1 + 4 * C::GROUPS);  // MMA commit + every epilogue warp
+            mbar_init(bar_qfull(q), 1);                    // producer arrival with the q8 block's tx bytes
+            mbar_init(bar_qempty(q), 1 + C::EPI_WARPS);    // MMA commit + every epilogue warp
         }
         for (int c = 0; c < C::ACC; ++c) {
             mbar_init(bar_tfull(c), 1);
-            mbar_init(bar_tempty(c), 4);
+            mbar_init(bar_tempty(c), 4 * C::NB);  // every warp of the stage's group, once its loads landed
         }
         sh->abort_flag = 0;
         fence_barrier_init();
@@ -254,8 +274,8 @@ __global__ void __launch_bounds__(IdxCfg<D_I, R>::THREADS, 1)
     if (warp == 0) {
         // ---------------- producer
         if (count > 0) {
-            TileCursor cur;
-            cur.start(a, sh->row0, sh->j0, C::STOK, R);
+            TileCursor<C::STOK, R> cur;
+            cur.start(a, sh->row0, sh->j0);
             int qi = -1;
             int issued = 0;
             for (int it = 0; it < count; ++it) {
@@ -305,8 +325,8 @@ __global__ void __launch_bounds__(IdxCfg<D_I, R>::THREADS, 1)
     } else if (warp == 1) {
         if (lane == 0 && count > 0) {
             // ---------------- MMA issuer
-            TileCursor cur;
-            cur.start(a, sh->row0, sh->j0, C::STOK, R);
+            TileCursor<C::STOK, R> cur;
+            cur.start(a, sh->row0, sh->j0);
             int qi = -1, qb = 0;
             int last_acc = -1, last_it = -1;
             for (int it = 0; it < count; ++it) {
@@ -318,7 +338,9 @@ __global__ void __launch_bounds__(IdxCfg<D_I, R>::THREADS, 1)
                 const int st = it % C::STAGES;
                 if (!mbar_wait(bar_full(st), (it / C::STAGES) & 1, abort_flag, a.status)) break;
                 const int acc = it % C::ACC;
-                if (it >= C::ACC && !mbar_wait(bar_tempty(acc), ((it / C::ACC) - 1) & 1, abort_flag, a.status))
+                // polled: the accumulator comes back while the epilogue warps compute, and a
+                // suspended wait would resume late on the tensor pipe's critical path
+                if (it >= C::ACC && !mbar_wait_spin(bar_tempty(acc), ((it / C::ACC) - 1) & 1, abort_flag, a.status))
                     break;
                 tc_fence_after();
                 const uint32_t b_addr = sQ + qb * C::Q_BYTES;
@@ -343,90 +365,107 @@ __global__ void __launch_bounds__(IdxCfg<D_I, R>::THREADS, 1)
                 mbar_wait(bar_tfull(last_acc), (last_it / C::ACC) & 1, nullptr, nullptr, 50000000ull);
         }
     } else {
-        // ---------------- epilogue: one token row per thread
-        const int g = (warp - C::EPI_WARP0) >> 2;  // epilogue group: tiles it with it % GROUPS == g
+        // ---------------- epilogue: one 64-column block of its group's accumulators per warp
+        // A warp reads its block (32 token lanes x 64 heads) in the 16x256b shape: thread t
+        // holds tokens g, g+8, g+16, g+24 (g = t/4) at the 16 heads 8k + 2(t%4) + {0, 1}, so
+        // its 16 folded weights stay in registers for the whole unit; four threads then
+        // combine their partial sums by shuffles.
+        const int q = (warp - C::EPI_WARP0) >> 2;  // quad
+        const int grp = q / C::NB;                 // group: stages it % QP == grp
+        const int blk = q % C::NB;                 // block of the group's accumulators
         const int sub = warp & 3;                  // TMEM sub-partition this warp may access
-        const int m = sub * 32 + lane;             // token row inside the tile
-        TileCursor cur;
-        if (count > 0) cur.start(a, sh->row0, sh->j0, C::STOK, R);
-        int qi = -1, qb = 0;
-        int nr[R];  // lengths of the unit's rows (0 past the last row)
+        const int h = R == 1 ? blk : 0;            // the block's tile within the stage
+        const int r = R == 1 ? 0 : blk;            // the block's query row within the unit
+        const int g = lane >> 2;
+        const int i4 = lane & 3;
+        // after the shuffles thread t owns token slot u = 2 (t%2) + (t%4)/2: token g + 8u of the
+        // warp's 32 lanes, i.e. token `tok` of every stage
+        const int tok = h * C::TILE + sub * 32 + g + 8 * (2 * (i4 & 1) + (i4 >> 1));
+        TileCursor<C::STOK, R> cur;
+        if (count > 0) cur.start(a, sh->row0, sh->j0);
+        int qi = -1;
+        int nrow = 0;               // this thread's scores exist for s < nrow (s = stage base + tok)
+        float* srow = nullptr;      // score row of the block's query row, offset by tok
+        int acc = 0, accph = 0;     // accumulator of stage `it` and its phase parity
+        uint64_t w2[8];             // folded weights of heads 8k + 2(t%4) + {0, 1}, packed in pairs
 #pragma unroll
-        for (int r = 0; r < R; ++r) nr[r] = 0;
-        const float* wq = wq_smem;
+        for (int k = 0; k < 8; ++k) w2[k] = 0;
         for (int it = 0; it < count; ++it) {
-            const bool seg_start = it == 0 || cur.j == 0;
-            const bool seg_end = cur.j == cur.nt - 1 || it == count - 1;
-            if (seg_start) {
+            if (it == 0 || cur.j == 0) {
                 ++qi;
-                qb = qi & 1;
+                const int qb = qi & 1;
+                const int64_t row = (int64_t)cur.row * R + r;
+                nrow = (R == 1 ? cur.n : (row < a.Nq ? max(0, min(a.q_len[row], cur.n)) : 0)) - tok;
+                srow = a.scores + row * a.ld + tok;
+                // folded weights of the unit: published by the producer with the q8 block
+                const bool okq = mbar_wait(bar_qfull(qb), (qi >> 1) & 1, abort_flag, a.status);
+                if (!__all_sync(0xffffffffu, okq)) break;
+                const float* wsrc = wq_smem + qb * C::NCOL + r * C::HEADS + 2 * i4;
 #pragma unroll
-                for (int r = 0; r < R; ++r) {
-                    const int row = cur.row * R + r;
-                    nr[r] = R == 1 ? cur.n : (row < a.Nq ? max(0, min(a.q_len[row], cur.n)) : 0);
-                }
+                for (int k = 0; k < 8; ++k) w2[k] = pack_f32x2(wsrc[8 * k], wsrc[8 * k + 1]);
+                // the weights are in registers: the producer may reuse the buffer
+                __syncwarp();
+                if (lane == 0) mbar_arrive(bar_qempty(qb));
             }
-            if (it % C::GROUPS == g) {
-                {
-                    // folded weights of this row: published by the producer with the q8 block
-                    // (cannot move on before this warp releases the row at its end)
-                    const bool okq = mbar_wait(bar_qfull(qb), (qi >> 1) & 1, abort_flag, a.status);
-                    if (!__all_sync(0xffffffffu, okq)) break;
-                    wq = wq_smem + qb * C::NCOL;
-                }
+            if (C::QP == 1 || it % C::QP == grp) {
                 const int st = it % C::STAGES;
-                const int acc = it % C::ACC;
-                bool ok = mbar_wait(bar_tfull(acc), (it / C::ACC) & 1, abort_flag, a.status);
+                bool ok = mbar_wait(bar_tfull(acc), accph, abort_flag, a.status);
                 ok = ok && mbar_wait(bar_full(st), (it / C::STAGES) & 1, abort_flag, a.status);
                 if (!__all_sync(0xffffffffu, ok)) break;
                 tc_fence_after();
-#pragma unroll
-                for (int h = 0; h < C::SUB; ++h) {
-                    // token h * TILE + m of the stage: TMEM lane m of accumulator h; the unit's
-                    // row r holds columns [r * HEADS, r * HEADS + HEADS)
-                    const int s = cur.j * C::STOK + h * C::TILE + m;
-                    const float ks = scale_smem[st * C::STOK + h * C::TILE + m];
-#pragma unroll 1
-                    for (int r = 0; r < R; ++r) {
-                        uint32_t v0[32], v1[32];
-                        const uint32_t taddr = tmem + ((uint32_t)(sub * 32) << 16) + acc * (C::SUB * C::NCOL) +
-                                               h * C::NCOL + r * C::HEADS;
-                        tmem_ld32(taddr, v0);
-                        tmem_ld32(taddr + 32, v1);
-                        tmem_wait_ld();
-                        const float* wr = wq + r * C::HEADS;
-                        float p0 = 0.f, p1 = 0.f, p2 = 0.f, p3 = 0.f;
-#pragma unroll
-                        for (int j = 0; j < 32; j += 4) {
-                            const float4 w4 = *reinterpret_cast<const float4*>(wr + j);
-                            p0 = fmaf(w4.x, fmaxf(__uint_as_float(v0[j + 0]), 0.f), p0);
-                            p1 = fmaf(w4.y, fmaxf(__uint_as_float(v0[j + 1]), 0.f), p1);
-                            p2 = fmaf(w4.z, fmaxf(__uint_as_float(v0[j + 2]), 0.f), p2);
-                            p3 = fmaf(w4.w, fmaxf(__uint_as_float(v0[j + 3]), 0.f), p3);
-                        }
-#pragma unroll
-                        for (int j = 0; j < 32; j += 4) {
-                            const float4 w4 = *reinterpret_cast<const float4*>(wr + 32 + j);
-                            p0 = fmaf(w4.x, fmaxf(__uint_as_float(v1[j + 0]), 0.f), p0);
-                            p1 = fmaf(w4.y, fmaxf(__uint_as_float(v1[j + 1]), 0.f), p1);
-                            p2 = fmaf(w4.z, fmaxf(__uint_as_float(v1[j + 2]), 0.f), p2);
-                            p3 = fmaf(w4.w, fmaxf(__uint_as_float(v1[j + 3]), 0.f), p3);
-                        }
-                        if (s < nr[r]) a.scores[(int64_t)(cur.row * R + r) * a.ld + s] = ks * ((p0 + p1) + (p2 + p3));
-                    }
+                uint32_t v[2][32];
+                {
+                    const uint32_t taddr =
+                        tmem + ((uint32_t)(sub * 32) << 16) + acc * (C::SUB * C::NCOL) + blk * C::HEADS;
+                    tmem_ld16x256b_x8(taddr, v[0]);
+                    tmem_ld16x256b_x8(taddr + (16u << 16), v[1]);
+                    tmem_wait_ld_regs(v[0]);
+                    tmem_wait_ld_regs(v[1]);
                 }
-                // TMEM and the key stage (its scales included) are free: the MMA has completed
+                const int sb = cur.j * C::STOK;
+                const float ks = scale_smem[st * C::STOK + tok];
+                // the accumulator is free (the values are in registers) and so is the key stage (the
+                // MMA that read it has completed; the scale is in a register)
                 tc_fence_before();
                 __syncwarp();
                 if (lane == 0) {
                     mbar_arrive(bar_tempty(acc));
                     mbar_arrive(bar_empty(st));
                 }
+                // p2[u]: this thread's 16 heads of token slot u (tokens g, g+8 from the first load,
+                // g+16, g+24 from the second), two heads per packed FMA
+                uint64_t p2[4] = {0, 0, 0, 0};
+#pragma unroll
+                for (int k = 0; k < 8; ++k) {
+#pragma unroll
+                    for (int u = 0; u < 4; ++u) {
+                        const uint32_t* x = &v[u >> 1][4 * k + 2 * (u & 1)];
+                        p2[u] = fma_f32x2(w2[k],
+                                          pack_f32x2(fmaxf(__uint_as_float(x[0]), 0.f),
+                                                     fmaxf(__uint_as_float(x[1]), 0.f)),
+                                          p2[u]);
+                    }
+                }
+                float s0, s1, s2, s3, t0, t1, t2, t3;
+                unpack_f32x2(p2[0], s0, t0);
+                unpack_f32x2(p2[1], s1, t1);
+                unpack_f32x2(p2[2], s2, t2);
+                unpack_f32x2(p2[3], s3, t3);
+                s0 += t0;
+                s1 += t1;
+                s2 += t2;
+                s3 += t3;
+                // sum over the four threads of a token group, leaving slot 2 (t%2) + (t%4)/2 here
+                const bool odd = i4 & 1;
+                const float qa = (odd ? s2 : s0) + __shfl_xor_sync(0xffffffffu, odd ? s0 : s2, 1);
+                const float qc = (odd ? s3 : s1) + __shfl_xor_sync(0xffffffffu, odd ? s1 : s3, 1);
+                const bool hi = i4 & 2;
+                const float sum = (hi ? qc : qa) + __shfl_xor_sync(0xffffffffu, hi ? qa : qc, 2);
+                if (sb < nrow) srow[sb] = ks * sum;
             }
-            if (seg_end) {
-                // this warp is done with the row's folded weights
-                __syncwarp();
-                if (lane == 0) mbar_arrive(bar_qempty(qb));
+            if (++acc == C::ACC) {
+                acc = 0;
+                accph ^= 1;
             }
             cur.advance(a);
         }
@@ -469,8 +508,8 @@ cudaError_t launch_indexer_fp8(const IndexerArgs& a, int grid, cudaStream_t st) 
 
 cudaError_t launch_indexer_fp8_units4(const IndexerArgs& a, int grid, cudaStream_t st) {
     if (a.Nq == 0) return cudaSuccess;
-    if (a.d_I == 64) return launch_fp8_impl<64, 4>(a, grid, st);
-    if (a.d_I == 128) return launch_fp8_impl<128, 4>(a, grid, st);
+    if (a.d_I == 64) return launch_fp8_impl<64, PREFILL_ROWS>(a, grid, st);
+    if (a.d_I == 128) return launch_fp8_impl<128, PREFILL_ROWS>(a, grid, st);
     return cudaErrorInvalidValue;
 }
 
