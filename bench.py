@@ -5,15 +5,24 @@ tokens each (H_I = 64, d_I = 64 FP8 indexer keys, top-2048, 128-head MLA over
 bf16 576-value latent rows), inputs resident in HBM.  Prints one JSON line.
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
+  python bench.py --workload prefill [--prefill-len L] [--steps K] [--warmup W]
 
 N > 1 is launched with torch.distributed.run (one process per GPU); every rank
 decodes its own batch (weak scaling, no data-path collective); the time is the
 max over ranks.  --impl reference times the CPU oracle (the only reference
 implementation there is) on a bounded sample of the same workload.
+
+--workload prefill times dsa_prefill over one causal prompt of L tokens
+(default 65,536: every position a query, top-2048, same shapes), then, in a
+second pass over the same row chunks, each stage through its own entry point
+(dsa_prefill_indexer_scores, dsa_topk, dsa_sparse_mla_attn) for the per-stage
+split and the indexer's tensor-core roofline (FP8 peak = 2 x the measured bf16
+peak).  It is a secondary line: the default run is the decode headline.
 """
 from __future__ import annotations
 
 import argparse
+import dataclasses
 import hashlib
 import json
 import math
@@ -44,6 +53,8 @@ def parse_args():
     p.add_argument("--warmup", type=int, default=20)
     p.add_argument("--impl", default="ours", choices=["ours", "reference"])
     p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--workload", default="long_decode", choices=["long_decode", "prefill"])
+    p.add_argument("--prefill-len", type=int, default=65536)
     return p.parse_args()
 
 
@@ -55,6 +66,16 @@ def peaks():
         return float(d["hbm_gbs"]), "measured"
     except Exception:
         return FALLBACK_HBM_GBS, "fallback"
+
+
+def tensor_peaks():
+    """FP8 dense peak (TFLOP/s) = 2 x the measured bf16 cuBLAS figures (the nominal fp8:bf16 ratio)."""
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            d = json.load(f)
+        return 2 * float(d["bf16_tflops"]), 2 * float(d["bf16_tflops_sustained"]), "measured"
+    except Exception:
+        return 2 * 1590.0, 2 * 1400.0, "fallback"
 
 
 def indexer_traffic():
@@ -346,6 +367,97 @@ def run_ours(args):
     return 0
 
 
+def run_prefill(args):
+    """Secondary line: one causal prompt of L tokens through dsa_prefill, with a per-stage split."""
+    import torch
+    from sparse_long_context_indexer_b200 import _lib, api, inputs
+
+    if args.gpus != 1:
+        raise SystemExit("--workload prefill runs on one GPU")
+    dev = torch.device("cuda", 0)
+    L = args.prefill_len
+    g = inputs.make_prefill_inputs(f"prefill_{L}", L, seed=4, device=dev)
+    dims = api.dims_of(g)
+    ws = api.make_workspace(dims, _lib.DSA_OP_PREFILL, dev)
+    out, lse = api.alloc_outputs(g)
+    idx = torch.empty((L, g.k), dtype=torch.int32, device=dev)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+
+    def whole():
+        api.prefill(dims, g.q_I, g.q_scale, g.w, g.k_I, g.k_scale, g.q, g.kv, g.q_seq, g.q_len, g.softmax_scale,
+                    out, lse, ws, idx_out=idx)
+
+    K, W = max(1, min(args.steps, 10)), args.warmup
+    for _ in range(W):
+        whole()
+    torch.cuda.synchronize()
+    ms = []
+    for _ in range(K):
+        flush.zero_()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        whole()
+        e1.record()
+        torch.cuda.synchronize()
+        ms.append(e0.elapsed_time(e1))
+    status = api.get_device_status(ws)
+    total_ms = statistics.median(ms)
+
+    # Stage pass: the same work, chunk by chunk, each stage through its own entry point.
+    chunk = max(1, min(L, (64 << 20) // (dims.ld_scores * 4)))
+    cd = api.Dims(B=1, Nq=chunk, H_I=g.H_I, d_I=g.d_I, H=g.H, k=g.k, T_max=g.T_max, idx_dtype=g.idx_dtype,
+                  kv_dtype=g.kv_dtype, ld_scores=dims.ld_scores)
+    cws = api.make_workspace(cd, _lib.DSA_OP_SPARSE_MLA, dev)
+    scores = torch.empty((chunk, dims.ld_scores), dtype=torch.float32, device=dev)
+    cidx = torch.empty((chunk, g.k), dtype=torch.int32, device=dev)
+    ev = []
+    for r0 in range(0, L, chunk):
+        r1 = min(L, r0 + chunk)
+        d = cd if r1 - r0 == chunk else dataclasses.replace(cd, Nq=r1 - r0)
+        e = [torch.cuda.Event(enable_timing=True) for _ in range(4)]
+        e[0].record()
+        api.prefill_indexer_scores(d, g.q_I[r0:r1], g.q_scale[r0:r1], g.w[r0:r1], g.k_I, g.k_scale, g.q_seq[r0:r1],
+                                   g.q_len[r0:r1], scores, cws)
+        e[1].record()
+        api.topk(d, scores, g.q_len[r0:r1], cidx, cws)
+        e[2].record()
+        api.sparse_mla_attn(d, g.q[r0:r1], g.kv, cidx, g.q_seq[r0:r1], g.q_len[r0:r1], g.softmax_scale,
+                            out[r0:r1], lse[r0:r1], cws)
+        e[3].record()
+        ev.append(e)
+    torch.cuda.synchronize()
+    stage_ms = [sum(e[j].elapsed_time(e[j + 1]) for e in ev) for j in range(3)]
+    status = status or api.get_device_status(cws)
+
+    pairs = int(g.q_len.sum().item())
+    idx_flop = pairs * 2.0 * g.H_I * g.d_I
+    sel = torch.clamp(g.q_len, max=g.k).sum().item()
+    mla_flop = sel * g.H * 2.0 * (576 + 512)
+    burst, sustained, src = tensor_peaks()
+    idx_tflops = idx_flop / (stage_ms[0] * 1e-3) / 1e12
+    line = {
+        "metric": f"prefill query-tok/s (one causal prompt of {L} tokens; index+top2048+sparse MLA)",
+        "value": L / (total_ms * 1e-3), "unit": "query-tok/s", "n_gpus": 1, "steps": K, "warmup": W,
+        "ms_per_step": total_ms, "higher_is_better": True, "scaling": "none", "vs_baseline": None,
+        "dtype": "fp8_e4m3/bf16", "data": "synthetic",
+        "config": {"workload": f"prefill_{L}", "H_I": g.H_I, "d_I": g.d_I, "top_k": g.k, "heads": g.H,
+                   "latent": "576 bf16 (512 + 64 rope)", "chunk_rows": chunk,
+                   "l2": "256 MiB written between steps, outside the timed events"},
+        "roofline": {"bound": "tensor", "kernel": "indexer_fp8_kernel (four rows per pass)",
+                     "achieved": idx_tflops, "peak": burst, "unit": "TFLOP/s", "frac": idx_tflops / burst,
+                     "frac_of_sustained": idx_tflops / sustained, "traffic": None,
+                     "peak_source": f"2 x {src} bf16_tflops (burst); sustained {sustained:.0f}",
+                     "algorithmic_flop": idx_flop},
+        "stages_ms": {"indexer": stage_ms[0], "topk": stage_ms[1], "sparse_mla": stage_ms[2]},
+        "sparse_mla_tflops": mla_flop / (stage_ms[2] * 1e-3) / 1e12,
+        "timing": {"step": "dsa_prefill between two events, median of the timed steps",
+                   "stages_ms": f"second pass of {len(ev)} chunks of {chunk} rows, two events per stage call"},
+        "device_status": status,
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
 def launches_per_step():
     """Kernels one decode step launches: indexer, top-k, attention, plus the split
     merge when the attention's split count is above the cluster limit (8)."""
@@ -443,6 +555,8 @@ def main():
     args = parse_args()
     if args.impl == "reference":
         return run_reference(args)
+    if args.workload == "prefill":
+        return run_prefill(args)
     return run_ours(args)
 
 

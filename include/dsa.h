@@ -125,6 +125,20 @@ dsa_status_t dsa_indexer_scores(const dsa_dims* dims, const void* q_I, const flo
                                 const int32_t* q_seq, const int32_t* q_len, float* scores,
                                 void* workspace, size_t ws_bytes, void* stream);
 
+/* Stage 1 for the rows of one prompt (prefill): the same scores as
+ * dsa_indexer_scores, with four consecutive query rows served by one
+ * tensor-core pass (MMA N = 4 x 64 heads), so that each cached key tile is read
+ * once per four rows.  Precondition: rows 4u .. 4u+3 belong to one sequence
+ * (q_seq equal); a group that does not is skipped and DSA_ERR_INVALID_ARG is
+ * recorded in the workspace's status word.  FP8 only (idx_dtype
+ * DSA_FP8_E4M3, H_I = 64, d_I 64 or 128); other dims return
+ * DSA_ERR_UNSUPPORTED.  Arguments, layouts and ownership as for
+ * dsa_indexer_scores. */
+dsa_status_t dsa_prefill_indexer_scores(const dsa_dims* dims, const void* q_I, const float* q_scale,
+                                        const void* w, const void* k_I, const float* k_scale,
+                                        const int32_t* q_seq, const int32_t* q_len, float* scores,
+                                        void* workspace, size_t ws_bytes, void* stream);
+
 /* Stage 2 -- per-row causal top-k (kgptalkie, "How Does the Selector Pick
  * 1,024?": keep the highest index_topk scores, min(budget, tokens so far),
  * redone for every query).  idx[t] holds the min(k, q_len[t]) positions of the

@@ -20,7 +20,8 @@ DSA_OP_INDEXER, DSA_OP_TOPK, DSA_OP_SPARSE_MLA, DSA_OP_DECODE, DSA_OP_PREFILL = 
 
 # every symbol include/dsa.h declares
 EXPORTS = (
-    "dsa_workspace_size", "dsa_workspace_init", "dsa_indexer_scores", "dsa_topk", "dsa_sparse_mla_attn",
+    "dsa_workspace_size", "dsa_workspace_init", "dsa_indexer_scores", "dsa_prefill_indexer_scores", "dsa_topk",
+    "dsa_sparse_mla_attn",
     "dsa_decode_step", "dsa_prefill", "dsa_get_device_status", "dsa_status_string", "dsa_last_cuda_error",
     "dsa_selftest_wait_timeout", "dsa_version", "dsa_sparse_mla_attn_noalloc",
 )
@@ -62,6 +63,7 @@ def _declare(lib):
     lib.dsa_workspace_size.argtypes = [D, I32, ctypes.POINTER(S)]
     lib.dsa_workspace_init.argtypes = [P, S, P]
     lib.dsa_indexer_scores.argtypes = [D, P, P, P, P, P, P, P, P, P, S, P]
+    lib.dsa_prefill_indexer_scores.argtypes = [D, P, P, P, P, P, P, P, P, P, S, P]
     lib.dsa_topk.argtypes = [D, P, P, P, P, S, P]
     lib.dsa_sparse_mla_attn.argtypes = [D, P, P, P, P, P, F, P, P, P, S, P]
     lib.dsa_sparse_mla_attn_noalloc.argtypes = [D, P, P, P, P, P, F, P, P, P]
@@ -70,7 +72,8 @@ def _declare(lib):
     lib.dsa_prefill.argtypes = [D, P, P, P, P, P, P, P, P, P, F, P, P, P, P, S, P]
     lib.dsa_get_device_status.argtypes = [P, P, ctypes.POINTER(I32)]
     lib.dsa_selftest_wait_timeout.argtypes = [P, S, I32, P]
-    for name in ("dsa_workspace_size", "dsa_workspace_init", "dsa_indexer_scores", "dsa_topk",
+    for name in ("dsa_workspace_size", "dsa_workspace_init", "dsa_indexer_scores", "dsa_prefill_indexer_scores",
+                 "dsa_topk",
                  "dsa_sparse_mla_attn", "dsa_decode_step", "dsa_prefill", "dsa_get_device_status",
                  "dsa_selftest_wait_timeout", "dsa_sparse_mla_attn_noalloc"):
         getattr(lib, name).restype = st

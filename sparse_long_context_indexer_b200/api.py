@@ -96,6 +96,17 @@ def indexer_scores(dims: Dims, q_I, q_scale, w, k_I, k_scale, q_seq, q_len, scor
     return scores
 
 
+def prefill_indexer_scores(dims: Dims, q_I, q_scale, w, k_I, k_scale, q_seq, q_len, scores, ws=None):
+    """Indexer scores for rows of one prompt: four consecutive rows per tensor-core pass."""
+    lib = _lib.load()
+    d = dims.c()
+    rc = lib.dsa_prefill_indexer_scores(ctypes.byref(d), _ptr(q_I), _ptr(q_scale), _ptr(w), _ptr(k_I), _ptr(k_scale),
+                                        _ptr(q_seq), _ptr(q_len), _ptr(scores), _ptr(ws),
+                                        0 if ws is None else ws.numel(), _stream_ptr())
+    _lib.check(lib, rc, "dsa_prefill_indexer_scores")
+    return scores
+
+
 def topk(dims: Dims, scores, q_len, idx, ws=None):
     lib = _lib.load()
     d = dims.c()

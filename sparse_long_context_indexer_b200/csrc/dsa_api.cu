@@ -270,6 +270,22 @@ dsa_status_t dsa_indexer_scores(const dsa_dims* dims, const void* q_I, const flo
                        workspace ? status_word(workspace) : nullptr, reinterpret_cast<cudaStream_t>(stream));
 }
 
+dsa_status_t dsa_prefill_indexer_scores(const dsa_dims* dims, const void* q_I, const float* q_scale, const void* w,
+                                        const void* k_I, const float* k_scale, const int32_t* q_seq,
+                                        const int32_t* q_len, float* scores, void* workspace, size_t ws_bytes,
+                                        void* stream) {
+    dsa_status_t s = check_dims(dims, true, false);
+    if (s != DSA_OK) return s;
+    if (dims->idx_dtype != DSA_FP8_E4M3 || dims->H_I != dsa::kIdxHeads || (dims->d_I != 64 && dims->d_I != 128))
+        return DSA_ERR_UNSUPPORTED;
+    if (dims->Nq == 0) return DSA_OK;
+    if (!q_I || !q_scale || !w || !k_I || !k_scale || !q_seq || !q_len || !scores) return DSA_ERR_INVALID_ARG;
+    if (!aligned16(q_I) || !aligned16(k_I) || !aligned16(scores) || !aligned16(w)) return DSA_ERR_INVALID_ARG;
+    if (workspace != nullptr && ws_bytes < kStatusBytes) return DSA_ERR_WORKSPACE;
+    return run_indexer(dims, dims->Nq, q_I, q_scale, w, k_I, k_scale, q_seq, q_len, scores,
+                       workspace ? status_word(workspace) : nullptr, reinterpret_cast<cudaStream_t>(stream), true);
+}
+
 dsa_status_t dsa_topk(const dsa_dims* dims, const float* scores, const int32_t* q_len, int32_t* idx, void* workspace,
                       size_t ws_bytes, void* stream) {
     dsa_status_t s = check_dims(dims, false, false);

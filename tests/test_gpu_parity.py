@@ -223,6 +223,57 @@ def test_prefill_matches_oracle(lib):
             assert np.array_equal(g_idx[i][: t + 1], np.arange(t + 1)) and np.all(g_idx[i][t + 1:] == -1)
 
 
+def oracle_scores_of_rows(inp, rows):
+    """Oracle indexer scores of the given query rows (whole rows, ld = the longest)."""
+    r = torch.as_tensor(list(rows), dtype=torch.long)
+    return oracle.indexer(inp, q_I=inp.q_I[r], q_scale=inp.q_scale[r], w=inp.w[r], q_seq=inp.q_seq[r],
+                          q_len=inp.q_len[r])
+
+
+def test_prefill_indexer_scores_match_oracle(lib):
+    # a prompt whose row count is not a multiple of four, several 128-token tiles and a ragged tail
+    L = 1283
+    inp = inputs.make_prefill_inputs("prefill_idx", L, seed=21)
+    g = inp.to("cuda")
+    dims = api.dims_of(g)
+    ws = api.make_workspace(dims, _lib.DSA_OP_INDEXER)
+    sc4 = torch.full((L, dims.ld_scores), float("nan"), dtype=torch.float32, device="cuda")
+    sc1 = torch.full_like(sc4, float("nan"))
+    api.prefill_indexer_scores(dims, g.q_I, g.q_scale, g.w, g.k_I, g.k_scale, g.q_seq, g.q_len, sc4, ws)
+    api.indexer_scores(dims, g.q_I, g.q_scale, g.w, g.k_I, g.k_scale, g.q_seq, g.q_len, sc1, ws)
+    torch.cuda.synchronize()
+    assert api.get_device_status(ws) == 0
+    rows = np.r_[0:6, 127:131, 640:644, 1279:1283]
+    sc_o = oracle_scores_of_rows(inp, rows)
+    got4 = np_scores(sc4)[rows][:, :sc_o.shape[1]]
+    q_len = inp.q_len.numpy()[rows]
+    check_scores(got4, sc_o, q_len)
+    got1 = np_scores(sc1)[rows][:, :sc_o.shape[1]]
+    for i, n in enumerate(q_len):
+        # the two entry points compute the same scores (the contraction and the epilogue are shared)
+        np.testing.assert_allclose(got4[i, :n], got1[i, :n], rtol=1e-6, atol=1e-6 * np.abs(got1[i, :n]).max())
+
+
+def test_prefill_indexer_flags_groups_that_mix_sequences(lib):
+    # rows 0-2 belong to sequence 0 and rows 3-7 to sequence 1: the group of rows 0-3 mixes two
+    # sequences (skipped and flagged), the group of rows 4-7 is computed
+    lens = [300, 301, 302, 200, 201, 202, 203, 204]
+    inp = inputs.make_decode_inputs("mixed", lens, T_max=384, seed=23)
+    q_seq = torch.tensor([0, 0, 0, 1, 1, 1, 1, 1], dtype=torch.int32)
+    inp.q_seq = q_seq
+    g = inp.to("cuda")
+    dims = api.dims_of(g)
+    ws = api.make_workspace(dims, _lib.DSA_OP_INDEXER)
+    sc = torch.full((len(lens), dims.ld_scores), float("nan"), dtype=torch.float32, device="cuda")
+    api.prefill_indexer_scores(dims, g.q_I, g.q_scale, g.w, g.k_I, g.k_scale, g.q_seq, g.q_len, sc, ws)
+    torch.cuda.synchronize()
+    assert api.get_device_status(ws) == _lib.DSA_ERR_INVALID_ARG
+    rows = [4, 5, 6, 7]
+    sc_o = oracle_scores_of_rows(inp, rows)
+    check_scores(np_scores(sc)[rows][:, :sc_o.shape[1]], sc_o, np.array(lens)[rows])
+    assert torch.isnan(sc[:4]).all(), "the mixed group must be left untouched"
+
+
 # ------------------------------------------------------------------ device-side error reporting
 
 def test_out_of_range_index_is_reported_and_masked(lib):
