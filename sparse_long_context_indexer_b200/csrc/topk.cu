@@ -16,9 +16,10 @@
 //     bins, so fixed digits would need several full passes).  CTA r of the
 //     cluster sums one range of bins over all CTAs (distributed shared
 //     memory); the owner of the threshold bin b* broadcasts it.
-//  2. The keys of bin b* are collected (usually a few dozen); CTA 0 gathers
-//     them from the cluster and finds tau among them with a radix select over
-//     four 8-bit digits.  If bin b* holds more than kCandMax keys (extremely
+//  2. The keys of bin b* are collected (usually a few dozen); every CTA
+//     gathers all of them from the cluster and finds tau itself, refining with
+//     2048-bin histograms of the bits below the bin's base (at most two
+//     levels).  If bin b* holds more than kCandMax keys (extremely
 //     concentrated scores) the kernel falls back to a radix select over four
 //     8-bit digits of all keys (warp-private histograms with match_any
 //     aggregation, merged across the cluster).  Rows whose keys are all equal
