@@ -147,6 +147,14 @@ __device__ __forceinline__ float4 ld_shared_cluster_v4_f32(uint32_t addr) {
                  : "memory");
     return v;
 }
+__device__ __forceinline__ uint4 ld_shared_cluster_v4_u32(uint32_t addr) {
+    uint4 v;
+    asm volatile("ld.shared::cluster.v4.u32 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+                 : "r"(addr)
+                 : "memory");
+    return v;
+}
 // Full cluster barrier (every thread of every CTA): shared-memory writes before
 // it are visible to the other CTAs' reads after it.
 __device__ __forceinline__ void cluster_sync_all() {

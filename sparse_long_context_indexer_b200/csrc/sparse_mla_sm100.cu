@@ -471,16 +471,23 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             const int col = c0 + 32 * hh;  // first output column of this piece
             if (kOut == kOutCluster) {
-                // fp32 rows for the peers: row h at h * 2048 bytes, 16-byte granule j at
-                // (j & ~7) | ((j ^ h) & 7)
-                const uint32_t row_addr = sKv + prow * (kDV * 4);
-                const int jb = col >> 2;  // a multiple of 8
+                // bf16 rows for the peers (half the bytes over the cluster network; the merge
+                // weights and sums stay fp32): row h at h * 1024 bytes, 16-byte granule j (eight
+                // values) at (j & ~7) | ((j ^ h) & 7)
+                const uint32_t row_addr = sKv + prow * (kDV * 2);
+                const int jb = col >> 3;  // a multiple of 4
 #pragma unroll
-                for (int g = 0; g < 8; ++g)
-                    asm volatile("st.shared.v4.f32 [%0], {%1, %2, %3, %4};" ::"r"(row_addr + ((jb | (g ^ (prow & 7))) << 4)),
-                                 "f"(__uint_as_float(ov[4 * g]) * inv_l), "f"(__uint_as_float(ov[4 * g + 1]) * inv_l),
-                                 "f"(__uint_as_float(ov[4 * g + 2]) * inv_l), "f"(__uint_as_float(ov[4 * g + 3]) * inv_l)
+                for (int q4 = 0; q4 < 4; ++q4) {
+                    uint32_t w[4];
+#pragma unroll
+                    for (int e = 0; e < 4; ++e)
+                        w[e] = pack_bf16x2(__uint_as_float(ov[8 * q4 + 2 * e]) * inv_l,
+                                           __uint_as_float(ov[8 * q4 + 2 * e + 1]) * inv_l);
+                    const int j = jb + q4;
+                    asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(row_addr + (((j & ~7) | ((j ^ prow) & 7)) << 4)),
+                                 "r"(w[0]), "r"(w[1]), "r"(w[2]), "r"(w[3])
                                  : "memory");
+                }
             } else if (kOut == kOutFinal) {
                 // bf16 TMA-store boxes of 64 heads x 64 columns: box k holds columns [64k, 64k + 64)
                 const uint32_t box = sKv + prow * 128 + (col >> 6) * kChunkBytes;
@@ -532,23 +539,26 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int hp = (kCtaHeads + S - 1) / S;
         const int h0 = rank * hp;
         const int nunits = 2 * max(0, min(kCtaHeads, h0 + hp) - h0);  // (head, half row) units
-        // every unit: lane j owns granules {j, j + 32} of its half row, i.e. two 16-byte pieces
-        // from each split, all loaded before any is used (the reads cross the cluster network)
+        // every unit: lane j owns granule j of its half row (eight bf16 values) from each
+        // split, all loaded before any is used (the reads cross the cluster network)
         for (int u = warp; u < nunits; u += kThreads / 32) {
             const int h = h0 + (u >> 1);
-            const int jh = (u & 1) * 64;  // first granule of the half row
+            const int jh = (u & 1) * 32;  // first granule of the half row
             const float ls = lane < S ? ld_shared_cluster_f32(mapa_shared(sP + h * 4, lane)) : -CUDART_INF_F;
             float x[kMlaClusterMaxSplits][8];
-            const uint32_t g0 = ((jh + lane) & ~7) | (((jh + lane) ^ h) & 7);
-            const uint32_t g1 = ((jh + lane + 32) & ~7) | (((jh + lane + 32) ^ h) & 7);
+            const int j = jh + lane;
+            const uint32_t g0 = (j & ~7) | ((j ^ h) & 7);
 #pragma unroll
             for (int sp = 0; sp < kMlaClusterMaxSplits; ++sp) {
                 if (sp < S) {
-                    const uint32_t rbase = mapa_shared(sKv + h * (kDV * 4), (uint32_t)sp);
-                    const float4 v0 = ld_shared_cluster_v4_f32(rbase + (g0 << 4));
-                    const float4 v1 = ld_shared_cluster_v4_f32(rbase + (g1 << 4));
-                    x[sp][0] = v0.x; x[sp][1] = v0.y; x[sp][2] = v0.z; x[sp][3] = v0.w;
-                    x[sp][4] = v1.x; x[sp][5] = v1.y; x[sp][6] = v1.z; x[sp][7] = v1.w;
+                    const uint32_t rbase = mapa_shared(sKv + h * (kDV * 2), (uint32_t)sp);
+                    const uint4 v = ld_shared_cluster_v4_u32(rbase + (g0 << 4));
+                    const uint32_t vw[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        x[sp][2 * e] = __uint_as_float(vw[e] << 16);
+                        x[sp][2 * e + 1] = __uint_as_float(vw[e] & 0xFFFF0000u);
+                    }
                 }
             }
             float L = ls;
@@ -569,9 +579,9 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             const float inv = esum > 0.f ? 1.f / esum : 0.f;
             const int64_t trow = (int64_t)t * kMlaHeads + half * kCtaHeads + h;
-            uint2* o = reinterpret_cast<uint2*>(reinterpret_cast<__nv_bfloat16*>(a.out) + trow * kDV);
-            o[jh + lane] = make_uint2(pack_bf16x2(acc[0] * inv, acc[1] * inv), pack_bf16x2(acc[2] * inv, acc[3] * inv));
-            o[jh + lane + 32] = make_uint2(pack_bf16x2(acc[4] * inv, acc[5] * inv), pack_bf16x2(acc[6] * inv, acc[7] * inv));
+            uint4* o = reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(a.out) + trow * kDV);
+            o[j] = make_uint4(pack_bf16x2(acc[0] * inv, acc[1] * inv), pack_bf16x2(acc[2] * inv, acc[3] * inv),
+                              pack_bf16x2(acc[4] * inv, acc[5] * inv), pack_bf16x2(acc[6] * inv, acc[7] * inv));
             if (lane == 0 && (u & 1) == 0 && a.lse) a.lse[trow] = esum > 0.f ? L + __logf(esum) : -CUDART_INF_F;
         }
         // peers keep reading this CTA's rows until every CTA of the cluster is done

@@ -52,7 +52,8 @@ constexpr int kOffScan = kOffMisc + 64;              // vector-scan scratch
 constexpr int kScanWords = kWarps * kRounds + kRounds + 16;
 constexpr int kFineBits = 11;
 constexpr int kFineBins = 1 << kFineBits;  // adaptive histogram bins
-constexpr int kCandMax = 2048;             // threshold-bin keys resolved on chip by CTA 0
+constexpr int kCandMax = 2048;             // threshold-bin keys resolved on chip by every CTA
+constexpr int kRankMax = 64;               // up to this many, tau is found by direct ranking
 // Keep a CTA small enough for two per SM at the long-decode chunk (16K keys): with one per
 // SM, 16 clusters of 8 no longer fit the GPCs in one wave.
 constexpr int kOffFine = (kOffScan + kScanWords + 3) & ~3;  // kFineBins counts (read remotely)
@@ -364,15 +365,48 @@ __global__ void __launch_bounds__(kThreads, 2) topk_radix_kernel(const TopkArgs 
             __syncthreads();
             cluster.sync();
             uint32_t* gbuf = sm + kOffGather;
+            // every CTA's candidate count in one round of remote reads, then all copies at once
+            int cnt_r[8], off_r[8];
             int off = 0;
-            for (int r = 0; r < C; ++r) {
-                const int cnt = cluster.map_shared_rank(misc, r)[13];
-                const uint32_t* rc = cluster.map_shared_rank(cand, r);
-                for (int i = tid; i < cnt; i += kThreads) gbuf[off + i] = rc[i];
-                off += cnt;
+#pragma unroll
+            for (int r = 0; r < 8; ++r) cnt_r[r] = r < C ? cluster.map_shared_rank(misc, r)[13] : 0;
+#pragma unroll
+            for (int r = 0; r < 8; ++r) {
+                off_r[r] = off;
+                off += cnt_r[r];
+            }
+            for (int i = tid; i < off; i += kThreads) {
+                int r = 0, base = 0;
+#pragma unroll
+                for (int q = 1; q < 8; ++q) {
+                    if (q < C && i >= off_r[q]) {
+                        r = q;
+                        base = off_r[q];
+                    }
+                }
+                gbuf[i] = cluster.map_shared_rank(cand, r)[i - base];
             }
             __syncthreads();
-            {
+            if (off <= kRankMax) {
+                // a few candidates: tau is the candidate c with #{> c} < rem <= #{>= c}, found by
+                // ranking every candidate against all others (quadratic, so only for small sets)
+                const int rem = a.k - above_total;
+                if (tid < off) {
+                    const uint32_t c = gbuf[tid];
+                    int gt = 0, ge = 0;
+                    for (int j = 0; j < off; ++j) {
+                        const uint32_t o = gbuf[j];
+                        gt += o > c;
+                        ge += o >= c;
+                    }
+                    if (gt < rem && rem <= ge) {
+                        // every thread holding a copy of tau writes the same values
+                        misc[11] = (int)c;
+                        misc[12] = rem - gt;  // candidates equal to tau that are taken
+                    }
+                }
+                __syncthreads();
+            } else {
                 // tau among the candidates (keys in [base, base + 2^shift)): refine by 2048-bin
                 // histograms of the bits below the bin base, at most two levels for shift <= 22;
                 // this CTA's own fine histogram is free now (peers read it only before the range merge)
