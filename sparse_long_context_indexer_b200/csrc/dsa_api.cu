@@ -94,7 +94,7 @@ int plan_topk_cluster(const dsa_dims* d, int nq) {
     const int fill = nq > 0 ? sms / nq : 8;
     if (fill > c) c = fill;
     if (c < 1) c = 1;
-    if (c > 8) c = 8;
+    if (c > dsa::kTopkMaxCluster) c = dsa::kTopkMaxCluster;
     return c;
 }
 

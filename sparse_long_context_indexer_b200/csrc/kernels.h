@@ -83,6 +83,9 @@ cudaError_t static_mla_scratch(void** ptr);
 
 // Largest row chunk kept in shared memory by one top-k CTA (elements).
 constexpr int kTopkSmemKeys = 45056;
+// Most CTAs (one thread-block cluster, the portable size) sharing one top-k row; 16-CTA
+// clusters were measured slower on the long decode (44 vs 32 us).
+constexpr int kTopkMaxCluster = 8;
 
 // cuTensorMapEncodeTiled through the runtime's driver entry point (no -lcuda).
 bool encode_tensor_map_2d(void* map, int dtype_bytes, const void* base, uint64_t inner, uint64_t outer,

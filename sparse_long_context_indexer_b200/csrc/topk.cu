@@ -40,6 +40,7 @@ namespace dsa {
 namespace {
 
 constexpr int kThreads = 512;
+constexpr int kMaxCluster = kTopkMaxCluster;
 constexpr int kWarps = kThreads / 32;
 constexpr int kBins = 256;
 constexpr int kRounds = 8;  // compaction: a thread owns 4 consecutive keys in each of kRounds rounds
@@ -242,15 +243,27 @@ __global__ void __launch_bounds__(kThreads, 2) topk_radix_kernel(const TopkArgs 
         return r;
     };
     cluster.sync();
-    uint32_t kmin = 0xFFFFFFFFu, kmax = 0u;
+    // the row's key range: lane r of warp 0 reads CTA r's min and max (one remote read each,
+    // instead of every thread reading every rank), shared through this CTA's memory
+    if (warp == 0) {
+        uint32_t mn = 0xFFFFFFFFu, mx = 0u;
+        if (lane < C) {
+            const int* rm = cluster.map_shared_rank(misc, lane);
+            mn = (uint32_t)rm[4];
+            mx = (uint32_t)rm[5];
+        }
 #pragma unroll
-    for (int r = 0; r < 8; ++r) {
-        if (r < C) {
-            const int* rm = cluster.map_shared_rank(misc, r);
-            kmin = min(kmin, (uint32_t)rm[4]);
-            kmax = max(kmax, (uint32_t)rm[5]);
+        for (int o = 16; o > 0; o >>= 1) {
+            mn = min(mn, __shfl_xor_sync(0xffffffffu, mn, o));
+            mx = max(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+        }
+        if (lane == 0) {
+            misc[22] = (int)mn;
+            misc[23] = (int)mx;
         }
     }
+    __syncthreads();
+    const uint32_t kmin = (uint32_t)misc[22], kmax = (uint32_t)misc[23];
 
     uint32_t tau;
     int take_eq_total;  // keys equal to tau that are selected, lowest positions first
@@ -284,10 +297,9 @@ __global__ void __launch_bounds__(kThreads, 2) topk_radix_kernel(const TopkArgs 
         const int b_lo = min(kFineBins, rank * per), b_hi = min(kFineBins, b_lo + per);
         int part = 0;
         for (int bb = b_lo + tid; bb < b_hi; bb += kThreads) {
-            uint32_t v[8];
+            uint32_t tot_b = 0u;
 #pragma unroll
-            for (int r = 0; r < 8; ++r) v[r] = r < C ? cluster.map_shared_rank(fine, r)[bb] : 0u;
-            const uint32_t tot_b = ((v[0] + v[1]) + (v[2] + v[3])) + ((v[4] + v[5]) + (v[6] + v[7]));
+            for (int r = 0; r < kMaxCluster; ++r) tot_b += r < C ? cluster.map_shared_rank(fine, r)[bb] : 0u;
             rng[bb - b_lo] = tot_b;
             part += (int)tot_b;
         }
@@ -298,25 +310,28 @@ __global__ void __launch_bounds__(kThreads, 2) topk_radix_kernel(const TopkArgs 
         cluster.sync();
         // every CTA finds b* itself: the range holding the k-th largest key (ranges of higher
         // ranks hold larger keys), then that range's bins read from its owner, top down
-        int above_r = 0, owner = 0;
-        {
-            int rs[8];
+        if (warp == 0) {
+            // lane r reads CTA r's range total; keys above range r = the totals of the ranges
+            // above it (a suffix sum); the owner's range holds the k-th largest key
+            const int rs = lane < C ? cluster.map_shared_rank(misc, lane)[6] : 0;
+            int suf = rs;  // inclusive suffix sum over lanes >= this one
 #pragma unroll
-            for (int r = 0; r < 8; ++r) rs[r] = r < C ? cluster.map_shared_rank(misc, r)[6] : 0;
-            int acc = 0;
-            bool found = false;
-#pragma unroll
-            for (int r = 7; r >= 0; --r) {
-                if (r < C && !found) {
-                    if (acc < a.k && a.k <= acc + rs[r]) {
-                        owner = r;
-                        above_r = acc;
-                        found = true;
-                    }
-                    acc += rs[r];
-                }
+            for (int o = 1; o < 32; o <<= 1) {
+                const int u = __shfl_down_sync(0xffffffffu, suf, o);
+                if (lane + o < 32) suf += u;
+            }
+            const int above = suf - rs;
+            const bool own = lane < C && above < a.k && a.k <= suf;
+            const unsigned m = __ballot_sync(0xffffffffu, own);
+            const int ow = m ? __ffs(m) - 1 : 0;
+            const int above_ow = __shfl_sync(0xffffffffu, above, ow);
+            if (lane == 0) {
+                misc[24] = ow;
+                misc[25] = above_ow;
             }
         }
+        __syncthreads();
+        const int owner = misc[24], above_r = misc[25];
         {
             const int o_lo = min(kFineBins, owner * per), o_hi = min(kFineBins, o_lo + per);
             const uint32_t* orng = cluster.map_shared_rank(rng, owner);
@@ -365,23 +380,29 @@ __global__ void __launch_bounds__(kThreads, 2) topk_radix_kernel(const TopkArgs 
             __syncthreads();
             cluster.sync();
             uint32_t* gbuf = sm + kOffGather;
-            // every CTA's candidate count in one round of remote reads, then all copies at once
-            int cnt_r[8], off_r[8];
-            int off = 0;
+            // every CTA's candidate count (lane r of warp 0 reads CTA r's) and their offsets in
+            // the gathered list, then all copies at once
+            if (warp == 0) {
+                const int c = lane < C ? cluster.map_shared_rank(misc, lane)[13] : 0;
+                int incl = c;
 #pragma unroll
-            for (int r = 0; r < 8; ++r) cnt_r[r] = r < C ? cluster.map_shared_rank(misc, r)[13] : 0;
-#pragma unroll
-            for (int r = 0; r < 8; ++r) {
-                off_r[r] = off;
-                off += cnt_r[r];
+                for (int o = 1; o < 32; o <<= 1) {
+                    const int u = __shfl_up_sync(0xffffffffu, incl, o);
+                    if (lane >= o) incl += u;
+                }
+                if (lane < kMaxCluster) misc[26 + lane] = incl - c;
+                if (lane == 31) misc[26 + kMaxCluster] = incl;
             }
+            __syncthreads();
+            const int off = misc[26 + kMaxCluster];
             for (int i = tid; i < off; i += kThreads) {
                 int r = 0, base = 0;
 #pragma unroll
-                for (int q = 1; q < 8; ++q) {
-                    if (q < C && i >= off_r[q]) {
+                for (int q = 1; q < kMaxCluster; ++q) {
+                    const int oq = misc[26 + q];
+                    if (q < C && i >= oq) {
                         r = q;
-                        base = off_r[q];
+                        base = oq;
                     }
                 }
                 gbuf[i] = cluster.map_shared_rank(cand, r)[i - base];
@@ -504,10 +525,10 @@ __global__ void __launch_bounds__(kThreads, 2) topk_radix_kernel(const TopkArgs 
                 }
                 cluster.sync();
                 if (tid < kBins) {
-                    uint32_t v[8];
+                    uint32_t sum_r = 0u;
 #pragma unroll
-                    for (int r = 0; r < 8; ++r) v[r] = r < C ? cluster.map_shared_rank(hist, r)[tid] : 0u;
-                    tot[tid] = ((v[0] + v[1]) + (v[2] + v[3])) + ((v[4] + v[5]) + (v[6] + v[7]));
+                    for (int r = 0; r < kMaxCluster; ++r) sum_r += r < C ? cluster.map_shared_rank(hist, r)[tid] : 0u;
+                    tot[tid] = sum_r;
                 }
                 __syncthreads();
                 // digit holding the remaining-th largest key: scan from the top digit down
@@ -542,23 +563,32 @@ __global__ void __launch_bounds__(kThreads, 2) topk_radix_kernel(const TopkArgs 
     }
     cluster.sync();
     int eq_before = 0, out_before = 0;
-    {
-        int rg[8], re[8];
-#pragma unroll
-        for (int r = 0; r < 8; ++r) {
-            const int* rm = cluster.map_shared_rank(misc, r < rank ? r : rank);
-            rg[r] = rm[2];
-            re[r] = rm[3];
+    if (warp == 0) {
+        // lane r < rank reads CTA r's counts; ties are taken lowest rank first
+        int g = 0, e = 0;
+        if (lane < rank) {
+            const int* rm = cluster.map_shared_rank(misc, lane);
+            g = rm[2];
+            e = rm[3];
         }
+        int e_incl = e;
 #pragma unroll
-        for (int r = 0; r < 8; ++r) {
-            if (r < rank) {
-                const int te = max(0, min(take_eq_total - eq_before, re[r]));
-                out_before += rg[r] + te;
-                eq_before += re[r];
-            }
+        for (int o = 1; o < 32; o <<= 1) {
+            const int u = __shfl_up_sync(0xffffffffu, e_incl, o);
+            if (lane >= o) e_incl += u;
+        }
+        const int te = max(0, min(take_eq_total - (e_incl - e), e));
+        int ob = g + te;
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) ob += __shfl_xor_sync(0xffffffffu, ob, o);
+        if (lane == 31) {
+            misc[20] = ob;
+            misc[21] = e_incl;  // the ties of all lower ranks
         }
     }
+    __syncthreads();
+    out_before = misc[20];
+    eq_before = misc[21];
     const int take_eq_local = max(0, min(take_eq_total - eq_before, local_eq));
     const bool all_ties = take_eq_local == local_eq;  // selection is then a plain threshold
     const uint64_t thr = take_eq_local > 0 ? (uint64_t)tau : (uint64_t)tau + 1u;
@@ -646,7 +676,7 @@ __global__ void __launch_bounds__(kThreads, 2) topk_radix_kernel(const TopkArgs 
 
 cudaError_t launch_topk(const TopkArgs& a, int cluster, cudaStream_t st) {
     if (a.Nq == 0) return cudaSuccess;
-    if (cluster < 1 || cluster > 8) return cudaErrorInvalidValue;
+    if (cluster < 1 || cluster > kMaxCluster) return cudaErrorInvalidValue;
     const int64_t row_max = a.ld < (int64_t)a.T_max ? a.ld : (int64_t)a.T_max;
     int64_t chunk = (row_max + cluster - 1) / cluster;
     chunk = (chunk + 3) & ~int64_t(3);
