@@ -74,7 +74,8 @@ typedef enum {
     DSA_OP_TOPK = 1,
     DSA_OP_SPARSE_MLA = 2,
     DSA_OP_DECODE = 3,
-    DSA_OP_PREFILL = 4
+    DSA_OP_PREFILL = 4,
+    DSA_OP_DENSE_MLA = 5
 } dsa_op_t;
 
 /* Problem sizes.  Supported builds:
@@ -164,6 +165,19 @@ dsa_status_t dsa_sparse_mla_attn(const dsa_dims* dims, const void* q, const void
                                  const int32_t* idx, const int32_t* q_seq, const int32_t* q_len,
                                  float softmax_scale, void* out, float* lse,
                                  void* workspace, size_t ws_bytes, void* stream);
+
+/* Dense MLA in MQA mode, the comparison the pages measure DSA against
+ * (kgptalkie "How Much Does DSA Save?": dense attention over every cached
+ * token vs the indexer plus attention over 2,048; kiadev "Efficiency,
+ * benchmarks and operational signals": decode cost at 128K).  Same formula and
+ * outputs as dsa_sparse_mla_attn with the selection replaced by every position
+ * s < q_len[t]: out[t,h,:] = sum_{s < q_len[t]} softmax_s(...) kv[b,s,0:512].
+ * The same kernel runs with each split walking a contiguous block of
+ * positions instead of an index list; dims->k is ignored (the plan uses T_max).
+ * kv_dtype DSA_BF16 only.  Workspace sized for DSA_OP_DENSE_MLA. */
+dsa_status_t dsa_dense_mla_attn(const dsa_dims* dims, const void* q, const void* kv,
+                                const int32_t* q_seq, const int32_t* q_len, float softmax_scale,
+                                void* out, float* lse, void* workspace, size_t ws_bytes, void* stream);
 
 /* Stage 3 for callers that cannot allocate device memory.  No counterpart in
  * the paper: it exists for callers embedded in a host that owns all device

@@ -16,12 +16,12 @@ LIB_PATH = os.path.join(HERE, "libdsa_b200.so")
 DSA_OK, DSA_ERR_INVALID_ARG, DSA_ERR_UNSUPPORTED, DSA_ERR_WORKSPACE, DSA_ERR_CUDA, DSA_ERR_TIMEOUT, \
     DSA_ERR_INDEX_OOB, DSA_ERR_LENGTH = range(8)
 DSA_F32, DSA_BF16, DSA_FP8_E4M3 = 0, 1, 2
-DSA_OP_INDEXER, DSA_OP_TOPK, DSA_OP_SPARSE_MLA, DSA_OP_DECODE, DSA_OP_PREFILL = range(5)
+DSA_OP_INDEXER, DSA_OP_TOPK, DSA_OP_SPARSE_MLA, DSA_OP_DECODE, DSA_OP_PREFILL, DSA_OP_DENSE_MLA = range(6)
 
 # every symbol include/dsa.h declares
 EXPORTS = (
     "dsa_workspace_size", "dsa_workspace_init", "dsa_indexer_scores", "dsa_prefill_indexer_scores", "dsa_topk",
-    "dsa_sparse_mla_attn",
+    "dsa_sparse_mla_attn", "dsa_dense_mla_attn",
     "dsa_decode_step", "dsa_prefill", "dsa_get_device_status", "dsa_status_string", "dsa_last_cuda_error",
     "dsa_selftest_wait_timeout", "dsa_version", "dsa_sparse_mla_attn_noalloc",
 )
@@ -67,6 +67,7 @@ def _declare(lib):
     lib.dsa_topk.argtypes = [D, P, P, P, P, S, P]
     lib.dsa_sparse_mla_attn.argtypes = [D, P, P, P, P, P, F, P, P, P, S, P]
     lib.dsa_sparse_mla_attn_noalloc.argtypes = [D, P, P, P, P, P, F, P, P, P]
+    lib.dsa_dense_mla_attn.argtypes = [D, P, P, P, P, F, P, P, P, S, P]
     lib.dsa_decode_step.argtypes = [D, P, P, P, P, P, P, P, P, P, F, P, P, P, P, P, S, P,
                                     ctypes.POINTER(DsaStageEvents)]
     lib.dsa_prefill.argtypes = [D, P, P, P, P, P, P, P, P, P, F, P, P, P, P, S, P]
@@ -75,7 +76,7 @@ def _declare(lib):
     for name in ("dsa_workspace_size", "dsa_workspace_init", "dsa_indexer_scores", "dsa_prefill_indexer_scores",
                  "dsa_topk",
                  "dsa_sparse_mla_attn", "dsa_decode_step", "dsa_prefill", "dsa_get_device_status",
-                 "dsa_selftest_wait_timeout", "dsa_sparse_mla_attn_noalloc"):
+                 "dsa_selftest_wait_timeout", "dsa_sparse_mla_attn_noalloc", "dsa_dense_mla_attn"):
         getattr(lib, name).restype = st
     lib.dsa_status_string.argtypes = [I32]
     lib.dsa_status_string.restype = ctypes.c_char_p

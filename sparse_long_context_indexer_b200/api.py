@@ -116,6 +116,17 @@ def topk(dims: Dims, scores, q_len, idx, ws=None):
     return idx
 
 
+def dense_mla_attn(dims: Dims, q, kv, q_seq, q_len, softmax_scale, out, lse, ws):
+    """Attention over every position s < q_len[t] (the dense comparison of the sparse path)."""
+    lib = _lib.load()
+    d = dims.c()
+    rc = lib.dsa_dense_mla_attn(ctypes.byref(d), _ptr(q), _ptr(kv), _ptr(q_seq), _ptr(q_len),
+                                ctypes.c_float(softmax_scale), _ptr(out), _ptr(lse), _ptr(ws), ws.numel(),
+                                _stream_ptr())
+    _lib.check(lib, rc, "dsa_dense_mla_attn")
+    return out
+
+
 def sparse_mla_attn(dims: Dims, q, kv, idx, q_seq, q_len, softmax_scale, out, lse, ws):
     lib = _lib.load()
     d = dims.c()

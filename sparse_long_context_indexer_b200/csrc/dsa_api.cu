@@ -119,10 +119,21 @@ void add_mla_partials(Layout& L, const dsa_dims* d, int nq, const MlaPlan& p) {
     }
 }
 
+// Dense attention plans its splits over every cached position: the selection length k is
+// T_max (rounded up to whole 64-row tiles).
+dsa_dims dense_dims(const dsa_dims* d) {
+    dsa_dims e = *d;
+    e.k = (d->T_max + dsa::kMlaTile - 1) / dsa::kMlaTile * dsa::kMlaTile;
+    return e;
+}
+
 Layout layout_for(const dsa_dims* d, int op) {
     Layout L;
     if (op == DSA_OP_SPARSE_MLA) {
         add_mla_partials(L, d, d->Nq, plan_mla(d, d->Nq));
+    } else if (op == DSA_OP_DENSE_MLA) {
+        const dsa_dims e = dense_dims(d);
+        add_mla_partials(L, &e, d->Nq, plan_mla(&e, d->Nq));
     } else if (op == DSA_OP_DECODE || op == DSA_OP_PREFILL) {
         const int rows = op == DSA_OP_PREFILL ? plan_prefill_chunk(d) : d->Nq;
         L.scores = L.total;
@@ -240,9 +251,9 @@ const char* dsa_status_string(int32_t s) {
 }
 
 dsa_status_t dsa_workspace_size(const dsa_dims* dims, int32_t op, size_t* bytes) {
-    if (bytes == nullptr || op < DSA_OP_INDEXER || op > DSA_OP_PREFILL) return DSA_ERR_INVALID_ARG;
+    if (bytes == nullptr || op < DSA_OP_INDEXER || op > DSA_OP_DENSE_MLA) return DSA_ERR_INVALID_ARG;
     const bool idx = op == DSA_OP_INDEXER || op == DSA_OP_DECODE || op == DSA_OP_PREFILL;
-    const bool mla = op == DSA_OP_SPARSE_MLA || op == DSA_OP_DECODE || op == DSA_OP_PREFILL;
+    const bool mla = op == DSA_OP_SPARSE_MLA || op == DSA_OP_DENSE_MLA || op == DSA_OP_DECODE || op == DSA_OP_PREFILL;
     dsa_status_t s = check_dims(dims, idx, mla, op == DSA_OP_PREFILL);
     if (s != DSA_OK) return s;
     *bytes = layout_for(dims, op).total;
@@ -310,6 +321,23 @@ dsa_status_t dsa_sparse_mla_attn(const dsa_dims* dims, const void* q, const void
     const Layout L = layout_for(dims, DSA_OP_SPARSE_MLA);
     if (workspace == nullptr || ws_bytes < L.total) return DSA_ERR_WORKSPACE;
     return run_mla(dims, dims->Nq, q, kv, idx, q_seq, q_len, softmax_scale, out, lse, workspace, L, nullptr,
+                   reinterpret_cast<cudaStream_t>(stream));
+}
+
+dsa_status_t dsa_dense_mla_attn(const dsa_dims* dims, const void* q, const void* kv, const int32_t* q_seq,
+                                const int32_t* q_len, float softmax_scale, void* out, float* lse, void* workspace,
+                                size_t ws_bytes, void* stream) {
+    dsa_status_t s = check_dims(dims, false, true);
+    if (s != DSA_OK) return s;
+    if (dims->kv_dtype != DSA_BF16) return DSA_ERR_UNSUPPORTED;
+    if (dims->Nq == 0) return DSA_OK;
+    if (!q || !kv || !q_seq || !q_len || !out || !std::isfinite(softmax_scale)) return DSA_ERR_INVALID_ARG;
+    if (!aligned16(q) || !aligned16(kv) || !aligned16(out)) return DSA_ERR_INVALID_ARG;
+    const Layout L = layout_for(dims, DSA_OP_DENSE_MLA);
+    if (workspace == nullptr || ws_bytes < L.total) return DSA_ERR_WORKSPACE;
+    const dsa_dims e = dense_dims(dims);
+    // no index list: the attention kernel takes entry j of a row as position j, j < q_len[t]
+    return run_mla(&e, dims->Nq, q, kv, nullptr, q_seq, q_len, softmax_scale, out, lse, workspace, L, nullptr,
                    reinterpret_cast<cudaStream_t>(stream));
 }
 

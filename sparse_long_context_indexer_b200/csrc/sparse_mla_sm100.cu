@@ -132,11 +132,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int split = blockIdx.x, half = blockIdx.y, t = blockIdx.z;
 
-    // rows of idx handled by this split
-    const int j_lo = split * a.rows_per_split;
-    const int j_hi = min(a.k, j_lo + a.rows_per_split);
-    const int nrows = max(0, j_hi - j_lo);
-    const int ntiles = (nrows + kTileRows - 1) / kTileRows;
     int n_t = a.q_len[t];
     const int b = a.q_seq[t];
     const bool row_ok = n_t >= 0 && n_t <= a.T_max && b >= 0 && b < a.B;
@@ -144,12 +139,20 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (split == 0 && half == 0 && tid == 0) record_status(a.status, DSA_STATUS_LENGTH);
         n_t = 0;
     }
-    const int32_t* idx_row = a.idx + (int64_t)t * a.k;
+    // Entries j of the row's selection handled by this split.  Dense mode (no index list):
+    // entry j is position j itself and the row has n_t entries, so attention runs over every
+    // position s < q_len[t].
+    const bool dense = a.idx == nullptr;
+    const int j_lo = split * a.rows_per_split;
+    const int j_hi = min(dense ? min(a.k, n_t) : a.k, j_lo + a.rows_per_split);
+    const int nrows = max(0, j_hi - j_lo);
+    const int ntiles = (nrows + kTileRows - 1) / kTileRows;
+    const int32_t* idx_row = dense ? nullptr : a.idx + (int64_t)t * a.k;
     const __nv_bfloat16* kv_seq = reinterpret_cast<const __nv_bfloat16*>(a.kv) + (int64_t)b * a.T_max * kDK;
-    // position r of tile i -> selected token, -1 past the end of the split
+    // entry r of tile i -> selected token, -1 past the end of the split
     auto load_pos = [&](int i, int r) -> int {
         const int j = j_lo + i * kTileRows + r;
-        return j < j_hi ? __ldg(idx_row + j) : -1;
+        return j < j_hi ? (dense ? j : __ldg(idx_row + j)) : -1;
     };
     auto valid = [&](int s) { return s >= 0 && s < n_t; };
 

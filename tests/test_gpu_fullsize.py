@@ -152,3 +152,23 @@ def test_prefill_64k_full_size(lib):
             check_sets(g_idx[i:i + 1], o_sel, sc_o[None], [n], g.k)
         o_out, o_lse = oracle_attention_on(g, t, g_idx[i])
         check_attention(g_out[i:i + 1], o_out[None], g_lse[i:i + 1], o_lse[None])
+
+
+def test_dense_attention_long_decode_sampled_rows(lib):
+    # dense attention over all 131,072 cached tokens of the long decode, launched as bench.py's
+    # dense line does; the oracle redoes two rows whole
+    g = inputs.long_decode(device="cuda")
+    dims = api.dims_of(g)
+    ws = api.make_workspace(dims, _lib.DSA_OP_DENSE_MLA)
+    out, lse = api.alloc_outputs(g)
+    api.dense_mla_attn(dims, g.q, g.kv, g.q_seq, g.q_len, g.softmax_scale, out, lse, ws)
+    torch.cuda.synchronize()
+    assert api.get_device_status(ws) == 0
+    for t in (0, 9):
+        n = int(g.q_len[t])
+        b = int(g.q_seq[t])
+        sub = SimpleNamespace(q=g.q[t:t + 1].cpu(), kv=g.kv[b:b + 1, :n].cpu(), q_seq=np.zeros(1, np.int32),
+                              q_len=np.array([n], np.int32), H=g.H, T_max=n, B=1, kv_dtype=g.kv_dtype,
+                              softmax_scale=g.softmax_scale)
+        o_out, o_lse = oracle.dense_attn(sub)
+        check_attention(out[t:t + 1].float().cpu().numpy(), o_out, lse[t:t + 1].cpu().numpy(), o_lse)

@@ -274,6 +274,41 @@ def test_prefill_indexer_flags_groups_that_mix_sequences(lib):
     assert torch.isnan(sc[:4]).all(), "the mixed group must be left untouched"
 
 
+def test_dense_attention_matches_oracle(lib):
+    # every position s < q_len[t]: ragged rows spanning several splits, a one-token row
+    inp = small_decode(seed=61, lens=[4097, 2500, 777, 1, 2049, 129])
+    out_o, lse_o = oracle.dense_attn(inp)
+    g = inp.to("cuda")
+    dims = api.dims_of(g)
+    ws = api.make_workspace(dims, _lib.DSA_OP_DENSE_MLA)
+    out, lse = api.alloc_outputs(g)
+    api.dense_mla_attn(dims, g.q, g.kv, g.q_seq, g.q_len, g.softmax_scale, out, lse, ws)
+    torch.cuda.synchronize()
+    assert api.get_device_status(ws) == 0
+    check_attention(out.float().cpu().numpy(), out_o, lse.cpu().numpy(), lse_o)
+
+
+def test_dense_equals_sparse_over_every_position(lib):
+    # with a budget covering the whole row the sparse path selects every position: the two
+    # entry points then compute the same attention
+    lens = [2048, 1500, 64, 65]
+    inp = small_decode(seed=62, lens=lens)
+    g = inp.to("cuda")
+    dims = api.dims_of(g)
+    idx = torch.full((len(lens), g.k), -1, dtype=torch.int32)
+    for t, n in enumerate(lens):
+        idx[t, :n] = torch.arange(n, dtype=torch.int32)
+    ws_s = api.make_workspace(dims, _lib.DSA_OP_SPARSE_MLA)
+    ws_d = api.make_workspace(dims, _lib.DSA_OP_DENSE_MLA)
+    out_s, lse_s = api.alloc_outputs(g)
+    out_d, lse_d = api.alloc_outputs(g)
+    api.sparse_mla_attn(dims, g.q, g.kv, idx.cuda(), g.q_seq, g.q_len, g.softmax_scale, out_s, lse_s, ws_s)
+    api.dense_mla_attn(dims, g.q, g.kv, g.q_seq, g.q_len, g.softmax_scale, out_d, lse_d, ws_d)
+    torch.cuda.synchronize()
+    assert api.get_device_status(ws_s) == 0 and api.get_device_status(ws_d) == 0
+    check_attention(out_d.float().cpu().numpy(), out_s.float().cpu().numpy(), lse_d.cpu().numpy(), lse_s.cpu().numpy())
+
+
 # ------------------------------------------------------------------ device-side error reporting
 
 def test_out_of_range_index_is_reported_and_masked(lib):
