@@ -209,7 +209,11 @@ dsa_status_t dsa_sparse_mla_attn_noalloc(const dsa_dims* dims, const void* q, co
  * section 3 sketch: indexer, top-K gather, attention over the K positions).
  * scores_out / idx_out may be NULL (then the workspace holds them; size the
  * workspace for DSA_OP_DECODE); when given they receive the intermediate
- * results.  events may be NULL. */
+ * results.  Short-context dispatch: a row with q_len[t] <= k selects every
+ * position (kgptalkie, "How Does the Selector Pick 1,024?": a short prompt is
+ * read in full), so when scores_out is NULL the indexer skips such rows and
+ * the top-k writes 0 .. q_len[t]-1 without reading scores; the outputs are
+ * the same.  events may be NULL. */
 dsa_status_t dsa_decode_step(const dsa_dims* dims,
                              const void* q_I, const float* q_scale, const void* w,
                              const void* k_I, const float* k_scale,
@@ -222,7 +226,8 @@ dsa_status_t dsa_decode_step(const dsa_dims* dims,
 /* Prefill: the same three stages for many query rows of ONE sequence (every
  * position of a prompt), processed in row chunks so the transient score rows
  * fit the workspace (size it for DSA_OP_PREFILL).  Semantics per row are
- * exactly those of dsa_decode_step; q_len[t] = t + 1 for a causal prompt.
+ * exactly those of dsa_decode_step; q_len[t] = t + 1 for a causal prompt
+ * (rows t < k skip the indexer, as in dsa_decode_step).
  * The indexer serves four consecutive rows per tensor-core pass, so every
  * q_seq[t] must name the same sequence: groups of four rows that do not are
  * skipped and DSA_ERR_INVALID_ARG is recorded in the device status word.

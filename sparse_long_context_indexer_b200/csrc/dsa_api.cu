@@ -153,7 +153,8 @@ void record_event(const dsa_stage_events* ev, int i, cudaStream_t st) {
 
 dsa_status_t run_indexer(const dsa_dims* d, int nq, const void* q_I, const float* q_scale, const void* w,
                          const void* k_I, const float* k_scale, const int32_t* q_seq, const int32_t* q_len,
-                         float* scores, int* status, cudaStream_t st, bool rows_of_one_sequence = false) {
+                         float* scores, int* status, cudaStream_t st, bool rows_of_one_sequence = false,
+                         int skip_upto = 0) {
     dsa::IndexerArgs a{};
     a.q_I = q_I;
     a.q_scale = q_scale;
@@ -170,6 +171,7 @@ dsa_status_t run_indexer(const dsa_dims* d, int nq, const void* q_I, const float
     a.H_I = d->H_I;
     a.d_I = d->d_I;
     a.status = status;
+    a.skip_upto = skip_upto;
     cudaError_t e = d->idx_dtype != DSA_FP8_E4M3 ? dsa::launch_indexer_f32(a, st)
                     : rows_of_one_sequence      ? dsa::launch_indexer_fp8_units4(a, device_sms(), st)
                                                 : dsa::launch_indexer_fp8(a, device_sms(), st);
@@ -194,7 +196,7 @@ dsa_status_t run_topk(const dsa_dims* d, int nq, const float* scores, const int3
 
 dsa_status_t run_mla(const dsa_dims* d, int nq, const void* q, const void* kv, const int32_t* idx, const int32_t* q_seq,
                      const int32_t* q_len, float scale, void* out, float* lse, void* ws, const Layout& L,
-                     const dsa_stage_events* ev, cudaStream_t st, bool pdl = false) {
+                     const dsa_stage_events* ev, cudaStream_t st, bool pdl = false, bool compact_idx = false) {
     const MlaPlan p = plan_mla(d, nq);
     dsa::MlaArgs a{};
     a.q = q;
@@ -216,6 +218,7 @@ dsa_status_t run_mla(const dsa_dims* d, int nq, const void* q, const void* kv, c
     a.softmax_scale = scale;
     a.status = ws ? status_word(ws) : nullptr;
     a.pdl = pdl ? 1 : 0;
+    a.compact = compact_idx ? 1 : 0;
     cudaError_t e;
     if (d->kv_dtype == DSA_BF16) {
         e = dsa::launch_sparse_mla_bf16(a, st);
@@ -405,7 +408,10 @@ dsa_status_t dsa_decode_step(const dsa_dims* dims, const void* q_I, const float*
     float* scores = scores_out ? scores_out : reinterpret_cast<float*>(ws + L.scores);
     int32_t* idx = idx_out ? idx_out : reinterpret_cast<int32_t*>(ws + L.idx);
     record_event(events, 0, st);
-    s = run_indexer(dims, dims->Nq, q_I, q_scale, w, k_I, k_scale, q_seq, q_len, scores, status, st);
+    // rows with at most k positions select all of them: unless the caller asked for the
+    // scores, the indexer skips those rows (short-context dispatch, same results)
+    s = run_indexer(dims, dims->Nq, q_I, q_scale, w, k_I, k_scale, q_seq, q_len, scores, status, st, false,
+                    scores_out ? 0 : dims->k);
     if (s != DSA_OK) return s;
     record_event(events, 1, st);
     // top-k and attention follow their producer as programmatic dependents: their setup
@@ -413,7 +419,8 @@ dsa_status_t dsa_decode_step(const dsa_dims* dims, const void* q_I, const float*
     s = run_topk(dims, dims->Nq, scores, q_len, idx, status, st, true);
     if (s != DSA_OK) return s;
     record_event(events, 2, st);
-    s = run_mla(dims, dims->Nq, q, kv, idx, q_seq, q_len, softmax_scale, out, lse, workspace, L, events, st, true);
+    s = run_mla(dims, dims->Nq, q, kv, idx, q_seq, q_len, softmax_scale, out, lse, workspace, L, events, st, true,
+                true);
     if (s != DSA_OK) return s;
     record_event(events, 4, st);
     return DSA_OK;
@@ -451,13 +458,14 @@ dsa_status_t dsa_prefill(const dsa_dims* dims, const void* q_I, const float* q_s
         const char* qi = static_cast<const char*>(q_I) + r0 * qi_row;
         const float* qs = fp8 ? q_scale + (size_t)r0 * dims->H_I : nullptr;
         const char* wr = static_cast<const char*>(w) + r0 * w_row;
-        s = run_indexer(dims, nq, qi, qs, wr, k_I, k_scale, q_seq + r0, q_len + r0, scores, status, st, true);
+        s = run_indexer(dims, nq, qi, qs, wr, k_I, k_scale, q_seq + r0, q_len + r0, scores, status, st, true,
+                        dims->k);
         if (s != DSA_OK) return s;
         s = run_topk(dims, nq, scores, q_len + r0, idx, status, st, true);
         if (s != DSA_OK) return s;
         s = run_mla(dims, nq, static_cast<const char*>(q) + r0 * q_row, kv, idx, q_seq + r0, q_len + r0,
                     softmax_scale, static_cast<char*>(out) + r0 * o_row, lse ? lse + (size_t)r0 * dims->H : nullptr,
-                    workspace, L, nullptr, st, true);
+                    workspace, L, nullptr, st, true, true);
         if (s != DSA_OK) return s;
     }
     return DSA_OK;

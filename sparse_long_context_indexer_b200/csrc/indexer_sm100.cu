@@ -128,10 +128,12 @@ __device__ __forceinline__ int unit_len(const IndexerArgs& a, int u, int R) {
     }
     return n;
 }
+// Stages scheduled for a unit: none for an invalid unit, and none for a unit whose longest
+// row is at most skip_upto (short rows: the top-k takes every position without scores).
 __device__ __forceinline__ int unit_tiles(const IndexerArgs& a, int u, int R, int stok) {
-    if (R == 1) return row_tiles(a, u, stok);
-    const int n = unit_len(a, u, R);
-    return n < 0 ? 0 : tiles_of(a, n, a.q_seq[u * R], stok);
+    const int n = R == 1 ? a.q_len[u] : unit_len(a, u, R);
+    if (n <= a.skip_upto) return 0;
+    return R == 1 ? row_tiles(a, u, stok) : (n < 0 ? 0 : tiles_of(a, n, a.q_seq[u * R], stok));
 }
 
 // Walks the flat (unit, stage) list.  The unit's sequence and length are read

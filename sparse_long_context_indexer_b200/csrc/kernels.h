@@ -26,6 +26,10 @@ struct IndexerArgs {
     int64_t ld;
     int Nq, B, T_max, H_I, d_I;
     int* status;
+    // rows (units) whose length is at most this get no scores: inside the library's pipelines,
+    // where the scores are intermediate, the top-k selects every position of such a row
+    // without reading them (0 = score every row)
+    int skip_upto;
 };
 
 struct TopkArgs {
@@ -53,6 +57,9 @@ struct MlaArgs {
     float softmax_scale;
     int* status;
     int pdl;  // launch as a programmatic dependent of the previous kernel (the library's own pipelines)
+    // the index list is the library's own top-k output: entries past min(k, q_len[t]) are -1,
+    // so the splits stop there
+    int compact;
 };
 
 cudaError_t launch_indexer_fp8(const IndexerArgs& a, int grid, cudaStream_t st);

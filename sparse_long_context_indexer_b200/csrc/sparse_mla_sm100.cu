@@ -141,10 +141,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     // Entries j of the row's selection handled by this split.  Dense mode (no index list):
     // entry j is position j itself and the row has n_t entries, so attention runs over every
-    // position s < q_len[t].
+    // position s < q_len[t].  A compact list (the library's top-k output) has min(k, n_t)
+    // entries before its -1 padding.
     const bool dense = a.idx == nullptr;
     const int j_lo = split * a.rows_per_split;
-    const int j_hi = min(dense ? min(a.k, n_t) : a.k, j_lo + a.rows_per_split);
+    const int j_hi = min((dense || a.compact) ? min(a.k, n_t) : a.k, j_lo + a.rows_per_split);
     const int nrows = max(0, j_hi - j_lo);
     const int ntiles = (nrows + kTileRows - 1) / kTileRows;
     const int32_t* idx_row = dense ? nullptr : a.idx + (int64_t)t * a.k;

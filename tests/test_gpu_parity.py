@@ -183,9 +183,13 @@ def run_decode_gpu(inp_gpu):
     return scores, idx, out, lse, status
 
 
-@pytest.mark.parametrize("which", ["small", "tiny"])
+@pytest.mark.parametrize("which", ["small", "tiny", "k512", "k1024", "dI128"])
 def test_decode_step_end_to_end(lib, which):
-    inp = small_decode(seed=41) if which == "small" else inputs.tiny()
+    # budgets 512 / 1024 and d_I = 128 are the width variants of kgptalkie "How Does the Selector
+    # Pick 1,024?" (V4 budgets) and its configuration table (d_I = 128)
+    inp = {"small": lambda: small_decode(seed=41), "tiny": inputs.tiny,
+           "k512": lambda: small_decode(seed=42, k=512), "k1024": lambda: small_decode(seed=43, k=1024),
+           "dI128": lambda: small_decode(seed=44, d_I=128)}[which]()
     sc_o, idx_o, out_o, lse_o = oracle.decode(inp)
     scores, idx, out, lse, status = run_decode_gpu(inp.to("cuda"))
     assert status == 0
@@ -195,6 +199,28 @@ def test_decode_step_end_to_end(lib, which):
     rows = [t for t in range(inp.Nq) if np.array_equal(g_idx[t], idx_o[t])]
     assert len(rows) >= max(1, total - 1), f"only {same}/{total} rows selected identical sets"
     check_attention(out.float().cpu().numpy(), out_o, lse.cpu().numpy(), lse_o, rows=rows)
+
+
+def test_short_rows_skip_the_indexer_with_the_same_outputs(lib):
+    # rows with q_len <= k: the decode step without scores_out skips their indexer work; the
+    # selection (every position) and the attention must not change
+    lens = [2048, 700, 1, 2049, 5000]
+    inp = small_decode(seed=45, lens=lens)
+    g = inp.to("cuda")
+    dims = api.dims_of(g)
+    ws = api.make_workspace(dims, _lib.DSA_OP_DECODE)
+    idx_a = torch.empty((len(lens), g.k), dtype=torch.int32, device="cuda")
+    idx_b = torch.empty_like(idx_a)
+    scores = torch.empty((len(lens), dims.ld_scores), device="cuda")
+    out_a, lse_a = api.run_decode(g, ws=ws, idx_out=idx_a, dims=dims)                    # skips short rows
+    out_b, lse_b = api.run_decode(g, ws=ws, idx_out=idx_b, scores_out=scores, dims=dims)  # scores every row
+    torch.cuda.synchronize()
+    assert api.get_device_status(ws) == 0
+    assert torch.equal(idx_a, idx_b)
+    for t, n in enumerate(lens):
+        if n <= g.k:
+            assert torch.equal(idx_a[t, :n].cpu(), torch.arange(n, dtype=torch.int32))
+    assert torch.equal(out_a, out_b) and torch.equal(lse_a, lse_b)
 
 
 def test_prefill_matches_oracle(lib):
