@@ -7,6 +7,7 @@ bf16 576-value latent rows), inputs resident in HBM.  Prints one JSON line.
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
   python bench.py --workload prefill [--prefill-len L] [--steps K] [--warmup W]
   python bench.py --workload dense [--steps K] [--warmup W]
+  python bench.py --workload paged [--block-size S] [--steps K] [--warmup W]
 
 N > 1 is launched with torch.distributed.run (one process per GPU); every rank
 decodes its own batch (weak scaling, no data-path collective); the time is the
@@ -24,6 +25,10 @@ peak).  It is a secondary line: the default run is the decode headline.
 batch (dsa_dense_mla_attn) and, in the same run, the DSA decode step on the
 same inputs, and reports the measured DSA-vs-dense ratio (the pages quote ~6x
 cheaper decode at 128K on H800 and a 13.4x arithmetic saving).
+
+--workload paged times dsa_decode_step_paged on the long-decode batch with its
+cache in blocks of a pool (seeded random physical order) and, in the same run,
+dsa_decode_step on the contiguous cache, and reports the cost of paging.
 """
 from __future__ import annotations
 
@@ -59,7 +64,8 @@ def parse_args():
     p.add_argument("--warmup", type=int, default=20)
     p.add_argument("--impl", default="ours", choices=["ours", "reference"])
     p.add_argument("--no-cpu-baseline", action="store_true")
-    p.add_argument("--workload", default="long_decode", choices=["long_decode", "prefill", "dense"])
+    p.add_argument("--workload", default="long_decode", choices=["long_decode", "prefill", "dense", "paged"])
+    p.add_argument("--block-size", type=int, default=64)
     p.add_argument("--prefill-len", type=int, default=65536)
     return p.parse_args()
 
@@ -537,6 +543,67 @@ def run_dense(args):
     return 0
 
 
+def run_paged(args):
+    """Secondary line: the decode step over a paged cache against the contiguous one."""
+    import torch
+    from sparse_long_context_indexer_b200 import _lib, api, inputs
+
+    if args.gpus != 1:
+        raise SystemExit("--workload paged runs on one GPU")
+    dev = torch.device("cuda", 0)
+    inp = inputs.make_decode_inputs(WORKLOAD, [CTX] * BATCH, T_max=CTX, n_anchors=32, recency=True, seed=3,
+                                    device=dev)
+    dims = api.dims_of(inp)
+    ws = api.make_workspace(dims, _lib.DSA_OP_DECODE, dev)
+    out, lse = api.alloc_outputs(inp)
+    out_p, lse_p = api.alloc_outputs(inp)
+    k_pool, s_pool, kv_pool, table = inputs.paged_layout(inp, args.block_size, seed=1)
+    cache = api.PagedCache(k_pool, s_pool, kv_pool, table, args.block_size)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    sweep = torch.ones(256 << 20, dtype=torch.uint8, device=dev)
+    K, W = max(1, min(args.steps, 2000)), args.warmup
+
+    def contiguous():
+        api.run_decode(inp, ws=ws, out=out, lse=lse, dims=dims)
+
+    def paged():
+        api.decode_step_paged(dims, inp.q_I, inp.q_scale, inp.w, cache, inp.q, inp.q_seq, inp.q_len,
+                              inp.softmax_scale, out_p, lse_p, ws)
+
+    def timed(fn):
+        for _ in range(W):
+            fn()
+        torch.cuda.synchronize()
+        ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(K)]
+        for i in range(K):
+            flush.zero_()
+            sweep.view(torch.int64).max()
+            ev[i][0].record()
+            fn()
+            ev[i][1].record()
+        torch.cuda.synchronize()
+        return sum(e[0].elapsed_time(e[1]) for e in ev) / K
+
+    c_ms = timed(contiguous)
+    p_ms = timed(paged)
+    status = api.get_device_status(ws)
+    same = bool(torch.equal(out, out_p) and torch.equal(lse, lse_p))
+    line = {
+        "metric": f"paged decode query-tok/s at 128K (blocks of {args.block_size} tokens)",
+        "value": BATCH / (p_ms * 1e-3), "unit": "query-tok/s", "n_gpus": 1, "steps": K, "warmup": W,
+        "ms_per_step": p_ms, "higher_is_better": True, "scaling": "none", "vs_baseline": None,
+        "dtype": "fp8_e4m3/bf16", "data": "synthetic",
+        "config": {"workload": WORKLOAD, "batch_per_gpu": BATCH, "cached_tokens": CTX, "block_size": args.block_size,
+                   "pool_blocks": int(kv_pool.shape[0]),
+                   "l2": "flushed between steps outside the timed events (write, then read of another buffer)"},
+        "paged_vs_contiguous": {"paged_ms": p_ms, "contiguous_ms": c_ms, "ratio": p_ms / c_ms,
+                                "outputs_identical": same},
+        "device_status": status,
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
 def launches_per_step():
     """Kernels one decode step launches: indexer, top-k, attention, plus the split
     merge when the attention's split count is above the cluster limit (8)."""
@@ -638,6 +705,8 @@ def main():
         return run_prefill(args)
     if args.workload == "dense":
         return run_dense(args)
+    if args.workload == "paged":
+        return run_paged(args)
     return run_ours(args)
 
 

@@ -223,6 +223,36 @@ dsa_status_t dsa_decode_step(const dsa_dims* dims,
                              void* workspace, size_t ws_bytes, void* stream,
                              const dsa_stage_events* events);
 
+/* A paged cache (kgptalkie "How Does the Selector Pick 1,024?": the selection
+ * is an address list into the paged KV cache).  Every sequence's cache lives in
+ * fixed-size blocks of shared pools, found through its row of a block table:
+ * token s of sequence b is row block_table[b * max_blocks + s / block_size] *
+ * block_size + s % block_size of each pool.  Caller-owned device memory. */
+typedef struct {
+    const void* k_I;             /* [num_blocks, block_size, d_I] e4m3 indexer keys */
+    const float* k_scale;        /* [num_blocks, block_size] fp32 key scales (16-byte aligned) */
+    const void* kv;              /* [num_blocks, block_size, 576] bf16 latent rows */
+    const int32_t* block_table;  /* [B, max_blocks] physical block of logical block j of sequence b */
+    int32_t block_size;          /* tokens per block: a power of two >= 64 */
+    int32_t num_blocks;          /* blocks in each pool */
+    int32_t max_blocks;          /* table row length; dims->T_max must equal max_blocks * block_size */
+    int32_t reserved;            /* must be 0 */
+} dsa_paged_cache;
+
+/* dsa_decode_step over a paged cache: the same stages and outputs, with the
+ * indexer's key and scale copies (one TMA box per block piece of a stage) and
+ * the attention's row gather translated through the block table.  Only blocks
+ * holding positions s < q_len[t] are read; a table entry outside
+ * [0, num_blocks) for such a block records DSA_ERR_INDEX_OOB in the status
+ * word (its rows are skipped).  FP8 indexer, bf16 latent. */
+dsa_status_t dsa_decode_step_paged(const dsa_dims* dims,
+                                   const void* q_I, const float* q_scale, const void* w,
+                                   const dsa_paged_cache* cache, const void* q,
+                                   const int32_t* q_seq, const int32_t* q_len, float softmax_scale,
+                                   void* out, float* lse, float* scores_out, int32_t* idx_out,
+                                   void* workspace, size_t ws_bytes, void* stream,
+                                   const dsa_stage_events* events);
+
 /* Prefill: the same three stages for many query rows of ONE sequence (every
  * position of a prompt), processed in row chunks so the transient score rows
  * fit the workspace (size it for DSA_OP_PREFILL).  Semantics per row are

@@ -22,7 +22,7 @@ DSA_OP_INDEXER, DSA_OP_TOPK, DSA_OP_SPARSE_MLA, DSA_OP_DECODE, DSA_OP_PREFILL, D
 EXPORTS = (
     "dsa_workspace_size", "dsa_workspace_init", "dsa_indexer_scores", "dsa_prefill_indexer_scores", "dsa_topk",
     "dsa_sparse_mla_attn", "dsa_dense_mla_attn",
-    "dsa_decode_step", "dsa_prefill", "dsa_get_device_status", "dsa_status_string", "dsa_last_cuda_error",
+    "dsa_decode_step", "dsa_decode_step_paged", "dsa_prefill", "dsa_get_device_status", "dsa_status_string", "dsa_last_cuda_error",
     "dsa_selftest_wait_timeout", "dsa_version", "dsa_sparse_mla_attn_noalloc",
 )
 
@@ -37,6 +37,12 @@ class DsaDims(ctypes.Structure):
 
 class DsaStageEvents(ctypes.Structure):
     _fields_ = [("ev", ctypes.c_void_p * 5)]
+
+
+class DsaPagedCache(ctypes.Structure):
+    _fields_ = [("k_I", ctypes.c_void_p), ("k_scale", ctypes.c_void_p), ("kv", ctypes.c_void_p),
+                ("block_table", ctypes.c_void_p), ("block_size", ctypes.c_int32), ("num_blocks", ctypes.c_int32),
+                ("max_blocks", ctypes.c_int32), ("reserved", ctypes.c_int32)]
 
 
 class DSAError(RuntimeError):
@@ -71,11 +77,14 @@ def _declare(lib):
     lib.dsa_decode_step.argtypes = [D, P, P, P, P, P, P, P, P, P, F, P, P, P, P, P, S, P,
                                     ctypes.POINTER(DsaStageEvents)]
     lib.dsa_prefill.argtypes = [D, P, P, P, P, P, P, P, P, P, F, P, P, P, P, S, P]
+    lib.dsa_decode_step_paged.argtypes = [D, P, P, P, ctypes.POINTER(DsaPagedCache), P, P, P, F, P, P, P, P, P, S,
+                                          P, ctypes.POINTER(DsaStageEvents)]
     lib.dsa_get_device_status.argtypes = [P, P, ctypes.POINTER(I32)]
     lib.dsa_selftest_wait_timeout.argtypes = [P, S, I32, P]
     for name in ("dsa_workspace_size", "dsa_workspace_init", "dsa_indexer_scores", "dsa_prefill_indexer_scores",
                  "dsa_topk",
-                 "dsa_sparse_mla_attn", "dsa_decode_step", "dsa_prefill", "dsa_get_device_status",
+                 "dsa_sparse_mla_attn", "dsa_decode_step", "dsa_decode_step_paged", "dsa_prefill",
+                 "dsa_get_device_status",
                  "dsa_selftest_wait_timeout", "dsa_sparse_mla_attn_noalloc", "dsa_dense_mla_attn"):
         getattr(lib, name).restype = st
     lib.dsa_status_string.argtypes = [I32]

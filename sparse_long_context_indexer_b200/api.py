@@ -137,6 +137,33 @@ def sparse_mla_attn(dims: Dims, q, kv, idx, q_seq, q_len, softmax_scale, out, ls
     return out, lse
 
 
+@dataclass
+class PagedCache:
+    """Block pools and block table of a paged cache (device tensors)."""
+    k_I: torch.Tensor          # [num_blocks, block_size, d_I] e4m3 (uint8)
+    k_scale: torch.Tensor      # [num_blocks, block_size] fp32
+    kv: torch.Tensor           # [num_blocks, block_size, 576] bf16
+    block_table: torch.Tensor  # [B, max_blocks] int32
+    block_size: int
+
+    def c(self) -> _lib.DsaPagedCache:
+        return _lib.DsaPagedCache(_ptr(self.k_I), _ptr(self.k_scale), _ptr(self.kv), _ptr(self.block_table),
+                                  self.block_size, self.kv.shape[0], self.block_table.shape[1], 0)
+
+
+def decode_step_paged(dims: Dims, q_I, q_scale, w, cache: PagedCache, q, q_seq, q_len, softmax_scale, out, lse, ws,
+                      scores_out=None, idx_out=None):
+    """One decode step over a paged cache on torch's current stream."""
+    lib = _lib.load()
+    d = dims.c()
+    pc = cache.c()
+    rc = lib.dsa_decode_step_paged(ctypes.byref(d), _ptr(q_I), _ptr(q_scale), _ptr(w), ctypes.byref(pc), _ptr(q),
+                                   _ptr(q_seq), _ptr(q_len), ctypes.c_float(softmax_scale), _ptr(out), _ptr(lse),
+                                   _ptr(scores_out), _ptr(idx_out), _ptr(ws), ws.numel(), _stream_ptr(), None)
+    _lib.check(lib, rc, "dsa_decode_step_paged")
+    return out, lse
+
+
 def decode_step(dims: Dims, q_I, q_scale, w, k_I, k_scale, q, kv, q_seq, q_len, softmax_scale, out, lse, ws,
                 scores_out=None, idx_out=None, events: Optional[Sequence] = None):
     """One decode step (indexer -> top-k -> sparse MLA) on torch's current stream.

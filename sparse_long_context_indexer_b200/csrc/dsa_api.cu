@@ -154,7 +154,7 @@ void record_event(const dsa_stage_events* ev, int i, cudaStream_t st) {
 dsa_status_t run_indexer(const dsa_dims* d, int nq, const void* q_I, const float* q_scale, const void* w,
                          const void* k_I, const float* k_scale, const int32_t* q_seq, const int32_t* q_len,
                          float* scores, int* status, cudaStream_t st, bool rows_of_one_sequence = false,
-                         int skip_upto = 0) {
+                         int skip_upto = 0, const dsa_paged_cache* paged = nullptr) {
     dsa::IndexerArgs a{};
     a.q_I = q_I;
     a.q_scale = q_scale;
@@ -172,6 +172,12 @@ dsa_status_t run_indexer(const dsa_dims* d, int nq, const void* q_I, const float
     a.d_I = d->d_I;
     a.status = status;
     a.skip_upto = skip_upto;
+    if (paged != nullptr) {
+        a.block_table = paged->block_table;
+        a.block_size = paged->block_size;
+        a.max_blocks = paged->max_blocks;
+        a.num_blocks = paged->num_blocks;
+    }
     cudaError_t e = d->idx_dtype != DSA_FP8_E4M3 ? dsa::launch_indexer_f32(a, st)
                     : rows_of_one_sequence      ? dsa::launch_indexer_fp8_units4(a, device_sms(), st)
                                                 : dsa::launch_indexer_fp8(a, device_sms(), st);
@@ -196,7 +202,8 @@ dsa_status_t run_topk(const dsa_dims* d, int nq, const float* scores, const int3
 
 dsa_status_t run_mla(const dsa_dims* d, int nq, const void* q, const void* kv, const int32_t* idx, const int32_t* q_seq,
                      const int32_t* q_len, float scale, void* out, float* lse, void* ws, const Layout& L,
-                     const dsa_stage_events* ev, cudaStream_t st, bool pdl = false, bool compact_idx = false) {
+                     const dsa_stage_events* ev, cudaStream_t st, bool pdl = false, bool compact_idx = false,
+                     const dsa_paged_cache* paged = nullptr) {
     const MlaPlan p = plan_mla(d, nq);
     dsa::MlaArgs a{};
     a.q = q;
@@ -219,6 +226,12 @@ dsa_status_t run_mla(const dsa_dims* d, int nq, const void* q, const void* kv, c
     a.status = ws ? status_word(ws) : nullptr;
     a.pdl = pdl ? 1 : 0;
     a.compact = compact_idx ? 1 : 0;
+    if (paged != nullptr) {
+        a.block_table = paged->block_table;
+        a.block_size = paged->block_size;
+        a.max_blocks = paged->max_blocks;
+        a.num_blocks = paged->num_blocks;
+    }
     cudaError_t e;
     if (d->kv_dtype == DSA_BF16) {
         e = dsa::launch_sparse_mla_bf16(a, st);
@@ -385,11 +398,17 @@ dsa_status_t dsa_sparse_mla_attn_noalloc(const dsa_dims* dims, const void* q, co
     return e == cudaSuccess ? DSA_OK : cuda_fail(e);
 }
 
-dsa_status_t dsa_decode_step(const dsa_dims* dims, const void* q_I, const float* q_scale, const void* w,
-                             const void* k_I, const float* k_scale, const void* q, const void* kv,
-                             const int32_t* q_seq, const int32_t* q_len, float softmax_scale, void* out, float* lse,
-                             float* scores_out, int32_t* idx_out, void* workspace, size_t ws_bytes, void* stream,
-                             const dsa_stage_events* events) {
+}  // extern "C"
+
+namespace {
+
+// The decode step over a contiguous cache (paged == nullptr) or a paged one (k_I, k_scale and
+// kv are then the pools and paged holds the block table).
+dsa_status_t decode_impl(const dsa_dims* dims, const void* q_I, const float* q_scale, const void* w, const void* k_I,
+                         const float* k_scale, const void* q, const void* kv, const dsa_paged_cache* paged,
+                         const int32_t* q_seq, const int32_t* q_len, float softmax_scale, void* out, float* lse,
+                         float* scores_out, int32_t* idx_out, void* workspace, size_t ws_bytes, void* stream,
+                         const dsa_stage_events* events) {
     dsa_status_t s = check_dims(dims, true, true);
     if (s != DSA_OK) return s;
     if (dims->Nq == 0) return DSA_OK;
@@ -411,7 +430,7 @@ dsa_status_t dsa_decode_step(const dsa_dims* dims, const void* q_I, const float*
     // rows with at most k positions select all of them: unless the caller asked for the
     // scores, the indexer skips those rows (short-context dispatch, same results)
     s = run_indexer(dims, dims->Nq, q_I, q_scale, w, k_I, k_scale, q_seq, q_len, scores, status, st, false,
-                    scores_out ? 0 : dims->k);
+                    scores_out ? 0 : dims->k, paged);
     if (s != DSA_OK) return s;
     record_event(events, 1, st);
     // top-k and attention follow their producer as programmatic dependents: their setup
@@ -420,10 +439,40 @@ dsa_status_t dsa_decode_step(const dsa_dims* dims, const void* q_I, const float*
     if (s != DSA_OK) return s;
     record_event(events, 2, st);
     s = run_mla(dims, dims->Nq, q, kv, idx, q_seq, q_len, softmax_scale, out, lse, workspace, L, events, st, true,
-                true);
+                true, paged);
     if (s != DSA_OK) return s;
     record_event(events, 4, st);
     return DSA_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+dsa_status_t dsa_decode_step(const dsa_dims* dims, const void* q_I, const float* q_scale, const void* w,
+                             const void* k_I, const float* k_scale, const void* q, const void* kv,
+                             const int32_t* q_seq, const int32_t* q_len, float softmax_scale, void* out, float* lse,
+                             float* scores_out, int32_t* idx_out, void* workspace, size_t ws_bytes, void* stream,
+                             const dsa_stage_events* events) {
+    return decode_impl(dims, q_I, q_scale, w, k_I, k_scale, q, kv, nullptr, q_seq, q_len, softmax_scale, out, lse,
+                       scores_out, idx_out, workspace, ws_bytes, stream, events);
+}
+
+dsa_status_t dsa_decode_step_paged(const dsa_dims* dims, const void* q_I, const float* q_scale, const void* w,
+                                   const dsa_paged_cache* cache, const void* q, const int32_t* q_seq,
+                                   const int32_t* q_len, float softmax_scale, void* out, float* lse,
+                                   float* scores_out, int32_t* idx_out, void* workspace, size_t ws_bytes,
+                                   void* stream, const dsa_stage_events* events) {
+    if (dims == nullptr || cache == nullptr || cache->block_table == nullptr || cache->reserved != 0)
+        return DSA_ERR_INVALID_ARG;
+    if (dims->idx_dtype != DSA_FP8_E4M3 || dims->kv_dtype != DSA_BF16) return DSA_ERR_UNSUPPORTED;
+    const int bs = cache->block_size;
+    if (bs < 64 || (bs & (bs - 1)) != 0 || cache->num_blocks < 1 || cache->max_blocks < 1) return DSA_ERR_INVALID_ARG;
+    if ((int64_t)cache->max_blocks * bs != dims->T_max) return DSA_ERR_INVALID_ARG;
+    if ((int64_t)cache->num_blocks * bs > (int64_t)INT32_MAX / 2) return DSA_ERR_UNSUPPORTED;
+    if (!aligned16(cache->k_scale)) return DSA_ERR_INVALID_ARG;
+    return decode_impl(dims, q_I, q_scale, w, cache->k_I, cache->k_scale, q, cache->kv, cache, q_seq, q_len,
+                       softmax_scale, out, lse, scores_out, idx_out, workspace, ws_bytes, stream, events);
 }
 
 dsa_status_t dsa_prefill(const dsa_dims* dims, const void* q_I, const float* q_scale, const void* w, const void* k_I,

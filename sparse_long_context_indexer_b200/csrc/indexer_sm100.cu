@@ -305,14 +305,43 @@ __global__ void __launch_bounds__(IdxCfg<D_I, R>::THREADS, 1)
                     const bool oke = mbar_wait(bar_empty(st), ((it / C::STAGES) - 1) & 1, abort_flag, a.status);
                     if (!__all_sync(0xffffffffu, oke)) break;
                 }
-                if (lane == 0) {
-                    mbar_arrive_expect_tx(bar_full(st), C::KTILE_BYTES + C::SC_BYTES);
+                if (a.block_table == nullptr) {
+                    if (lane == 0) {
+                        mbar_arrive_expect_tx(bar_full(st), C::KTILE_BYTES + C::SC_BYTES);
 #pragma unroll
-                    for (int q = 0; q < C::NBOX; ++q) {
-                        const int tok = cur.j * C::STOK + q * C::BOX;
-                        tma_load_2d(sK + st * C::KTILE_BYTES + q * (C::BOX * D_I), &tmap_k, 0, cur.b * a.T_max + tok,
-                                    bar_full(st));
-                        tma_load_2d(sS + st * C::SC_BYTES + q * (C::BOX * 4), &tmap_s, tok, cur.b, bar_full(st));
+                        for (int q = 0; q < C::NBOX; ++q) {
+                            const int tok = cur.j * C::STOK + q * C::BOX;
+                            tma_load_2d(sK + st * C::KTILE_BYTES + q * (C::BOX * D_I), &tmap_k, 0,
+                                        cur.b * a.T_max + tok, bar_full(st));
+                            tma_load_2d(sS + st * C::SC_BYTES + q * (C::BOX * 4), &tmap_s, tok, cur.b, bar_full(st));
+                        }
+                    }
+                } else {
+                    // paged cache: one key box and one scale box per block piece of the stage, for
+                    // the pieces that hold tokens of the unit (later pieces may have no block; their
+                    // stale rows only reach scores that are never stored).  Lane q reads piece q's
+                    // block id, so the table reads overlap.
+                    const int kb = a.page_box;
+                    const int tok0 = cur.j * C::STOK;
+                    const int live = min(C::STOK / kb, (cur.n - tok0 + kb - 1) / kb);
+                    int pb_l = 0;
+                    if (lane < live) {
+                        pb_l = a.block_table[(int64_t)cur.b * a.max_blocks + (tok0 + lane * kb) / a.block_size];
+                        if (pb_l < 0 || pb_l >= a.num_blocks) {
+                            record_status(a.status, DSA_STATUS_INDEX_OOB);
+                            pb_l = 0;
+                        }
+                    }
+                    if (lane == 0) mbar_arrive_expect_tx(bar_full(st), (uint32_t)live * kb * (D_I + 4));
+#pragma unroll
+                    for (int q = 0; q < C::STOK / 64; ++q) {  // kb >= 64: at most STOK / 64 pieces
+                        const int pb = __shfl_sync(0xffffffffu, pb_l, q);
+                        if (lane == 0 && q < live) {
+                            const int off = (tok0 + q * kb) % a.block_size;
+                            tma_load_2d(sK + st * C::KTILE_BYTES + q * (kb * D_I), &tmap_k, 0, pb * a.block_size + off,
+                                        bar_full(st));
+                            tma_load_2d(sS + st * C::SC_BYTES + q * (kb * 4), &tmap_s, off, pb, bar_full(st));
+                        }
                     }
                 }
                 ++issued;
@@ -485,17 +514,32 @@ cudaError_t launch_fp8_impl(const IndexerArgs& a, int grid, cudaStream_t st) {
     using C = IdxCfg<D_I, R>;
     alignas(64) CUtensorMap tk, tq, ts;
     const int swz = D_I;  // 64-byte rows -> 64B swizzle, 128-byte rows -> 128B swizzle
-    if (!encode_tensor_map_2d(&tk, 1, a.k_I, D_I, (uint64_t)a.B * a.T_max, D_I, D_I, C::BOX, swz))
-        return cudaErrorInvalidValue;
+    IndexerArgs b = a;
+    if (a.block_table == nullptr) {
+        if (!encode_tensor_map_2d(&tk, 1, a.k_I, D_I, (uint64_t)a.B * a.T_max, D_I, D_I, C::BOX, swz))
+            return cudaErrorInvalidValue;
+        if (!encode_tensor_map_2d(&ts, 4, a.k_scale, a.T_max, (uint64_t)a.B, (uint64_t)a.T_max * 4, C::BOX, 1, 0))
+            return cudaErrorInvalidValue;
+    } else {
+        // pools of num_blocks blocks: keys [num_blocks * block_size, d_I], scales [num_blocks, block_size]
+        if (a.block_size < 64 || (a.block_size & (a.block_size - 1)) != 0 || a.num_blocks < 1)
+            return cudaErrorInvalidValue;
+        b.page_box = a.block_size < C::BOX ? a.block_size : C::BOX;
+        if (C::STOK % b.page_box != 0) return cudaErrorInvalidValue;
+        if (!encode_tensor_map_2d(&tk, 1, a.k_I, D_I, (uint64_t)a.num_blocks * a.block_size, D_I, D_I,
+                                  (uint32_t)b.page_box, swz))
+            return cudaErrorInvalidValue;
+        if (!encode_tensor_map_2d(&ts, 4, a.k_scale, (uint64_t)a.block_size, (uint64_t)a.num_blocks,
+                                  (uint64_t)a.block_size * 4, (uint32_t)b.page_box, 1, 0))
+            return cudaErrorInvalidValue;
+    }
     // q8 rows of a unit are consecutive: [Nq * HEADS, d_I], boxes of NCOL rows
     if (!encode_tensor_map_2d(&tq, 1, a.q_I, D_I, (uint64_t)a.Nq * C::HEADS, D_I, D_I, C::NCOL, swz))
-        return cudaErrorInvalidValue;
-    if (!encode_tensor_map_2d(&ts, 4, a.k_scale, a.T_max, (uint64_t)a.B, (uint64_t)a.T_max * 4, C::BOX, 1, 0))
         return cudaErrorInvalidValue;
     auto kern = indexer_fp8_kernel<D_I, R>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
     if (e != cudaSuccess) return e;
-    kern<<<grid, C::THREADS, C::SMEM_BYTES, st>>>(a, tk, tq, ts);
+    kern<<<grid, C::THREADS, C::SMEM_BYTES, st>>>(b, tk, tq, ts);
     return cudaGetLastError();
 }
 

@@ -30,6 +30,12 @@ struct IndexerArgs {
     // where the scores are intermediate, the top-k selects every position of such a row
     // without reading them (0 = score every row)
     int skip_upto;
+    // Paged cache (block_table != nullptr): token s of sequence b lives in pool row
+    // block_table[b * max_blocks + s / block_size] * block_size + s % block_size of k_I
+    // ([num_blocks * block_size, d_I]) and k_scale ([num_blocks, block_size]).
+    const int32_t* block_table;
+    int block_size, max_blocks, num_blocks;
+    int page_box;  // key rows per TMA box in paged mode (set by the launcher)
 };
 
 struct TopkArgs {
@@ -60,6 +66,10 @@ struct MlaArgs {
     // the index list is the library's own top-k output: entries past min(k, q_len[t]) are -1,
     // so the splits stop there
     int compact;
+    // paged latent cache (block_table != nullptr): token s of sequence b is kv row
+    // block_table[b * max_blocks + s / block_size] * block_size + s % block_size
+    const int32_t* block_table;
+    int block_size, max_blocks, num_blocks;
 };
 
 cudaError_t launch_indexer_fp8(const IndexerArgs& a, int grid, cudaStream_t st);

@@ -149,7 +149,17 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int nrows = max(0, j_hi - j_lo);
     const int ntiles = (nrows + kTileRows - 1) / kTileRows;
     const int32_t* idx_row = dense ? nullptr : a.idx + (int64_t)t * a.k;
-    const __nv_bfloat16* kv_seq = reinterpret_cast<const __nv_bfloat16*>(a.kv) + (int64_t)b * a.T_max * kDK;
+    const __nv_bfloat16* kv_base = reinterpret_cast<const __nv_bfloat16*>(a.kv);
+    const __nv_bfloat16* kv_seq = kv_base + (int64_t)b * a.T_max * kDK;
+    const int32_t* btab = a.block_table ? a.block_table + (int64_t)b * a.max_blocks : nullptr;
+    // latent row of token s (contiguous cache, or through the block table of a paged one);
+    // nullptr for a block id outside the pool
+    auto kv_row = [&](int s) -> const __nv_bfloat16* {
+        if (btab == nullptr) return kv_seq + (int64_t)s * kDK;
+        const int pb = __ldg(btab + s / a.block_size);
+        if (pb < 0 || pb >= a.num_blocks) return nullptr;
+        return kv_base + ((int64_t)pb * a.block_size + s % a.block_size) * kDK;
+    };
     // entry r of tile i -> selected token, -1 past the end of the split
     auto load_pos = [&](int i, int r) -> int {
         const int j = j_lo + i * kTileRows + r;
@@ -213,7 +223,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         // thread p copies 16-byte granule (p & 7) of every 128-byte piece of rows
         // (p >> 3) and (p >> 3) + 32 of each tile.
         auto prefetch_row = [&](int s) {
-            if (valid(s)) l2_prefetch_bulk(kv_seq + (int64_t)s * kDK, kDK * 2);
+            if (valid(s)) {
+                const __nv_bfloat16* r = kv_row(s);
+                if (r) l2_prefetch_bulk(r, kDK * 2);
+            }
         };
         if (pf_lane) prefetch_row(pf_first);
         for (int i = 0; i < ntiles; ++i) {
@@ -226,9 +239,10 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (int h2 = 0; h2 < 2; ++h2) {
                 const int s = h2 ? cur1 : cur0;
                 const int r = rr + 32 * h2;
-                const bool ok_row = valid(s);
-                const __nv_bfloat16* src =
-                    ok_row ? kv_seq + (int64_t)s * kDK + gl * 8 : reinterpret_cast<const __nv_bfloat16*>(a.kv);
+                const __nv_bfloat16* row = valid(s) ? kv_row(s) : nullptr;
+                if (valid(s) && row == nullptr && gl == 0) record_status(a.status, DSA_STATUS_INDEX_OOB);
+                const bool ok_row = row != nullptr;
+                const __nv_bfloat16* src = ok_row ? row + gl * 8 : kv_base;
                 const uint32_t dst = stage + r * 128 + ((gl ^ (r & 7)) << 4);
 #pragma unroll
                 for (int c = 0; c < kChunks; ++c) cp_async16_zfill(dst + c * kChunkBytes, src + c * 64, ok_row ? 16u : 0u);

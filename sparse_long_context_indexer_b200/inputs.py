@@ -238,6 +238,40 @@ def make_prefill_inputs(name: str, L: int, *, H_I=64, d_I=64, H=128, k=2048, see
 
 # ---- the five workloads ------------------------------------------------------
 
+def paged_layout(inp: DSAInputs, block_size: int, seed: int = 0, spare_blocks: int = 3):
+    """The same cache in paged form: pools of blocks in a seeded random physical order.
+
+    Returns (k_I_pool, k_scale_pool, kv_pool, block_table) with block_table[b, j] the pool
+    block holding tokens [j * block_size, (j + 1) * block_size) of sequence b; blocks past a
+    sequence's longest query length get -1 (never read).  Pure data movement.
+    """
+    B, T_max = inp.kv.shape[0], inp.kv.shape[1]
+    assert T_max % block_size == 0
+    mb = T_max // block_size
+    nb = B * mb + spare_blocks
+    gen = torch.Generator().manual_seed(seed)
+    perm = torch.randperm(nb, generator=gen)
+    dev = inp.kv.device
+    k_pool = torch.zeros((nb, block_size) + tuple(inp.k_I.shape[2:]), dtype=inp.k_I.dtype, device=dev)
+    s_pool = torch.zeros((nb, block_size), dtype=torch.float32, device=dev)
+    kv_pool = torch.zeros((nb, block_size, inp.kv.shape[2]), dtype=inp.kv.dtype, device=dev)
+    table = torch.full((B, mb), -1, dtype=torch.int32)
+    q_seq = inp.q_seq.cpu()
+    q_len = inp.q_len.cpu()
+    for b in range(B):
+        rows = q_seq == b
+        need = int(q_len[rows].max()) if bool(rows.any()) else 0
+        for j in range((need + block_size - 1) // block_size):
+            pb = int(perm[b * mb + j])
+            table[b, j] = pb
+            sl = slice(j * block_size, (j + 1) * block_size)
+            k_pool[pb] = inp.k_I[b, sl]
+            if inp.k_scale is not None:
+                s_pool[pb] = inp.k_scale[b, sl]
+            kv_pool[pb] = inp.kv[b, sl]
+    return k_pool, s_pool, kv_pool, table.to(dev)
+
+
 def tiny(device="cpu"):
     """Tiny decode: 1 query over 4096 cached tokens, fp32, H_I=4, top-256, 16 heads, 16 anchors."""
     return make_decode_inputs("tiny_decode_4k_fp32", [4096], H_I=4, d_I=64, H=16, k=256,

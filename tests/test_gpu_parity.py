@@ -223,6 +223,34 @@ def test_short_rows_skip_the_indexer_with_the_same_outputs(lib):
     assert torch.equal(out_a, out_b) and torch.equal(lse_a, lse_b)
 
 
+@pytest.mark.parametrize("block_size", [64, 256])
+def test_paged_decode_matches_contiguous(lib, block_size):
+    # the same cache in blocks of a pool, in a random physical order, read through a block
+    # table (kgptalkie: the selection is an address list into the paged KV cache); the
+    # contiguous path is pinned to the oracle, the paged one must give identical outputs
+    lens = [4097, 2500, 777, 2048, 2049, 129, 1]
+    inp = inputs.make_decode_inputs("paged", lens, T_max=4352, anchor_frac=0.01, seed=71)
+    g = inp.to("cuda")
+    dims = api.dims_of(g)
+    ws = api.make_workspace(dims, _lib.DSA_OP_DECODE)
+    idx_c = torch.empty((len(lens), g.k), dtype=torch.int32, device="cuda")
+    sc_c = torch.empty((len(lens), dims.ld_scores), device="cuda")
+    out_c, lse_c = api.run_decode(g, ws=ws, idx_out=idx_c, scores_out=sc_c, dims=dims)
+    k_pool, s_pool, kv_pool, table = inputs.paged_layout(g, block_size, seed=block_size)
+    cache = api.PagedCache(k_pool, s_pool, kv_pool, table, block_size)
+    out_p, lse_p = api.alloc_outputs(g)
+    idx_p = torch.empty_like(idx_c)
+    sc_p = torch.full_like(sc_c, float("nan"))
+    api.decode_step_paged(dims, g.q_I, g.q_scale, g.w, cache, g.q, g.q_seq, g.q_len, g.softmax_scale, out_p, lse_p, ws,
+                          scores_out=sc_p, idx_out=idx_p)
+    torch.cuda.synchronize()
+    assert api.get_device_status(ws) == 0
+    for t, n in enumerate(lens):
+        assert torch.equal(sc_p[t, :n], sc_c[t, :n]), f"row {t}: paged scores differ"
+    assert torch.equal(idx_p, idx_c)
+    assert torch.equal(out_p, out_c) and torch.equal(lse_p, lse_c)
+
+
 def test_prefill_matches_oracle(lib):
     L = 3000
     inp = inputs.make_prefill_inputs("prefill_small", L, seed=7)
