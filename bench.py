@@ -422,7 +422,11 @@ def run_prefill(args):
     total_ms = statistics.median(ms)
 
     # Stage pass: the same work, chunk by chunk, each stage through its own entry point.
-    chunk = max(1, min(L, (64 << 20) // (dims.ld_scores * 4)))
+    sms = torch.cuda.get_device_properties(0).multi_processor_count
+    chunk = max(1, (64 << 20) // (dims.ld_scores * 4))
+    if chunk >= sms // 2:
+        chunk = chunk // (sms // 2) * (sms // 2) // 4 * 4   # the library's plan: whole attention waves
+    chunk = max(1, min(L, chunk))
     cd = api.Dims(B=1, Nq=chunk, H_I=g.H_I, d_I=g.d_I, H=g.H, k=g.k, T_max=g.T_max, idx_dtype=g.idx_dtype,
                   kv_dtype=g.kv_dtype, ld_scores=dims.ld_scores)
     cws = api.make_workspace(cd, _lib.DSA_OP_SPARSE_MLA, dev)

@@ -101,6 +101,12 @@ int plan_topk_cluster(const dsa_dims* d, int nq) {
 int plan_prefill_chunk(const dsa_dims* d) {
     int64_t rows = (int64_t)(kPrefillChunkScoreBytes / ((size_t)d->ld_scores * sizeof(float)));
     if (rows < 1) rows = 1;
+    // The attention of a chunk runs one CTA per (row, head half) on one SM each: a chunk of
+    // whole waves (2 rows x SMs / 2 per wave) in multiples of four rows (the indexer's units)
+    // keeps the last wave full.
+    const int64_t per_wave = device_sms() / 2;
+    if (rows >= per_wave) rows = rows / per_wave * per_wave / 4 * 4;
+    if (rows < 1) rows = 1;
     if (rows > d->Nq) rows = d->Nq;
     if (rows > 65535) rows = 65535;
     return (int)(rows < 1 ? 1 : rows);
