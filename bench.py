@@ -8,6 +8,7 @@ bf16 576-value latent rows), inputs resident in HBM.  Prints one JSON line.
   python bench.py --workload prefill [--prefill-len L] [--steps K] [--warmup W]
   python bench.py --workload dense [--steps K] [--warmup W]
   python bench.py --workload paged [--block-size S] [--steps K] [--warmup W]
+  python bench.py --workload fp8kv [--steps K] [--warmup W]
 
 N > 1 is launched with torch.distributed.run (one process per GPU); every rank
 decodes its own batch (weak scaling, no data-path collective); the time is the
@@ -29,6 +30,10 @@ cheaper decode at 128K on H800 and a 13.4x arithmetic saving).
 --workload paged times dsa_decode_step_paged on the long-decode batch with its
 cache in blocks of a pool (seeded random physical order) and, in the same run,
 dsa_decode_step on the contiguous cache, and reports the cost of paging.
+
+--workload fp8kv times the decode step with the latent cache in 656-byte FP8
+entries (512 e4m3 values, 4 fp32 scales, 64 bf16 rope values) against the
+bf16 cache on the same inputs, same run.
 """
 from __future__ import annotations
 
@@ -64,7 +69,7 @@ def parse_args():
     p.add_argument("--warmup", type=int, default=20)
     p.add_argument("--impl", default="ours", choices=["ours", "reference"])
     p.add_argument("--no-cpu-baseline", action="store_true")
-    p.add_argument("--workload", default="long_decode", choices=["long_decode", "prefill", "dense", "paged"])
+    p.add_argument("--workload", default="long_decode", choices=["long_decode", "prefill", "dense", "paged", "fp8kv"])
     p.add_argument("--block-size", type=int, default=64)
     p.add_argument("--prefill-len", type=int, default=65536)
     return p.parse_args()
@@ -614,6 +619,62 @@ def run_paged(args):
     return 0
 
 
+def run_fp8kv(args):
+    """Secondary line: the decode step over the FP8 latent cache against the bf16 one."""
+    import torch
+    from sparse_long_context_indexer_b200 import _lib, accounting, api, inputs
+
+    if args.gpus != 1:
+        raise SystemExit("--workload fp8kv runs on one GPU")
+    dev = torch.device("cuda", 0)
+    inp = inputs.make_decode_inputs(WORKLOAD, [CTX] * BATCH, T_max=CTX, n_anchors=32, recency=True, seed=3,
+                                    device=dev)
+    inp8 = inputs.with_fp8_latent(inp)
+    dims, dims8 = api.dims_of(inp), api.dims_of(inp8)
+    ws = api.make_workspace(dims, _lib.DSA_OP_DECODE, dev)
+    out, lse = api.alloc_outputs(inp)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    sweep = torch.ones(256 << 20, dtype=torch.uint8, device=dev)
+    K, W = max(1, min(args.steps, 2000)), args.warmup
+
+    def timed(g, d):
+        for _ in range(W):
+            api.run_decode(g, ws=ws, out=out, lse=lse, dims=d)
+        torch.cuda.synchronize()
+        ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(K)]
+        for i in range(K):
+            flush.zero_()
+            sweep.view(torch.int64).max()
+            ev[i][0].record()
+            api.run_decode(g, ws=ws, out=out, lse=lse, dims=d)
+            ev[i][1].record()
+        torch.cuda.synchronize()
+        return sum(e[0].elapsed_time(e[1]) for e in ev) / K
+
+    bf16_ms = timed(inp, dims)
+    fp8_ms = timed(inp8, dims8)
+    status = api.get_device_status(ws)
+    by = accounting.decode_step_bytes([CTX] * BATCH)
+    gather_bf16 = BATCH * 2048 * 1152
+    fp8_bytes = by["total"] - gather_bf16 + BATCH * 2048 * 656
+    line = {
+        "metric": "decode query-tok/s at 128K with the FP8 latent cache (656-byte entries)",
+        "value": BATCH / (fp8_ms * 1e-3), "unit": "query-tok/s", "n_gpus": 1, "steps": K, "warmup": W,
+        "ms_per_step": fp8_ms, "higher_is_better": True, "scaling": "none", "vs_baseline": None,
+        "dtype": "fp8_e4m3 (indexer and latent)/bf16", "data": "synthetic",
+        "config": {"workload": WORKLOAD + "_fp8kv", "batch_per_gpu": BATCH, "cached_tokens": CTX,
+                   "latent": "656 B: 512 e4m3 + 4 fp32 scales + 64 bf16 rope",
+                   "l2": "flushed between steps outside the timed events (write, then read of another buffer)"},
+        "step_roofline": {"achieved": fp8_bytes / (fp8_ms * 1e-3) / 1e9, "peak": peaks()[0], "unit": "GB/s",
+                          "algorithmic_bytes": fp8_bytes},
+        "fp8_vs_bf16_latent": {"fp8_ms": fp8_ms, "bf16_ms": bf16_ms, "ratio": fp8_ms / bf16_ms,
+                               "gather_bytes_per_row": {"fp8": 2048 * 656, "bf16": 2048 * 1152}},
+        "device_status": status,
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
 def launches_per_step():
     """Kernels one decode step launches: indexer, top-k, attention, plus the split
     merge when the attention's split count is above the cluster limit (8)."""
@@ -717,6 +778,8 @@ def main():
         return run_dense(args)
     if args.workload == "paged":
         return run_paged(args)
+    if args.workload == "fp8kv":
+        return run_fp8kv(args)
     return run_ours(args)
 
 

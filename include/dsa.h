@@ -39,7 +39,12 @@
  *   k_I      [B, T_max, d_I]  FP8 e4m3 bytes or float
  *   k_scale  [B, T_max]       float, > 0 (FP8 only; may be NULL for float)
  *   q        [Nq, H, 576]     bfloat16 or float (absorbed MLA query: 512 latent + 64 rope)
- *   kv       [B, T_max, 576]  bfloat16 or float (latent cache; value = first 512)
+ *   kv       [B, T_max, 576]  bfloat16 or float (latent cache; value = first 512), or
+ *            [B, T_max, 656]  bytes with kv_dtype DSA_FP8_E4M3: the FP8 latent entry of
+ *                             kgptalkie "What Does the GPU Actually Run?" -- bytes 0..511 the
+ *                             e4m3 codes of latent values 0..511, bytes 512..527 four fp32
+ *                             scales (value i = e4m3(code i) * scale[i / 128]), bytes
+ *                             528..655 the 64 rope values in bf16; q and out stay bf16
  *   out      [Nq, H, 512]     same element type as kv
  *   lse      [Nq, H]          float, natural-log sum of exp(scale * q.c) over the selection
  *   scores   [Nq, ld_scores]  float, entries s >= q_len[t] are not written
@@ -82,7 +87,7 @@ typedef enum {
  *   idx_dtype DSA_FP8_E4M3: d_I in {64, 128}, H_I = 64 (the MMA N dimension of the
  *                           tensor-core kernel), T_max a multiple of 4; w is bfloat16.
  *   idx_dtype DSA_F32:      d_I in {64, 128}, 1 <= H_I <= 64; w is float.
- *   kv_dtype  DSA_BF16:     H = 128 (MMA M dimension).
+ *   kv_dtype  DSA_BF16 or DSA_FP8_E4M3 (656-byte entries): H = 128 (MMA M dimension).
  *   kv_dtype  DSA_F32:      1 <= H <= 128.
  *   1 <= k <= 2048; 1 <= T_max; ld_scores >= 1 and a multiple of 4. */
 typedef struct {
@@ -94,7 +99,7 @@ typedef struct {
     int32_t k;          /* top-k budget */
     int32_t T_max;      /* cache capacity per sequence, tokens (row stride of k_I/kv per sequence) */
     int32_t idx_dtype;  /* dsa_dtype_t of q_I/k_I: DSA_FP8_E4M3 or DSA_F32 */
-    int32_t kv_dtype;   /* dsa_dtype_t of q/kv/out: DSA_BF16 or DSA_F32 */
+    int32_t kv_dtype;   /* dsa_dtype_t of the cache: DSA_BF16, DSA_F32 or DSA_FP8_E4M3 (656-byte entries) */
     int32_t reserved;   /* must be 0 */
     int64_t ld_scores;  /* row stride of the scores matrix, elements */
 } dsa_dims;
@@ -174,7 +179,7 @@ dsa_status_t dsa_sparse_mla_attn(const dsa_dims* dims, const void* q, const void
  * s < q_len[t]: out[t,h,:] = sum_{s < q_len[t]} softmax_s(...) kv[b,s,0:512].
  * The same kernel runs with each split walking a contiguous block of
  * positions instead of an index list; dims->k is ignored (the plan uses T_max).
- * kv_dtype DSA_BF16 only.  Workspace sized for DSA_OP_DENSE_MLA. */
+ * kv_dtype DSA_BF16 or DSA_FP8_E4M3.  Workspace sized for DSA_OP_DENSE_MLA. */
 dsa_status_t dsa_dense_mla_attn(const dsa_dims* dims, const void* q, const void* kv,
                                 const int32_t* q_seq, const int32_t* q_len, float softmax_scale,
                                 void* out, float* lse, void* workspace, size_t ws_bytes, void* stream);
@@ -185,7 +190,7 @@ dsa_status_t dsa_dense_mla_attn(const dsa_dims* dims, const void* q, const void*
  * buffers, or serving loops whose device-memory budget is fixed at start-up --
  * and so can neither call cudaMalloc nor size a workspace for
  * dsa_sparse_mla_attn.  Same arguments and results as dsa_sparse_mla_attn with
- * kv_dtype DSA_BF16, minus the workspace: the split partials live in a buffer
+ * kv_dtype DSA_BF16 or DSA_FP8_E4M3, minus the workspace: the split partials live in a buffer
  * the library holds statically on every GPU that loads it (about 16.1 MiB,
  * kept until the process exits).
  * Limit: when the split count is above 8 (the partials path of
@@ -231,7 +236,7 @@ dsa_status_t dsa_decode_step(const dsa_dims* dims,
 typedef struct {
     const void* k_I;             /* [num_blocks, block_size, d_I] e4m3 indexer keys */
     const float* k_scale;        /* [num_blocks, block_size] fp32 key scales (16-byte aligned) */
-    const void* kv;              /* [num_blocks, block_size, 576] bf16 latent rows */
+    const void* kv;              /* [num_blocks, block_size, 576] bf16 or [.., 656] FP8 latent entries */
     const int32_t* block_table;  /* [B, max_blocks] physical block of logical block j of sequence b */
     int32_t block_size;          /* tokens per block: a power of two >= 64 */
     int32_t num_blocks;          /* blocks in each pool */
@@ -244,7 +249,8 @@ typedef struct {
  * the attention's row gather translated through the block table.  Only blocks
  * holding positions s < q_len[t] are read; a table entry outside
  * [0, num_blocks) for such a block records DSA_ERR_INDEX_OOB in the status
- * word (its rows are skipped).  FP8 indexer, bf16 latent. */
+ * word (its rows are skipped).  FP8 indexer; bf16 or FP8 (656-byte) latent pool
+ * ([num_blocks, block_size, 576] bf16 or [num_blocks, block_size, 656] bytes). */
 dsa_status_t dsa_decode_step_paged(const dsa_dims* dims,
                                    const void* q_I, const float* q_scale, const void* w,
                                    const dsa_paged_cache* cache, const void* q,

@@ -137,10 +137,39 @@ def topk(scores, q_len, k, nthreads=0):
     return idx
 
 
+def _bf16_bits_to_f32(bits):
+    """bf16 bit patterns -> float32: a bf16 value is the upper half of an IEEE binary32."""
+    return (np.asarray(bits).astype(np.uint16).astype(np.uint32) << 16).view(np.float32)
+
+
+def dequant_latent_fp8(entries):
+    """656-byte FP8 latent entries (kgptalkie "What Does the GPU Actually Run?": 512 values
+    in e4m3, 4 float32 scale factors, the 64 rope values in bf16) -> float32 [..., 576].
+
+    Latent value i = e4m3(code_i) * scale[i // 128] (this oracle's own e4m3 decoding,
+    products formed in float64 and stored as float32); rope values widened from bf16."""
+    e = np.ascontiguousarray(_np(entries, np.uint8))
+    lead = e.shape[:-1]
+    e = e.reshape(-1, 656)
+    table = np.array([e4m3_decode(c) for c in range(256)], dtype=np.float64)
+    scales = e[:, 512:528].copy().view(np.float32).astype(np.float64)  # [n, 4]
+    lat = table[e[:, :512]].reshape(-1, 4, 128) * scales[:, :, None]
+    rope = _bf16_bits_to_f32(e[:, 528:656].copy().view(np.uint16))
+    out = np.concatenate([lat.reshape(-1, 512).astype(np.float32), rope.reshape(-1, 64)], axis=1)
+    return out.reshape(*lead, 576)
+
+
+def _attn_operands(inp, q, kv):
+    """(q, kv, element type) for the C attention routines; an FP8 latent cache is dequantised
+    here and the query widened to float32 with it (exact), so both go in as float32."""
+    if inp.kv_dtype == FP8:
+        return _bf16_bits_to_f32(_np(q)), dequant_latent_fp8(kv), F32
+    return _np(q), _np(kv), inp.kv_dtype
+
+
 def sparse_attn(inp, idx, q=None, kv=None, q_seq=None, q_len=None, scale=None, nthreads=0):
     """(out [Nq, H, 512] float64, lse [Nq, H] float64) over the positions in idx."""
-    q = _np(inp.q if q is None else q)
-    kv = _np(inp.kv if kv is None else kv)
+    q, kv, kvdt = _attn_operands(inp, inp.q if q is None else q, inp.kv if kv is None else kv)
     idx = _np(idx, np.int32)
     q_seq = _np(inp.q_seq if q_seq is None else q_seq, np.int32)
     q_len = _np(inp.q_len if q_len is None else q_len, np.int32)
@@ -149,7 +178,7 @@ def sparse_attn(inp, idx, q=None, kv=None, q_seq=None, q_len=None, scale=None, n
     out = np.zeros((Nq, inp.H, 512), dtype=np.float64)
     lse = np.zeros((Nq, inp.H), dtype=np.float64)
     sc = inp.softmax_scale if scale is None else scale
-    rc = _load().dsa_oracle_sparse_attn(Nq, inp.H, inp.T_max, inp.B, k, inp.kv_dtype, _ptr(q), _ptr(kv),
+    rc = _load().dsa_oracle_sparse_attn(Nq, inp.H, inp.T_max, inp.B, k, kvdt, _ptr(q), _ptr(kv),
                                        _ptr(idx), _ptr(q_seq), _ptr(q_len), sc, _ptr(out), _ptr(lse),
                                        nthreads)
     if rc != 0:
@@ -158,8 +187,7 @@ def sparse_attn(inp, idx, q=None, kv=None, q_seq=None, q_len=None, scale=None, n
 
 
 def masked_dense_attn(inp, idx, scale=None, nthreads=0):
-    q = _np(inp.q)
-    kv = _np(inp.kv)
+    q, kv, kvdt = _attn_operands(inp, inp.q, inp.kv)
     idx = _np(idx, np.int32)
     q_seq = _np(inp.q_seq, np.int32)
     q_len = _np(inp.q_len, np.int32)
@@ -167,7 +195,7 @@ def masked_dense_attn(inp, idx, scale=None, nthreads=0):
     out = np.zeros((Nq, inp.H, 512), dtype=np.float64)
     lse = np.zeros((Nq, inp.H), dtype=np.float64)
     sc = inp.softmax_scale if scale is None else scale
-    rc = _load().dsa_oracle_masked_dense_attn(Nq, inp.H, inp.T_max, inp.B, idx.shape[1], inp.kv_dtype,
+    rc = _load().dsa_oracle_masked_dense_attn(Nq, inp.H, inp.T_max, inp.B, idx.shape[1], kvdt,
                                              _ptr(q), _ptr(kv), _ptr(idx), _ptr(q_seq), _ptr(q_len),
                                              sc, _ptr(out), _ptr(lse), nthreads)
     if rc != 0:
@@ -176,15 +204,14 @@ def masked_dense_attn(inp, idx, scale=None, nthreads=0):
 
 
 def dense_attn(inp, scale=None, nthreads=0):
-    q = _np(inp.q)
-    kv = _np(inp.kv)
+    q, kv, kvdt = _attn_operands(inp, inp.q, inp.kv)
     q_seq = _np(inp.q_seq, np.int32)
     q_len = _np(inp.q_len, np.int32)
     Nq = q_seq.shape[0]
     out = np.zeros((Nq, inp.H, 512), dtype=np.float64)
     lse = np.zeros((Nq, inp.H), dtype=np.float64)
     sc = inp.softmax_scale if scale is None else scale
-    rc = _load().dsa_oracle_dense_attn(Nq, inp.H, inp.T_max, inp.B, inp.kv_dtype, _ptr(q), _ptr(kv),
+    rc = _load().dsa_oracle_dense_attn(Nq, inp.H, inp.T_max, inp.B, kvdt, _ptr(q), _ptr(kv),
                                       _ptr(q_seq), _ptr(q_len), sc, _ptr(out), _ptr(lse), nthreads)
     if rc != 0:
         raise ValueError(f"oracle dense attention failed (rc={rc})")

@@ -209,7 +209,7 @@ def selftest_wait_timeout(ws: torch.Tensor, timeout_us: int = 200000):
 
 def alloc_outputs(inp, device=None):
     dev = device or inp.device
-    odt = torch.bfloat16 if inp.kv_dtype == _lib.DSA_BF16 else torch.float32
+    odt = torch.float32 if inp.kv_dtype == _lib.DSA_F32 else torch.bfloat16
     out = torch.empty((inp.Nq, inp.H, D_V), dtype=odt, device=dev)
     lse = torch.empty((inp.Nq, inp.H), dtype=torch.float32, device=dev)
     return out, lse

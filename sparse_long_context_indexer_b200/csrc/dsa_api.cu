@@ -53,7 +53,7 @@ dsa_status_t check_dims(const dsa_dims* d, bool need_indexer, bool need_mla, boo
         if ((int64_t)d->Nq * d->H_I > INT32_MAX / 2) return DSA_ERR_UNSUPPORTED;
     }
     if (need_mla) {
-        if (d->kv_dtype == DSA_BF16) {
+        if (d->kv_dtype == DSA_BF16 || d->kv_dtype == DSA_FP8_E4M3) {  // FP8: the 656-byte latent entry
             if (d->H != dsa::kMlaHeads) return DSA_ERR_UNSUPPORTED;
         } else if (d->kv_dtype == DSA_F32) {
             if (d->H < 1 || d->H > 128) return DSA_ERR_UNSUPPORTED;
@@ -72,7 +72,7 @@ struct MlaPlan {
 
 MlaPlan plan_mla(const dsa_dims* d, int nq) {
     MlaPlan p;
-    if (d->kv_dtype != DSA_BF16 || nq <= 0) {
+    if (d->kv_dtype == DSA_F32 || nq <= 0) {
         p.rows_per_split = d->k;
         return p;
     }
@@ -238,8 +238,9 @@ dsa_status_t run_mla(const dsa_dims* d, int nq, const void* q, const void* kv, c
         a.max_blocks = paged->max_blocks;
         a.num_blocks = paged->num_blocks;
     }
+    a.kv_fp8 = d->kv_dtype == DSA_FP8_E4M3 ? 1 : 0;
     cudaError_t e;
-    if (d->kv_dtype == DSA_BF16) {
+    if (d->kv_dtype != DSA_F32) {
         e = dsa::launch_sparse_mla_bf16(a, st);
         record_event(ev, 3, st);
         if (e == cudaSuccess) e = dsa::launch_mla_combine(a, st);
@@ -351,7 +352,7 @@ dsa_status_t dsa_dense_mla_attn(const dsa_dims* dims, const void* q, const void*
                                 size_t ws_bytes, void* stream) {
     dsa_status_t s = check_dims(dims, false, true);
     if (s != DSA_OK) return s;
-    if (dims->kv_dtype != DSA_BF16) return DSA_ERR_UNSUPPORTED;
+    if (dims->kv_dtype == DSA_F32) return DSA_ERR_UNSUPPORTED;
     if (dims->Nq == 0) return DSA_OK;
     if (!q || !kv || !q_seq || !q_len || !out || !std::isfinite(softmax_scale)) return DSA_ERR_INVALID_ARG;
     if (!aligned16(q) || !aligned16(kv) || !aligned16(out)) return DSA_ERR_INVALID_ARG;
@@ -368,7 +369,7 @@ dsa_status_t dsa_sparse_mla_attn_noalloc(const dsa_dims* dims, const void* q, co
                                          float* lse, void* stream) {
     dsa_status_t s = check_dims(dims, false, true);
     if (s != DSA_OK) return s;
-    if (dims->kv_dtype != DSA_BF16) return DSA_ERR_UNSUPPORTED;
+    if (dims->kv_dtype == DSA_F32) return DSA_ERR_UNSUPPORTED;
     if (dims->Nq == 0) return DSA_OK;
     if (!q || !kv || !idx || !q_seq || !q_len || !out || !std::isfinite(softmax_scale)) return DSA_ERR_INVALID_ARG;
     if (!aligned16(q) || !aligned16(kv) || !aligned16(out)) return DSA_ERR_INVALID_ARG;
@@ -396,6 +397,7 @@ dsa_status_t dsa_sparse_mla_attn_noalloc(const dsa_dims* dims, const void* q, co
     a.H = dims->H;
     a.splits = p.splits;
     a.rows_per_split = p.rows_per_split;
+    a.kv_fp8 = dims->kv_dtype == DSA_FP8_E4M3 ? 1 : 0;
     a.softmax_scale = softmax_scale;
     a.status = nullptr;  // no caller memory to report device-side errors into
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
@@ -471,7 +473,7 @@ dsa_status_t dsa_decode_step_paged(const dsa_dims* dims, const void* q_I, const 
                                    void* stream, const dsa_stage_events* events) {
     if (dims == nullptr || cache == nullptr || cache->block_table == nullptr || cache->reserved != 0)
         return DSA_ERR_INVALID_ARG;
-    if (dims->idx_dtype != DSA_FP8_E4M3 || dims->kv_dtype != DSA_BF16) return DSA_ERR_UNSUPPORTED;
+    if (dims->idx_dtype != DSA_FP8_E4M3 || dims->kv_dtype == DSA_F32) return DSA_ERR_UNSUPPORTED;
     const int bs = cache->block_size;
     if (bs < 64 || (bs & (bs - 1)) != 0 || cache->num_blocks < 1 || cache->max_blocks < 1) return DSA_ERR_INVALID_ARG;
     if ((int64_t)cache->max_blocks * bs != dims->T_max) return DSA_ERR_INVALID_ARG;
@@ -503,7 +505,7 @@ dsa_status_t dsa_prefill(const dsa_dims* dims, const void* q_I, const float* q_s
     const int chunk = plan_prefill_chunk(dims);
     const size_t qi_row = (size_t)dims->H_I * dims->d_I * (fp8 ? 1 : 4);
     const size_t w_row = (size_t)dims->H_I * (fp8 ? 2 : 4);
-    const size_t kv_esz = dims->kv_dtype == DSA_BF16 ? 2 : 4;
+    const size_t kv_esz = dims->kv_dtype == DSA_F32 ? 4 : 2;  // q and out are bf16 unless the cache is f32
     const size_t q_row = (size_t)dims->H * dsa::kDK * kv_esz;
     const size_t o_row = (size_t)dims->H * dsa::kDV * kv_esz;
     for (int r0 = 0; r0 < dims->Nq; r0 += chunk) {

@@ -70,7 +70,13 @@ struct MlaArgs {
     // block_table[b * max_blocks + s / block_size] * block_size + s % block_size
     const int32_t* block_table;
     int block_size, max_blocks, num_blocks;
+    // FP8 latent cache: 656-byte entries of 512 e4m3 values, 4 fp32 scales (one per 128
+    // values) and the 64 rope values in bf16; dequantised to bf16 by the gather
+    int kv_fp8;
 };
+constexpr int kFp8EntryBytes = 656;  // 512 + 4 * 4 + 64 * 2
+constexpr int kFp8ScaleOff = 512;
+constexpr int kFp8RopeOff = 528;
 
 cudaError_t launch_indexer_fp8(const IndexerArgs& a, int grid, cudaStream_t st);
 // Same scores, four consecutive query rows per tensor-core pass: every group of four

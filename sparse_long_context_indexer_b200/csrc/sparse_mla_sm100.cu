@@ -52,6 +52,8 @@
 
 #include <mutex>
 
+#include <cuda_fp8.h>
+
 #include "kernels.h"
 #include "ptx.cuh"
 
@@ -160,6 +162,19 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (pb < 0 || pb >= a.num_blocks) return nullptr;
         return kv_base + ((int64_t)pb * a.block_size + s % a.block_size) * kDK;
     };
+    // the same for the 656-byte FP8 entries
+    const uint8_t* kv8_base = reinterpret_cast<const uint8_t*>(a.kv);
+    auto kv8_row = [&](int s) -> const uint8_t* {
+        int64_t row;
+        if (btab == nullptr) {
+            row = (int64_t)b * a.T_max + s;
+        } else {
+            const int pb = __ldg(btab + s / a.block_size);
+            if (pb < 0 || pb >= a.num_blocks) return nullptr;
+            row = (int64_t)pb * a.block_size + s % a.block_size;
+        }
+        return kv8_base + row * kFp8EntryBytes;
+    };
     // entry r of tile i -> selected token, -1 past the end of the split
     auto load_pos = [&](int i, int r) -> int {
         const int j = j_lo + i * kTileRows + r;
@@ -224,11 +239,107 @@ __global__ void __launch_bounds__(kThreads, 1)
         // (p >> 3) and (p >> 3) + 32 of each tile.
         auto prefetch_row = [&](int s) {
             if (valid(s)) {
-                const __nv_bfloat16* r = kv_row(s);
-                if (r) l2_prefetch_bulk(r, kDK * 2);
+                if (a.kv_fp8) {
+                    const uint8_t* r = kv8_row(s);
+                    if (r) l2_prefetch_bulk(r, kFp8EntryBytes);
+                } else {
+                    const __nv_bfloat16* r = kv_row(s);
+                    if (r) l2_prefetch_bulk(r, kDK * 2);
+                }
             }
         };
         if (pf_lane) prefetch_row(pf_first);
+        if (a.kv_fp8) {
+            // FP8 entries: thread p owns row p / 4 of each tile and its 128-value group p % 4:
+            // eight 16-byte loads of e4m3 codes and one scale into registers a tile ahead,
+            // dequantised to bf16 into the tile the MMAs read (chunks 2q and 2q + 1); the rope
+            // values (chunk 8) go by asynchronous copies.
+            const int r8 = p >> 2, q8 = p & 3;
+            uint4 lat[8];
+            float scl = 0.f;
+            bool has = false;
+            auto load_tile = [&](int i) {
+                const int s = load_pos(i, r8);
+                const uint8_t* row = valid(s) ? kv8_row(s) : nullptr;
+                if (valid(s) && row == nullptr && q8 == 0) record_status(a.status, DSA_STATUS_INDEX_OOB);
+                if (valid(s) == false && s != -1 && q8 == 0 && row_ok && half == 0)
+                    record_status(a.status, DSA_STATUS_INDEX_OOB);
+                has = row != nullptr;
+                if (has) {
+                    const uint4* src = reinterpret_cast<const uint4*>(row + q8 * 128);
+#pragma unroll
+                    for (int k = 0; k < 8; ++k) lat[k] = __ldg(src + k);
+                    scl = __ldg(reinterpret_cast<const float*>(row + kFp8ScaleOff) + q8);
+                }
+                return row;
+            };
+            const uint8_t* row_cur = load_tile(0);
+            for (int i = 0; i < ntiles; ++i) {
+                const int st = i % kStages;
+                const uint32_t stage = sKv + st * kKvStageBytes;
+                // rope: granules 2 q8 and 2 q8 + 1 of the row's 128 bytes, chunk 8
+#pragma unroll
+                for (int g2 = 0; g2 < 2; ++g2) {
+                    const int g = 2 * q8 + g2;
+                    const uint8_t* src = row_cur ? row_cur + kFp8RopeOff + 16 * g : kv8_base;
+                    cp_async16_zfill(stage + 8 * kChunkBytes + r8 * 128 + ((g ^ (r8 & 7)) << 4), src, row_cur ? 16u : 0u);
+                }
+                // dequantise this tile's codes (taken out of the registers before the next loads)
+                uint4 cur[8];
+                const float sc = scl;
+                const bool cur_has = has;
+#pragma unroll
+                for (int k = 0; k < 8; ++k) cur[k] = lat[k];
+                if (pf_lane && i + kPrefetchTiles < ntiles) prefetch_row(pf);
+                if (i + 1 < ntiles) {
+                    row_cur = load_tile(i + 1);
+                    if (pf_lane && i + 1 + kPrefetchTiles < ntiles) pf = load_pos(i + 1 + kPrefetchTiles, rr + 32 * half);
+                }
+#pragma unroll
+                for (int k = 0; k < 8; ++k) {
+                    // 16 codes = values 128 q8 + 16 k .. + 15: chunk 2 q8 + k / 4, granules 2 (k % 4), + 1
+                    const uint32_t w[4] = {cur[k].x, cur[k].y, cur[k].z, cur[k].w};
+                    uint32_t o[8];
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const __half2_raw lo = __nv_cvt_fp8x2_to_halfraw2((__nv_fp8x2_storage_t)(w[e] & 0xFFFFu), __NV_E4M3);
+                        const __half2_raw hi = __nv_cvt_fp8x2_to_halfraw2((__nv_fp8x2_storage_t)(w[e] >> 16), __NV_E4M3);
+                        const float2 flo = __half22float2(*reinterpret_cast<const __half2*>(&lo));
+                        const float2 fhi = __half22float2(*reinterpret_cast<const __half2*>(&hi));
+                        o[2 * e] = cur_has ? pack_bf16x2(flo.x * sc, flo.y * sc) : 0u;
+                        o[2 * e + 1] = cur_has ? pack_bf16x2(fhi.x * sc, fhi.y * sc) : 0u;
+                    }
+                    const int c = 2 * q8 + (k >> 2);
+#pragma unroll
+                    for (int g2 = 0; g2 < 2; ++g2) {
+                        const int g = 2 * (k & 3) + g2;
+                        asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(stage + c * kChunkBytes + r8 * 128 +
+                                                                                     ((g ^ (r8 & 7)) << 4)),
+                                     "r"(o[4 * g2]), "r"(o[4 * g2 + 1]), "r"(o[4 * g2 + 2]), "r"(o[4 * g2 + 3])
+                                     : "memory");
+                    }
+                }
+                // the tile is complete for this thread: its rope copies have landed and its stores are
+                // visible to the tensor cores
+                cp_async_wait_all();
+                fence_proxy_async_smem();
+                mbar_arrive(bar_kv_full(st));
+                if (i + 1 < ntiles) {
+                    const int nx = i + 1;
+                    bool ok = true;
+                    if (lane == 0) {
+                        if (nx == kQStage) {
+                            ok = mbar_wait_spin(bar_q, 0, abort_flag, a.status);
+                        } else if (nx >= kStages) {
+                            ok = mbar_wait_spin(bar_kv_empty(nx % kStages), ((nx / kStages) - 1) & 1, abort_flag,
+                                                a.status);
+                        }
+                    }
+                    ok = __shfl_sync(0xffffffffu, ok, 0);
+                    if (!ok) break;
+                }
+            }
+        } else
         for (int i = 0; i < ntiles; ++i) {
             const int st = i % kStages;
             if (gl == 0 && row_ok && half == 0 &&

@@ -94,6 +94,37 @@ def quantize_e4m3_per_row(x: torch.Tensor):
     return q.view(torch.uint8).reshape(x.shape), scale.float()
 
 
+FP8_ENTRY_BYTES = 656      # 512 e4m3 latent values, 4 fp32 scales, 64 bf16 rope values
+FP8_GROUP = 128            # latent values per scale
+
+
+def pack_fp8_latent(kv: torch.Tensor) -> torch.Tensor:
+    """The FP8 latent cache entry of kgptalkie "What Does the GPU Actually Run?": per token
+    512 e4m3 codes (four groups of 128, each scaled by its amax / 448, round-to-nearest-even),
+    the 4 fp32 scales, then the 64 rope values left in bf16.  kv: [..., 576] bf16 -> uint8
+    [..., 656].  Input preparation only: the hot path and the oracle receive the bytes."""
+    lead = kv.shape[:-1]
+    x = kv.reshape(-1, 576)
+    lat = x[:, :512].float().reshape(-1, 4, FP8_GROUP)
+    amax = lat.abs().amax(dim=2)
+    scale = torch.where(amax > 0, amax / FP8_MAX, torch.ones_like(amax)).float()
+    codes = (lat / scale[:, :, None]).clamp(-FP8_MAX, FP8_MAX).to(torch.float8_e4m3fn).view(torch.uint8)
+    out = torch.empty((x.shape[0], FP8_ENTRY_BYTES), dtype=torch.uint8, device=kv.device)
+    out[:, :512] = codes.reshape(-1, 512)
+    out[:, 512:528] = scale.contiguous().view(torch.uint8).reshape(-1, 16)
+    out[:, 528:] = x[:, 512:].contiguous().view(torch.uint8).reshape(-1, 128)
+    return out.reshape(*lead, FP8_ENTRY_BYTES)
+
+
+def with_fp8_latent(inp: "DSAInputs") -> "DSAInputs":
+    """The same workload with its latent cache in 656-byte FP8 entries (kv_dtype FP8)."""
+    out = DSAInputs(**{f: getattr(inp, f) for f in inp.__dataclass_fields__})
+    out.kv = pack_fp8_latent(inp.kv)
+    out.kv_dtype = FP8
+    out.name = inp.name + "_fp8kv"
+    return out
+
+
 def _unit(v: torch.Tensor) -> torch.Tensor:
     n = v.norm()
     return v / n if float(n) > 0 else v

@@ -113,6 +113,12 @@ def test_long_decode_16x128k_full_size(lib):
     check_decode_workload(g, full_rows=[0, 11], window_rows=[5])
 
 
+def test_long_decode_fp8_latent_full_size(lib):
+    # the long decode with its latent cache in 656-byte FP8 entries
+    g = inputs.with_fp8_latent(inputs.long_decode(device="cuda"))
+    check_decode_workload(g, full_rows=[3], window_rows=[])
+
+
 def test_decode_batch32_full_size(lib):
     g = inputs.decode32(device="cuda")
     check_decode_workload(g, full_rows=[0, 17, 31], window_rows=[])

@@ -251,6 +251,65 @@ def test_paged_decode_matches_contiguous(lib, block_size):
     assert torch.equal(out_p, out_c) and torch.equal(lse_p, lse_c)
 
 
+def test_fp8_latent_attention_matches_oracle(lib):
+    # the 656-byte FP8 latent entries, dequantised by the gather; random selections with -1
+    # tails, an empty row
+    inp = inputs.with_fp8_latent(small_decode(seed=81, lens=[5000, 5000, 300, 0], k=2048))
+    rng = np.random.default_rng(3)
+    idx = np.full((4, 2048), -1, np.int32)
+    idx[0] = np.sort(rng.choice(5000, 2048, replace=False))
+    idx[1, :1000] = np.sort(rng.choice(5000, 1000, replace=False))
+    idx[2, :300] = np.arange(300)
+    o_out, o_lse = oracle.sparse_attn(inp, idx)
+    g = inp.to("cuda")
+    dims = api.dims_of(g)
+    ws = api.make_workspace(dims, _lib.DSA_OP_SPARSE_MLA)
+    out, lse = api.alloc_outputs(g)
+    api.sparse_mla_attn(dims, g.q, g.kv, torch.from_numpy(idx).cuda(), g.q_seq, g.q_len, g.softmax_scale, out, lse, ws)
+    torch.cuda.synchronize()
+    assert api.get_device_status(ws) == 0
+    check_attention(out.float().cpu().numpy(), o_out, lse.cpu().numpy(), o_lse)
+    assert torch.all(out[3] == 0) and torch.all(torch.isneginf(lse[3]))
+
+
+def test_fp8_latent_decode_end_to_end(lib):
+    inp = inputs.with_fp8_latent(small_decode(seed=82))
+    sc_o, idx_o, out_o, lse_o = oracle.decode(inp)
+    scores, idx, out, lse, status = run_decode_gpu(inp.to("cuda"))
+    assert status == 0
+    check_scores(np_scores(scores), sc_o, inp.q_len.numpy())
+    same, total = check_sets(idx.cpu().numpy(), idx_o, sc_o, inp.q_len.numpy(), inp.k)
+    g_idx = idx.cpu().numpy()
+    rows = [t for t in range(inp.Nq) if np.array_equal(g_idx[t], idx_o[t])]
+    assert len(rows) >= max(1, total - 1)
+    check_attention(out.float().cpu().numpy(), out_o, lse.cpu().numpy(), lse_o, rows=rows)
+
+
+def test_fp8_latent_dense_and_paged(lib):
+    # the dense comparison and the paged cache read the same 656-byte entries
+    lens = [3000, 2049, 64, 1]
+    inp = inputs.with_fp8_latent(inputs.make_decode_inputs("fp8_paged", lens, T_max=3072, seed=83))
+    out_o, lse_o = oracle.dense_attn(inp)
+    g = inp.to("cuda")
+    dims = api.dims_of(g)
+    ws_d = api.make_workspace(dims, _lib.DSA_OP_DENSE_MLA)
+    out, lse = api.alloc_outputs(g)
+    api.dense_mla_attn(dims, g.q, g.kv, g.q_seq, g.q_len, g.softmax_scale, out, lse, ws_d)
+    ws = api.make_workspace(dims, _lib.DSA_OP_DECODE)
+    idx_c = torch.empty((len(lens), g.k), dtype=torch.int32, device="cuda")
+    out_c, lse_c = api.run_decode(g, ws=ws, idx_out=idx_c, dims=dims)
+    k_pool, s_pool, kv_pool, table = inputs.paged_layout(g, 64, seed=5)
+    cache = api.PagedCache(k_pool, s_pool, kv_pool, table, 64)
+    out_p, lse_p = api.alloc_outputs(g)
+    idx_p = torch.empty_like(idx_c)
+    api.decode_step_paged(dims, g.q_I, g.q_scale, g.w, cache, g.q, g.q_seq, g.q_len, g.softmax_scale, out_p, lse_p,
+                          ws, idx_out=idx_p)
+    torch.cuda.synchronize()
+    assert api.get_device_status(ws_d) == 0 and api.get_device_status(ws) == 0
+    check_attention(out.float().cpu().numpy(), out_o, lse.cpu().numpy(), lse_o)
+    assert torch.equal(idx_p, idx_c) and torch.equal(out_p, out_c) and torch.equal(lse_p, lse_c)
+
+
 def test_prefill_matches_oracle(lib):
     L = 3000
     inp = inputs.make_prefill_inputs("prefill_small", L, seed=7)

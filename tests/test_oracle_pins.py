@@ -350,3 +350,50 @@ def test_attention_rejects_index_beyond_causal_length():
     inp = ns_attn(q, kv, [10, 10], 0.1)
     with pytest.raises(ValueError):
         oracle.sparse_attn(inp, np.array([[10], [0]], np.int32))
+
+
+# ------------------------------------------------------------------ FP8 latent cache entry
+
+def _entry(codes, scales, rope_bits):
+    e = np.zeros(656, np.uint8)
+    e[:512] = codes
+    e[512:528] = np.asarray(scales, np.float32).view(np.uint8)
+    e[528:] = np.asarray(rope_bits, np.uint16).view(np.uint8)
+    return e
+
+
+def test_fp8_latent_entry_hand_decoded():
+    # kgptalkie "What Does the GPU Actually Run?": 512 e4m3 values, 4 fp32 scales, 64 bf16 rope
+    # values.  Codes by the format definition: 0x38 = 1.0, 0x40 = 2.0, 0xB8 = -1.0,
+    # 0x01 = 2^-9 (smallest subnormal), 0x7E = 448; group g = values [128 g, 128 g + 128).
+    codes = np.zeros(512, np.uint8)
+    codes[0], codes[127] = 0x38, 0x40          # group 0, scale 0.5
+    codes[128], codes[255] = 0xB8, 0x01        # group 1, scale 2.0
+    codes[256] = 0x7E                          # group 2, scale 1.0
+    codes[511] = 0x38                          # group 3, scale 0.25
+    rope = np.zeros(64, np.uint16)
+    rope[0], rope[63] = 0x3FC0, 0xC020         # bf16 1.5, -2.5
+    d = oracle.dequant_latent_fp8(_entry(codes, [0.5, 2.0, 1.0, 0.25], rope)[None])[0]
+    want = np.zeros(576)
+    want[0], want[127] = 0.5, 1.0
+    want[128], want[255] = -2.0, 2.0 * 2.0 ** -9
+    want[256] = 448.0
+    want[511] = 0.25
+    want[512], want[575] = 1.5, -2.5
+    assert np.array_equal(d.astype(np.float64), want)
+
+
+def test_fp8_latent_round_trip_within_e4m3_half_ulp():
+    # quantise a bf16 latent cache (input preparation) and decode it with the oracle: every
+    # latent value is within half an e4m3 step of the original (relative 2^-4 for normals,
+    # 2^-10 of the group scale in the subnormal range); rope values are untouched
+    from sparse_long_context_indexer_b200 import inputs
+    inp = inputs.make_decode_inputs("fp8_round_trip", [500, 130], T_max=512, seed=9)
+    entries = inputs.pack_fp8_latent(inp.kv)
+    d = oracle.dequant_latent_fp8(entries).astype(np.float64)
+    ref = inp.kv.float().numpy().astype(np.float64)
+    scales = entries[..., 512:528].contiguous().view(torch.float32).numpy().astype(np.float64)
+    s_of = np.repeat(scales, 128, axis=-1)
+    bound = np.maximum(2.0 ** -4 * np.abs(ref[..., :512]), 2.0 ** -10 * s_of)
+    assert np.all(np.abs(d[..., :512] - ref[..., :512]) <= bound * (1 + 1e-6))
+    assert np.array_equal(d[..., 512:], ref[..., 512:])
