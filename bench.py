@@ -691,8 +691,9 @@ def launches_per_step():
 
 def measure_e2e(inp, dims, ws, dev, steps, warmup):
     """End to end through the public API, as a serving loop would run it.  Per step:
-    one H2D copy of all of the step's inputs (query-side tensors and the new token's
-    cache entries, packed in one pinned buffer), the cache append, the decode step,
+    one H2D copy of all of the step's inputs (query-side tensors, the new token's position,
+    bf16 latent row and fp32 indexer key, packed in one pinned buffer), the cache append
+    (dsa_append_tokens, which quantises the key on the device), the decode step,
     and the D2H copy of out and lse.  Two buffer slots on separate copy-in, compute and
     copy-out streams: the copies of step i+1 and step i-1 overlap the compute of step
     i; each step's append and decode stay in order on the compute stream.  Each stage
@@ -702,10 +703,13 @@ def measure_e2e(inp, dims, ws, dev, steps, warmup):
     from sparse_long_context_indexer_b200 import api
     B = inp.B
     pos = (inp.q_len - 1).long()
+    rows = torch.arange(B, device=dev)
+    # the new token of each sequence: its bf16 latent row and its fp32 indexer key (the
+    # library quantises it on the device), written at position q_len - 1
+    k_new = inp.k_I[rows, pos].view(torch.float8_e4m3fn).float() * inp.k_scale[rows, pos][:, None]
     fields = {
         "q": inp.q, "q_I": inp.q_I, "q_scale": inp.q_scale, "w": inp.w, "q_len": inp.q_len,
-        "kv_new": inp.kv[torch.arange(B, device=dev), pos], "k_new": inp.k_I[torch.arange(B, device=dev), pos],
-        "ks_new": inp.k_scale[torch.arange(B, device=dev), pos],
+        "pos": pos.to(torch.int32), "kv_new": inp.kv[rows, pos], "k_new": k_new,
     }
     offs, off = {}, 0
     for k, v in fields.items():
@@ -731,16 +735,15 @@ def measure_e2e(inp, dims, ws, dev, steps, warmup):
         slots[0]["lse_h"].numel() * slots[0]["lse_h"].element_size()
     s_in, s_out = torch.cuda.Stream(device=dev), torch.cuda.Stream(device=dev)
     s_c = torch.cuda.current_stream(dev)
-    bidx = torch.arange(B, device=dev)
 
     def copy_in(sl):
         sl["dbuf"].copy_(host_pack, non_blocking=True)
 
+    seq = torch.arange(B, dtype=torch.int32, device=dev)
+
     def compute(sl):
         v = sl["v"]
-        inp.kv[bidx, pos] = v["kv_new"]
-        inp.k_I[bidx, pos] = v["k_new"]
-        inp.k_scale[bidx, pos] = v["ks_new"]
+        api.append_tokens(dims, seq, v["pos"], v["kv_new"], v["k_new"], inp.kv, inp.k_I, inp.k_scale, ws=ws)
         api.decode_step(dims, v["q_I"], v["q_scale"], v["w"], inp.k_I, inp.k_scale, v["q"], inp.kv, inp.q_seq,
                         v["q_len"], inp.softmax_scale, sl["out"], sl["lse"], ws)
 

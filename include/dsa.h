@@ -259,6 +259,25 @@ dsa_status_t dsa_decode_step_paged(const dsa_dims* dims,
                                    void* workspace, size_t ws_bytes, void* stream,
                                    const dsa_stage_events* events);
 
+/* Write n new tokens into the caches (kgptalkie, "What Does the Whole Block
+ * Look Like?": on the precise path the token is compressed and written to the
+ * KV cache; "What Does the GPU Actually Run?": FP8 entries with fp32 scales).
+ * Token i goes to sequence seq[i], position pos[i] (0 <= pos < T_max):
+ *   k_new [n, d_I] fp32 -> with idx_dtype DSA_FP8_E4M3, e4m3 codes of
+ *       k_new / s, s = max|k_new| / 448 (1 if all zero), round to nearest even,
+ *       clamped to +-448, into k_I, and s into k_scale; with DSA_F32 copied;
+ *   kv_new [n, 576] bf16 -> copied (kv_dtype DSA_BF16) or packed into the
+ *       656-byte FP8 entry (kv_dtype DSA_FP8_E4M3: each 128-value latent group
+ *       quantised like the key with its own scale; rope values copied).
+ * paged == NULL: kv, k_I, k_scale are the contiguous caches ([B, T_max, ..]);
+ * otherwise the pools and block table of *paged are used and kv, k_I,
+ * k_scale are ignored.  A token whose sequence or position is out of range,
+ * or whose block id is outside the pool, is skipped and recorded in the
+ * workspace's status word (workspace may be NULL).  n <= 65535. */
+dsa_status_t dsa_append_tokens(const dsa_dims* dims, int32_t n, const int32_t* seq, const int32_t* pos,
+                               const void* kv_new, const float* k_new, void* kv, void* k_I, float* k_scale,
+                               const dsa_paged_cache* paged, void* workspace, size_t ws_bytes, void* stream);
+
 /* Prefill: the same three stages for many query rows of ONE sequence (every
  * position of a prompt), processed in row chunks so the transient score rows
  * fit the workspace (size it for DSA_OP_PREFILL).  Semantics per row are

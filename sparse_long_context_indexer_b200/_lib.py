@@ -22,7 +22,7 @@ DSA_OP_INDEXER, DSA_OP_TOPK, DSA_OP_SPARSE_MLA, DSA_OP_DECODE, DSA_OP_PREFILL, D
 EXPORTS = (
     "dsa_workspace_size", "dsa_workspace_init", "dsa_indexer_scores", "dsa_prefill_indexer_scores", "dsa_topk",
     "dsa_sparse_mla_attn", "dsa_dense_mla_attn",
-    "dsa_decode_step", "dsa_decode_step_paged", "dsa_prefill", "dsa_get_device_status", "dsa_status_string", "dsa_last_cuda_error",
+    "dsa_decode_step", "dsa_decode_step_paged", "dsa_append_tokens", "dsa_prefill", "dsa_get_device_status", "dsa_status_string", "dsa_last_cuda_error",
     "dsa_selftest_wait_timeout", "dsa_version", "dsa_sparse_mla_attn_noalloc",
 )
 
@@ -77,13 +77,16 @@ def _declare(lib):
     lib.dsa_decode_step.argtypes = [D, P, P, P, P, P, P, P, P, P, F, P, P, P, P, P, S, P,
                                     ctypes.POINTER(DsaStageEvents)]
     lib.dsa_prefill.argtypes = [D, P, P, P, P, P, P, P, P, P, F, P, P, P, P, S, P]
+    lib.dsa_append_tokens.argtypes = [D, ctypes.c_int32, P, P, P, P, P, P, P, ctypes.POINTER(DsaPagedCache), P,
+                                       S, P]
     lib.dsa_decode_step_paged.argtypes = [D, P, P, P, ctypes.POINTER(DsaPagedCache), P, P, P, F, P, P, P, P, P, S,
                                           P, ctypes.POINTER(DsaStageEvents)]
     lib.dsa_get_device_status.argtypes = [P, P, ctypes.POINTER(I32)]
     lib.dsa_selftest_wait_timeout.argtypes = [P, S, I32, P]
     for name in ("dsa_workspace_size", "dsa_workspace_init", "dsa_indexer_scores", "dsa_prefill_indexer_scores",
                  "dsa_topk",
-                 "dsa_sparse_mla_attn", "dsa_decode_step", "dsa_decode_step_paged", "dsa_prefill",
+                 "dsa_sparse_mla_attn", "dsa_decode_step", "dsa_decode_step_paged", "dsa_append_tokens",
+                 "dsa_prefill",
                  "dsa_get_device_status",
                  "dsa_selftest_wait_timeout", "dsa_sparse_mla_attn_noalloc", "dsa_dense_mla_attn"):
         getattr(lib, name).restype = st

@@ -151,6 +151,19 @@ class PagedCache:
                                   self.block_size, self.kv.shape[0], self.block_table.shape[1], 0)
 
 
+def append_tokens(dims: Dims, seq, pos, kv_new, k_new, kv=None, k_I=None, k_scale=None,
+                  cache: Optional["PagedCache"] = None, ws=None):
+    """Write new tokens (bf16 latent rows, fp32 indexer keys) into the caches, quantising as
+    the caches' types require; contiguous caches (kv, k_I, k_scale) or a paged cache."""
+    lib = _lib.load()
+    d = dims.c()
+    pc = cache.c() if cache is not None else None
+    rc = lib.dsa_append_tokens(ctypes.byref(d), int(seq.numel()), _ptr(seq), _ptr(pos), _ptr(kv_new), _ptr(k_new),
+                               _ptr(kv), _ptr(k_I), _ptr(k_scale), ctypes.byref(pc) if pc is not None else None,
+                               _ptr(ws), 0 if ws is None else ws.numel(), _stream_ptr())
+    _lib.check(lib, rc, "dsa_append_tokens")
+
+
 def decode_step_paged(dims: Dims, q_I, q_scale, w, cache: PagedCache, q, q_seq, q_len, softmax_scale, out, lse, ws,
                       scores_out=None, idx_out=None):
     """One decode step over a paged cache on torch's current stream."""

@@ -528,6 +528,52 @@ dsa_status_t dsa_prefill(const dsa_dims* dims, const void* q_I, const float* q_s
     return DSA_OK;
 }
 
+dsa_status_t dsa_append_tokens(const dsa_dims* dims, int32_t n, const int32_t* seq, const int32_t* pos,
+                               const void* kv_new, const float* k_new, void* kv, void* k_I, float* k_scale,
+                               const dsa_paged_cache* paged, void* workspace, size_t ws_bytes, void* stream) {
+    dsa_status_t s = check_dims(dims, true, true);
+    if (s != DSA_OK) return s;
+    if (n < 0 || n > 65535) return n < 0 ? DSA_ERR_INVALID_ARG : DSA_ERR_UNSUPPORTED;
+    if (n == 0) return DSA_OK;
+    const bool fp8 = dims->idx_dtype == DSA_FP8_E4M3;
+    if (dims->kv_dtype == DSA_F32) return DSA_ERR_UNSUPPORTED;
+    if (paged != nullptr) {
+        if (paged->block_table == nullptr || paged->reserved != 0) return DSA_ERR_INVALID_ARG;
+        const int bs = paged->block_size;
+        if (bs < 64 || (bs & (bs - 1)) != 0 || paged->num_blocks < 1 ||
+            (int64_t)paged->max_blocks * bs != dims->T_max)
+            return DSA_ERR_INVALID_ARG;
+        kv = const_cast<void*>(paged->kv);
+        k_I = const_cast<void*>(paged->k_I);
+        k_scale = const_cast<float*>(paged->k_scale);
+    }
+    if (!seq || !pos || !kv_new || !k_new || !kv || !k_I || (fp8 && !k_scale)) return DSA_ERR_INVALID_ARG;
+    if (workspace != nullptr && ws_bytes < kStatusBytes) return DSA_ERR_WORKSPACE;
+    dsa::AppendArgs a{};
+    a.n = n;
+    a.seq = seq;
+    a.pos = pos;
+    a.kv_new = kv_new;
+    a.k_new = k_new;
+    a.kv = kv;
+    a.k_I = k_I;
+    a.k_scale = k_scale;
+    a.B = dims->B;
+    a.T_max = dims->T_max;
+    a.d_I = dims->d_I;
+    a.idx_fp8 = fp8 ? 1 : 0;
+    a.kv_fp8 = dims->kv_dtype == DSA_FP8_E4M3 ? 1 : 0;
+    if (paged != nullptr) {
+        a.block_table = paged->block_table;
+        a.block_size = paged->block_size;
+        a.max_blocks = paged->max_blocks;
+        a.num_blocks = paged->num_blocks;
+    }
+    a.status = workspace ? status_word(workspace) : nullptr;
+    const cudaError_t e = dsa::launch_append_tokens(a, reinterpret_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? DSA_OK : cuda_fail(e);
+}
+
 dsa_status_t dsa_get_device_status(void* workspace, void* stream, int32_t* status) {
     if (workspace == nullptr || status == nullptr) return DSA_ERR_INVALID_ARG;
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);

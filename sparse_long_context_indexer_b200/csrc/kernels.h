@@ -78,6 +78,24 @@ constexpr int kFp8EntryBytes = 656;  // 512 + 4 * 4 + 64 * 2
 constexpr int kFp8ScaleOff = 512;
 constexpr int kFp8RopeOff = 528;
 
+// New tokens into the caches (contiguous when block_table is null, else pools of blocks).
+struct AppendArgs {
+    int n;                     // new tokens
+    const int32_t* seq;        // [n] sequence of token i
+    const int32_t* pos;        // [n] its position
+    const void* kv_new;        // [n, 576] bf16 latent rows
+    const float* k_new;        // [n, d_I] fp32 indexer keys
+    void* kv;                  // latent cache: [.., 576] bf16 or [.., 656] FP8 entries
+    void* k_I;                 // indexer keys: e4m3 codes (idx_fp8) or fp32
+    float* k_scale;            // per-token key scales (idx_fp8)
+    int B, T_max, d_I;
+    int idx_fp8, kv_fp8;
+    const int32_t* block_table;
+    int block_size, max_blocks, num_blocks;
+    int* status;
+};
+cudaError_t launch_append_tokens(const AppendArgs& a, cudaStream_t st);
+
 cudaError_t launch_indexer_fp8(const IndexerArgs& a, int grid, cudaStream_t st);
 // Same scores, four consecutive query rows per tensor-core pass: every group of four
 // rows (row 4u .. 4u+3) must belong to one sequence (prefill).

@@ -310,6 +310,61 @@ def test_fp8_latent_dense_and_paged(lib):
     assert torch.equal(idx_p, idx_c) and torch.equal(out_p, out_c) and torch.equal(lse_p, lse_c)
 
 
+@pytest.mark.parametrize("fp8_latent", [False, True])
+def test_append_tokens_matches_the_input_quantisers(lib, fp8_latent):
+    # kgptalkie "What Does the Whole Block Look Like?": the new token is compressed and written to
+    # the cache.  The device's bytes must equal the input preparation's (torch's RNE e4m3 cast:
+    # keys with one scale per token, the latent in four 128-value groups); a token at an
+    # out-of-range position is skipped and reported.
+    lens = [700, 300, 129]
+    inp = inputs.make_decode_inputs("append", lens, T_max=768, seed=91)
+    if fp8_latent:
+        inp = inputs.with_fp8_latent(inp)
+    g = inp.to("cuda")
+    dims = api.dims_of(g)
+    ws = api.make_workspace(dims, _lib.DSA_OP_DECODE)
+    gen = torch.Generator().manual_seed(5)
+    seq = torch.tensor([0, 1, 2, 1, 2], dtype=torch.int32)
+    pos = torch.tensor([700, 10, 128, 767, 768], dtype=torch.int32)   # the last is out of range
+    k_new = torch.randn((5, g.d_I), generator=gen) / 8
+    k_new[2] = 0.0                                                   # all-zero key: scale 1
+    kv_new = (torch.randn((5, 576), generator=gen) / 8).to(torch.bfloat16)
+    # contiguous caches
+    kv, k_I, k_scale = g.kv.clone(), g.k_I.clone(), g.k_scale.clone()
+    api.append_tokens(dims, seq.cuda(), pos.cuda(), kv_new.cuda(), k_new.cuda(), kv, k_I, k_scale, ws=ws)
+    torch.cuda.synchronize()
+    assert api.get_device_status(ws) == _lib.DSA_ERR_LENGTH
+    codes, scales = inputs.quantize_e4m3_per_row(k_new)
+    want_kv = inputs.pack_fp8_latent(kv_new) if fp8_latent else kv_new
+    for i in range(4):
+        b, s_ = int(seq[i]), int(pos[i])
+        assert torch.equal(k_I[b, s_].cpu(), codes[i]), f"token {i}: key codes"
+        assert float(k_scale[b, s_]) == float(scales[i]), f"token {i}: key scale"
+        assert torch.equal(kv[b, s_].cpu(), want_kv[i]), f"token {i}: latent entry"
+    # everything else is untouched
+    mask = torch.ones(kv.shape[:2], dtype=torch.bool)
+    for i in range(4):
+        mask[int(seq[i]), int(pos[i])] = False
+    assert torch.equal(kv.cpu()[mask], g.kv.cpu()[mask]) and torch.equal(k_I.cpu()[mask], g.k_I.cpu()[mask])
+    # the same appends into the paged form of the original cache
+    k_pool, s_pool, kv_pool, table = inputs.paged_layout(g, 64, seed=2)
+    full = table.clone()
+    free = [p_ for p_ in range(kv_pool.shape[0]) if p_ not in set(table[table >= 0].tolist())]
+    for b in range(3):                        # blocks for every position the appends may touch
+        for j in range(full.shape[1]):
+            if full[b, j] < 0:
+                full[b, j] = free.pop()
+    cache = api.PagedCache(k_pool, s_pool, kv_pool, full.cuda(), 64)
+    api.append_tokens(dims, seq.cuda(), pos.cuda(), kv_new.cuda(), k_new.cuda(), cache=cache, ws=ws)
+    torch.cuda.synchronize()
+    assert api.get_device_status(ws) == _lib.DSA_ERR_LENGTH
+    for i in range(4):
+        b, s_ = int(seq[i]), int(pos[i])
+        pr = int(full[b, s_ // 64]), s_ % 64
+        assert torch.equal(k_pool[pr].cpu(), codes[i]) and float(s_pool[pr]) == float(scales[i])
+        assert torch.equal(kv_pool[pr].cpu(), want_kv[i])
+
+
 def test_prefill_matches_oracle(lib):
     L = 3000
     inp = inputs.make_prefill_inputs("prefill_small", L, seed=7)
