@@ -87,9 +87,10 @@ MlaPlan plan_mla(const dsa_dims* d, int nq) {
     return p;
 }
 
-int plan_topk_cluster(const dsa_dims* d, int nq) {
+int plan_topk_cluster(const dsa_dims* d, int nq, int64_t row_len_hint = 0) {
     const int sms = device_sms();
-    const int64_t rowmax = d->ld_scores < d->T_max ? d->ld_scores : d->T_max;
+    int64_t rowmax = d->ld_scores < d->T_max ? d->ld_scores : d->T_max;
+    if (row_len_hint > 0 && row_len_hint < rowmax) rowmax = row_len_hint;
     int c = (int)((rowmax + dsa::kTopkSmemKeys - 1) / dsa::kTopkSmemKeys);
     const int fill = nq > 0 ? sms / nq : 8;
     if (fill > c) c = fill;
@@ -191,7 +192,7 @@ dsa_status_t run_indexer(const dsa_dims* d, int nq, const void* q_I, const float
 }
 
 dsa_status_t run_topk(const dsa_dims* d, int nq, const float* scores, const int32_t* q_len, int32_t* idx, int* status,
-                      cudaStream_t st, bool pdl = false) {
+                      cudaStream_t st, bool pdl = false, int64_t row_len_hint = 0) {
     dsa::TopkArgs a{};
     a.scores = scores;
     a.ld = d->ld_scores;
@@ -202,7 +203,8 @@ dsa_status_t run_topk(const dsa_dims* d, int nq, const float* scores, const int3
     a.T_max = d->T_max;
     a.status = status;
     a.pdl = pdl ? 1 : 0;
-    cudaError_t e = dsa::launch_topk(a, plan_topk_cluster(d, nq), st);
+    a.row_len_hint = row_len_hint;
+    cudaError_t e = dsa::launch_topk(a, plan_topk_cluster(d, nq, row_len_hint), st);
     return e == cudaSuccess ? DSA_OK : cuda_fail(e);
 }
 
@@ -518,7 +520,9 @@ dsa_status_t dsa_prefill(const dsa_dims* dims, const void* q_I, const float* q_s
         s = run_indexer(dims, nq, qi, qs, wr, k_I, k_scale, q_seq + r0, q_len + r0, scores, status, st, true,
                         dims->k);
         if (s != DSA_OK) return s;
-        s = run_topk(dims, nq, scores, q_len + r0, idx, status, st, true);
+        // a causal prompt's rows r0 .. r0 + nq - 1 hold at most r0 + nq positions: the top-k's
+        // clusters and slices are planned for that (longer rows stay correct, only slower)
+        s = run_topk(dims, nq, scores, q_len + r0, idx, status, st, true, (int64_t)r0 + nq);
         if (s != DSA_OK) return s;
         s = run_mla(dims, nq, static_cast<const char*>(q) + r0 * q_row, kv, idx, q_seq + r0, q_len + r0,
                     softmax_scale, static_cast<char*>(out) + r0 * o_row, lse ? lse + (size_t)r0 * dims->H : nullptr,

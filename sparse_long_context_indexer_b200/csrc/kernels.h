@@ -46,6 +46,9 @@ struct TopkArgs {
     int Nq, k, T_max;
     int* status;
     int pdl;  // launch as a programmatic dependent of the previous kernel (the library's own pipelines)
+    // expected longest row (0: ld / T_max): sizes the cluster and each CTA's shared-memory slice;
+    // a longer row stays correct (its slices beyond the cached size are read from global memory)
+    int64_t row_len_hint;
 };
 
 struct MlaArgs {

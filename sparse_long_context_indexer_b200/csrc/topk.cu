@@ -677,7 +677,8 @@ __global__ void __launch_bounds__(kThreads, 2) topk_radix_kernel(const TopkArgs 
 cudaError_t launch_topk(const TopkArgs& a, int cluster, cudaStream_t st) {
     if (a.Nq == 0) return cudaSuccess;
     if (cluster < 1 || cluster > kMaxCluster) return cudaErrorInvalidValue;
-    const int64_t row_max = a.ld < (int64_t)a.T_max ? a.ld : (int64_t)a.T_max;
+    int64_t row_max = a.ld < (int64_t)a.T_max ? a.ld : (int64_t)a.T_max;
+    if (a.row_len_hint > 0 && a.row_len_hint < row_max) row_max = a.row_len_hint;
     int64_t chunk = (row_max + cluster - 1) / cluster;
     chunk = (chunk + 3) & ~int64_t(3);
     const int cap = (int)(chunk < kTopkSmemKeys ? chunk : kTopkSmemKeys);
