@@ -449,8 +449,8 @@ def run_prefill(args):
         api.prefill_indexer_scores(d, g.q_I[r0:r1], g.q_scale[r0:r1], g.w[r0:r1], g.k_I, g.k_scale, g.q_seq[r0:r1],
                                    g.q_len[r0:r1], scores, cws)
         e[1].record()
-        # a causal chunk's rows hold at most r1 positions: the same bound dsa_prefill plans its top-k with
-        api.topk(dataclasses.replace(d, T_max=r1), scores, g.q_len[r0:r1], cidx, cws)
+        # the chunk's rows hold at most (T_max - L) + r1 positions: the bound dsa_prefill plans its top-k with
+        api.topk(dataclasses.replace(d, T_max=g.T_max - L + r1), scores, g.q_len[r0:r1], cidx, cws)
         e[2].record()
         api.sparse_mla_attn(d, g.q[r0:r1], g.kv, cidx, g.q_seq[r0:r1], g.q_len[r0:r1], g.softmax_scale,
                             out[r0:r1], lse[r0:r1], cws)

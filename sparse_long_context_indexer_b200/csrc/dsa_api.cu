@@ -520,9 +520,12 @@ dsa_status_t dsa_prefill(const dsa_dims* dims, const void* q_I, const float* q_s
         s = run_indexer(dims, nq, qi, qs, wr, k_I, k_scale, q_seq + r0, q_len + r0, scores, status, st, true,
                         dims->k);
         if (s != DSA_OK) return s;
-        // a causal prompt's rows r0 .. r0 + nq - 1 hold at most r0 + nq positions: the top-k's
-        // clusters and slices are planned for that (longer rows stay correct, only slower)
-        s = run_topk(dims, nq, scores, q_len + r0, idx, status, st, true, (int64_t)r0 + nq);
+        // prompt rows at the end of the cache (a causal prompt, or a chunk of one after a cached
+        // context: q_len[t] = T_max - Nq + t + 1 at most) hold at most T_max - Nq + r0 + nq
+        // positions in rows r0 .. r0 + nq - 1; the top-k's clusters and slices are planned for
+        // that (a longer row stays correct, only slower)
+        const int64_t before = dims->T_max > dims->Nq ? (int64_t)dims->T_max - dims->Nq : 0;
+        s = run_topk(dims, nq, scores, q_len + r0, idx, status, st, true, before + r0 + nq);
         if (s != DSA_OK) return s;
         s = run_mla(dims, nq, static_cast<const char*>(q) + r0 * q_row, kv, idx, q_seq + r0, q_len + r0,
                     softmax_scale, static_cast<char*>(out) + r0 * o_row, lse ? lse + (size_t)r0 * dims->H : nullptr,

@@ -391,6 +391,32 @@ def test_prefill_matches_oracle(lib):
             assert np.array_equal(g_idx[i][: t + 1], np.arange(t + 1)) and np.all(g_idx[i][t + 1:] == -1)
 
 
+def test_prefill_chunk_after_a_cached_context_matches_oracle(lib):
+    # the last 1,200 rows of a 7,200-token prompt (a prefill chunk after 6,000 cached tokens):
+    # rows hold 6,001..7,200 positions, far more than the chunk's own row count
+    offset, L = 6000, 1200
+    rows_all = list(range(offset, offset + L))
+    inp = inputs.make_prefill_inputs("prefill_after_ctx", offset + L, seed=9, rows=rows_all)
+    pick = np.r_[0:4, 597:601, 1196:1200]
+    sub = inputs.make_prefill_inputs("prefill_after_ctx", offset + L, seed=9, rows=[rows_all[i] for i in pick])
+    sc_o, idx_o, out_o, lse_o = oracle.decode(sub)
+    g = inp.to("cuda")
+    dims = api.dims_of(g)
+    assert dims.Nq == L and int(inp.q_len.min()) == offset + 1
+    ws = api.make_workspace(dims, _lib.DSA_OP_PREFILL)
+    out, lse = api.alloc_outputs(g)
+    idx = torch.empty((L, g.k), dtype=torch.int32, device="cuda")
+    api.prefill(dims, g.q_I, g.q_scale, g.w, g.k_I, g.k_scale, g.q, g.kv, g.q_seq, g.q_len, g.softmax_scale,
+                out, lse, ws, idx_out=idx)
+    torch.cuda.synchronize()
+    assert api.get_device_status(ws) == 0
+    g_idx = idx.cpu().numpy()[pick]
+    check_sets(g_idx, idx_o, sc_o, sub.q_len.numpy(), sub.k)
+    same = [i for i in range(len(pick)) if np.array_equal(g_idx[i], idx_o[i])]
+    assert len(same) >= len(pick) - 2
+    check_attention(out.float().cpu().numpy()[pick], out_o, lse.cpu().numpy()[pick], lse_o, rows=same)
+
+
 def oracle_scores_of_rows(inp, rows):
     """Oracle indexer scores of the given query rows (whole rows, ld = the longest)."""
     r = torch.as_tensor(list(rows), dtype=torch.long)
