@@ -101,3 +101,72 @@ def test_python_layer_has_no_compute_fallback():
     src = open(os.path.join(ROOT, "sparse_long_context_indexer_b200", "api.py")).read()
     for forbidden in ("torch.topk", "torch.softmax", "torch.einsum", "torch.matmul", "@ ", "relu", "oracle"):
         assert forbidden not in src, forbidden
+
+
+def _paged(block_size=64, max_blocks=2048, num_blocks=4096, k_scale=1 << 20, table=1 << 21, reserved=0):
+    return _lib.DsaPagedCache(k_I=1 << 20, k_scale=k_scale, kv=1 << 22, block_table=table, block_size=block_size,
+                              num_blocks=num_blocks, max_blocks=max_blocks, reserved=reserved)
+
+
+@pytest.mark.parametrize("case,code", [
+    (dict(n=-1), _lib.DSA_ERR_INVALID_ARG),
+    (dict(n=70000), _lib.DSA_ERR_UNSUPPORTED),
+    (dict(seq=None), _lib.DSA_ERR_INVALID_ARG),
+    (dict(k_scale=None), _lib.DSA_ERR_INVALID_ARG),
+    (dict(paged=_paged(block_size=48)), _lib.DSA_ERR_INVALID_ARG),
+    (dict(paged=_paged(max_blocks=1000)), _lib.DSA_ERR_INVALID_ARG),
+    (dict(paged=_paged(reserved=1)), _lib.DSA_ERR_INVALID_ARG),
+    (dict(dims=dict(kv_dtype=_lib.DSA_F32)), _lib.DSA_ERR_UNSUPPORTED),
+    (dict(ws_bytes=64), _lib.DSA_ERR_WORKSPACE),
+    (dict(n=0), _lib.DSA_OK),
+])
+def test_append_tokens_host_checks(lib, case, code):
+    P = 1 << 20
+    d = decode_dims(**case.get("dims", {})).c()
+    paged = case.get("paged")
+    rc = lib.dsa_append_tokens(ctypes.byref(d), case.get("n", 4), case.get("seq", P), P, P, P, P, P,
+                               case.get("k_scale", P), ctypes.byref(paged) if paged is not None else None, P,
+                               case.get("ws_bytes", 256), None)
+    assert rc == code
+
+
+@pytest.mark.parametrize("case,code", [
+    (dict(cache=None), _lib.DSA_ERR_INVALID_ARG),
+    (dict(cache=_paged(table=None)), _lib.DSA_ERR_INVALID_ARG),
+    (dict(cache=_paged(block_size=96)), _lib.DSA_ERR_INVALID_ARG),
+    (dict(cache=_paged(block_size=32, max_blocks=4096)), _lib.DSA_ERR_INVALID_ARG),
+    (dict(cache=_paged(max_blocks=1024)), _lib.DSA_ERR_INVALID_ARG),
+    (dict(cache=_paged(k_scale=(1 << 20) + 4)), _lib.DSA_ERR_INVALID_ARG),
+    (dict(cache=_paged(), dims=dict(idx_dtype=_lib.DSA_F32)), _lib.DSA_ERR_UNSUPPORTED),
+    (dict(cache=_paged(), ws_bytes=1024), _lib.DSA_ERR_WORKSPACE),
+])
+def test_paged_decode_host_checks(lib, case, code):
+    P = 1 << 20
+    d = decode_dims(**case.get("dims", {})).c()
+    cache = case["cache"]
+    rc = lib.dsa_decode_step_paged(ctypes.byref(d), P, P, P, ctypes.byref(cache) if cache is not None else None, P,
+                                   P, P, ctypes.c_float(0.07), P, P, None, None, P, case.get("ws_bytes", 1 << 30),
+                                   None, None)
+    assert rc == code
+
+
+def test_dense_and_prefill_host_checks(lib):
+    P = 1 << 20
+    d = decode_dims().c()
+    # dense attention: NULL query, then a workspace below its plan
+    assert lib.dsa_dense_mla_attn(ctypes.byref(d), None, P, P, P, ctypes.c_float(0.07), P, P, P, 1 << 30,
+                                  None) == _lib.DSA_ERR_INVALID_ARG
+    assert lib.dsa_dense_mla_attn(ctypes.byref(d), P, P, P, P, ctypes.c_float(0.07), P, P, P, 16,
+                                  None) == _lib.DSA_ERR_WORKSPACE
+    # prefill: misaligned w, non-finite scale, an empty batch (no launch)
+    one = decode_dims(B=1, Nq=4096, T_max=4096, ld_scores=4096).c()
+    args = [P, P, P, P, P, P, P, P, P]
+    bad = list(args)
+    bad[2] = P + 2
+    assert lib.dsa_prefill(ctypes.byref(one), *bad, ctypes.c_float(0.07), P, P, None, P, 1 << 30,
+                           None) == _lib.DSA_ERR_INVALID_ARG
+    assert lib.dsa_prefill(ctypes.byref(one), *args, ctypes.c_float(float("inf")), P, P, None, P, 1 << 30,
+                           None) == _lib.DSA_ERR_INVALID_ARG
+    empty = decode_dims(B=1, Nq=0, T_max=4096, ld_scores=4096).c()
+    assert lib.dsa_prefill(ctypes.byref(empty), *args, ctypes.c_float(0.07), P, P, None, P, 1 << 30,
+                           None) == _lib.DSA_OK
