@@ -20,18 +20,25 @@ import numpy as np
 _HERE = os.path.dirname(os.path.abspath(__file__))
 _SRC = os.path.join(_HERE, "dsa_oracle.c")
 _LIB_PATH = os.path.join(_HERE, "libdsa_oracle.so")
+# A prebuilt oracle library to load instead (used only by the test that plants mistakes in a
+# copy of the oracle source and checks that the pins catch each one).
+_LIB_OVERRIDE = os.environ.get("DSA_ORACLE_LIB")
 _lock = threading.Lock()
 _lib = None
 
 F32, BF16, FP8 = 0, 1, 2
 
 
+GCC_FLAGS = ["-O2", "-std=c11", "-fopenmp", "-fPIC", "-shared", "-fno-fast-math", "-ffp-contract=off"]
+
+
 def build(force: bool = False) -> str:
     """Compile dsa_oracle.c with gcc (-O2, OpenMP, IEEE arithmetic, no fast-math)."""
+    if _LIB_OVERRIDE:
+        return _LIB_OVERRIDE
     if force or not os.path.exists(_LIB_PATH) or os.path.getmtime(_LIB_PATH) < os.path.getmtime(_SRC):
         tmp = _LIB_PATH + f".tmp{os.getpid()}"
-        cmd = ["gcc", "-O2", "-std=c11", "-fopenmp", "-fPIC", "-shared", "-fno-fast-math",
-               "-ffp-contract=off", _SRC, "-o", tmp, "-lm"]
+        cmd = ["gcc"] + GCC_FLAGS + [_SRC, "-o", tmp, "-lm"]
         subprocess.check_call(cmd)
         os.replace(tmp, _LIB_PATH)
     return _LIB_PATH
@@ -41,8 +48,7 @@ def _load():
     global _lib
     with _lock:
         if _lib is None:
-            build()
-            lib = ctypes.CDLL(_LIB_PATH)
+            lib = ctypes.CDLL(build())
             P = ctypes.c_void_p
             I = ctypes.c_int
             L = ctypes.c_int64
