@@ -55,6 +55,7 @@ constexpr int kFineBits = 11;
 constexpr int kFineBins = 1 << kFineBits;  // adaptive histogram bins
 constexpr int kCandMax = 2048;             // threshold-bin keys resolved on chip by every CTA
 constexpr int kRankMax = 64;               // up to this many, tau is found by direct ranking
+constexpr uint32_t kFloorOctaves = 8;      // the first histogram's floor: 2^-8 of the row's largest score
 // Keep a CTA small enough for two per SM at the long-decode chunk (16K keys): with one per
 // SM, 16 clusters of 8 no longer fit the GPCs in one wave.
 constexpr int kOffFine = (kOffScan + kScanWords + 3) & ~3;  // kFineBins counts (read remotely)
@@ -276,11 +277,27 @@ __global__ void __launch_bounds__(kThreads, 2) topk_radix_kernel(const TopkArgs 
         local_eq = len;
     } else {
         // ---- 1. adaptive histogram over the row's key range, cluster totals per range of
-        // bins, threshold bin b*
-        const uint32_t span = kmax - kmin;
-        const int shift = max(0, 32 - __clz((int)span) - kFineBits);
+        // bins, threshold bin b*.  The bins cover [kbase, kmax]: kbase is the row's minimum,
+        // raised to 2^-kFloorOctaves of the largest score when that is positive (the k-th
+        // largest score of a row almost always lies within those octaves of the largest, and
+        // the narrower range leaves a few keys in b* instead of hundreds); keys below kbase
+        // count in bin 0.  Should b* be bin 0 all the same, the histogram is rebuilt over the
+        // full range.
+        constexpr uint32_t kFloorStep = kFloorOctaves << 23;  // the exponent field of a key
+        uint32_t kbase = kmin;
+        if (kmax > 0x80000000u + kFloorStep && kmax - kFloorStep > kmin) kbase = kmax - kFloorStep;
+        int shift = 0;
+        auto bin_of = [&](uint32_t kk) -> int {
+            return kk <= kbase ? 0 : min(kFineBins - 1, (int)((kk - kbase) >> shift));
+        };
         uint32_t* fine = sm + kOffFine;
         uint32_t* rng = sm + kOffRange;
+        // CTA rank owns bins [b_lo, b_hi): their totals over the cluster
+        const int per = (kFineBins + C - 1) / C;
+        const int b_lo = min(kFineBins, rank * per), b_hi = min(kFineBins, b_lo + per);
+#pragma unroll 1
+        while (true) {
+        shift = max(0, 32 - __clz((int)(kmax - kbase)) - kFineBits);
         for (int i = tid; i < kFineBins; i += kThreads) fine[i] = 0u;
         __syncthreads();
         for (int i0 = 4 * tid; i0 < len; i0 += 4 * kThreads) {
@@ -288,13 +305,10 @@ __global__ void __launch_bounds__(kThreads, 2) topk_radix_kernel(const TopkArgs 
             const uint32_t kv[4] = {k4.x, k4.y, k4.z, k4.w};
 #pragma unroll
             for (int u = 0; u < 4; ++u)
-                if (i0 + u < len) atomicAdd(&fine[(kv[u] - kmin) >> shift], 1u);
+                if (i0 + u < len) atomicAdd(&fine[bin_of(kv[u])], 1u);
         }
         __syncthreads();
         cluster.sync();
-        // CTA rank owns bins [b_lo, b_hi): their totals over the cluster
-        const int per = (kFineBins + C - 1) / C;
-        const int b_lo = min(kFineBins, rank * per), b_hi = min(kFineBins, b_lo + per);
         int part = 0;
         for (int bb = b_lo + tid; bb < b_hi; bb += kThreads) {
             uint32_t tot_b = 0u;
@@ -359,6 +373,14 @@ __global__ void __launch_bounds__(kThreads, 2) topk_radix_kernel(const TopkArgs 
             }
             __syncthreads();
         }
+        // the same b* in every CTA of the cluster (read from the same totals): a uniform exit
+        if (misc[8] != 0 || kbase == kmin) break;
+        // b* fell to the floor bin: rebuild over the full range once every peer has read this
+        // CTA's range totals
+        kbase = kmin;
+        cluster.sync();
+        if (tid == 0) misc[6] = 0;
+        }
         const int bstar = misc[8];
         const int above_total = misc[9];
         const int Tc = misc[10];
@@ -375,7 +397,7 @@ __global__ void __launch_bounds__(kThreads, 2) topk_radix_kernel(const TopkArgs 
                 const uint32_t kv[4] = {k4.x, k4.y, k4.z, k4.w};
 #pragma unroll
                 for (int u = 0; u < 4; ++u)
-                    if (i0 + u < len && (int)((kv[u] - kmin) >> shift) == bstar) cand[atomicAdd(misc + 13, 1)] = kv[u];
+                    if (i0 + u < len && bin_of(kv[u]) == bstar) cand[atomicAdd(misc + 13, 1)] = kv[u];
             }
             __syncthreads();
             cluster.sync();
@@ -432,7 +454,7 @@ __global__ void __launch_bounds__(kThreads, 2) topk_radix_kernel(const TopkArgs 
                 // histograms of the bits below the bin base, at most two levels for shift <= 22;
                 // this CTA's own fine histogram is free now (peers read it only before the range merge)
                 int rem = a.k - above_total;
-                uint64_t base = (uint64_t)kmin + ((uint64_t)bstar << shift);
+                uint64_t base = (uint64_t)kbase + ((uint64_t)bstar << shift);
                 int sh = shift;
 #pragma unroll 1
                 while (sh > 0) {
