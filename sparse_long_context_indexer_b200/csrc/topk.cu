@@ -10,10 +10,13 @@
 // the k-th largest key tau plus how many keys equal to tau are taken.  A row is
 // split across a thread-block cluster of C CTAs (C <= 8); every CTA keeps its
 // slice of the row in shared memory as keys and tracks their min and max.
-//  1. One histogram of 2048 bins over (key - min) >> shift, the shift chosen
-//     so that the row's key range fills the bins (the top digits of a float
-//     key -- sign and exponent -- put most scores of a row in a handful of
-//     bins, so fixed digits would need several full passes).  CTA r of the
+//  1. One histogram of 2048 bins over (key - base) >> shift, the shift chosen
+//     so that [base, max] fills the bins (the top digits of a float key --
+//     sign and exponent -- put most scores of a row in a handful of bins, so
+//     fixed digits would need several full passes).  base is the row's
+//     minimum key, raised to 2^-8 of its largest score when that is positive
+//     (keys below count in bin 0; if the threshold lands there the histogram
+//     is rebuilt from the minimum).  CTA r of the
 //     cluster sums one range of bins over all CTAs (distributed shared
 //     memory); the owner of the threshold bin b* broadcasts it.
 //  2. The keys of bin b* are collected (usually a few dozen); every CTA
