@@ -60,6 +60,7 @@ BATCH, CTX = 16, 131072
 FALLBACK_HBM_GBS = 6650.0
 INDEXER_SRC = os.path.join(ROOT, "sparse_long_context_indexer_b200", "csrc", "indexer_sm100.cu")
 TRAFFIC_FILE = os.path.join(ROOT, "profiles", "indexer_long_decode_b16_128k.md")
+E2E_STEPS = 400          # end-to-end steps timed, whatever --steps is
 
 
 def parse_args():
@@ -69,6 +70,8 @@ def parse_args():
     p.add_argument("--warmup", type=int, default=20)
     p.add_argument("--impl", default="ours", choices=["ours", "reference"])
     p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--no-secondary", action="store_true",
+                   help="skip the secondary workloads (decode batch 32, 1M-context decode, prefill) of the default line")
     p.add_argument("--workload", default="long_decode", choices=["long_decode", "prefill", "dense", "paged", "fp8kv"])
     p.add_argument("--block-size", type=int, default=64)
     p.add_argument("--prefill-len", type=int, default=65536)
@@ -167,6 +170,39 @@ class ClockSampler:
                     reasons.add(nm)
         return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": smax,
                 "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def nvml_reading(gpu_index):
+    """One read-only NVML sample of the SM clock and the active clock-event reasons."""
+    try:
+        import pynvml
+        pynvml.nvmlInit()
+        try:
+            h = pynvml.nvmlDeviceGetHandleByIndex(int(gpu_index))
+            sm = pynvml.nvmlDeviceGetClockInfo(h, pynvml.NVML_CLOCK_SM)
+            smax = pynvml.nvmlDeviceGetMaxClockInfo(h, pynvml.NVML_CLOCK_SM)
+            r = pynvml.nvmlDeviceGetCurrentClocksEventReasons(h)
+            names = {"hw_slowdown": pynvml.nvmlClocksEventReasonHwSlowdown,
+                     "hw_thermal_slowdown": pynvml.nvmlClocksEventReasonHwThermalSlowdown,
+                     "sw_thermal_slowdown": pynvml.nvmlClocksEventReasonSwThermalSlowdown,
+                     "sw_power_cap": pynvml.nvmlClocksEventReasonSwPowerCap}
+            return {"sm_mhz": float(sm), "sm_max_mhz": float(smax),
+                    "reasons": sorted(k for k, v in names.items() if r & v)}
+        finally:
+            pynvml.nvmlShutdown()
+    except Exception as e:  # reading only; a missing NVML is reported, not fatal
+        return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [f"nvml unavailable: {type(e).__name__}"]}
+
+
+def cpu_model():
+    try:
+        with open("/proc/cpuinfo") as f:
+            for ln in f:
+                if ln.startswith("model name"):
+                    return ln.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return None
 
 
 def dist_setup(n):
@@ -279,6 +315,17 @@ def run_ours(args):
         sweep.view(torch.int64).max()
     K, W = args.steps, args.warmup
 
+    vis = os.environ.get("CUDA_VISIBLE_DEVICES", "")
+    ids = [x for x in vis.split(",") if x.strip()]
+    li = local if world > 1 else 0
+    gpu_index = ids[li] if li < len(ids) else str(li)
+    # clocks are sampled from the warm-up through the end-to-end pass (seconds, not only the
+    # few milliseconds of the timed loop), plus one NVML reading on each side of the timed loop
+    sampler = ClockSampler(gpu_index)
+    sampler.start()
+    sampler.wait_first()
+    window0 = time.perf_counter()
+
     for _ in range(W):
         flush_l2()
         api.run_decode(inp, ws=ws, out=out, lse=lse, dims=dims)
@@ -291,14 +338,9 @@ def run_ours(args):
     # stages cost ~2 us of GPU time each, so the per-stage breakdown (and the indexer
     # duration the roofline uses) comes from a second pass right after this one.
     evs = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(K)]
-    vis = os.environ.get("CUDA_VISIBLE_DEVICES", "")
-    ids = [x for x in vis.split(",") if x.strip()]
-    li = local if world > 1 else 0
-    sampler = ClockSampler(ids[li] if li < len(ids) else str(li))
     barrier(world)
     torch.cuda.synchronize()
-    sampler.start()
-    sampler.wait_first()
+    nvml_before = nvml_reading(gpu_index)
     wall0 = time.perf_counter()
     for i in range(K):
         flush_l2()   # outside the timed events
@@ -307,15 +349,15 @@ def run_ours(args):
         evs[i][1].record()
     torch.cuda.synchronize()
     wall1 = time.perf_counter()
+    nvml_after = nvml_reading(gpu_index)
     wall = wall1 - wall0
     barrier(world)
-    clocks = sampler.stop(window=(wall0, wall1))
     step_ms = [evs[i][0].elapsed_time(evs[i][1]) for i in range(K)]
     mean_ms = sum(step_ms) / K
     mean_ms = max_over_ranks(mean_ms, world)
 
     # Stage pass: the same steps with an event before the indexer and after every stage.
-    KS = min(K, 1000)
+    KS = min(max(K, 200), 1000)
     sev = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(KS)]
     for i in range(KS):
         flush_l2()
@@ -326,10 +368,12 @@ def run_ours(args):
     status = api.get_device_status(ws)
 
     # ---- end to end through the C interface with host buffers
-    e2e = measure_e2e(inp, dims, ws, dev, steps=min(K, 200), warmup=min(W, 10))
+    e2e = measure_e2e(inp, dims, dev, steps=E2E_STEPS, warmup=max(W, 10))
     if not e2e["readback_ok"]:
         raise SystemExit("end-to-end loop: the host copy of the last step's output differs from the device's")
     e2e_ms = max_over_ranks(e2e["ms"], world)
+    window1 = time.perf_counter()
+    clocks = sampler.stop(window=(window0, window1))
 
     hbm, peak_kind = peaks()
     lens = [CTX] * BATCH
@@ -341,6 +385,18 @@ def run_ours(args):
     value = BATCH * world / (mean_ms * 1e-3)
     step_gbs = by["total"] / (mean_ms * 1e-3) / 1e9
 
+    # ---- secondary workloads (one GPU): decode batch 32 (ragged 16K-32K), 1M-context decode, prefill
+    secondary = {}
+    if world == 1 and not args.no_secondary:
+        del inp, ws, out, lse
+        torch.cuda.empty_cache()
+        for key, make in (("decode32", inputs.decode32), ("million", inputs.million)):
+            secondary[key] = measure_secondary_decode(make, dev, K=max(K, 20), W=max(W, 3), flush_l2=flush_l2,
+                                                      hbm=hbm, peak_kind=peak_kind)
+            torch.cuda.empty_cache()
+        secondary["prefill"] = measure_prefill(65536, dev, K=2, W=1)
+        torch.cuda.empty_cache()
+
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         import oracle
@@ -348,9 +404,16 @@ def run_ours(args):
         cores = oracle.max_threads()
         rows = BATCH
         t, passes = oracle_sample(rows, cores, min_seconds=10.0, max_passes=40)
+        t1, p1 = oracle_sample(1, 1, min_seconds=4.0, max_passes=5)
         cpu = {"value": rows * passes / t, "unit": UNIT, "cores": cores, "kind": "oracle",
+               "cpu_model": cpu_model(),
                "sample": f"the {rows} query rows of {WORKLOAD} (each a 131072-token sequence), full path, "
-                         f"fp64 C oracle with OpenMP, {passes} passes in {t:.1f} s"}
+                         f"fp64 C oracle with OpenMP on {cores} threads, {passes} passes in {t:.1f} s",
+               "single_thread": {"value": p1 / t1, "unit": UNIT, "cores": 1,
+                                 "sample": f"1 query row of {WORKLOAD}, full path, fp64 C oracle on one thread, "
+                                           f"{p1} passes in {t1:.1f} s"}}
+        if "prefill" in secondary:
+            secondary["prefill"]["cpu_baseline"] = prefill_cpu_baseline(65536, cores, dev)
     if world > 1:
         import torch.distributed as dist
         dist.destroy_process_group()
@@ -373,35 +436,89 @@ def run_ours(args):
         "stages_us": {"indexer": stage_us[0], "topk": stage_us[1], "sparse_mla": stage_us[2],
                       "merge": stage_us[3]},
         "e2e": {"value": BATCH * world / (e2e_ms * 1e-3), "unit": UNIT, "h2d_bytes_per_step": e2e["h2d"],
-                "d2h_bytes_per_step": e2e["d2h"], "ms_per_step": e2e_ms,
-                "pipeline": "one packed H2D copy per step; copy-in, compute (cache append + dsa_decode_step) "
-                            "and copy-out streams with two buffer slots (copies of neighbouring steps "
-                            "overlap a step's compute); each stage replayed from a CUDA graph captured "
-                            "from the same calls; the last step's read-back checked against the device "
-                            "copy and against a direct dsa_decode_step call"},
+                "d2h_bytes_per_step": e2e["d2h"], "ms_per_step": e2e_ms, "steps": E2E_STEPS,
+                "pipeline": "one CUDA-graph replay per step, captured once per buffer slot from the public calls: "
+                            "the step's cache append + dsa_decode_step on its slot, the H2D copy of the next "
+                            "step's inputs (one packed pinned buffer) and the D2H copy of the previous step's "
+                            "out and lse, as three concurrent branches of the graph; the timed region also "
+                            "holds the first copy-in and the last copy-out; the last read-back is checked "
+                            "against the device copy and against a direct dsa_decode_step call"},
         "gpu_launches": launches_per_step() * K,
         "timing": {"step": "one start and one end event per step on the launching stream",
                    "stages_us": f"separate pass of {KS} steps with an event between stages (each adds ~2 us)"},
         "clocks": {"sm_mhz": clocks["sm_mhz"], "sm_max_mhz": clocks["sm_max_mhz"], "reasons": clocks["reasons"],
-                   "samples": clocks["samples"]},
+                   "samples": clocks["samples"], "window_s": window1 - window0,
+                   "window": "nvidia-smi every 100 ms from the warm-up through the end-to-end pass",
+                   "nvml_before_timed_loop": nvml_before, "nvml_after_timed_loop": nvml_after},
         "device_status": status,
         "wall_s_timed_loop": wall,
     }
     if cpu is not None:
         line["cpu_baseline"] = cpu
+    for key, v in secondary.items():
+        line[key] = v
     print(json.dumps(line), flush=True)
     return 0
+
+
+def measure_secondary_decode(make, dev, K, W, flush_l2, hbm, peak_kind):
+    """A secondary decode workload (labelled as such in the line): the same decode step timed
+    like the headline (one start/end event per step, L2 flushed outside the timed events)."""
+    import torch
+    from sparse_long_context_indexer_b200 import _lib, accounting, api
+    inp = make(device=dev)
+    dims = api.dims_of(inp)
+    ws = api.make_workspace(dims, _lib.DSA_OP_DECODE, dev)
+    out, lse = api.alloc_outputs(inp)
+    for _ in range(W):
+        flush_l2()
+        api.run_decode(inp, ws=ws, out=out, lse=lse, dims=dims)
+    torch.cuda.synchronize()
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(K)]
+    for i in range(K):
+        flush_l2()
+        evs[i][0].record()
+        api.run_decode(inp, ws=ws, out=out, lse=lse, dims=dims)
+        evs[i][1].record()
+    torch.cuda.synchronize()
+    ms = sum(e[0].elapsed_time(e[1]) for e in evs) / K
+    status = api.get_device_status(ws)
+    lens = list(inp.seq_lens)
+    by = accounting.decode_step_bytes(lens)
+    gbs = by["total"] / (ms * 1e-3) / 1e9
+    return {"label": "secondary workload (the headline is the long decode above)",
+            "workload": inp.name, "batch": inp.B, "cached_tokens": {"min": min(lens), "max": max(lens),
+                                                                    "sum": sum(lens)},
+            "value": inp.B / (ms * 1e-3), "unit": UNIT, "ms_per_step": ms, "steps": K, "warmup": W,
+            "step_roofline": {"bound": "hbm", "achieved": gbs, "peak": hbm, "unit": "GB/s", "frac": gbs / hbm,
+                              "algorithmic_bytes": by["total"], "peak_source": f"{peak_kind} hbm_gbs"},
+            "device_status": status}
 
 
 def run_prefill(args):
     """Secondary line: one causal prompt of L tokens through dsa_prefill, with a per-stage split."""
     import torch
-    from sparse_long_context_indexer_b200 import _lib, api, inputs
-
     if args.gpus != 1:
         raise SystemExit("--workload prefill runs on one GPU")
-    dev = torch.device("cuda", 0)
-    L = args.prefill_len
+    line = measure_prefill(args.prefill_len, torch.device("cuda", 0), K=max(1, min(args.steps, 10)), W=args.warmup)
+    line["metric"] = f"prefill query-tok/s (one causal prompt of {args.prefill_len} tokens; index+top2048+sparse MLA)"
+    line.update({"n_gpus": 1, "higher_is_better": True, "scaling": "none", "vs_baseline": None,
+                 "dtype": "fp8_e4m3/bf16", "data": "synthetic"})
+    if not args.no_cpu_baseline:
+        import oracle
+        oracle.build()
+        line["cpu_baseline"] = prefill_cpu_baseline(args.prefill_len, oracle.max_threads(), torch.device("cuda", 0))
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def measure_prefill(L, dev, K, W):
+    """dsa_prefill over one causal prompt of L tokens (median of K timed prompts), then a second
+    pass over the same row chunks calling each stage's own entry point for the stage split and
+    the indexer's tensor-core roofline."""
+    import torch
+    from sparse_long_context_indexer_b200 import _lib, api, inputs
+
     g = inputs.make_prefill_inputs(f"prefill_{L}", L, seed=4, device=dev)
     dims = api.dims_of(g)
     ws = api.make_workspace(dims, _lib.DSA_OP_PREFILL, dev)
@@ -413,7 +530,6 @@ def run_prefill(args):
         api.prefill(dims, g.q_I, g.q_scale, g.w, g.k_I, g.k_scale, g.q, g.kv, g.q_seq, g.q_len, g.softmax_scale,
                     out, lse, ws, idx_out=idx)
 
-    K, W = max(1, min(args.steps, 10)), args.warmup
     for _ in range(W):
         whole()
     torch.cuda.synchronize()
@@ -430,7 +546,7 @@ def run_prefill(args):
     total_ms = statistics.median(ms)
 
     # Stage pass: the same work, chunk by chunk, each stage through its own entry point.
-    sms = torch.cuda.get_device_properties(0).multi_processor_count
+    sms = torch.cuda.get_device_properties(dev).multi_processor_count
     chunk = max(1, (64 << 20) // (dims.ld_scores * 4))
     if chunk >= sms // 2:
         chunk = chunk // (sms // 2) * (sms // 2) // 4 * 4   # the library's plan: whole attention waves
@@ -466,14 +582,13 @@ def run_prefill(args):
     mla_flop = sel * g.H * 2.0 * (576 + 512)
     burst, sustained, src = tensor_peaks()
     idx_tflops = idx_flop / (stage_ms[0] * 1e-3) / 1e12
-    line = {
-        "metric": f"prefill query-tok/s (one causal prompt of {L} tokens; index+top2048+sparse MLA)",
-        "value": L / (total_ms * 1e-3), "unit": "query-tok/s", "n_gpus": 1, "steps": K, "warmup": W,
-        "ms_per_step": total_ms, "higher_is_better": True, "scaling": "none", "vs_baseline": None,
-        "dtype": "fp8_e4m3/bf16", "data": "synthetic",
-        "config": {"workload": f"prefill_{L}", "H_I": g.H_I, "d_I": g.d_I, "top_k": g.k, "heads": g.H,
+    del g, out, lse, idx, scores, cidx
+    return {
+        "label": "secondary workload (the headline is the long decode above)",
+        "value": L / (total_ms * 1e-3), "unit": "query-tok/s", "steps": K, "warmup": W, "ms_per_step": total_ms,
+        "config": {"workload": f"prefill_{L}", "H_I": dims.H_I, "d_I": dims.d_I, "top_k": dims.k, "heads": dims.H,
                    "latent": "576 bf16 (512 + 64 rope)", "chunk_rows": chunk,
-                   "l2": "256 MiB written between steps, outside the timed events"},
+                   "l2": "256 MiB written between prompts, outside the timed events"},
         "roofline": {"bound": "tensor", "kernel": "indexer_fp8_kernel (four rows per pass)",
                      "achieved": idx_tflops, "peak": burst, "unit": "TFLOP/s", "frac": idx_tflops / burst,
                      "frac_of_sustained": idx_tflops / sustained, "traffic": None,
@@ -481,12 +596,78 @@ def run_prefill(args):
                      "algorithmic_flop": idx_flop},
         "stages_ms": {"indexer": stage_ms[0], "topk": stage_ms[1], "sparse_mla": stage_ms[2]},
         "sparse_mla_tflops": mla_flop / (stage_ms[2] * 1e-3) / 1e12,
-        "timing": {"step": "dsa_prefill between two events, median of the timed steps",
+        "timing": {"step": "dsa_prefill between two events, median of the timed prompts",
                    "stages_ms": f"second pass of {len(ev)} chunks of {chunk} rows, two events per stage call"},
         "device_status": status,
     }
-    print(json.dumps(line), flush=True)
-    return 0
+
+
+def prefill_sample_rows(L, k=2048):
+    """The fixed 512-row oracle sample of the prefill prompt: rows 0-63 (short rows that take
+    every position), 2000-2111 (around the budget), 32 rows spread evenly, and the last 304."""
+    spread = [int(round(x)) for x in [(i + 0.5) * L / 32 for i in range(32)]]
+    rows = sorted(set(list(range(0, 64)) + list(range(2000, 2112)) + spread + list(range(L - 304, L))))
+    return [r for r in rows if 0 <= r < L]
+
+
+def prefill_cpu_baseline(L, cores, dev=None):
+    """The oracle (full path) on the fixed 512-row sample of the prefill prompt, with OpenMP on
+    all host cores, timed per group of rows.  The whole prompt is then EXTRAPOLATED with a
+    per-row cost a * (t + 1) + b * min(t + 1, k) fitted to the groups (non-negative least
+    squares); the line says so."""
+    import numpy as np
+    import oracle
+    from sparse_long_context_indexer_b200 import inputs
+    k = 2048
+    rows = prefill_sample_rows(L, k)
+    # drawn on the device the GPU leg uses (same generator, so the sample rows are the GPU
+    # workload's own rows), then handed to the oracle on the host
+    sub = inputs.make_prefill_inputs(f"prefill_{L}", L, seed=4, rows=rows, device=dev or "cpu").to("cpu")
+    groups = {"0-63": [r for r in rows if r < 64], "2000-2111": [r for r in rows if 2000 <= r < 2112],
+              f"last 304": [r for r in rows if r >= L - 304]}
+    used = set(sum(groups.values(), []))
+    groups["spread"] = [r for r in rows if r not in used]
+    pos = {r: i for i, r in enumerate(rows)}
+    times, feats = {}, []
+    for name, rr in groups.items():
+        sel = [pos[r] for r in rr]
+        part = subset_rows(sub, sel)
+        t0 = time.perf_counter()
+        oracle.decode(part, nthreads=cores)
+        times[name] = time.perf_counter() - t0
+        n = np.array(rr, dtype=np.float64) + 1
+        feats.append([n.sum(), np.minimum(n, k).sum()])
+    A = np.array(feats)
+    y = np.array(list(times.values()))
+    from scipy.optimize import nnls
+    coef, _ = nnls(A, y)                       # non-negative costs per key and per selected row
+    n_all = np.arange(1, L + 1, dtype=np.float64)
+    extrap = float(coef[0] * n_all.sum() + coef[1] * np.minimum(n_all, k).sum())
+    total = sum(times.values())
+    return {"value": len(rows) / total, "unit": "query-tok/s", "cores": cores, "kind": "oracle",
+            "cpu_model": cpu_model(),
+            "sample": f"{len(rows)} fixed rows of the {L}-token prompt (0-63, 2000-2111, 32 spread, last 304), "
+                      f"full path (indexer over t+1 keys, top-2048, 128-head sparse MLA), fp64 C oracle, "
+                      f"OpenMP on {cores} threads, {total:.1f} s",
+            "seconds_per_group": times, "rows_per_group": {kk: len(v) for kk, v in groups.items()},
+            "extrapolated_prompt_s": extrap,
+            "extrapolation": "EXTRAPOLATED, not measured: per-row cost a*(t+1) + b*min(t+1, 2048) fitted to the "
+                             f"group times (a = {coef[0]:.3e} s per key, b = {coef[1]:.3e} s per selected row), "
+                             f"summed over all {L} rows"}
+
+
+def subset_rows(inp, sel):
+    """The same inputs restricted to the query rows `sel` (the cache is shared)."""
+    import torch
+    from sparse_long_context_indexer_b200 import inputs
+    r = torch.as_tensor(sel, dtype=torch.long)
+    out = inputs.DSAInputs(**{f: getattr(inp, f) for f in inp.__dataclass_fields__})
+    for f in ("q_I", "q_scale", "w", "q", "q_seq", "q_len"):
+        v = getattr(inp, f)
+        if v is not None:
+            setattr(out, f, v[r].contiguous())
+    out.Nq = len(sel)
+    return out
 
 
 def run_dense(args):
@@ -690,18 +871,21 @@ def launches_per_step():
     return 4 if splits > 8 else 3
 
 
-def measure_e2e(inp, dims, ws, dev, steps, warmup):
-    """End to end through the public API, as a serving loop would run it.  Per step:
-    one H2D copy of all of the step's inputs (query-side tensors, the new token's position,
-    bf16 latent row and fp32 indexer key, packed in one pinned buffer), the cache append
-    (dsa_append_tokens, which quantises the key on the device), the decode step,
-    and the D2H copy of out and lse.  Two buffer slots on separate copy-in, compute and
-    copy-out streams: the copies of step i+1 and step i-1 overlap the compute of step
-    i; each step's append and decode stay in order on the compute stream.  Each stage
-    of each slot is captured once into a CUDA graph from these calls and replayed, so
-    the host's issue cost per step stays below the step's GPU time."""
+def measure_e2e(inp, dims, dev, steps, warmup):
+    """End to end through the public API, as a serving loop would run it.  Per step: the H2D
+    copy of all of the step's inputs (query-side tensors, the new token's position, bf16
+    latent row and fp32 indexer key, packed in one pinned buffer), the cache append
+    (dsa_append_tokens, which quantises the key on the device), the decode step, and the D2H
+    copy of out and lse.
+
+    Two buffer slots.  Step i runs one CUDA graph, captured once per slot from the public
+    calls, with three concurrent branches: the append + decode of step i on its slot, the
+    H2D copy of step i+1's inputs into the other slot, and the D2H copy of step i-1's
+    outputs from the other slot.  Graph launches on one stream run one after another, which
+    orders the slots' reuse; the first copy-in and the last copy-out are inside the timed
+    region too.  One host call per step keeps the host's issue cost off the step time."""
     import torch
-    from sparse_long_context_indexer_b200 import api
+    from sparse_long_context_indexer_b200 import _lib, api
     B = inp.B
     pos = (inp.q_len - 1).long()
     rows = torch.arange(B, device=dev)
@@ -722,6 +906,7 @@ def measure_e2e(inp, dims, ws, dev, steps, warmup):
     for k, v in fields.items():
         nb = v.numel() * v.element_size()
         host_pack[offs[k]:offs[k] + nb].copy_(v.contiguous().cpu().view(-1).view(torch.uint8))
+    ws = api.make_workspace(dims, _lib.DSA_OP_DECODE, dev)
     slots = []
     for _ in range(2):
         dbuf = torch.empty(total, dtype=torch.uint8, device=dev)
@@ -730,17 +915,15 @@ def measure_e2e(inp, dims, ws, dev, steps, warmup):
         o, l = api.alloc_outputs(inp)
         slots.append({"dbuf": dbuf, "v": views, "out": o, "lse": l,
                       "out_h": torch.empty(o.shape, dtype=o.dtype).pin_memory(),
-                      "lse_h": torch.empty(l.shape, dtype=l.dtype).pin_memory(),
-                      "in_done": torch.cuda.Event(), "comp_done": torch.cuda.Event(), "out_done": torch.cuda.Event()})
+                      "lse_h": torch.empty(l.shape, dtype=l.dtype).pin_memory()})
     d2h = slots[0]["out_h"].numel() * slots[0]["out_h"].element_size() + \
         slots[0]["lse_h"].numel() * slots[0]["lse_h"].element_size()
+    main = torch.cuda.Stream(device=dev)
     s_in, s_out = torch.cuda.Stream(device=dev), torch.cuda.Stream(device=dev)
-    s_c = torch.cuda.current_stream(dev)
+    seq = torch.arange(B, dtype=torch.int32, device=dev)
 
     def copy_in(sl):
         sl["dbuf"].copy_(host_pack, non_blocking=True)
-
-    seq = torch.arange(B, dtype=torch.int32, device=dev)
 
     def compute(sl):
         v = sl["v"]
@@ -752,55 +935,58 @@ def measure_e2e(inp, dims, ws, dev, steps, warmup):
         sl["out_h"].copy_(sl["out"], non_blocking=True)
         sl["lse_h"].copy_(sl["lse"], non_blocking=True)
 
-    # Each stage of each slot is captured once from the same public calls into a CUDA graph
-    # and replayed (a serving loop's usual way to keep the host out of the step time).
-    for sl in slots:
-        for fn in (copy_in, compute, copy_out):      # eager run first (lazy initialisation)
-            fn(sl)
-    torch.cuda.synchronize(dev)
-    for sl in slots:
-        sl["graphs"] = []
-        for fn in (copy_in, compute, copy_out):
-            g = torch.cuda.CUDAGraph()
-            with torch.cuda.graph(g, capture_error_mode="relaxed"):
-                fn(sl)
-            sl["graphs"].append(g)
-    torch.cuda.synchronize(dev)
-    first = [True, True]
-
-    def step(i):
-        sl = slots[i % 2]
-        g_in, g_c, g_out = sl["graphs"]
+    def step_body(s):
+        # fork: the other slot's copies run beside this slot's compute; join before the end
+        cur, other = slots[s], slots[1 - s]
+        fork = torch.cuda.Event()
+        fork.record(main)
+        s_in.wait_event(fork)
+        s_out.wait_event(fork)
         with torch.cuda.stream(s_in):
-            if not first[i % 2]:
-                s_in.wait_event(sl["comp_done"])       # the slot's previous decode has read its inputs
-            g_in.replay()
-            sl["in_done"].record(s_in)
-        s_c.wait_event(sl["in_done"])
-        if not first[i % 2]:
-            s_c.wait_event(sl["out_done"])             # the slot's previous outputs have been read back
-        with torch.cuda.stream(s_c):
-            g_c.replay()
-        sl["comp_done"].record(s_c)
+            copy_in(other)
+            in_done = torch.cuda.Event()
+            in_done.record(s_in)
         with torch.cuda.stream(s_out):
-            s_out.wait_event(sl["comp_done"])
-            g_out.replay()
-            sl["out_done"].record(s_out)
-        first[i % 2] = False
+            copy_out(other)
+            out_done = torch.cuda.Event()
+            out_done.record(s_out)
+        with torch.cuda.stream(main):
+            compute(cur)
+        main.wait_event(in_done)
+        main.wait_event(out_done)
 
-    for i in range(warmup):
-        step(i)
+    with torch.cuda.stream(main):                   # eager run first (lazy initialisation)
+        copy_in(slots[0])
+        copy_in(slots[1])
+    main.synchronize()
+    for s in (0, 1):
+        with torch.cuda.stream(main):
+            step_body(s)
+    torch.cuda.synchronize(dev)
+    graphs = []
+    for s in (0, 1):
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=main, capture_error_mode="relaxed"):
+            step_body(s)
+        graphs.append(g)
+    torch.cuda.synchronize(dev)
+
+    def run(n):
+        with torch.cuda.stream(main):
+            copy_in(slots[0])                       # the first step's inputs
+            for i in range(n):
+                graphs[i % 2].replay()
+            copy_out(slots[(n - 1) % 2])            # the last step's outputs
+
+    run(warmup)
     torch.cuda.synchronize(dev)
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record(s_in)
-    for i in range(steps):
-        step(i)
-    # the last step's read-back ends the timed region
-    s_in.wait_stream(s_out)
-    e1.record(s_in)
+    e0.record(main)
+    run(steps)
+    e1.record(main)
     torch.cuda.synchronize(dev)
     last = slots[(steps - 1) % 2]
-    ok = torch.equal(last["out_h"], last["out"].cpu())
+    ok = torch.equal(last["out_h"], last["out"].cpu()) and torch.equal(last["lse_h"], last["lse"].cpu())
     # the replayed step computes what a direct call computes on the same inputs
     ref_out, ref_lse = api.alloc_outputs(inp)
     v = last["v"]
@@ -808,11 +994,14 @@ def measure_e2e(inp, dims, ws, dev, steps, warmup):
                     v["q_len"], inp.softmax_scale, ref_out, ref_lse, ws)
     torch.cuda.synchronize(dev)
     ok = ok and torch.equal(ref_out.cpu(), last["out_h"]) and torch.equal(ref_lse.cpu(), last["lse_h"])
-    return {"ms": e0.elapsed_time(e1) / steps, "h2d": h2d, "d2h": d2h, "readback_ok": ok}
+    status = api.get_device_status(ws)
+    return {"ms": e0.elapsed_time(e1) / steps, "h2d": h2d, "d2h": d2h, "readback_ok": ok and status == 0}
 
 
 def main():
     args = parse_args()
+    if os.environ.get("DSA_ORACLE_LIB") or os.environ.get("DSA_ORACLE_MUTANT_RUN"):
+        raise SystemExit("bench.py times the committed oracle only: unset DSA_ORACLE_LIB / DSA_ORACLE_MUTANT_RUN")
     if args.impl == "reference":
         return run_reference(args)
     if args.workload == "prefill":

@@ -195,17 +195,23 @@ dsa_status_t dsa_dense_mla_attn(const dsa_dims* dims, const void* q, const void*
  * kept until the process exits).
  * Limit: when the split count is above 8 (the partials path of
  * dsa_sparse_mla_attn), (number of splits) x Nq <= 64 partial rows of 128
- * heads; the split count is the one dsa_sparse_mla_attn would use (it depends
- * on Nq and the device's SM count).  1 to 8 splits need no scratch at all.
+ * heads.  The split count is the one dsa_sparse_mla_attn uses:
+ * S = clamp(SMs / (2 Nq), 1, 16), rows per split = ceil(k / S) rounded up to
+ * a multiple of 64, splits = ceil(k / rows per split).  1 to 8 splits merge on
+ * chip and need no scratch at all.  At k = 2048 on a 148-SM B200 that means:
+ * Nq <= 5 uses the buffer (Nq 1..4: 16 splits, Nq 5: 11), Nq = 6 (11 splits,
+ * 66 partial rows) is refused, Nq >= 7 merges on chip.
  * Larger requests return DSA_ERR_UNSUPPORTED before any launch.  kv_dtype
  * DSA_F32 returns DSA_ERR_UNSUPPORTED.
  * The first call on a device looks up the buffer's device address (once per
  * device, with that device current); make that first call before any stream
  * capture.  All calls share the buffer, so calls whose kernels overlap on the
  * GPU (other streams, other host threads) race on it: serialise them.  No
- * status word exists here: device-side index errors are not reported (entries
- * outside [-1, q_len[t]) are still treated as -1).  Allocates nothing; calls no
- * cudaMalloc or cudaFree. */
+ * status word exists here, so device-side errors are not reported: entries
+ * outside [-1, q_len[t]) are still treated as -1 without a flag, and a
+ * bounded wait that runs out (a stalled GPU) ends the kernel early with
+ * incomplete outputs and no error code.  Callers that need those reports use
+ * dsa_sparse_mla_attn.  Allocates nothing; calls no cudaMalloc or cudaFree. */
 dsa_status_t dsa_sparse_mla_attn_noalloc(const dsa_dims* dims, const void* q, const void* kv,
                                          const int32_t* idx, const int32_t* q_seq, const int32_t* q_len,
                                          float softmax_scale, void* out, float* lse, void* stream);

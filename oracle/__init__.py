@@ -20,9 +20,14 @@ import numpy as np
 _HERE = os.path.dirname(os.path.abspath(__file__))
 _SRC = os.path.join(_HERE, "dsa_oracle.c")
 _LIB_PATH = os.path.join(_HERE, "libdsa_oracle.so")
-# A prebuilt oracle library to load instead (used only by the test that plants mistakes in a
-# copy of the oracle source and checks that the pins catch each one).
+# A prebuilt oracle library to load instead.  Only the test that plants mistakes in a copy of
+# the oracle source (and checks that the pins catch each one) uses it, in a child process that
+# also sets DSA_ORACLE_MUTANT_RUN=1; anywhere else a stray DSA_ORACLE_LIB would swap the
+# checker, so it is refused.
 _LIB_OVERRIDE = os.environ.get("DSA_ORACLE_LIB")
+if _LIB_OVERRIDE and os.environ.get("DSA_ORACLE_MUTANT_RUN") != "1":
+    raise RuntimeError("DSA_ORACLE_LIB is honoured only inside the oracle mutation test's child process "
+                       "(DSA_ORACLE_MUTANT_RUN=1); unset it")
 _lock = threading.Lock()
 _lib = None
 

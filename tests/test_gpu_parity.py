@@ -75,6 +75,51 @@ def test_topk_bit_exact_on_identical_scores(lib, lens, k):
         assert np.array_equal(got[t], want[t]), f"row {t} (n={lens[t]}): first diff at {np.argmax(got[t] != want[t])}"
 
 
+def anchored_scores(seed):
+    """Long rows for the first histogram's floor (2^-8 of the row's largest score) and its
+    full-range rebuild: (scores [4, 131072], lengths).
+      row 0 (131,072 keys) and row 1 (40,000 keys): N(0,1) scores plus a few anchors about
+        1e4 times larger, so almost every key lies below the floor and the k-th largest too;
+      row 2: exactly k-1 keys above the floor (the k-th largest sits just below it);
+      row 3: exactly k keys above the floor (the k-th largest is the lowest of them)."""
+    k, ld = 2048, 131072
+    g = torch.Generator().manual_seed(seed)
+    sc = torch.randn((4, ld), generator=g)
+    for t, n_anchor in ((0, 24), (1, 7)):
+        pos = torch.randperm(131072 if t == 0 else 40000, generator=g)[:n_anchor]
+        sc[t, pos] = 1e4 * (1 + torch.rand(n_anchor, generator=g))
+    for t, above in ((2, k - 1), (3, k)):
+        row = torch.clamp(torch.randn(ld, generator=g), -3.5, 3.5)      # all below 1000 / 256
+        pos = torch.randperm(ld, generator=g)[:above]
+        row[pos] = 10 + 990 * torch.rand(above, generator=g)             # above the floor
+        row[pos[0]] = 1000.0                                             # the row's largest
+        row[pos[1:4]] = 500.0                                            # a few ties above it
+        sc[t] = row
+    sc[:, 5:9] = sc[:, 5:6]                                              # ties in the tail
+    return sc.float(), [131072, 40000, 131072, 131072]
+
+
+def test_topk_bit_exact_on_long_rows_with_anchors_and_floor_rebuild(lib):
+    k = 2048
+    sc, lens = anchored_scores(77)
+    ld = sc.shape[1]
+    q_len = torch.tensor(lens, dtype=torch.int32)
+    want = oracle.topk(sc.double().numpy(), q_len.numpy(), k)
+    # the rows really exercise the floor: their k-th largest score lies at or below max / 256
+    for t in (0, 1, 2):
+        row = np.sort(sc[t, :lens[t]].numpy())[::-1]
+        assert row[k - 1] <= row[0] / 256
+    dims = api.Dims(B=1, Nq=len(lens), H_I=64, d_I=64, H=128, k=k, T_max=ld, idx_dtype=2, kv_dtype=1, ld_scores=ld)
+    ws = api.make_workspace(dims, _lib.DSA_OP_TOPK)
+    idx = torch.full((len(lens), k), -7, dtype=torch.int32, device="cuda")
+    api.topk(dims, sc.cuda(), q_len.cuda(), idx, ws)
+    torch.cuda.synchronize()
+    assert api.get_device_status(ws) == 0
+    got = idx.cpu().numpy()
+    for t in range(len(lens)):
+        assert np.array_equal(got[t], want[t]), f"row {t} (n={lens[t]}): first diff at {np.argmax(got[t] != want[t])}"
+
+
 def test_topk_all_equal_scores_take_lowest_positions(lib):
     n, k = 70000, 2048
     sc = torch.full((2, n), 0.25)
@@ -206,6 +251,7 @@ def test_short_rows_skip_the_indexer_with_the_same_outputs(lib):
     # selection (every position) and the attention must not change
     lens = [2048, 700, 1, 2049, 5000]
     inp = small_decode(seed=45, lens=lens)
+    sc_o, idx_o, out_o, lse_o = oracle.decode(inp)
     g = inp.to("cuda")
     dims = api.dims_of(g)
     ws = api.make_workspace(dims, _lib.DSA_OP_DECODE)
@@ -221,15 +267,24 @@ def test_short_rows_skip_the_indexer_with_the_same_outputs(lib):
         if n <= g.k:
             assert torch.equal(idx_a[t, :n].cpu(), torch.arange(n, dtype=torch.int32))
     assert torch.equal(out_a, out_b) and torch.equal(lse_a, lse_b)
+    # the dispatched step against the oracle (the short rows attend over every position)
+    g_idx = idx_a.cpu().numpy()
+    check_sets(g_idx, idx_o, sc_o, inp.q_len.numpy(), inp.k)
+    rows = [t for t in range(len(lens)) if np.array_equal(g_idx[t], idx_o[t])]
+    assert all(t in rows for t, n in enumerate(lens) if n <= g.k)
+    assert len(rows) >= len(lens) - 1
+    check_attention(out_a.float().cpu().numpy(), out_o, lse_a.cpu().numpy(), lse_o, rows=rows)
 
 
 @pytest.mark.parametrize("block_size", [64, 256])
-def test_paged_decode_matches_contiguous(lib, block_size):
+def test_paged_decode_matches_oracle_and_contiguous(lib, block_size):
     # the same cache in blocks of a pool, in a random physical order, read through a block
-    # table (kgptalkie: the selection is an address list into the paged KV cache); the
-    # contiguous path is pinned to the oracle, the paged one must give identical outputs
+    # table (kgptalkie "How Does the Selector Pick 1,024?": the selection is an address list
+    # into the paged KV cache).  The paged outputs are checked against the oracle on the same
+    # logical cache, and must equal the contiguous path's bit for bit.
     lens = [4097, 2500, 777, 2048, 2049, 129, 1]
     inp = inputs.make_decode_inputs("paged", lens, T_max=4352, anchor_frac=0.01, seed=71)
+    sc_o, idx_o, out_o, lse_o = oracle.decode(inp)
     g = inp.to("cuda")
     dims = api.dims_of(g)
     ws = api.make_workspace(dims, _lib.DSA_OP_DECODE)
@@ -245,6 +300,14 @@ def test_paged_decode_matches_contiguous(lib, block_size):
                           scores_out=sc_p, idx_out=idx_p)
     torch.cuda.synchronize()
     assert api.get_device_status(ws) == 0
+    # against the oracle
+    check_scores(np_scores(sc_p), sc_o, inp.q_len.numpy())
+    g_idx = idx_p.cpu().numpy()
+    same, total = check_sets(g_idx, idx_o, sc_o, inp.q_len.numpy(), inp.k)
+    rows = [t for t in range(inp.Nq) if np.array_equal(g_idx[t], idx_o[t])]
+    assert len(rows) >= max(1, total - 1), f"only {same}/{total} rows selected identical sets"
+    check_attention(out_p.float().cpu().numpy(), out_o, lse_p.cpu().numpy(), lse_o, rows=rows)
+    # and against the contiguous path
     for t, n in enumerate(lens):
         assert torch.equal(sc_p[t, :n], sc_c[t, :n]), f"row {t}: paged scores differ"
     assert torch.equal(idx_p, idx_c)
@@ -290,6 +353,7 @@ def test_fp8_latent_dense_and_paged(lib):
     lens = [3000, 2049, 64, 1]
     inp = inputs.with_fp8_latent(inputs.make_decode_inputs("fp8_paged", lens, T_max=3072, seed=83))
     out_o, lse_o = oracle.dense_attn(inp)
+    sc_d, idx_d, out_dec, lse_dec = oracle.decode(inp)
     g = inp.to("cuda")
     dims = api.dims_of(g)
     ws_d = api.make_workspace(dims, _lib.DSA_OP_DENSE_MLA)
@@ -307,6 +371,12 @@ def test_fp8_latent_dense_and_paged(lib):
     torch.cuda.synchronize()
     assert api.get_device_status(ws_d) == 0 and api.get_device_status(ws) == 0
     check_attention(out.float().cpu().numpy(), out_o, lse.cpu().numpy(), lse_o)
+    # the paged decode against the oracle's decode of the same logical FP8 cache
+    g_idx = idx_p.cpu().numpy()
+    check_sets(g_idx, idx_d, sc_d, inp.q_len.numpy(), inp.k)
+    rows = [t for t in range(len(lens)) if np.array_equal(g_idx[t], idx_d[t])]
+    assert len(rows) >= len(lens) - 1
+    check_attention(out_p.float().cpu().numpy(), out_dec, lse_p.cpu().numpy(), lse_dec, rows=rows)
     assert torch.equal(idx_p, idx_c) and torch.equal(out_p, out_c) and torch.equal(lse_p, lse_c)
 
 
@@ -334,6 +404,9 @@ def test_append_tokens_matches_the_input_quantisers(lib, fp8_latent):
     api.append_tokens(dims, seq.cuda(), pos.cuda(), kv_new.cuda(), k_new.cuda(), kv, k_I, k_scale, ws=ws)
     torch.cuda.synchronize()
     assert api.get_device_status(ws) == _lib.DSA_ERR_LENGTH
+    # the format definition, through the oracle's own e4m3 decoder: every written key value is
+    # within half an e4m3 step of its fp32 input, and the scale is amax / 448 in fp32
+    check_appended_against_format(k_I.cpu(), k_scale.cpu(), kv.cpu(), seq, pos, k_new, kv_new, fp8_latent)
     codes, scales = inputs.quantize_e4m3_per_row(k_new)
     want_kv = inputs.pack_fp8_latent(kv_new) if fp8_latent else kv_new
     for i in range(4):
@@ -363,6 +436,41 @@ def test_append_tokens_matches_the_input_quantisers(lib, fp8_latent):
         pr = int(full[b, s_ // 64]), s_ % 64
         assert torch.equal(k_pool[pr].cpu(), codes[i]) and float(s_pool[pr]) == float(scales[i])
         assert torch.equal(kv_pool[pr].cpu(), want_kv[i])
+
+
+E4M3_MAX = 448.0
+
+
+def e4m3_half_step_bound(ref, scale):
+    """Largest error of one round-to-nearest e4m3 code times `scale` against `ref`: half a step,
+    i.e. 2^-4 of |ref| in the normal range and 2^-10 of the scale in the subnormal range."""
+    return np.maximum(2.0 ** -4 * np.abs(ref), 2.0 ** -10 * scale) * (1 + 1e-6)
+
+
+def check_appended_against_format(k_I, k_scale, kv, seq, pos, k_new, kv_new, fp8_latent):
+    """The appended token's stored bytes, decoded by the oracle, against the fp32/bf16 inputs."""
+    table = np.array([oracle.e4m3_decode(c) for c in range(256)], dtype=np.float64)
+    for i in range(4):
+        b, s_ = int(seq[i]), int(pos[i])
+        x = k_new[i].double().numpy()
+        amax = np.float32(np.abs(k_new[i].numpy()).max())
+        want_scale = np.float32(amax / np.float32(E4M3_MAX)) if amax > 0 else np.float32(1.0)
+        got_scale = np.float32(k_scale[b, s_])
+        assert got_scale == want_scale, f"token {i}: key scale {got_scale} != amax/448 = {want_scale}"
+        dec = table[k_I[b, s_].numpy()] * float(got_scale)
+        assert np.all(np.abs(dec - x) <= e4m3_half_step_bound(x, float(got_scale))), f"token {i}: key codes"
+        ref = kv_new[i].float().numpy().astype(np.float64)
+        if fp8_latent:
+            d = oracle.dequant_latent_fp8(kv[b, s_]).astype(np.float64)
+            grp = np.abs(kv_new[i, :512].float().numpy()).reshape(4, 128).max(axis=1).astype(np.float32)
+            want = np.where(grp > 0, grp / np.float32(E4M3_MAX), np.float32(1.0)).astype(np.float32)
+            got = kv[b, s_, 512:528].contiguous().view(torch.float32).numpy()
+            assert np.array_equal(got, want), f"token {i}: latent group scales"
+            bound = e4m3_half_step_bound(ref[:512], np.repeat(got.astype(np.float64), 128))
+            assert np.all(np.abs(d[:512] - ref[:512]) <= bound), f"token {i}: latent codes"
+            assert np.array_equal(d[512:], ref[512:]), f"token {i}: rope values"
+        else:
+            assert torch.equal(kv[b, s_], kv_new[i]), f"token {i}: latent row"
 
 
 def test_prefill_matches_oracle(lib):

@@ -45,7 +45,7 @@ def test_pins_catch_a_planted_mistake(tmp_path, name, old, new):
     mutant.write_text(src.replace(old, new))
     so = tmp_path / "libdsa_oracle_mutant.so"
     subprocess.check_call(["gcc"] + oracle.GCC_FLAGS + [str(mutant), "-o", str(so), "-lm"])
-    env = dict(os.environ, DSA_ORACLE_LIB=str(so))
+    env = dict(os.environ, DSA_ORACLE_LIB=str(so), DSA_ORACLE_MUTANT_RUN="1")
     r = subprocess.run([sys.executable, "-m", "pytest", "-x", "-q", "-p", "no:cacheprovider", "-m", "not gpu",
                         os.path.join("tests", "test_oracle_pins.py")],
                        cwd=ROOT, env=env, capture_output=True, text=True, timeout=900)
@@ -59,7 +59,7 @@ def test_unmodified_copy_passes_the_pins(tmp_path):
         pytest.skip("gcc not available")
     so = tmp_path / "libdsa_oracle_copy.so"
     subprocess.check_call(["gcc"] + oracle.GCC_FLAGS + [SRC, "-o", str(so), "-lm"])
-    env = dict(os.environ, DSA_ORACLE_LIB=str(so))
+    env = dict(os.environ, DSA_ORACLE_LIB=str(so), DSA_ORACLE_MUTANT_RUN="1")
     r = subprocess.run([sys.executable, "-m", "pytest", "-q", "-p", "no:cacheprovider", "-m", "not gpu",
                         os.path.join("tests", "test_oracle_pins.py")],
                        cwd=ROOT, env=env, capture_output=True, text=True, timeout=900)
