@@ -84,7 +84,19 @@ struct IdxCfg {
     // quads covers an accumulator, and with QP groups group g takes the stages it % QP == g.
     static constexpr int NB = SUB * R;
     static constexpr int QP = R == 2 ? 2 : 1;
-    static constexpr int EPI_WARP0 = 2;
+    // Decode streams its keys with 16-byte cp.async copies from two producer warps, which write
+    // the swizzled tile themselves (measured on B200: the long decode's 142.7 MB of keys and
+    // scales stream in 27.6 us with plain 16-byte loads against 33.6 us with 64-byte TMA box
+    // rows); prefill, bound by its epilogue, keeps one TMA producer lane.
+    static constexpr bool CPASYNC = R == 1;
+    static constexpr int PROD_WARPS = CPASYNC ? 2 : 1;
+    static constexpr int PROD_THREADS = 32 * PROD_WARPS;
+    static constexpr int MMA_WARP = PROD_WARPS;
+    static constexpr int EPI_WARP0 = PROD_WARPS + 1;
+    static constexpr int KCHUNKS = STOK * D_I / 16;  // 16-byte pieces of a key stage
+    static constexpr int SCHUNKS = STOK / 4;         // 16-byte pieces of its scales
+    static_assert(!CPASYNC || (KCHUNKS % PROD_THREADS == 0 && SCHUNKS % PROD_THREADS == 0),
+                  "every producer thread copies the same number of pieces per stage");
     static constexpr int EPI_WARPS = 4 * NB * QP;
     static constexpr int THREADS = (EPI_WARP0 + EPI_WARPS) * 32;
     static constexpr int K_STEPS = D_I / 32;      // kind::f8f6f4 consumes 32 bytes of K per MMA
@@ -197,7 +209,9 @@ __global__ void __launch_bounds__(IdxCfg<D_I, R>::THREADS, 1)
 
     if (tid == 0) {
         for (int s = 0; s < C::STAGES; ++s) {
-            mbar_init(bar_full(s), 1);
+            // TMA: one arrival with the stage's bytes; cp.async: one arrival per producer thread
+            // once its copies of the stage have landed
+            mbar_init(bar_full(s), C::CPASYNC ? C::PROD_THREADS : 1);
             mbar_init(bar_empty(s), 4 * C::NB);  // every warp of the stage's epilogue group, once it
                                                  // has its scales (the MMA that read the keys has
                                                  // completed before)
@@ -216,13 +230,14 @@ __global__ void __launch_bounds__(IdxCfg<D_I, R>::THREADS, 1)
         tma_prefetch_desc(&tmap_q);
         tma_prefetch_desc(&tmap_s);
     }
-    if (warp == 1) {
+    if (warp == C::MMA_WARP) {
         tmem_alloc(smem_u32(&sh->tmem_base), C::TMEM_COLS);
         tmem_relinquish();
     }
-    // Work range: this CTA's slice of the flat (unit, stage) list (warp 2 scans the units).
+    // Work range: this CTA's slice of the flat (unit, stage) list (the first epilogue warp
+    // scans the units).
     const int nunits = (a.Nq + R - 1) / R;
-    if (warp == 2) {
+    if (warp == C::EPI_WARP0) {
         if (blockIdx.x == 0) {
             for (int r = lane; r < a.Nq; r += 32) {
                 if (a.q_len[r] != 0 && row_tiles(a, r, C::STOK) == 0) record_status(a.status, DSA_STATUS_LENGTH);
@@ -273,31 +288,34 @@ __global__ void __launch_bounds__(IdxCfg<D_I, R>::THREADS, 1)
     const int count = sh->count;
     griddep_launch_dependents();  // the top-k may start its setup on SMs this grid leaves free
 
-    if (warp == 0) {
+    if (warp < C::PROD_WARPS) {
         // ---------------- producer
         if (count > 0) {
             TileCursor<C::STOK, R> cur;
             cur.start(a, sh->row0, sh->j0);
             int qi = -1;
             int issued = 0;
+            const uint64_t stream_policy = l2_policy_evict_first();
             for (int it = 0; it < count; ++it) {
                 if (it == 0 || cur.j == 0) {
                     ++qi;
                     const int qb = qi & 1;
-                    if (qi >= 2) {
-                        const bool okq = mbar_wait(bar_qempty(qb), ((qi - 2) >> 1) & 1, abort_flag, a.status);
-                        if (!__all_sync(0xffffffffu, okq)) break;
-                    }
-                    // folded weights w * q_scale of the unit's rows (0 past the last row)
-                    const int64_t o = (int64_t)cur.row * C::NCOL;
-                    const __nv_bfloat16* wr = reinterpret_cast<const __nv_bfloat16*>(a.w) + o;
-                    const int64_t lim = (int64_t)a.Nq * C::HEADS - o;
-                    for (int i = lane; i < C::NCOL; i += 32)
-                        wq_smem[qb * C::NCOL + i] = i < lim ? __bfloat162float(wr[i]) * a.q_scale[o + i] : 0.f;
-                    __syncwarp();
-                    if (lane == 0) {
-                        mbar_arrive_expect_tx(bar_qfull(qb), C::Q_BYTES);
-                        tma_load_2d(sQ + qb * C::Q_BYTES, &tmap_q, 0, cur.row * C::NCOL, bar_qfull(qb));
+                    if (warp == 0) {
+                        if (qi >= 2) {
+                            const bool okq = mbar_wait(bar_qempty(qb), ((qi - 2) >> 1) & 1, abort_flag, a.status);
+                            if (!__all_sync(0xffffffffu, okq)) break;
+                        }
+                        // folded weights w * q_scale of the unit's rows (0 past the last row)
+                        const int64_t o = (int64_t)cur.row * C::NCOL;
+                        const __nv_bfloat16* wr = reinterpret_cast<const __nv_bfloat16*>(a.w) + o;
+                        const int64_t lim = (int64_t)a.Nq * C::HEADS - o;
+                        for (int i = lane; i < C::NCOL; i += 32)
+                            wq_smem[qb * C::NCOL + i] = i < lim ? __bfloat162float(wr[i]) * a.q_scale[o + i] : 0.f;
+                        __syncwarp();
+                        if (lane == 0) {
+                            mbar_arrive_expect_tx(bar_qfull(qb), C::Q_BYTES);
+                            tma_load_2d(sQ + qb * C::Q_BYTES, &tmap_q, 0, cur.row * C::NCOL, bar_qfull(qb));
+                        }
                     }
                 }
                 const int st = it % C::STAGES;
@@ -305,55 +323,125 @@ __global__ void __launch_bounds__(IdxCfg<D_I, R>::THREADS, 1)
                     const bool oke = mbar_wait(bar_empty(st), ((it / C::STAGES) - 1) & 1, abort_flag, a.status);
                     if (!__all_sync(0xffffffffu, oke)) break;
                 }
-                if (a.block_table == nullptr) {
-                    if (lane == 0) {
-                        mbar_arrive_expect_tx(bar_full(st), C::KTILE_BYTES + C::SC_BYTES);
-#pragma unroll
-                        for (int q = 0; q < C::NBOX; ++q) {
-                            const int tok = cur.j * C::STOK + q * C::BOX;
-                            tma_load_2d(sK + st * C::KTILE_BYTES + q * (C::BOX * D_I), &tmap_k, 0,
-                                        cur.b * a.T_max + tok, bar_full(st));
-                            tma_load_2d(sS + st * C::SC_BYTES + q * (C::BOX * 4), &tmap_s, tok, cur.b, bar_full(st));
-                        }
-                    }
-                } else {
-                    // paged cache: one key box and one scale box per block piece of the stage, for
-                    // the pieces that hold tokens of the unit (later pieces may have no block; their
-                    // stale rows only reach scores that are never stored).  Lane q reads piece q's
-                    // block id, so the table reads overlap.
-                    const int kb = a.page_box;
+                if constexpr (C::CPASYNC) {
+                    // Piece i of the stage = 16 bytes of token row r = i / (D_I / 16), chunk c; it goes
+                    // to the K-major swizzled slot the MMA reads: 64B swizzle (d_I = 64) XORs the
+                    // chunk with bits 1-2 of the row, 128B swizzle (d_I = 128) with bits 0-2.  Rows
+                    // at or past the unit's length are zero-filled without a read.
+                    constexpr int CPR = D_I / 16;
                     const int tok0 = cur.j * C::STOK;
-                    const int live = min(C::STOK / kb, (cur.n - tok0 + kb - 1) / kb);
-                    int pb_l = 0;
-                    if (lane < live) {
-                        pb_l = a.block_table[(int64_t)cur.b * a.max_blocks + (tok0 + lane * kb) / a.block_size];
-                        if (pb_l < 0 || pb_l >= a.num_blocks) {
-                            record_status(a.status, DSA_STATUS_INDEX_OOB);
-                            pb_l = 0;
+                    const int live = max(0, min(C::STOK, cur.n - tok0));
+                    const int pt = tid;  // 0 .. PROD_THREADS - 1
+                    const uint32_t kdst = sK + st * C::KTILE_BYTES;
+                    const uint32_t sdst = sS + st * C::SC_BYTES;
+                    const uint8_t* kbase = reinterpret_cast<const uint8_t*>(a.k_I);
+                    if (a.block_table == nullptr) {
+                        const uint8_t* ksrc = kbase + ((int64_t)cur.b * a.T_max + tok0) * D_I;
+                        const float* ssrc = a.k_scale + (int64_t)cur.b * a.T_max + tok0;
+#pragma unroll 4
+                        for (int i = pt; i < C::KCHUNKS; i += C::PROD_THREADS) {
+                            const int r = i / CPR, c = i % CPR;
+                            const int sw = D_I == 64 ? ((r >> 1) & 3) : (r & 7);
+                            const bool ok = r < live;
+                            cp_async16_zfill_hint(kdst + r * D_I + ((c ^ sw) << 4), ok ? ksrc + 16 * i : kbase,
+                                                  ok ? 16u : 0u, stream_policy);
+                        }
+#pragma unroll
+                        for (int i = pt; i < C::SCHUNKS; i += C::PROD_THREADS) {
+                            const bool ok = 4 * i < live;
+                            cp_async16_zfill_hint(sdst + 16 * i, ok ? ssrc + 4 * i : a.k_scale, ok ? 16u : 0u,
+                                                  stream_policy);
+                        }
+                    } else {
+                        // paged cache: lane q holds the pool block of the stage's q-th block-sized piece
+                        // (block_size >= 64 is a power of two, so a 16-byte piece never straddles blocks)
+                        const int bs = a.block_size;
+                        const int nblk = bs >= C::STOK ? 1 : C::STOK / bs;
+                        int pb_l = 0;
+                        if (lane < nblk && tok0 + lane * bs < cur.n) {
+                            pb_l = a.block_table[(int64_t)cur.b * a.max_blocks + (tok0 + lane * bs) / bs];
+                            if (pb_l < 0 || pb_l >= a.num_blocks) {
+                                if (warp == 0) record_status(a.status, DSA_STATUS_INDEX_OOB);
+                                pb_l = 0;
+                            }
+                        }
+#pragma unroll 4
+                        for (int i = pt; i < C::KCHUNKS; i += C::PROD_THREADS) {
+                            const int r = i / CPR, c = i % CPR;
+                            const int sw = D_I == 64 ? ((r >> 1) & 3) : (r & 7);
+                            const bool ok = r < live;
+                            const int pb = __shfl_sync(0xffffffffu, pb_l, nblk == 1 ? 0 : r / bs);
+                            const int64_t prow = (int64_t)pb * bs + ((tok0 + r) & (bs - 1));
+                            cp_async16_zfill_hint(kdst + r * D_I + ((c ^ sw) << 4),
+                                                  ok ? kbase + prow * D_I + 16 * c : kbase, ok ? 16u : 0u,
+                                                  stream_policy);
+                        }
+#pragma unroll
+                        for (int i = pt; i < C::SCHUNKS; i += C::PROD_THREADS) {
+                            const int r = 4 * i;
+                            const bool ok = r < live;
+                            const int pb = __shfl_sync(0xffffffffu, pb_l, nblk == 1 ? 0 : r / bs);
+                            const int64_t prow = (int64_t)pb * bs + ((tok0 + r) & (bs - 1));
+                            cp_async16_zfill_hint(sdst + 16 * i, ok ? a.k_scale + prow : a.k_scale, ok ? 16u : 0u,
+                                                  stream_policy);
                         }
                     }
-                    if (lane == 0) mbar_arrive_expect_tx(bar_full(st), (uint32_t)live * kb * (D_I + 4));
+                    cp_async_arrive_noinc(bar_full(st));
+                } else {
+                    if (a.block_table == nullptr) {
+                        if (lane == 0) {
+                            mbar_arrive_expect_tx(bar_full(st), C::KTILE_BYTES + C::SC_BYTES);
 #pragma unroll
-                    for (int q = 0; q < C::STOK / 64; ++q) {  // kb >= 64: at most STOK / 64 pieces
-                        const int pb = __shfl_sync(0xffffffffu, pb_l, q);
-                        if (lane == 0 && q < live) {
-                            const int off = (tok0 + q * kb) % a.block_size;
-                            tma_load_2d(sK + st * C::KTILE_BYTES + q * (kb * D_I), &tmap_k, 0, pb * a.block_size + off,
-                                        bar_full(st));
-                            tma_load_2d(sS + st * C::SC_BYTES + q * (kb * 4), &tmap_s, off, pb, bar_full(st));
+                            for (int q = 0; q < C::NBOX; ++q) {
+                                const int tok = cur.j * C::STOK + q * C::BOX;
+                                tma_load_2d(sK + st * C::KTILE_BYTES + q * (C::BOX * D_I), &tmap_k, 0,
+                                            cur.b * a.T_max + tok, bar_full(st));
+                                tma_load_2d(sS + st * C::SC_BYTES + q * (C::BOX * 4), &tmap_s, tok, cur.b,
+                                            bar_full(st));
+                            }
+                        }
+                    } else {
+                        // paged cache: one key box and one scale box per block piece of the stage, for
+                        // the pieces that hold tokens of the unit (later pieces may have no block; their
+                        // stale rows only reach scores that are never stored).  Lane q reads piece q's
+                        // block id, so the table reads overlap.
+                        const int kb = a.page_box;
+                        const int tok0 = cur.j * C::STOK;
+                        const int live = min(C::STOK / kb, (cur.n - tok0 + kb - 1) / kb);
+                        int pb_l = 0;
+                        if (lane < live) {
+                            pb_l = a.block_table[(int64_t)cur.b * a.max_blocks + (tok0 + lane * kb) / a.block_size];
+                            if (pb_l < 0 || pb_l >= a.num_blocks) {
+                                record_status(a.status, DSA_STATUS_INDEX_OOB);
+                                pb_l = 0;
+                            }
+                        }
+                        if (lane == 0) mbar_arrive_expect_tx(bar_full(st), (uint32_t)live * kb * (D_I + 4));
+#pragma unroll
+                        for (int q = 0; q < C::STOK / 64; ++q) {  // kb >= 64: at most STOK / 64 pieces
+                            const int pb = __shfl_sync(0xffffffffu, pb_l, q);
+                            if (lane == 0 && q < live) {
+                                const int off = (tok0 + q * kb) % a.block_size;
+                                tma_load_2d(sK + st * C::KTILE_BYTES + q * (kb * D_I), &tmap_k, 0,
+                                            pb * a.block_size + off, bar_full(st));
+                                tma_load_2d(sS + st * C::SC_BYTES + q * (kb * 4), &tmap_s, off, pb, bar_full(st));
+                            }
                         }
                     }
                 }
                 ++issued;
                 cur.advance(a);
             }
-            if (lane == 0 && *abort_flag) {
+            if constexpr (C::CPASYNC) {
+                // copies still in flight land before the CTA's shared memory is released
+                cp_async_wait_all();
+            } else if (lane == 0 && *abort_flag) {
                 // drain copies still in flight before the CTA's shared memory is released
                 for (int it = issued - C::STAGES < 0 ? 0 : issued - C::STAGES; it < issued; ++it)
                     mbar_wait(bar_full(it % C::STAGES), (it / C::STAGES) & 1, nullptr, nullptr, 50000000ull);
             }
         }
-    } else if (warp == 1) {
+    } else if (warp == C::MMA_WARP) {
         if (lane == 0 && count > 0) {
             // ---------------- MMA issuer
             TileCursor<C::STOK, R> cur;
@@ -368,6 +456,8 @@ __global__ void __launch_bounds__(IdxCfg<D_I, R>::THREADS, 1)
                 }
                 const int st = it % C::STAGES;
                 if (!mbar_wait(bar_full(st), (it / C::STAGES) & 1, abort_flag, a.status)) break;
+                // keys written by cp.async (generic proxy) are read by the tensor core (async proxy)
+                if constexpr (C::CPASYNC) fence_proxy_async_smem();
                 const int acc = it % C::ACC;
                 // polled: the accumulator comes back while the epilogue warps compute, and a
                 // suspended wait would resume late on the tensor pipe's critical path
@@ -503,7 +593,7 @@ __global__ void __launch_bounds__(IdxCfg<D_I, R>::THREADS, 1)
     }
     tc_fence_before();
     __syncthreads();
-    if (warp == 1) {
+    if (warp == C::MMA_WARP) {
         tc_fence_after();
         tmem_dealloc(tmem, C::TMEM_COLS);
     }

@@ -185,6 +185,20 @@ __device__ __forceinline__ void cp_async16_zfill(uint32_t dst, const void* src, 
                  "r"(src_bytes)
                  : "memory");
 }
+// L2 policy for data read once (a streamed cache): its lines are the first to go, so
+// that data written for the next kernel stays in L2.
+__device__ __forceinline__ uint64_t l2_policy_evict_first() {
+    uint64_t p;
+    asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(p));
+    return p;
+}
+// The same 16-byte copy with an L2 cache policy.
+__device__ __forceinline__ void cp_async16_zfill_hint(uint32_t dst, const void* src, uint32_t src_bytes,
+                                                      uint64_t policy) {
+    asm volatile("cp.async.cg.shared.global.L2::cache_hint [%0], [%1], 16, %2, %3;" ::"r"(dst),
+                 "l"(reinterpret_cast<uint64_t>(src)), "r"(src_bytes), "l"(policy)
+                 : "memory");
+}
 // Arrive on the mbarrier once every cp.async this thread issued so far has
 // landed; the arrival is counted in the barrier's expected count (noinc).
 __device__ __forceinline__ void cp_async_arrive_noinc(uint32_t bar) {
