@@ -115,6 +115,7 @@ struct IdxCfg {
 
 struct IdxShared {
     int row0, j0, count;
+    int n0, b0, nt0;  // the first unit's longest row, sequence and stage count
     int tmem_base;
     int abort_flag;
 };
@@ -169,6 +170,14 @@ struct TileCursor {
         j = j0;
         load_row(a);
     }
+    // the same start from values another warp loaded (no global reads on the way in)
+    __device__ void start(int r0, int j0, int n0, int b0, int nt0) {
+        row = r0;
+        j = j0;
+        n = n0;
+        b = b0;
+        nt = nt0;
+    }
     __device__ void advance(const IndexerArgs& a) {
         if (++j >= nt) {
             j = 0;
@@ -217,7 +226,9 @@ __global__ void __launch_bounds__(IdxCfg<D_I, R>::THREADS, 1)
                                                  // completed before)
         }
         for (int q = 0; q < 2; ++q) {
-            mbar_init(bar_qfull(q), 1);                    // producer arrival with the q8 block's tx bytes
+            // producer arrivals: one with the q8 block's tx bytes (issued first), one once the
+            // folded weights are in shared memory (written after the unit's first key copies)
+            mbar_init(bar_qfull(q), 2);
             mbar_init(bar_qempty(q), 1 + C::EPI_WARPS);    // MMA commit + every epilogue warp
         }
         for (int c = 0; c < C::ACC; ++c) {
@@ -279,6 +290,11 @@ __global__ void __launch_bounds__(IdxCfg<D_I, R>::THREADS, 1)
             sh->row0 = row0;
             sh->j0 = j0;
             sh->count = (int)(end - begin);
+            TileCursor<C::STOK, R> first;
+            first.start(a, row0, j0);
+            sh->n0 = first.n;
+            sh->b0 = first.b;
+            sh->nt0 = first.nt;
         }
     }
     tc_fence_before();
@@ -292,26 +308,22 @@ __global__ void __launch_bounds__(IdxCfg<D_I, R>::THREADS, 1)
         // ---------------- producer
         if (count > 0) {
             TileCursor<C::STOK, R> cur;
-            cur.start(a, sh->row0, sh->j0);
+            cur.start(sh->row0, sh->j0, sh->n0, sh->b0, sh->nt0);
             int qi = -1;
             int issued = 0;
             const uint64_t stream_policy = l2_policy_evict_first();
             for (int it = 0; it < count; ++it) {
-                if (it == 0 || cur.j == 0) {
+                const bool new_unit = it == 0 || cur.j == 0;
+                int qb = 0;
+                if (new_unit) {
                     ++qi;
-                    const int qb = qi & 1;
+                    qb = qi & 1;
                     if (warp == 0) {
                         if (qi >= 2) {
                             const bool okq = mbar_wait(bar_qempty(qb), ((qi - 2) >> 1) & 1, abort_flag, a.status);
                             if (!__all_sync(0xffffffffu, okq)) break;
                         }
-                        // folded weights w * q_scale of the unit's rows (0 past the last row)
-                        const int64_t o = (int64_t)cur.row * C::NCOL;
-                        const __nv_bfloat16* wr = reinterpret_cast<const __nv_bfloat16*>(a.w) + o;
-                        const int64_t lim = (int64_t)a.Nq * C::HEADS - o;
-                        for (int i = lane; i < C::NCOL; i += 32)
-                            wq_smem[qb * C::NCOL + i] = i < lim ? __bfloat162float(wr[i]) * a.q_scale[o + i] : 0.f;
-                        __syncwarp();
+                        // the unit's q8 block first: it depends on nothing the copies below need
                         if (lane == 0) {
                             mbar_arrive_expect_tx(bar_qfull(qb), C::Q_BYTES);
                             tma_load_2d(sQ + qb * C::Q_BYTES, &tmap_q, 0, cur.row * C::NCOL, bar_qfull(qb));
@@ -326,35 +338,53 @@ __global__ void __launch_bounds__(IdxCfg<D_I, R>::THREADS, 1)
                 if constexpr (C::CPASYNC) {
                     // Piece i of the stage = 16 bytes of token row r = i / (D_I / 16), chunk c; it goes
                     // to the K-major swizzled slot the MMA reads: 64B swizzle (d_I = 64) XORs the
-                    // chunk with bits 1-2 of the row, 128B swizzle (d_I = 128) with bits 0-2.  Rows
-                    // at or past the unit's length are zero-filled without a read.
+                    // chunk with bits 1-2 of the row, 128B swizzle (d_I = 128) with bits 0-2.  Thread
+                    // pt copies pieces pt + k * PROD_THREADS: its chunk c and its rows' swizzle are the
+                    // same for every k (the row step is a multiple of 8), so each copy is a fixed offset
+                    // from the first.  Rows at or past the unit's length are zero-filled without a read.
                     constexpr int CPR = D_I / 16;
+                    constexpr int RSTEP = C::PROD_THREADS / CPR;        // rows between a thread's pieces
+                    constexpr int NIT = C::KCHUNKS / C::PROD_THREADS;   // pieces per thread per stage
+                    constexpr int STEP = RSTEP * D_I;                   // bytes between them (1024)
+                    static_assert(RSTEP % 8 == 0, "the swizzle phase repeats every 8 rows");
                     const int tok0 = cur.j * C::STOK;
                     const int live = max(0, min(C::STOK, cur.n - tok0));
                     const int pt = tid;  // 0 .. PROD_THREADS - 1
-                    const uint32_t kdst = sK + st * C::KTILE_BYTES;
-                    const uint32_t sdst = sS + st * C::SC_BYTES;
+                    const int c = pt % CPR, r0 = pt / CPR;
+                    const int sw = D_I == 64 ? ((r0 >> 1) & 3) : (r0 & 7);
+                    const uint32_t kd0 = sK + st * C::KTILE_BYTES + r0 * D_I + ((c ^ sw) << 4);
+                    const uint32_t sd0 = sS + st * C::SC_BYTES + 16 * pt;
                     const uint8_t* kbase = reinterpret_cast<const uint8_t*>(a.k_I);
                     if (a.block_table == nullptr) {
-                        const uint8_t* ksrc = kbase + ((int64_t)cur.b * a.T_max + tok0) * D_I;
-                        const float* ssrc = a.k_scale + (int64_t)cur.b * a.T_max + tok0;
-#pragma unroll 4
-                        for (int i = pt; i < C::KCHUNKS; i += C::PROD_THREADS) {
-                            const int r = i / CPR, c = i % CPR;
-                            const int sw = D_I == 64 ? ((r >> 1) & 3) : (r & 7);
-                            const bool ok = r < live;
-                            cp_async16_zfill_hint(kdst + r * D_I + ((c ^ sw) << 4), ok ? ksrc + 16 * i : kbase,
-                                                  ok ? 16u : 0u, stream_policy);
-                        }
+                        const uint8_t* ks0 = kbase + ((int64_t)cur.b * a.T_max + tok0) * D_I + 16 * pt;
+                        const float* ss0 = a.k_scale + (int64_t)cur.b * a.T_max + tok0 + 4 * pt;
+                        if (live == C::STOK) {
 #pragma unroll
-                        for (int i = pt; i < C::SCHUNKS; i += C::PROD_THREADS) {
-                            const bool ok = 4 * i < live;
-                            cp_async16_zfill_hint(sdst + 16 * i, ok ? ssrc + 4 * i : a.k_scale, ok ? 16u : 0u,
-                                                  stream_policy);
+                            for (int k = 0; k < NIT; ++k) cp_async16_hint(kd0 + k * STEP, ks0 + k * STEP, stream_policy);
+#pragma unroll
+                            for (int k = 0; k < C::SCHUNKS / C::PROD_THREADS; ++k)
+                                cp_async16_hint(sd0 + k * 16 * C::PROD_THREADS, ss0 + k * 4 * C::PROD_THREADS,
+                                                stream_policy);
+                        } else {
+#pragma unroll
+                            for (int k = 0; k < NIT; ++k) {
+                                const bool ok = r0 + k * RSTEP < live;
+                                cp_async16_zfill_hint(kd0 + k * STEP, ok ? ks0 + k * STEP : kbase, ok ? 16u : 0u,
+                                                      stream_policy);
+                            }
+#pragma unroll
+                            for (int k = 0; k < C::SCHUNKS / C::PROD_THREADS; ++k) {
+                                const bool ok = 4 * (pt + k * C::PROD_THREADS) < live;
+                                cp_async16_zfill_hint(sd0 + k * 16 * C::PROD_THREADS,
+                                                      ok ? ss0 + k * 4 * C::PROD_THREADS : a.k_scale, ok ? 16u : 0u,
+                                                      stream_policy);
+                            }
                         }
                     } else {
                         // paged cache: lane q holds the pool block of the stage's q-th block-sized piece
-                        // (block_size >= 64 is a power of two, so a 16-byte piece never straddles blocks)
+                        // (block_size >= 64 is a power of two; a thread's rows r0 + k * RSTEP with
+                        // r0 < RSTEP never straddle a block, so piece k lies in block slot
+                        // (k * RSTEP) / block_size)
                         const int bs = a.block_size;
                         const int nblk = bs >= C::STOK ? 1 : C::STOK / bs;
                         int pb_l = 0;
@@ -365,25 +395,25 @@ __global__ void __launch_bounds__(IdxCfg<D_I, R>::THREADS, 1)
                                 pb_l = 0;
                             }
                         }
-#pragma unroll 4
-                        for (int i = pt; i < C::KCHUNKS; i += C::PROD_THREADS) {
-                            const int r = i / CPR, c = i % CPR;
-                            const int sw = D_I == 64 ? ((r >> 1) & 3) : (r & 7);
+                        const int lbs = 31 - __clz(bs);
+                        const int off0 = tok0 & (bs - 1);  // the stage's offset inside its first block
+#pragma unroll
+                        for (int k = 0; k < NIT; ++k) {
+                            const int r = r0 + k * RSTEP;
                             const bool ok = r < live;
-                            const int pb = __shfl_sync(0xffffffffu, pb_l, nblk == 1 ? 0 : r / bs);
-                            const int64_t prow = (int64_t)pb * bs + ((tok0 + r) & (bs - 1));
-                            cp_async16_zfill_hint(kdst + r * D_I + ((c ^ sw) << 4),
-                                                  ok ? kbase + prow * D_I + 16 * c : kbase, ok ? 16u : 0u,
-                                                  stream_policy);
+                            const int pb = __shfl_sync(0xffffffffu, pb_l, (k * RSTEP) >> lbs);
+                            const int64_t prow = ((int64_t)pb << lbs) + ((off0 + r) & (bs - 1));
+                            cp_async16_zfill_hint(kd0 + k * STEP, ok ? kbase + prow * D_I + 16 * c : kbase,
+                                                  ok ? 16u : 0u, stream_policy);
                         }
 #pragma unroll
-                        for (int i = pt; i < C::SCHUNKS; i += C::PROD_THREADS) {
-                            const int r = 4 * i;
+                        for (int k = 0; k < C::SCHUNKS / C::PROD_THREADS; ++k) {
+                            const int r = 4 * (pt + k * C::PROD_THREADS);
                             const bool ok = r < live;
-                            const int pb = __shfl_sync(0xffffffffu, pb_l, nblk == 1 ? 0 : r / bs);
-                            const int64_t prow = (int64_t)pb * bs + ((tok0 + r) & (bs - 1));
-                            cp_async16_zfill_hint(sdst + 16 * i, ok ? a.k_scale + prow : a.k_scale, ok ? 16u : 0u,
-                                                  stream_policy);
+                            const int pb = __shfl_sync(0xffffffffu, pb_l, r >> lbs);
+                            const int64_t prow = ((int64_t)pb << lbs) + ((off0 + r) & (bs - 1));
+                            cp_async16_zfill_hint(sd0 + k * 16 * C::PROD_THREADS, ok ? a.k_scale + prow : a.k_scale,
+                                                  ok ? 16u : 0u, stream_policy);
                         }
                     }
                     cp_async_arrive_noinc(bar_full(st));
@@ -429,6 +459,17 @@ __global__ void __launch_bounds__(IdxCfg<D_I, R>::THREADS, 1)
                         }
                     }
                 }
+                if (new_unit && warp == 0) {
+                    // folded weights w * q_scale of the unit's rows (0 past the last row), after the
+                    // stage's copies so that their load latency does not delay the key stream
+                    const int64_t o = (int64_t)cur.row * C::NCOL;
+                    const __nv_bfloat16* wr = reinterpret_cast<const __nv_bfloat16*>(a.w) + o;
+                    const int64_t lim = (int64_t)a.Nq * C::HEADS - o;
+                    for (int i = lane; i < C::NCOL; i += 32)
+                        wq_smem[qb * C::NCOL + i] = i < lim ? __bfloat162float(wr[i]) * a.q_scale[o + i] : 0.f;
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(bar_qfull(qb));
+                }
                 ++issued;
                 cur.advance(a);
             }
@@ -445,7 +486,7 @@ __global__ void __launch_bounds__(IdxCfg<D_I, R>::THREADS, 1)
         if (lane == 0 && count > 0) {
             // ---------------- MMA issuer
             TileCursor<C::STOK, R> cur;
-            cur.start(a, sh->row0, sh->j0);
+            cur.start(sh->row0, sh->j0, sh->n0, sh->b0, sh->nt0);
             int qi = -1, qb = 0;
             int last_acc = -1, last_it = -1;
             for (int it = 0; it < count; ++it) {
@@ -503,7 +544,7 @@ __global__ void __launch_bounds__(IdxCfg<D_I, R>::THREADS, 1)
         // warp's 32 lanes, i.e. token `tok` of every stage
         const int tok = h * C::TILE + sub * 32 + g + 8 * (2 * (i4 & 1) + (i4 >> 1));
         TileCursor<C::STOK, R> cur;
-        if (count > 0) cur.start(a, sh->row0, sh->j0);
+        if (count > 0) cur.start(sh->row0, sh->j0, sh->n0, sh->b0, sh->nt0);
         int qi = -1;
         int nrow = 0;               // this thread's scores exist for s < nrow (s = stage base + tok)
         float* srow = nullptr;      // score row of the block's query row, offset by tok

@@ -155,10 +155,29 @@ __device__ __forceinline__ uint4 ld_shared_cluster_v4_u32(uint32_t addr) {
                  : "memory");
     return v;
 }
+// Stores into another CTA's shared memory (address from mapa_shared); made visible to the
+// owner by a cluster barrier (release on arrive, acquire on wait).
+__device__ __forceinline__ void st_shared_cluster_v4_u32(uint32_t addr, uint32_t x, uint32_t y, uint32_t z, uint32_t w) {
+    asm volatile("st.shared::cluster.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(x), "r"(y), "r"(z), "r"(w)
+                 : "memory");
+}
+__device__ __forceinline__ void st_shared_cluster_f32(uint32_t addr, float v) {
+    asm volatile("st.shared::cluster.f32 [%0], %1;" ::"r"(addr), "f"(v) : "memory");
+}
 // Full cluster barrier (every thread of every CTA): shared-memory writes before
 // it are visible to the other CTAs' reads after it.
 __device__ __forceinline__ void cluster_sync_all() {
     asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+
+// The two halves of a cluster barrier, for work that can run between them: arrive once
+// this thread's accesses to other CTAs' shared memory are done, wait before the CTA's own
+// shared memory may go away.  Every thread of every CTA executes both, in this order.
+__device__ __forceinline__ void cluster_arrive_release() {
+    asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void cluster_wait_acquire() {
+    asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory");
 }
 
 // ---------------------------------------------------------------- TMA (tiled, no multicast)
@@ -192,7 +211,13 @@ __device__ __forceinline__ uint64_t l2_policy_evict_first() {
     asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(p));
     return p;
 }
-// The same 16-byte copy with an L2 cache policy.
+// 16-byte copy with an L2 cache policy (every byte read).
+__device__ __forceinline__ void cp_async16_hint(uint32_t dst, const void* src, uint64_t policy) {
+    asm volatile("cp.async.cg.shared.global.L2::cache_hint [%0], [%1], 16, %2;" ::"r"(dst),
+                 "l"(reinterpret_cast<uint64_t>(src)), "l"(policy)
+                 : "memory");
+}
+// The same 16-byte copy with an L2 cache policy and a source size (0 = zero-fill, no read).
 __device__ __forceinline__ void cp_async16_zfill_hint(uint32_t dst, const void* src, uint32_t src_bytes,
                                                       uint64_t policy) {
     asm volatile("cp.async.cg.shared.global.L2::cache_hint [%0], [%1], 16, %2, %3;" ::"r"(dst),

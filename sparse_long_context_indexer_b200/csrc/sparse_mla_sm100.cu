@@ -87,6 +87,10 @@ constexpr uint32_t kColQ = 0;            // Q: 288 columns (576 bf16), low lanes
 constexpr uint32_t kColS = 384;          // S buffers: [384, 448), [448, 512), low lanes
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
 constexpr int kPrefetchTiles = kStages + 1;  // L2 prefetch distance of the gather, in tiles
+// split merge: received rows (at most 70 slots of (split, owned head), 1 KB each) and then their
+// lse values, inside the idle gather stages
+constexpr int kMergeLseOff = 72 * 1024;
+static_assert(kMergeLseOff + 4 * 72 <= kStages * kKvStageBytes, "merge slots fit the gather stages");
 constexpr uint32_t kIdescQK = make_idesc(kCtaHeads, kTileRows, 1 /*bf16*/, 1 /*bf16*/, 0, 0);
 constexpr uint32_t kIdescPV = make_idesc(kCtaHeads, 256, 1 /*bf16*/, 1 /*bf16*/, 0 /*A K-major*/, 1 /*B MN-major*/);
 
@@ -579,17 +583,24 @@ __global__ void __launch_bounds__(kThreads, 1)
         const bool read_o = have_o && ok;
         if (read_o) tc_fence_after();
         const int64_t th = (int64_t)t * kMlaHeads + half * kCtaHeads + prow;
-        if (hh == 0) {
-            if (kOut == kOutCluster) {
-                reinterpret_cast<float*>(smem + kOffP)[prow] = lse_v;  // beside P's (now idle) tile
-            } else if (kOut == kOutFinal) {
+        if (kOut == kOutCluster) {
+            // every warp of the CTA stages the rows after the role loops: publish this head's
+            // normaliser and lse, and whether its O may be read (in P's idle tile)
+            if (hh == 0) {
+                float* pub = reinterpret_cast<float*>(smem + kOffP);
+                pub[prow] = read_o ? inv_l : 0.f;
+                pub[kCtaHeads + prow] = lse_v;
+                if (r == 0) reinterpret_cast<int*>(pub)[2 * kCtaHeads + warp] = read_o ? 1 : 0;
+            }
+        } else if (hh == 0) {
+            if (kOut == kOutFinal) {
                 if (a.lse) a.lse[th] = lse_v;
             } else {
                 a.part_lse[(int64_t)split * a.Nq * kMlaHeads + th] = lse_v;
             }
         }
 #pragma unroll 1
-        for (int c0 = 0; c0 < kDV; c0 += 64) {
+        for (int c0 = 0; c0 < (kOut == kOutCluster ? 0 : kDV); c0 += 64) {
             uint32_t ov[32];
             if (read_o) {
                 tmem_ld16x2_32(o_base + c0, ov);
@@ -599,25 +610,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 for (int c = 0; c < 32; ++c) ov[c] = 0u;
             }
             const int col = c0 + 32 * hh;  // first output column of this piece
-            if (kOut == kOutCluster) {
-                // bf16 rows for the peers (half the bytes over the cluster network; the merge
-                // weights and sums stay fp32): row h at h * 1024 bytes, 16-byte granule j (eight
-                // values) at (j & ~7) | ((j ^ h) & 7)
-                const uint32_t row_addr = sKv + prow * (kDV * 2);
-                const int jb = col >> 3;  // a multiple of 4
-#pragma unroll
-                for (int q4 = 0; q4 < 4; ++q4) {
-                    uint32_t w[4];
-#pragma unroll
-                    for (int e = 0; e < 4; ++e)
-                        w[e] = pack_bf16x2(__uint_as_float(ov[8 * q4 + 2 * e]) * inv_l,
-                                           __uint_as_float(ov[8 * q4 + 2 * e + 1]) * inv_l);
-                    const int j = jb + q4;
-                    asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(row_addr + (((j & ~7) | ((j ^ prow) & 7)) << 4)),
-                                 "r"(w[0]), "r"(w[1]), "r"(w[2]), "r"(w[3])
-                                 : "memory");
-                }
-            } else if (kOut == kOutFinal) {
+            if (kOut == kOutFinal) {
                 // bf16 TMA-store boxes of 64 heads x 64 columns: box k holds columns [64k, 64k + 64)
                 const uint32_t box = sKv + prow * 128 + (col >> 6) * kChunkBytes;
                 const int g0 = (col & 63) >> 3;
@@ -659,37 +652,73 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
     }
     if (kOut == kOutCluster) {
-        // ---- merge of the splits: CTA `rank` of the cluster owns heads [rank * hp, rank * hp + hp)
+        // ---- merge of the splits.  CTA `rank` of the cluster owns heads [rank * hp, rank * hp + hp)
         // O = sum_s exp(lse_s - L) O_s / sum_s exp(lse_s - L),  lse = L + ln sum_s exp(lse_s - L)
-        __syncthreads();
-        cluster_sync_all();
+        // Every CTA pushes its normalised bf16 rows (and lse values) straight into the shared
+        // memory of the head's owner -- stores cross the cluster network without a round trip
+        // each -- and every owner then merges from its own shared memory.  The first barrier
+        // makes sure no peer still reads its gather stages (the push lands there).
         const int S = a.splits;
         const int rank = (int)cluster_ctarank();
         const int hp = (kCtaHeads + S - 1) / S;
-        const int h0 = rank * hp;
-        const int nunits = 2 * max(0, min(kCtaHeads, h0 + hp) - h0);  // (head, half row) units
-        // every unit: lane j owns granule j of its half row (eight bf16 values) from each
-        // split, all loaded before any is used (the reads cross the cluster network)
-        for (int u = warp; u < nunits; u += kThreads / 32) {
-            const int h = h0 + (u >> 1);
-            const int jh = (u & 1) * 32;  // first granule of the half row
-            const float ls = lane < S ? ld_shared_cluster_f32(mapa_shared(sP + h * 4, lane)) : -CUDART_INF_F;
-            float x[kMlaClusterMaxSplits][8];
-            const int j = jh + lane;
-            const uint32_t g0 = (j & ~7) | ((j ^ h) & 7);
+        const float* pub = reinterpret_cast<const float*>(smem + kOffP);
+        __syncthreads();
+        cluster_sync_all();
+        tc_fence_after();
+        {
+            // receive slot of (split s, owned head hl): 1 KB row at sKv + (s * hp + hl) * 1024, its
+            // 16-byte granule j (eight values) at (j & ~7) | ((j ^ row) & 7); its lse at
+            // sKv + kMergeLseOff + 4 * (s * hp + hl)
+            const int sub = warp & 3;                      // TMEM sub-partition this warp may read
+            const int nw = sub == 0 ? 4 : 3;               // warps 0..12 per sub-partition
+            const int iw = warp >> 2;
+            const int r = lane & 15, hh = lane >> 4;
+            const int prow = sub * 16 + r;                 // head within this CTA
+            const int owner = prow / hp, hl = prow - owner * hp;
+            const int slot = split * hp + hl;
+            const uint32_t dst_row = mapa_shared(sKv + slot * (kDV * 2), (uint32_t)owner);
+            const float inv_l = pub[prow];
+            const bool sub_ok = reinterpret_cast<const int*>(pub)[2 * kCtaHeads + sub] != 0;
+            const uint32_t o_sub = tmem + ((uint32_t)(sub * 32) << 16) + kLaneHi;
+#pragma unroll 1
+            for (int ck = iw; ck < kDV / 64; ck += nw) {
+                const int c0 = ck * 64;
+                uint32_t ov[32];
+                if (sub_ok) {
+                    tmem_ld16x2_32(o_sub + c0, ov);
+                    tmem_wait_ld();
+                } else {
 #pragma unroll
-            for (int sp = 0; sp < kMlaClusterMaxSplits; ++sp) {
-                if (sp < S) {
-                    const uint32_t rbase = mapa_shared(sKv + h * (kDV * 2), (uint32_t)sp);
-                    const uint4 v = ld_shared_cluster_v4_u32(rbase + (g0 << 4));
-                    const uint32_t vw[4] = {v.x, v.y, v.z, v.w};
+                    for (int c = 0; c < 32; ++c) ov[c] = 0u;
+                }
+                const int jb = (c0 + 32 * hh) >> 3;  // first granule of this thread's 32 columns
 #pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        x[sp][2 * e] = __uint_as_float(vw[e] << 16);
-                        x[sp][2 * e + 1] = __uint_as_float(vw[e] & 0xFFFF0000u);
-                    }
+                for (int q4 = 0; q4 < 4; ++q4) {
+                    uint32_t w[4];
+#pragma unroll
+                    for (int e = 0; e < 4; ++e)
+                        w[e] = pack_bf16x2(__uint_as_float(ov[8 * q4 + 2 * e]) * inv_l,
+                                           __uint_as_float(ov[8 * q4 + 2 * e + 1]) * inv_l);
+                    const int j = jb + q4;
+                    st_shared_cluster_v4_u32(dst_row + ((((j & ~7) | ((j ^ slot) & 7))) << 4), w[0], w[1], w[2], w[3]);
                 }
             }
+        }
+        if (tid < kCtaHeads) {
+            const int ow = tid / hp;
+            st_shared_cluster_f32(mapa_shared(sKv + kMergeLseOff + 4 * (split * hp + tid - ow * hp), (uint32_t)ow),
+                                  pub[kCtaHeads + tid]);
+        }
+        cluster_sync_all();  // every push has landed
+        const int h0 = rank * hp;
+        const int nh = max(0, min(kCtaHeads, h0 + hp) - h0);
+        const int nunits = 2 * nh;  // (head, half row) units
+        const float* lse_in = reinterpret_cast<const float*>(smem + kOffKv + kMergeLseOff);
+        for (int u = warp; u < nunits; u += kThreads / 32) {
+            const int hl = u >> 1;
+            const int jh = (u & 1) * 32;  // first granule of the half row
+            const int j = jh + lane;
+            const float ls = lane < S ? lse_in[lane * hp + hl] : -CUDART_INF_F;
             float L = ls;
 #pragma unroll
             for (int o = 16; o > 0; o >>= 1) L = fmaxf(L, __shfl_xor_sync(0xffffffffu, L, o));
@@ -702,19 +731,27 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (int sp = 0; sp < kMlaClusterMaxSplits; ++sp) {
                 const float es = __shfl_sync(0xffffffffu, e, sp);  // 0 for absent or empty splits
                 if (sp < S) {
+                    const int slot = sp * hp + hl;
+                    uint4 v;
+                    asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
+                                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+                                 : "r"(sKv + slot * (kDV * 2) + ((((j & ~7) | ((j ^ slot) & 7))) << 4)));
+                    const uint32_t vw[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
-                    for (int c = 0; c < 8; ++c) acc[c] = fmaf(es, x[sp][c], acc[c]);
+                    for (int q = 0; q < 4; ++q) {
+                        acc[2 * q] = fmaf(es, __uint_as_float(vw[q] << 16), acc[2 * q]);
+                        acc[2 * q + 1] = fmaf(es, __uint_as_float(vw[q] & 0xFFFF0000u), acc[2 * q + 1]);
+                    }
                 }
             }
             const float inv = esum > 0.f ? 1.f / esum : 0.f;
-            const int64_t trow = (int64_t)t * kMlaHeads + half * kCtaHeads + h;
+            const int64_t trow = (int64_t)t * kMlaHeads + half * kCtaHeads + h0 + hl;
             uint4* o = reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(a.out) + trow * kDV);
             o[j] = make_uint4(pack_bf16x2(acc[0] * inv, acc[1] * inv), pack_bf16x2(acc[2] * inv, acc[3] * inv),
                               pack_bf16x2(acc[4] * inv, acc[5] * inv), pack_bf16x2(acc[6] * inv, acc[7] * inv));
             if (lane == 0 && (u & 1) == 0 && a.lse) a.lse[trow] = esum > 0.f ? L + __logf(esum) : -CUDART_INF_F;
         }
-        // peers keep reading this CTA's rows until every CTA of the cluster is done
-        cluster_sync_all();
+        // no peer touches this CTA's shared memory after the last barrier: no exit barrier
     }
     tc_fence_before();
     __syncthreads();

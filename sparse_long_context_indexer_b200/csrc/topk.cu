@@ -27,10 +27,12 @@
 //     8-bit digits of all keys (warp-private histograms with match_any
 //     aggregation, merged across the cluster).  Rows whose keys are all equal
 //     take the first k positions directly.
-//  3. A final pass compacts the selected positions in position order with one
-//     block-wide vector scan per sweep; CTA r learns from the lower-ranked CTAs
-//     how many ties and outputs precede it, which gives the lower-index tie
-//     rule across the whole row.
+//  3. A final pass compacts the selected positions in position order: each warp
+//     owns a contiguous segment of the CTA's keys, counts them in a first pass,
+//     and writes its selected positions in a second, with ballots ranking the
+//     keys inside each step.  CTA r knows from the gathered threshold-bin keys
+//     how many ties and outputs the lower-ranked CTAs hold, which gives the
+//     lower-index tie rule across the whole row.
 #include <cooperative_groups.h>
 #include <cuda_runtime.h>
 
@@ -42,31 +44,34 @@ namespace cg = cooperative_groups;
 namespace dsa {
 namespace {
 
-constexpr int kThreads = 512;
 constexpr int kMaxCluster = kTopkMaxCluster;
-constexpr int kWarps = kThreads / 32;
 constexpr int kBins = 256;
-constexpr int kRounds = 8;  // compaction: a thread owns 4 consecutive keys in each of kRounds rounds
-// shared memory map (32-bit words)
-constexpr int kOffPriv = 0;                          // kWarps x kBins warp-private histograms
-constexpr int kOffHist = kOffPriv + kWarps * kBins;  // 2 x kBins per-CTA histogram (ping-pong, read remotely)
-constexpr int kOffTot = kOffHist + 2 * kBins;        // kBins cluster-wide histogram
-constexpr int kOffMisc = kOffTot + kBins;            // 64 words: results, counts (read remotely), scan scratch
-constexpr int kOffScan = kOffMisc + 64;              // vector-scan scratch
-constexpr int kScanWords = kWarps * kRounds + kRounds + 16;
+constexpr int kLoadBatch = 8;  // 16-byte score loads in flight per thread
 constexpr int kFineBits = 11;
 constexpr int kFineBins = 1 << kFineBits;  // adaptive histogram bins
 constexpr int kCandMax = 2048;             // threshold-bin keys resolved on chip by every CTA
 constexpr int kRankMax = 64;               // up to this many, tau is found by direct ranking
 constexpr uint32_t kFloorOctaves = 8;      // the first histogram's floor: 2^-8 of the row's largest score
-// Keep a CTA small enough for two per SM at the long-decode chunk (16K keys): with one per
-// SM, 16 clusters of 8 no longer fit the GPCs in one wave.
-constexpr int kOffFine = (kOffScan + kScanWords + 3) & ~3;  // kFineBins counts (read remotely)
-constexpr int kOffRange = kOffFine + kFineBins;            // this CTA's range of cluster-wide bin totals
-constexpr int kOffGather = kOffRange + kFineBins;          // all candidates of the row
-constexpr int kOffKeys = (kOffGather + kCandMax + 3) & ~3;
-static_assert(kWarps * kBins >= kCandMax, "the local candidate list lives in the warp-private histograms");
-constexpr int kBaseWords = kOffKeys;
+
+// Shared-memory map (32-bit words) of a CTA of T threads.  512-thread CTAs fit two per SM
+// (launches with more rows than one wave holds); 1024-thread CTAs take a whole SM (launches
+// whose clusters all fit one wave: decode).
+template <int T>
+struct TopkLayout {
+    static constexpr int kWarps = T / 32;
+    static constexpr int kOffPriv = 0;                          // kWarps x kBins warp-private histograms
+    static constexpr int kOffHist = kOffPriv + kWarps * kBins;  // 2 x kBins per-CTA histogram (ping-pong, read remotely)
+    static constexpr int kOffTot = kOffHist + 2 * kBins;        // kBins cluster-wide histogram
+    static constexpr int kOffMisc = kOffTot + kBins;            // 64 words: results, counts (read remotely)
+    static constexpr int kOffScan = kOffMisc + 64;              // block-scan and compaction scratch
+    static constexpr int kScanWords = 4 * kWarps + 16;
+    static constexpr int kOffFine = (kOffScan + kScanWords + 3) & ~3;  // kFineBins counts (read remotely)
+    static constexpr int kOffRange = kOffFine + kFineBins;            // this CTA's range of cluster-wide bin totals
+    static constexpr int kOffGather = kOffRange + kFineBins;          // all candidates of the row
+    static constexpr int kOffKeys = (kOffGather + kCandMax + 3) & ~3;
+    static constexpr int kBaseWords = kOffKeys;
+    static_assert(kWarps * kBins >= kCandMax, "the local candidate list lives in the warp-private histograms");
+};
 
 __device__ __forceinline__ uint32_t score_key(float f) {
     uint32_t u = __float_as_uint(f);
@@ -75,7 +80,9 @@ __device__ __forceinline__ uint32_t score_key(float f) {
 }
 
 // Block-wide exclusive scan of one int per thread.  scratch >= kWarps + 1 ints.
+template <int T>
 __device__ __forceinline__ int block_scan1(int v, int* scratch, int* total) {
+    constexpr int kWarps = T / 32;
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     int incl = v;
 #pragma unroll
@@ -103,48 +110,14 @@ __device__ __forceinline__ int block_scan1(int v, int* scratch, int* total) {
     return r;
 }
 
-// Block-wide exclusive scan of kRounds ints per thread, rounds in order:
-// element (rr, tid) is preceded by all of rounds < rr and by threads < tid of
-// round rr.  Returns exclusive prefixes in pre[] (offset by base) and the new base.
-__device__ __forceinline__ int block_scan_rounds(const int (&v)[kRounds], int (&pre)[kRounds], int base, int* scr) {
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    int incl[kRounds];
-#pragma unroll
-    for (int rr = 0; rr < kRounds; ++rr) incl[rr] = v[rr];
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-#pragma unroll
-        for (int rr = 0; rr < kRounds; ++rr) {
-            const int u = __shfl_up_sync(0xffffffffu, incl[rr], o);
-            if (lane >= o) incl[rr] += u;
-        }
-    }
-    if (lane == 31) {
-#pragma unroll
-        for (int rr = 0; rr < kRounds; ++rr) scr[warp * kRounds + rr] = incl[rr];
-    }
-    __syncthreads();
-    if (threadIdx.x < kRounds) {
-        int run = 0;
-        for (int w = 0; w < kWarps; ++w) {
-            const int x = scr[w * kRounds + threadIdx.x];
-            scr[w * kRounds + threadIdx.x] = run;
-            run += x;
-        }
-        scr[kWarps * kRounds + threadIdx.x] = run;
-    }
-    __syncthreads();
-    int b = base;
-#pragma unroll
-    for (int rr = 0; rr < kRounds; ++rr) {
-        pre[rr] = b + scr[warp * kRounds + rr] + incl[rr] - v[rr];
-        b += scr[kWarps * kRounds + rr];
-    }
-    __syncthreads();
-    return b;
-}
-
-__global__ void __launch_bounds__(kThreads, 2) topk_radix_kernel(const TopkArgs a, int cached_cap) {
+template <int T>
+__global__ void __launch_bounds__(T, T == 512 ? 2 : 1) topk_radix_kernel(const TopkArgs a, int cached_cap) {
+    using L = TopkLayout<T>;
+    constexpr int kThreads = T;
+    constexpr int kWarps = L::kWarps;
+    constexpr int kOffPriv = L::kOffPriv, kOffHist = L::kOffHist, kOffTot = L::kOffTot, kOffMisc = L::kOffMisc;
+    constexpr int kOffScan = L::kOffScan, kOffFine = L::kOffFine, kOffRange = L::kOffRange;
+    constexpr int kOffGather = L::kOffGather, kOffKeys = L::kOffKeys;
     cg::cluster_group cluster = cg::this_cluster();
     const int C = (int)cluster.num_blocks();
     const int rank = (int)cluster.block_rank();
@@ -189,19 +162,20 @@ __global__ void __launch_bounds__(kThreads, 2) topk_radix_kernel(const TopkArgs 
     __syncthreads();
     uint32_t kmn = 0xFFFFFFFFu, kmx = 0u;
     if (cached) {
-        // 16-byte loads, four in flight per thread, keys written in place
+        // 16-byte loads, eight in flight per thread (a 16 K-key slice in one round trip), keys
+        // written in place
         const int nv = len >> 2;
         const float4* r4 = reinterpret_cast<const float4*>(row + lo);
         uint4* k4 = reinterpret_cast<uint4*>(keys);
-        for (int i0 = 0; i0 < nv; i0 += 4 * kThreads) {
-            float4 f[4];
+        for (int i0 = 0; i0 < nv; i0 += kLoadBatch * kThreads) {
+            float4 f[kLoadBatch];
 #pragma unroll
-            for (int u = 0; u < 4; ++u) {
+            for (int u = 0; u < kLoadBatch; ++u) {
                 const int i = i0 + u * kThreads + tid;
                 f[u] = i < nv ? __ldg(r4 + i) : make_float4(0.f, 0.f, 0.f, 0.f);
             }
 #pragma unroll
-            for (int u = 0; u < 4; ++u) {
+            for (int u = 0; u < kLoadBatch; ++u) {
                 const int i = i0 + u * kThreads + tid;
                 if (i < nv) {
                     const uint4 kk = make_uint4(score_key(f[u].x), score_key(f[u].y), score_key(f[u].z), score_key(f[u].w));
@@ -273,6 +247,8 @@ __global__ void __launch_bounds__(kThreads, 2) topk_radix_kernel(const TopkArgs 
     int take_eq_total;  // keys equal to tau that are selected, lowest positions first
     int local_gt = 0;   // keys of this CTA above tau
     int local_eq = 0;   // keys of this CTA equal to tau
+    int eq_before = 0, out_before = 0;  // ties / outputs of the lower ranks
+    bool counts_done = false;           // (cluster-uniform) the lower ranks' counts are known
     if (kmin == kmax) {
         // every key of the row is equal: the first k positions
         tau = kmin;
@@ -303,13 +279,25 @@ __global__ void __launch_bounds__(kThreads, 2) topk_radix_kernel(const TopkArgs 
         shift = max(0, 32 - __clz((int)(kmax - kbase)) - kFineBits);
         for (int i = tid; i < kFineBins; i += kThreads) fine[i] = 0u;
         __syncthreads();
+        // keys at or below the base (most of a row's keys once the base is raised) are counted
+        // in registers: one shared-memory address taking every one of them serialises the atomics
+        int below = 0;
         for (int i0 = 4 * tid; i0 < len; i0 += 4 * kThreads) {
             const uint4 k4 = keys4_at(i0);
             const uint32_t kv[4] = {k4.x, k4.y, k4.z, k4.w};
 #pragma unroll
-            for (int u = 0; u < 4; ++u)
-                if (i0 + u < len) atomicAdd(&fine[bin_of(kv[u])], 1u);
+            for (int u = 0; u < 4; ++u) {
+                if (i0 + u < len) {
+                    if (kv[u] <= kbase)
+                        ++below;
+                    else
+                        atomicAdd(&fine[bin_of(kv[u])], 1u);
+                }
+            }
         }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) below += __shfl_xor_sync(0xffffffffu, below, o);
+        if (lane == 0 && below > 0) atomicAdd(&fine[0], (uint32_t)below);
         __syncthreads();
         cluster.sync();
         int part = 0;
@@ -361,7 +349,7 @@ __global__ void __launch_bounds__(kThreads, 2) topk_radix_kernel(const TopkArgs 
                 c4 += cb[u];
             }
             int tsum;
-            const int before = block_scan1(c4, scr, &tsum);
+            const int before = block_scan1<T>(c4, scr, &tsum);
             if (before < need && need <= before + c4) {
                 int run = before;
 #pragma unroll
@@ -391,7 +379,8 @@ __global__ void __launch_bounds__(kThreads, 2) topk_radix_kernel(const TopkArgs 
         int la = 0;
         for (int bb = bstar + 1 + tid; bb < kFineBins; bb += kThreads) la += (int)fine[bb];
         int latot;
-        block_scan1(la, scr, &latot);
+        block_scan1<T>(la, scr, &latot);
+        if (tid == 0) misc[7] = latot;  // read by the higher ranks after the candidate barrier
         if (Tc <= kCandMax) {
             // ---- 2. the keys of bin b*: every CTA gathers them all and finds tau itself
             uint32_t* cand = priv;
@@ -478,7 +467,7 @@ __global__ void __launch_bounds__(kThreads, 2) topk_radix_kernel(const TopkArgs 
                         c4 += cb[u];
                     }
                     int tsum;
-                    const int before = block_scan1(c4, scr, &tsum);
+                    const int before = block_scan1<T>(c4, scr, &tsum);
                     if (before < rem && rem <= before + c4) {
                         int run = before;
 #pragma unroll
@@ -504,17 +493,43 @@ __global__ void __launch_bounds__(kThreads, 2) topk_radix_kernel(const TopkArgs 
             }
             tau = (uint32_t)misc[11];
             take_eq_total = misc[12];
-            const int nc = misc[13];
-            int g = 0, e = 0;
-            for (int i = tid; i < nc; i += kThreads) {
-                g += cand[i] > tau;
-                e += cand[i] == tau;
+            // Every rank's counts come from the gathered list (rank r's candidates are
+            // gbuf[misc[26 + r], misc[27 + r])) and from its keys above b* (its misc[7]): lane r
+            // of warp 0 counts rank r; ties are taken lowest rank first.  No further exchange.
+            if (warp == 0) {
+                int g = 0, e = 0;
+                if (lane < C) {
+                    g = lane == rank ? latot : cluster.map_shared_rank(misc, lane)[7];
+                    const int b0 = misc[26 + lane], b1 = misc[27 + lane];
+                    for (int i = b0; i < b1; ++i) {
+                        g += gbuf[i] > tau;
+                        e += gbuf[i] == tau;
+                    }
+                }
+                int e_incl = e;
+#pragma unroll
+                for (int o = 1; o < 32; o <<= 1) {
+                    const int u = __shfl_up_sync(0xffffffffu, e_incl, o);
+                    if (lane >= o) e_incl += u;
+                }
+                const int e_excl = e_incl - e;
+                const int te = max(0, min(take_eq_total - e_excl, e));
+                int ob = lane < rank ? g + te : 0;
+#pragma unroll
+                for (int o = 16; o > 0; o >>= 1) ob += __shfl_xor_sync(0xffffffffu, ob, o);
+                if (lane == rank) {
+                    misc[16] = g;
+                    misc[17] = e;
+                    misc[20] = ob;
+                    misc[21] = e_excl;
+                }
             }
-            int gtot, etot;
-            block_scan1(g, scr, &gtot);
-            block_scan1(e, scr, &etot);
-            local_gt = latot + gtot;
-            local_eq = etot;
+            __syncthreads();
+            local_gt = misc[16];
+            local_eq = misc[17];
+            out_before = misc[20];
+            eq_before = misc[21];
+            counts_done = true;
         } else {
             // ---- fallback: radix select over four 8-bit digits of all keys
             uint32_t prefix = 0, pmask = 0;
@@ -560,7 +575,7 @@ __global__ void __launch_bounds__(kThreads, 2) topk_radix_kernel(const TopkArgs 
                 const int d = kBins - 1 - tid;
                 const int c = tid < kBins ? (int)tot[d] : 0;
                 int tsum;
-                const int before = block_scan1(c, scr, &tsum);
+                const int before = block_scan1<T>(c, scr, &tsum);
                 if (tid < kBins && before < remaining && remaining <= before + c) {
                     misc[0] = d;
                     misc[1] = before;
@@ -570,7 +585,7 @@ __global__ void __launch_bounds__(kThreads, 2) topk_radix_kernel(const TopkArgs 
                 const int above = misc[1];
                 // this CTA's keys in digits above the chosen one (same prefix) are above tau
                 int atot;
-                block_scan1((tid < kBins && d > dsel) ? (int)hist[d] : 0, scr, &atot);
+                block_scan1<T>((tid < kBins && d > dsel) ? (int)hist[d] : 0, scr, &atot);
                 local_gt += atot;
                 if (p == 3) local_eq = (int)hist[dsel];
                 prefix |= (uint32_t)dsel << sh;
@@ -582,137 +597,159 @@ __global__ void __launch_bounds__(kThreads, 2) topk_radix_kernel(const TopkArgs 
         }
     }
 
-    if (tid == 0) {
-        misc[2] = local_gt;
-        misc[3] = local_eq;
-    }
-    cluster.sync();
-    int eq_before = 0, out_before = 0;
-    if (warp == 0) {
-        // lane r < rank reads CTA r's counts; ties are taken lowest rank first
-        int g = 0, e = 0;
-        if (lane < rank) {
-            const int* rm = cluster.map_shared_rank(misc, lane);
-            g = rm[2];
-            e = rm[3];
+    if (!counts_done) {
+        // all-equal rows and the radix fallback: exchange the counts through the cluster
+        if (tid == 0) {
+            misc[2] = local_gt;
+            misc[3] = local_eq;
         }
-        int e_incl = e;
+        cluster.sync();
+        if (warp == 0) {
+            // lane r < rank reads CTA r's counts; ties are taken lowest rank first
+            int g = 0, e = 0;
+            if (lane < rank) {
+                const int* rm = cluster.map_shared_rank(misc, lane);
+                g = rm[2];
+                e = rm[3];
+            }
+            int e_incl = e;
 #pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-            const int u = __shfl_up_sync(0xffffffffu, e_incl, o);
-            if (lane >= o) e_incl += u;
-        }
-        const int te = max(0, min(take_eq_total - (e_incl - e), e));
-        int ob = g + te;
+            for (int o = 1; o < 32; o <<= 1) {
+                const int u = __shfl_up_sync(0xffffffffu, e_incl, o);
+                if (lane >= o) e_incl += u;
+            }
+            const int te = max(0, min(take_eq_total - (e_incl - e), e));
+            int ob = g + te;
 #pragma unroll
-        for (int o = 16; o > 0; o >>= 1) ob += __shfl_xor_sync(0xffffffffu, ob, o);
-        if (lane == 31) {
-            misc[20] = ob;
-            misc[21] = e_incl;  // the ties of all lower ranks
+            for (int o = 16; o > 0; o >>= 1) ob += __shfl_xor_sync(0xffffffffu, ob, o);
+            if (lane == 31) {
+                misc[20] = ob;
+                misc[21] = e_incl;  // the ties of all lower ranks
+            }
         }
+        __syncthreads();
+        out_before = misc[20];
+        eq_before = misc[21];
     }
+    // This CTA reads no peer's shared memory from here on: arrive now, wait before exiting
+    // (peers may still be reading this CTA's candidates and counts until they arrive).
     __syncthreads();
-    out_before = misc[20];
-    eq_before = misc[21];
+    cluster_arrive_release();
     const int take_eq_local = max(0, min(take_eq_total - eq_before, local_eq));
-    const bool all_ties = take_eq_local == local_eq;  // selection is then a plain threshold
-    const uint64_t thr = take_eq_local > 0 ? (uint64_t)tau : (uint64_t)tau + 1u;
 
-    // ordered compaction in sweeps of kRounds x 4 x kThreads keys
-    const int sweep = kRounds * 4 * kThreads;
-    int out_run = out_before, eq_run = 0;
-    for (int s0 = 0; s0 < len; s0 += sweep) {
-        uint32_t sel = 0;  // bit 4*rr+u: key (rr, u) of this thread selected
-        int cnt[kRounds];
-        if (all_ties) {
-#pragma unroll
-            for (int rr = 0; rr < kRounds; ++rr) {
-                cnt[rr] = 0;
-                const int i0 = s0 + (rr * kThreads + tid) * 4;
-                const uint4 k4 = keys4_at(i0);
-                const uint32_t kv[4] = {k4.x, k4.y, k4.z, k4.w};
-#pragma unroll
-                for (int u = 0; u < 4; ++u) {
-                    if (i0 + u < len && (uint64_t)kv[u] >= thr) {
-                        sel |= 1u << (4 * rr + u);
-                        ++cnt[rr];
-                    }
-                }
-            }
-        } else {
-            // rank of each tie among this CTA's ties decides it
-            int ceq[kRounds], pre[kRounds];
-            uint32_t eqm = 0;
-#pragma unroll
-            for (int rr = 0; rr < kRounds; ++rr) {
-                cnt[rr] = 0;
-                ceq[rr] = 0;
-                const int i0 = s0 + (rr * kThreads + tid) * 4;
-                const uint4 k4 = keys4_at(i0);
-                const uint32_t kv[4] = {k4.x, k4.y, k4.z, k4.w};
-#pragma unroll
-                for (int u = 0; u < 4; ++u) {
-                    if (i0 + u < len) {
-                        const uint32_t kk = kv[u];
-                        if (kk > tau) {
-                            sel |= 1u << (4 * rr + u);
-                            ++cnt[rr];
-                        } else if (kk == tau) {
-                            eqm |= 1u << (4 * rr + u);
-                            ++ceq[rr];
-                        }
-                    }
-                }
-            }
-            eq_run = block_scan_rounds(ceq, pre, eq_run, scr);
-#pragma unroll
-            for (int rr = 0; rr < kRounds; ++rr) {
-                int e = pre[rr];
-#pragma unroll
-                for (int u = 0; u < 4; ++u) {
-                    if ((eqm >> (4 * rr + u)) & 1u) {
-                        if (e < take_eq_local) {
-                            sel |= 1u << (4 * rr + u);
-                            ++cnt[rr];
-                        }
-                        ++e;
-                    }
-                }
-            }
-        }
-        int pos[kRounds];
-        out_run = block_scan_rounds(cnt, pos, out_run, scr);
-#pragma unroll
-        for (int rr = 0; rr < kRounds; ++rr) {
-            int o = pos[rr];
+    // ordered compaction: warp w owns the contiguous segment [w * seg, w * seg + seg) of this
+    // CTA's keys, read four consecutive keys per lane (128 per warp step).  Pass 1 counts each
+    // warp's keys above tau and equal to it; one warp turns the counts into the warp's first tie
+    // rank and first output slot; pass 2 writes the selected positions in position order
+    // (ballots give every key its rank inside the step).  A tie is selected while its rank
+    // among this CTA's ties is below take_eq_local.
+    {
+        const int seg = ((len + kWarps - 1) / kWarps + 127) & ~127;
+        const int w_lo = min(len, warp * seg), w_hi = min(len, w_lo + seg);
+        int gt = 0, eq = 0;
+#pragma unroll 1
+        for (int base = w_lo; base < w_hi; base += 128) {  // warp-uniform steps
+            const int i0 = base + 4 * lane;
+            const uint4 k4 = keys4_at(i0);
+            const uint32_t kv[4] = {k4.x, k4.y, k4.z, k4.w};
 #pragma unroll
             for (int u = 0; u < 4; ++u) {
-                if ((sel >> (4 * rr + u)) & 1u) {
-                    if (o < a.k) out[o] = lo + s0 + (rr * kThreads + tid) * 4 + u;
+                const bool in = i0 + u < w_hi;
+                gt += in && kv[u] > tau;
+                eq += in && kv[u] == tau;
+            }
+        }
+        gt = __reduce_add_sync(0xffffffffu, gt);
+        eq = __reduce_add_sync(0xffffffffu, eq);
+        if (lane == 0) {
+            scr[warp] = gt;
+            scr[kWarps + warp] = eq;
+        }
+        __syncthreads();
+        if (warp == 0) {
+            // lane w: warp w's first tie rank and first output slot
+            const int g = lane < kWarps ? scr[lane] : 0;
+            const int e = lane < kWarps ? scr[kWarps + lane] : 0;
+            int e_incl = e;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const int v = __shfl_up_sync(0xffffffffu, e_incl, o);
+                if (lane >= o) e_incl += v;
+            }
+            const int e_excl = e_incl - e;
+            const int taken = g + max(0, min(take_eq_local - e_excl, e));
+            int t_incl = taken;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const int v = __shfl_up_sync(0xffffffffu, t_incl, o);
+                if (lane >= o) t_incl += v;
+            }
+            if (lane < kWarps) {
+                scr[2 * kWarps + lane] = e_excl;
+                scr[3 * kWarps + lane] = out_before + t_incl - taken;
+            }
+        }
+        __syncthreads();
+        int eq_run = scr[2 * kWarps + warp];
+        int out_run = scr[3 * kWarps + warp];
+        const unsigned lt = (1u << lane) - 1u;
+#pragma unroll 1
+        for (int base = w_lo; base < w_hi; base += 128) {  // warp-uniform steps (ballots below)
+            const int i0 = base + 4 * lane;
+            const uint4 k4 = keys4_at(i0);
+            const uint32_t kv[4] = {k4.x, k4.y, k4.z, k4.w};
+            unsigned eb[4];
+#pragma unroll
+            for (int u = 0; u < 4; ++u) eb[u] = __ballot_sync(0xffffffffu, i0 + u < w_hi && kv[u] == tau);
+            // ties at lower positions in this step: lower lanes (all four keys), then this lane's
+            int eq_before = eq_run + __popc(eb[0] & lt) + __popc(eb[1] & lt) + __popc(eb[2] & lt) + __popc(eb[3] & lt);
+            bool sel[4];
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                const bool in = i0 + u < w_hi;
+                const bool is_eq = (eb[u] >> lane) & 1u;
+                sel[u] = in && (kv[u] > tau || (is_eq && eq_before < take_eq_local));
+                eq_before += is_eq;
+            }
+            eq_run += __popc(eb[0]) + __popc(eb[1]) + __popc(eb[2]) + __popc(eb[3]);
+            unsigned sb[4];
+#pragma unroll
+            for (int u = 0; u < 4; ++u) sb[u] = __ballot_sync(0xffffffffu, sel[u]);
+            int o = out_run + __popc(sb[0] & lt) + __popc(sb[1] & lt) + __popc(sb[2] & lt) + __popc(sb[3] & lt);
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                if (sel[u]) {
+                    if (o < a.k) out[o] = lo + i0 + u;
                     ++o;
                 }
             }
+            out_run += __popc(sb[0]) + __popc(sb[1]) + __popc(sb[2]) + __popc(sb[3]);
         }
     }
-    cluster.sync();  // keep this CTA's shared memory alive until every peer has read it
+    cluster_wait_acquire();  // keep this CTA's shared memory alive until every peer has read it
 }
 
 }  // namespace
 
-cudaError_t launch_topk(const TopkArgs& a, int cluster, cudaStream_t st) {
-    if (a.Nq == 0) return cudaSuccess;
-    if (cluster < 1 || cluster > kMaxCluster) return cudaErrorInvalidValue;
-    int64_t row_max = a.ld < (int64_t)a.T_max ? a.ld : (int64_t)a.T_max;
-    if (a.row_len_hint > 0 && a.row_len_hint < row_max) row_max = a.row_len_hint;
+namespace {
+
+// Largest shared-memory slice (keys) of one CTA: what fits beside the CTA's own map.
+template <int T>
+constexpr int smem_keys_cap() {
+    return T == 512 ? kTopkSmemKeys : 40960;
+}
+
+template <int T>
+cudaError_t launch_topk_impl(const TopkArgs& a, int cluster, int64_t row_max, cudaStream_t st) {
     int64_t chunk = (row_max + cluster - 1) / cluster;
     chunk = (chunk + 3) & ~int64_t(3);
-    const int cap = (int)(chunk < kTopkSmemKeys ? chunk : kTopkSmemKeys);
-    const size_t smem = (size_t)(kBaseWords + cap) * sizeof(uint32_t);
-    cudaError_t e = cudaFuncSetAttribute(topk_radix_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    const int cap = (int)(chunk < smem_keys_cap<T>() ? chunk : smem_keys_cap<T>());
+    const size_t smem = (size_t)(TopkLayout<T>::kBaseWords + cap) * sizeof(uint32_t);
+    cudaError_t e = cudaFuncSetAttribute(topk_radix_kernel<T>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(cluster, a.Nq, 1);
-    cfg.blockDim = dim3(kThreads, 1, 1);
+    cfg.blockDim = dim3(T, 1, 1);
     cfg.dynamicSmemBytes = smem;
     cfg.stream = st;
     cudaLaunchAttribute attr[2];
@@ -724,9 +761,68 @@ cudaError_t launch_topk(const TopkArgs& a, int cluster, cudaStream_t st) {
     attr[1].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = a.pdl ? 2 : 1;
-    e = cudaLaunchKernelEx(&cfg, topk_radix_kernel, a, cap);
+    e = cudaLaunchKernelEx(&cfg, topk_radix_kernel<T>, a, cap);
     if (e != cudaSuccess) return e;
     return cudaGetLastError();
+}
+
+// How many clusters of c 1024-thread CTAs (one per SM) the device holds at once: cluster
+// placement is per GPC, so this can be below SMs / c.  Asked once per device and size.
+constexpr int kMaxTopkDevices = 64;
+int g_wide_clusters[kMaxTopkDevices][kTopkMaxCluster + 1];
+
+int max_wide_clusters(int c) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxTopkDevices) return 0;
+    int& slot = g_wide_clusters[dev][c];
+    if (slot == 0) {
+        constexpr int T = 1024;
+        const size_t smem = (size_t)(TopkLayout<T>::kBaseWords + smem_keys_cap<T>()) * sizeof(uint32_t);
+        int n = -1;
+        if (cudaFuncSetAttribute(topk_radix_kernel<T>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) ==
+            cudaSuccess) {
+            cudaLaunchConfig_t cfg = {};
+            cfg.gridDim = dim3(c, 1, 1);
+            cfg.blockDim = dim3(T, 1, 1);
+            cfg.dynamicSmemBytes = smem;
+            cudaLaunchAttribute attr[1];
+            attr[0].id = cudaLaunchAttributeClusterDimension;
+            attr[0].val.clusterDim.x = c;
+            attr[0].val.clusterDim.y = 1;
+            attr[0].val.clusterDim.z = 1;
+            cfg.attrs = attr;
+            cfg.numAttrs = 1;
+            int m = 0;
+            if (cudaOccupancyMaxActiveClusters(&m, topk_radix_kernel<T>, &cfg) == cudaSuccess && m > 0) n = m;
+        }
+        (void)cudaGetLastError();  // a refused query only means: no wide launch
+        slot = n;
+    }
+    return slot > 0 ? slot : 0;
+}
+
+}  // namespace
+
+cudaError_t launch_topk(const TopkArgs& a, int cluster, cudaStream_t st) {
+    if (a.Nq == 0) return cudaSuccess;
+    if (cluster < 1 || cluster > kMaxCluster) return cudaErrorInvalidValue;
+    int64_t row_max = a.ld < (int64_t)a.T_max ? a.ld : (int64_t)a.T_max;
+    if (a.row_len_hint > 0 && a.row_len_hint < row_max) row_max = a.row_len_hint;
+    // When every row's cluster fits one wave at one CTA per SM, a 1024-thread CTA per SM runs
+    // the same chain with twice the threads and no SM shared by two CTAs: the largest cluster
+    // size up to the planned one whose Nq clusters the device holds at once, provided the
+    // slices still fit shared memory wherever the planned launch's would.
+    int sms = 0, dev = 0;
+    if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    if (sms > 0 && (int64_t)a.Nq * cluster <= sms) {
+        const bool planned_fits = (row_max + cluster - 1) / cluster <= smem_keys_cap<512>();
+        for (int c = cluster; c >= 1; --c) {
+            const bool fits = (row_max + c - 1) / c <= smem_keys_cap<1024>();
+            if (planned_fits && !fits) break;
+            if (a.Nq <= max_wide_clusters(c)) return launch_topk_impl<1024>(a, c, row_max, st);
+        }
+    }
+    return launch_topk_impl<512>(a, cluster, row_max, st);
 }
 
 }  // namespace dsa
