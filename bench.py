@@ -72,6 +72,9 @@ def parse_args():
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--no-secondary", action="store_true",
                    help="skip the secondary workloads (decode batch 32, 1M-context decode, prefill) of the default line")
+    p.add_argument("--soak-seconds", type=float, default=2.0,
+                   help="seconds of back-to-back steps inside the clock-sampled window (0 under a profiler)")
+    p.add_argument("--e2e-steps", type=int, default=E2E_STEPS, help="steps of the end-to-end pass")
     p.add_argument("--workload", default="long_decode", choices=["long_decode", "prefill", "dense", "paged", "fp8kv"])
     p.add_argument("--block-size", type=int, default=64)
     p.add_argument("--prefill-len", type=int, default=65536)
@@ -359,7 +362,7 @@ def run_ours(args):
     # Clock soak: the same step back to back for ~2 s of wall time while nvidia-smi samples
     # (the timed loop itself lasts a few milliseconds, too short for 100 ms samples)
     t_soak = time.perf_counter()
-    while time.perf_counter() - t_soak < 2.0:
+    while time.perf_counter() - t_soak < args.soak_seconds:
         for _ in range(200):
             flush_l2()
             api.run_decode(inp, ws=ws, out=out, lse=lse, dims=dims)
@@ -377,7 +380,7 @@ def run_ours(args):
     status = api.get_device_status(ws)
 
     # ---- end to end through the C interface with host buffers
-    e2e = measure_e2e(inp, dims, dev, steps=E2E_STEPS, warmup=max(W, 10))
+    e2e = measure_e2e(inp, dims, dev, steps=args.e2e_steps, warmup=max(W, 10))
     if not e2e["readback_ok"]:
         raise SystemExit("end-to-end loop: the host copy of the last step's output differs from the device's")
     e2e_ms = max_over_ranks(e2e["ms"], world)
@@ -445,7 +448,7 @@ def run_ours(args):
         "stages_us": {"indexer": stage_us[0], "topk": stage_us[1], "sparse_mla": stage_us[2],
                       "merge": stage_us[3]},
         "e2e": {"value": BATCH * world / (e2e_ms * 1e-3), "unit": UNIT, "h2d_bytes_per_step": e2e["h2d"],
-                "d2h_bytes_per_step": e2e["d2h"], "ms_per_step": e2e_ms, "steps": E2E_STEPS,
+                "d2h_bytes_per_step": e2e["d2h"], "ms_per_step": e2e_ms, "steps": args.e2e_steps,
                 "pipeline": "one CUDA-graph replay per step, captured once per buffer slot from the public calls: "
                             "the step's cache append + dsa_decode_step on its slot, the H2D copy of the next "
                             "step's inputs (one packed pinned buffer) and the D2H copy of the previous step's "
@@ -458,7 +461,7 @@ def run_ours(args):
         "clocks": {"sm_mhz": clocks["sm_mhz"], "sm_max_mhz": clocks["sm_max_mhz"], "reasons": clocks["reasons"],
                    "samples": clocks["samples"], "window_s": window1 - window0,
                    "window": "nvidia-smi every 100 ms from the warm-up through the end-to-end pass, which "
-                             "includes ~2 s of the same step back to back",
+                             f"includes ~{args.soak_seconds:g} s of the same step back to back",
                    "nvml_before_timed_loop": nvml_before, "nvml_after_timed_loop": nvml_after},
         "device_status": status,
         "wall_s_timed_loop": wall,

@@ -319,6 +319,21 @@ int32_t dsa_last_cuda_error(void);
 dsa_status_t dsa_selftest_wait_timeout(void* workspace, size_t ws_bytes, int32_t timeout_us,
                                        void* stream);
 
+/* Self-test of a production kernel's bounded waits: dsa_sparse_mla_attn's
+ * kernel (kv_dtype DSA_BF16, same arguments and workspace) with one fault
+ * planted on the host's request: its gather warps never signal that the
+ * first tile has landed.  The MMA warp's wait for that tile runs out after
+ * about `timeout_us` microseconds (1 .. 5,000,000); the kernel then records
+ * DSA_ERR_TIMEOUT in the workspace status word, every role of every CTA
+ * leaves its loop, copies still in flight land, tensor memory is freed and the
+ * kernel exits.  out and lse hold zeros / -inf or partial results afterwards.
+ * The CUDA context stays usable.  No counterpart on the pages: it checks the
+ * failure handling that every kernel's waits rely on. */
+dsa_status_t dsa_selftest_attention_stall(const dsa_dims* dims, const void* q, const void* kv, const int32_t* idx,
+                                          const int32_t* q_seq, const int32_t* q_len, float softmax_scale,
+                                          void* out, float* lse, void* workspace, size_t ws_bytes,
+                                          int32_t timeout_us, void* stream);
+
 /* Library version string. */
 const char* dsa_version(void);
 

@@ -23,7 +23,7 @@ EXPORTS = (
     "dsa_workspace_size", "dsa_workspace_init", "dsa_indexer_scores", "dsa_prefill_indexer_scores", "dsa_topk",
     "dsa_sparse_mla_attn", "dsa_dense_mla_attn",
     "dsa_decode_step", "dsa_decode_step_paged", "dsa_append_tokens", "dsa_prefill", "dsa_get_device_status", "dsa_status_string", "dsa_last_cuda_error",
-    "dsa_selftest_wait_timeout", "dsa_version", "dsa_sparse_mla_attn_noalloc",
+    "dsa_selftest_wait_timeout", "dsa_selftest_attention_stall", "dsa_version", "dsa_sparse_mla_attn_noalloc",
 )
 
 
@@ -83,12 +83,14 @@ def _declare(lib):
                                           P, ctypes.POINTER(DsaStageEvents)]
     lib.dsa_get_device_status.argtypes = [P, P, ctypes.POINTER(I32)]
     lib.dsa_selftest_wait_timeout.argtypes = [P, S, I32, P]
+    lib.dsa_selftest_attention_stall.argtypes = [D, P, P, P, P, P, F, P, P, P, S, I32, P]
     for name in ("dsa_workspace_size", "dsa_workspace_init", "dsa_indexer_scores", "dsa_prefill_indexer_scores",
                  "dsa_topk",
                  "dsa_sparse_mla_attn", "dsa_decode_step", "dsa_decode_step_paged", "dsa_append_tokens",
                  "dsa_prefill",
                  "dsa_get_device_status",
-                 "dsa_selftest_wait_timeout", "dsa_sparse_mla_attn_noalloc", "dsa_dense_mla_attn"):
+                 "dsa_selftest_wait_timeout", "dsa_selftest_attention_stall", "dsa_sparse_mla_attn_noalloc",
+                 "dsa_dense_mla_attn"):
         getattr(lib, name).restype = st
     lib.dsa_status_string.argtypes = [I32]
     lib.dsa_status_string.restype = ctypes.c_char_p

@@ -218,6 +218,17 @@ def selftest_wait_timeout(ws: torch.Tensor, timeout_us: int = 200000):
     _lib.check(lib, rc, "dsa_selftest_wait_timeout")
 
 
+def selftest_attention_stall(dims: Dims, q, kv, idx, q_seq, q_len, softmax_scale, out, lse, ws,
+                             timeout_us: int = 100000):
+    """The attention kernel with its first tile never signalled: its bounded wait runs out."""
+    lib = _lib.load()
+    d = dims.c()
+    rc = lib.dsa_selftest_attention_stall(ctypes.byref(d), _ptr(q), _ptr(kv), _ptr(idx), _ptr(q_seq), _ptr(q_len),
+                                          ctypes.c_float(softmax_scale), _ptr(out), _ptr(lse), _ptr(ws), ws.numel(),
+                                          int(timeout_us), _stream_ptr())
+    _lib.check(lib, rc, "dsa_selftest_attention_stall")
+
+
 # ---- conveniences over an inputs.DSAInputs workload --------------------------
 
 def alloc_outputs(inp, device=None):

@@ -595,6 +595,47 @@ dsa_status_t dsa_get_device_status(void* workspace, void* stream, int32_t* statu
     return DSA_OK;
 }
 
+dsa_status_t dsa_selftest_attention_stall(const dsa_dims* dims, const void* q, const void* kv, const int32_t* idx,
+                                          const int32_t* q_seq, const int32_t* q_len, float softmax_scale, void* out,
+                                          float* lse, void* workspace, size_t ws_bytes, int32_t timeout_us,
+                                          void* stream) {
+    dsa_status_t s = check_dims(dims, false, true);
+    if (s != DSA_OK) return s;
+    if (dims->kv_dtype != DSA_BF16) return DSA_ERR_UNSUPPORTED;
+    if (timeout_us < 1 || timeout_us > 5000000) return DSA_ERR_INVALID_ARG;
+    if (dims->Nq == 0) return DSA_OK;
+    if (!q || !kv || !idx || !q_seq || !q_len || !out || !std::isfinite(softmax_scale)) return DSA_ERR_INVALID_ARG;
+    if (!aligned16(q) || !aligned16(kv) || !aligned16(out)) return DSA_ERR_INVALID_ARG;
+    const Layout L = layout_for(dims, DSA_OP_SPARSE_MLA);
+    if (workspace == nullptr || ws_bytes < L.total) return DSA_ERR_WORKSPACE;
+    const MlaPlan p = plan_mla(dims, dims->Nq);
+    dsa::MlaArgs a{};
+    a.q = q;
+    a.kv = kv;
+    a.idx = idx;
+    a.q_seq = q_seq;
+    a.q_len = q_len;
+    a.out = out;
+    a.lse = lse;
+    a.part_o = p.splits > 1 ? reinterpret_cast<float*>(static_cast<char*>(workspace) + L.part_o) : nullptr;
+    a.part_lse = p.splits > 1 ? reinterpret_cast<float*>(static_cast<char*>(workspace) + L.part_lse) : nullptr;
+    a.Nq = dims->Nq;
+    a.B = dims->B;
+    a.T_max = dims->T_max;
+    a.k = dims->k;
+    a.H = dims->H;
+    a.splits = p.splits;
+    a.rows_per_split = p.rows_per_split;
+    a.softmax_scale = softmax_scale;
+    a.status = status_word(workspace);
+    a.selftest_stall = 1;
+    a.wait_budget_ns = (uint64_t)timeout_us * 1000ull;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    cudaError_t e = dsa::launch_sparse_mla_bf16(a, st);
+    if (e == cudaSuccess) e = dsa::launch_mla_combine(a, st);
+    return e == cudaSuccess ? DSA_OK : cuda_fail(e);
+}
+
 dsa_status_t dsa_selftest_wait_timeout(void* workspace, size_t ws_bytes, int32_t timeout_us, void* stream) {
     if (workspace == nullptr || ws_bytes < kStatusBytes) return DSA_ERR_WORKSPACE;
     if (timeout_us < 1 || timeout_us > 5000000) return DSA_ERR_INVALID_ARG;

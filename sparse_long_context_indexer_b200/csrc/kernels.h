@@ -76,6 +76,11 @@ struct MlaArgs {
     // FP8 latent cache: 656-byte entries of 512 e4m3 values, 4 fp32 scales (one per 128
     // values) and the 64 rope values in bf16; dequantised to bf16 by the gather
     int kv_fp8;
+    // Self-test of the bounded waits (0 in every production call): the gather never signals
+    // the first tile, so the MMA warp's wait on it runs out after wait_budget_ns (0 = the
+    // default budget) and the kernel records DSA_ERR_TIMEOUT and drains.
+    int selftest_stall;
+    uint64_t wait_budget_ns;
 };
 constexpr int kFp8EntryBytes = 656;  // 512 + 4 * 4 + 64 * 2
 constexpr int kFp8ScaleOff = 512;

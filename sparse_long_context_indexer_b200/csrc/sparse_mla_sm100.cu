@@ -362,7 +362,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
                 for (int c = 0; c < kChunks; ++c) cp_async16_zfill(dst + c * kChunkBytes, src + c * 64, ok_row ? 16u : 0u);
             }
-            cp_async_arrive_noinc(bar_kv_full(st));
+            if (!(a.selftest_stall && i == 0)) cp_async_arrive_noinc(bar_kv_full(st));
             if (pf_lane && i + kPrefetchTiles < ntiles) prefetch_row(pf);
             if (i + 1 < ntiles) {
                 cur0 = load_pos(i + 1, rr);
@@ -451,7 +451,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     bool stop = false;
                     if (*abort_flag) {
                         stop = true;
-                    } else if (globaltimer_ns() - t_last > kWaitBudgetNs) {
+                    } else if (globaltimer_ns() - t_last > (a.wait_budget_ns ? a.wait_budget_ns : kWaitBudgetNs)) {
                         if (lane == 0) {
                             record_status(a.status, DSA_STATUS_TIMEOUT);
                             *abort_flag = 1;

@@ -639,6 +639,31 @@ def test_length_beyond_cache_is_reported(lib):
     assert status == _lib.DSA_ERR_LENGTH
 
 
+@pytest.mark.parametrize("lens", [[4096] * 16, [4096] * 2])
+def test_production_attention_wait_times_out_and_context_survives(lib, lens):
+    # the attention kernel itself (a cluster of 4 splits for 16 rows; 16 splits and the merge
+    # kernel for 2 rows) with its first tile never signalled: the MMA warp's bounded wait runs
+    # out after 50 ms, the kernel records DSA_ERR_TIMEOUT, drains and exits; afterwards the same
+    # kernel on the same buffers matches the oracle
+    inp = small_decode(seed=57, lens=lens)
+    sc = oracle.indexer(inp, ld=inp.T_max)
+    idx = oracle.topk(sc, inp.q_len.numpy(), inp.k)
+    o_out, o_lse = oracle.sparse_attn(inp, idx)
+    g = inp.to("cuda")
+    dims = api.dims_of(g)
+    ws = api.make_workspace(dims, _lib.DSA_OP_SPARSE_MLA)
+    out, lse = api.alloc_outputs(g)
+    idx_d = torch.from_numpy(idx).cuda()
+    api.selftest_attention_stall(dims, g.q, g.kv, idx_d, g.q_seq, g.q_len, g.softmax_scale, out, lse, ws,
+                                 timeout_us=50000)
+    assert api.get_device_status(ws) == _lib.DSA_ERR_TIMEOUT
+    out.zero_()
+    api.sparse_mla_attn(dims, g.q, g.kv, idx_d, g.q_seq, g.q_len, g.softmax_scale, out, lse, ws)
+    torch.cuda.synchronize()
+    assert api.get_device_status(ws) == 0
+    check_attention(out.float().cpu().numpy(), o_out, lse.cpu().numpy(), o_lse)
+
+
 def test_bounded_wait_times_out_with_status(lib):
     dims = api.Dims(B=1, Nq=1, H_I=64, d_I=64, H=128, k=16, T_max=128, idx_dtype=2, kv_dtype=1, ld_scores=128)
     ws = api.make_workspace(dims, _lib.DSA_OP_TOPK)
