@@ -197,6 +197,45 @@ def nvml_reading(gpu_index):
         return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [f"nvml unavailable: {type(e).__name__}"]}
 
 
+def gpu_local_cpus(gpu_index):
+    """The host cores NVML lists as local to this GPU (its NUMA node), within the cores this
+    process may use; None when NVML cannot tell.  Read-only."""
+    try:
+        import pynvml
+        pynvml.nvmlInit()
+        try:
+            h = pynvml.nvmlDeviceGetHandleByIndex(int(gpu_index))
+            words = pynvml.nvmlDeviceGetCpuAffinity(h, (os.cpu_count() + 63) // 64)
+        finally:
+            pynvml.nvmlShutdown()
+        cpus = {64 * i + b for i, w in enumerate(words) for b in range(64) if (int(w) >> b) & 1}
+        cpus &= os.sched_getaffinity(0)
+        return cpus or None
+    except Exception:
+        return None
+
+
+class near_gpu_memory:
+    """Runs its body on the GPU's local cores, so that pinned host buffers allocated inside it
+    are placed (first touch) on the GPU's NUMA node; the process's affinity is restored on
+    exit.  The DMA engines then read and write memory next to the GPU's PCIe root."""
+
+    def __init__(self, gpu_index):
+        self.cpus = gpu_local_cpus(gpu_index)
+        self.saved = None
+
+    def __enter__(self):
+        if self.cpus:
+            self.saved = os.sched_getaffinity(0)
+            os.sched_setaffinity(0, self.cpus)
+        return self
+
+    def __exit__(self, *exc):
+        if self.saved is not None:
+            os.sched_setaffinity(0, self.saved)
+        return False
+
+
 def cpu_model():
     try:
         with open("/proc/cpuinfo") as f:
@@ -380,7 +419,7 @@ def run_ours(args):
     status = api.get_device_status(ws)
 
     # ---- end to end through the C interface with host buffers
-    e2e = measure_e2e(inp, dims, dev, steps=args.e2e_steps, warmup=max(W, 10))
+    e2e = measure_e2e(inp, dims, dev, steps=args.e2e_steps, warmup=max(W, 10), gpu_index=gpu_index)
     if not e2e["readback_ok"]:
         raise SystemExit("end-to-end loop: the host copy of the last step's output differs from the device's")
     e2e_ms = max_over_ranks(e2e["ms"], world)
@@ -454,7 +493,8 @@ def run_ours(args):
                             "step's inputs (one packed pinned buffer) and the D2H copy of the previous step's "
                             "out and lse, as three concurrent branches of the graph; the timed region also "
                             "holds the first copy-in and the last copy-out; the last read-back is checked "
-                            "against the device copy and against a direct dsa_decode_step call"},
+                            "against the device copy and against a direct dsa_decode_step call",
+                "host_link": e2e["link"]},
         "gpu_launches": launches_per_step() * K,
         "timing": {"step": "one start and one end event per step on the launching stream",
                    "stages_us": f"separate pass of {KS} steps with an event between stages (each adds ~2 us)"},
@@ -884,7 +924,7 @@ def launches_per_step():
     return 4 if splits > 8 else 3
 
 
-def measure_e2e(inp, dims, dev, steps, warmup):
+def measure_e2e(inp, dims, dev, steps, warmup, gpu_index="0"):
     """End to end through the public API, as a serving loop would run it.  Per step: the H2D
     copy of all of the step's inputs (query-side tensors, the new token's position, bf16
     latent row and fp32 indexer key, packed in one pinned buffer), the cache append
@@ -915,20 +955,22 @@ def measure_e2e(inp, dims, dev, steps, warmup):
         off += (v.numel() * v.element_size() + 255) // 256 * 256
     total = off
     h2d = sum(v.numel() * v.element_size() for v in fields.values())
-    host_pack = torch.empty(total, dtype=torch.uint8).pin_memory()
-    for k, v in fields.items():
-        nb = v.numel() * v.element_size()
-        host_pack[offs[k]:offs[k] + nb].copy_(v.contiguous().cpu().view(-1).view(torch.uint8))
-    ws = api.make_workspace(dims, _lib.DSA_OP_DECODE, dev)
-    slots = []
-    for _ in range(2):
-        dbuf = torch.empty(total, dtype=torch.uint8, device=dev)
-        views = {k: dbuf[offs[k]:offs[k] + v.numel() * v.element_size()].view(v.dtype).view(v.shape)
-                 for k, v in fields.items()}
-        o, l = api.alloc_outputs(inp)
-        slots.append({"dbuf": dbuf, "v": views, "out": o, "lse": l,
-                      "out_h": torch.empty(o.shape, dtype=o.dtype).pin_memory(),
-                      "lse_h": torch.empty(l.shape, dtype=l.dtype).pin_memory()})
+    near = near_gpu_memory(gpu_index)
+    with near:                                      # pinned buffers on the GPU's NUMA node
+        host_pack = torch.empty(total, dtype=torch.uint8).pin_memory()
+        for k, v in fields.items():
+            nb = v.numel() * v.element_size()
+            host_pack[offs[k]:offs[k] + nb].copy_(v.contiguous().cpu().view(-1).view(torch.uint8))
+        ws = api.make_workspace(dims, _lib.DSA_OP_DECODE, dev)
+        slots = []
+        for _ in range(2):
+            dbuf = torch.empty(total, dtype=torch.uint8, device=dev)
+            views = {k: dbuf[offs[k]:offs[k] + v.numel() * v.element_size()].view(v.dtype).view(v.shape)
+                     for k, v in fields.items()}
+            o, l = api.alloc_outputs(inp)
+            slots.append({"dbuf": dbuf, "v": views, "out": o, "lse": l,
+                          "out_h": torch.empty(o.shape, dtype=o.dtype).pin_memory(),
+                          "lse_h": torch.empty(l.shape, dtype=l.dtype).pin_memory()})
     d2h = slots[0]["out_h"].numel() * slots[0]["out_h"].element_size() + \
         slots[0]["lse_h"].numel() * slots[0]["lse_h"].element_size()
     main = torch.cuda.Stream(device=dev)
@@ -991,6 +1033,22 @@ def measure_e2e(inp, dims, dev, steps, warmup):
                 graphs[i % 2].replay()
             copy_out(slots[(n - 1) % 2])            # the last step's outputs
 
+    def link_rate(copy, nbytes, reps=50):
+        # the host link alone: the same copies back to back on one stream, GB/s
+        with torch.cuda.stream(main):
+            for _ in range(5):
+                copy()
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(main)
+            for _ in range(reps):
+                copy()
+            b.record(main)
+        b.synchronize()
+        return nbytes * reps / (a.elapsed_time(b) * 1e-3) / 1e9
+
+    h2d_gbs = link_rate(lambda: copy_in(slots[0]), total)
+    d2h_gbs = link_rate(lambda: copy_out(slots[0]), d2h)
+
     run(warmup)
     torch.cuda.synchronize(dev)
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -1008,7 +1066,10 @@ def measure_e2e(inp, dims, dev, steps, warmup):
     torch.cuda.synchronize(dev)
     ok = ok and torch.equal(ref_out.cpu(), last["out_h"]) and torch.equal(ref_lse.cpu(), last["lse_h"])
     status = api.get_device_status(ws)
-    return {"ms": e0.elapsed_time(e1) / steps, "h2d": h2d, "d2h": d2h, "readback_ok": ok and status == 0}
+    return {"ms": e0.elapsed_time(e1) / steps, "h2d": h2d, "d2h": d2h, "readback_ok": ok and status == 0,
+            "link": {"h2d_gbs": round(h2d_gbs, 1), "d2h_gbs": round(d2h_gbs, 1),
+                     "pinned_on": (f"the GPU's NUMA node ({len(near.cpus)} local cores)" if near.cpus
+                                   else "the allocating thread's node (NVML gave no CPU affinity)")}}
 
 
 def main():
