@@ -300,7 +300,8 @@ dsa_status_t dsa_indexer_scores(const dsa_dims* dims, const void* q_I, const flo
     const bool fp8 = dims->idx_dtype == DSA_FP8_E4M3;
     if (!q_I || !w || !k_I || !q_seq || !q_len || !scores || (fp8 && (!q_scale || !k_scale)))
         return DSA_ERR_INVALID_ARG;
-    if (!aligned16(q_I) || !aligned16(k_I) || !aligned16(scores) || !aligned16(w) || (fp8 && !aligned16(k_scale)))
+    if (!aligned16(q_I) || !aligned16(k_I) || !aligned16(scores) || !aligned16(w) ||
+        (fp8 && (!aligned16(k_scale) || !aligned16(q_scale))))
         return DSA_ERR_INVALID_ARG;
     if (workspace != nullptr && ws_bytes < kStatusBytes) return DSA_ERR_WORKSPACE;
     return run_indexer(dims, dims->Nq, q_I, q_scale, w, k_I, k_scale, q_seq, q_len, scores,
@@ -317,7 +318,8 @@ dsa_status_t dsa_prefill_indexer_scores(const dsa_dims* dims, const void* q_I, c
         return DSA_ERR_UNSUPPORTED;
     if (dims->Nq == 0) return DSA_OK;
     if (!q_I || !q_scale || !w || !k_I || !k_scale || !q_seq || !q_len || !scores) return DSA_ERR_INVALID_ARG;
-    if (!aligned16(q_I) || !aligned16(k_I) || !aligned16(scores) || !aligned16(w) || !aligned16(k_scale))
+    if (!aligned16(q_I) || !aligned16(k_I) || !aligned16(scores) || !aligned16(w) || !aligned16(k_scale) ||
+        !aligned16(q_scale))
         return DSA_ERR_INVALID_ARG;
     if (workspace != nullptr && ws_bytes < kStatusBytes) return DSA_ERR_WORKSPACE;
     return run_indexer(dims, dims->Nq, q_I, q_scale, w, k_I, k_scale, q_seq, q_len, scores,
@@ -429,7 +431,8 @@ dsa_status_t decode_impl(const dsa_dims* dims, const void* q_I, const float* q_s
         !std::isfinite(softmax_scale))
         return DSA_ERR_INVALID_ARG;
     if (!aligned16(q_I) || !aligned16(k_I) || !aligned16(w) || !aligned16(q) || !aligned16(kv) || !aligned16(out) ||
-        (fp8 && !aligned16(k_scale)) || (scores_out && !aligned16(scores_out)) || (idx_out && !aligned16(idx_out)))
+        (fp8 && (!aligned16(k_scale) || !aligned16(q_scale))) || (scores_out && !aligned16(scores_out)) ||
+        (idx_out && !aligned16(idx_out)))
         return DSA_ERR_INVALID_ARG;
     const Layout L = layout_for(dims, DSA_OP_DECODE);
     if (workspace == nullptr || ws_bytes < L.total) return DSA_ERR_WORKSPACE;
@@ -499,7 +502,7 @@ dsa_status_t dsa_prefill(const dsa_dims* dims, const void* q_I, const float* q_s
         !std::isfinite(softmax_scale))
         return DSA_ERR_INVALID_ARG;
     if (!aligned16(q_I) || !aligned16(k_I) || !aligned16(w) || !aligned16(q) || !aligned16(kv) || !aligned16(out) ||
-        (fp8 && !aligned16(k_scale)) || (idx_out && !aligned16(idx_out)))
+        (fp8 && (!aligned16(k_scale) || !aligned16(q_scale))) || (idx_out && !aligned16(idx_out)))
         return DSA_ERR_INVALID_ARG;
     const Layout L = layout_for(dims, DSA_OP_PREFILL);
     if (workspace == nullptr || ws_bytes < L.total) return DSA_ERR_WORKSPACE;
