@@ -87,6 +87,11 @@ def test_null_and_misaligned_pointers_rejected_before_launch(lib):
     bad[6] = P + 8  # kv
     rc = lib.dsa_decode_step(ctypes.byref(d), *bad, ctypes.c_float(0.07), P, P, None, None, P, 1 << 30, None, None)
     assert rc == _lib.DSA_ERR_INVALID_ARG
+    # misaligned q_scale (every tensor base must be 16-byte aligned)
+    bad = list(args)
+    bad[1] = P + 4  # q_scale
+    rc = lib.dsa_decode_step(ctypes.byref(d), *bad, ctypes.c_float(0.07), P, P, None, None, P, 1 << 30, None, None)
+    assert rc == _lib.DSA_ERR_INVALID_ARG
     # workspace too small
     rc = lib.dsa_decode_step(ctypes.byref(d), *args, ctypes.c_float(0.07), P, P, None, None, P, 1024, None, None)
     assert rc == _lib.DSA_ERR_WORKSPACE
