@@ -447,6 +447,8 @@ def run_ours(args):
             torch.cuda.empty_cache()
         secondary["prefill"] = measure_prefill(65536, dev, K=2, W=1)
         torch.cuda.empty_cache()
+        secondary["dense_crossover"] = measure_crossover(dev, K=3, W=1)
+        torch.cuda.empty_cache()
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -723,6 +725,76 @@ def subset_rows(inp, sel):
     return out
 
 
+def measure_crossover(dev, K=5, W=2, decode_lens=(2048, 4096, 8192, 16384, 32768, 65536, 131072),
+                      prefill_lens=(2048, 4096, 8192, 16384, 32768)):
+    """Where DSA starts to beat dense attention on this GPU: the DSA decode step (indexer +
+    top-2048 + sparse MLA) against dense MLA over every cached token, for a batch of 16 rows
+    of each length, and dsa_prefill against dense causal MLA for one prompt of each length.
+    Medians of K event-timed runs, L2 flushed between runs (outside the events)."""
+    import torch
+    from sparse_long_context_indexer_b200 import _lib, api, inputs
+
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+
+    def timed(fn):
+        for _ in range(W):
+            flush.zero_()
+            fn()
+        torch.cuda.synchronize()
+        ms = []
+        for _ in range(K):
+            flush.zero_()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            fn()
+            e1.record()
+            torch.cuda.synchronize()
+            ms.append(e0.elapsed_time(e1))
+        return statistics.median(ms)
+
+    def point(L, dsa_ms, dense_ms):
+        return {"tokens": L, "dsa_ms": round(dsa_ms, 4), "dense_ms": round(dense_ms, 4),
+                "dense_over_dsa": round(dense_ms / dsa_ms, 3)}
+
+    status = 0
+    dec = []
+    for L in decode_lens:
+        g = inputs.make_decode_inputs(f"crossover_decode_{L}", [L] * BATCH, T_max=L, n_anchors=32, recency=True,
+                                      seed=3, device=dev)
+        dims = api.dims_of(g)
+        ws, ws_d = api.make_workspace(dims, _lib.DSA_OP_DECODE, dev), api.make_workspace(dims, _lib.DSA_OP_DENSE_MLA, dev)
+        out, lse = api.alloc_outputs(g)
+        dsa_ms = timed(lambda: api.run_decode(g, ws=ws, out=out, lse=lse, dims=dims))
+        dense_ms = timed(lambda: api.dense_mla_attn(dims, g.q, g.kv, g.q_seq, g.q_len, g.softmax_scale, out, lse, ws_d))
+        status = status or api.get_device_status(ws) or api.get_device_status(ws_d)
+        dec.append(point(L, dsa_ms, dense_ms))
+        del g, ws, ws_d, out, lse
+        torch.cuda.empty_cache()
+    pre = []
+    for L in prefill_lens:
+        g = inputs.make_prefill_inputs(f"crossover_prefill_{L}", L, seed=4, device=dev)
+        dims = api.dims_of(g)
+        ws, ws_d = api.make_workspace(dims, _lib.DSA_OP_PREFILL, dev), api.make_workspace(dims, _lib.DSA_OP_DENSE_MLA, dev)
+        out, lse = api.alloc_outputs(g)
+        dsa_ms = timed(lambda: api.prefill(dims, g.q_I, g.q_scale, g.w, g.k_I, g.k_scale, g.q, g.kv, g.q_seq, g.q_len,
+                                           g.softmax_scale, out, lse, ws))
+        dense_ms = timed(lambda: api.dense_mla_attn(dims, g.q, g.kv, g.q_seq, g.q_len, g.softmax_scale, out, lse, ws_d))
+        status = status or api.get_device_status(ws) or api.get_device_status(ws_d)
+        pre.append(point(L, dsa_ms, dense_ms))
+        del g, ws, ws_d, out, lse
+        torch.cuda.empty_cache()
+
+    def first_win(pts):
+        return next((p["tokens"] for p in pts if p["dense_over_dsa"] > 1.0), None)
+
+    return {"label": "secondary measurement (the headline is the long decode above)",
+            "decode": {"batch": BATCH, "points": dec, "dsa_faster_from_tokens": first_win(dec)},
+            "prefill": {"points": pre, "dsa_faster_from_tokens": first_win(pre),
+                        "note": "one causal prompt; dense = every row over its whole causal prefix"},
+            "k": 2048, "timing": f"median of {K} event-timed runs per point, L2 flushed between runs",
+            "device_status": status}
+
+
 def run_dense(args):
     """Secondary line: dense MLA over all cached tokens of the long decode, against the DSA step."""
     import torch
@@ -792,6 +864,9 @@ def run_dense(args):
                          "note": "DSA = indexer + top-2048 + sparse MLA on the same batch, same run"},
         "device_status": status,
     }
+    del inp, ws, ws_d, out, lse
+    torch.cuda.empty_cache()
+    line["crossover"] = measure_crossover(dev)
     print(json.dumps(line), flush=True)
     return 0
 
