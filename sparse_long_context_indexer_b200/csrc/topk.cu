@@ -28,9 +28,11 @@
 //     aggregation, merged across the cluster).  Rows whose keys are all equal
 //     take the first k positions directly.
 //  3. A final pass compacts the selected positions in position order: each warp
-//     owns a contiguous segment of the CTA's keys, counts them in a first pass,
-//     and writes its selected positions in a second, with ballots ranking the
-//     keys inside each step.  CTA r knows from the gathered threshold-bin keys
+//     owns a contiguous segment of the CTA's keys and writes its selected
+//     positions, with ballots ranking the keys inside each step.  Its counts
+//     come from the candidate pass of step 2, which reads the same segments
+//     (keys above b*, and its own candidates against tau); the rare paths
+//     without that pass (all-equal rows, the radix fallback) count first.  CTA r knows from the gathered threshold-bin keys
 //     how many ties and outputs the lower-ranked CTAs hold, which gives the
 //     lower-index tie rule across the whole row.
 #include <cooperative_groups.h>
@@ -70,7 +72,8 @@ struct TopkLayout {
     static constexpr int kOffGather = kOffRange + kFineBins;          // all candidates of the row
     static constexpr int kOffKeys = (kOffGather + kCandMax + 3) & ~3;
     static constexpr int kBaseWords = kOffKeys;
-    static_assert(kWarps * kBins >= kCandMax, "the local candidate list lives in the warp-private histograms");
+    static_assert(kWarps * kBins >= 2 * kCandMax,
+                  "the local candidate list and its warps live in the warp-private histograms");
 };
 
 __device__ __forceinline__ uint32_t score_key(float f) {
@@ -249,6 +252,7 @@ __global__ void __launch_bounds__(T, T == 512 ? 2 : 1) topk_radix_kernel(const T
     int local_eq = 0;   // keys of this CTA equal to tau
     int eq_before = 0, out_before = 0;  // ties / outputs of the lower ranks
     bool counts_done = false;           // (cluster-uniform) the lower ranks' counts are known
+    bool warp_counts = false;           // (block-uniform) scr holds every warp's counts for the compaction
     if (kmin == kmax) {
         // every key of the row is equal: the first k positions
         tau = kmin;
@@ -382,14 +386,37 @@ __global__ void __launch_bounds__(T, T == 512 ? 2 : 1) topk_radix_kernel(const T
         block_scan1<T>(la, scr, &latot);
         if (tid == 0) misc[7] = latot;  // read by the higher ranks after the candidate barrier
         if (Tc <= kCandMax) {
-            // ---- 2. the keys of bin b*: every CTA gathers them all and finds tau itself
+            // ---- 2. the keys of bin b*: every CTA gathers them all and finds tau itself.  Each
+            // warp reads the segment of keys it compacts at the end (see below), counts its keys
+            // above b* (all above tau) and records with each of its candidates its warp, so that
+            // the compaction needs no counting pass of its own.
             uint32_t* cand = priv;
-            for (int i0 = 4 * tid; i0 < len; i0 += 4 * kThreads) {
-                const uint4 k4 = keys4_at(i0);
-                const uint32_t kv[4] = {k4.x, k4.y, k4.z, k4.w};
+            uint32_t* cand_w = priv + kCandMax;
+            {
+                const int seg = ((len + kWarps - 1) / kWarps + 127) & ~127;
+                const int w_lo = min(len, warp * seg), w_hi = min(len, w_lo + seg);
+                int above = 0;
+#pragma unroll 1
+                for (int base = w_lo; base < w_hi; base += 128) {
+                    const int i0 = base + 4 * lane;
+                    const uint4 k4 = keys4_at(i0);
+                    const uint32_t kv[4] = {k4.x, k4.y, k4.z, k4.w};
 #pragma unroll
-                for (int u = 0; u < 4; ++u)
-                    if (i0 + u < len && bin_of(kv[u]) == bstar) cand[atomicAdd(misc + 13, 1)] = kv[u];
+                    for (int u = 0; u < 4; ++u) {
+                        if (i0 + u < w_hi) {
+                            const int bb = bin_of(kv[u]);
+                            if (bb > bstar) {
+                                ++above;
+                            } else if (bb == bstar) {
+                                const int slot = atomicAdd(misc + 13, 1);
+                                cand[slot] = kv[u];
+                                cand_w[slot] = (uint32_t)warp;
+                            }
+                        }
+                    }
+                }
+                above = __reduce_add_sync(0xffffffffu, above);
+                if (lane == 0) scr[2 * kWarps + warp] = above;  // block_scan1 uses scr[0 .. kWarps] only
             }
             __syncthreads();
             cluster.sync();
@@ -524,7 +551,21 @@ __global__ void __launch_bounds__(T, T == 512 ? 2 : 1) topk_radix_kernel(const T
                     misc[21] = e_excl;
                 }
             }
+            // every warp's counts for the compaction: its keys above b* plus its own candidates
+            // above and equal to tau
+            if (tid < kWarps) {
+                scr[tid] = scr[2 * kWarps + tid];
+                scr[kWarps + tid] = 0;
+            }
             __syncthreads();
+            for (int i = tid; i < misc[13]; i += kThreads) {
+                const uint32_t kk = cand[i];
+                if (kk > tau)
+                    atomicAdd(&scr[cand_w[i]], 1);
+                else if (kk == tau)
+                    atomicAdd(&scr[kWarps + cand_w[i]], 1);
+            }
+            warp_counts = true;
             local_gt = misc[16];
             local_eq = misc[17];
             out_before = misc[20];
@@ -646,24 +687,26 @@ __global__ void __launch_bounds__(T, T == 512 ? 2 : 1) topk_radix_kernel(const T
     {
         const int seg = ((len + kWarps - 1) / kWarps + 127) & ~127;
         const int w_lo = min(len, warp * seg), w_hi = min(len, w_lo + seg);
-        int gt = 0, eq = 0;
+        if (!warp_counts) {
+            int gt = 0, eq = 0;
 #pragma unroll 1
-        for (int base = w_lo; base < w_hi; base += 128) {  // warp-uniform steps
-            const int i0 = base + 4 * lane;
-            const uint4 k4 = keys4_at(i0);
-            const uint32_t kv[4] = {k4.x, k4.y, k4.z, k4.w};
+            for (int base = w_lo; base < w_hi; base += 128) {  // warp-uniform steps
+                const int i0 = base + 4 * lane;
+                const uint4 k4 = keys4_at(i0);
+                const uint32_t kv[4] = {k4.x, k4.y, k4.z, k4.w};
 #pragma unroll
-            for (int u = 0; u < 4; ++u) {
-                const bool in = i0 + u < w_hi;
-                gt += in && kv[u] > tau;
-                eq += in && kv[u] == tau;
+                for (int u = 0; u < 4; ++u) {
+                    const bool in = i0 + u < w_hi;
+                    gt += in && kv[u] > tau;
+                    eq += in && kv[u] == tau;
+                }
             }
-        }
-        gt = __reduce_add_sync(0xffffffffu, gt);
-        eq = __reduce_add_sync(0xffffffffu, eq);
-        if (lane == 0) {
-            scr[warp] = gt;
-            scr[kWarps + warp] = eq;
+            gt = __reduce_add_sync(0xffffffffu, gt);
+            eq = __reduce_add_sync(0xffffffffu, eq);
+            if (lane == 0) {
+                scr[warp] = gt;
+                scr[kWarps + warp] = eq;
+            }
         }
         __syncthreads();
         if (warp == 0) {
@@ -693,6 +736,28 @@ __global__ void __launch_bounds__(T, T == 512 ? 2 : 1) topk_radix_kernel(const T
         int eq_run = scr[2 * kWarps + warp];
         int out_run = scr[3 * kWarps + warp];
         const unsigned lt = (1u << lane) - 1u;
+        if (scr[kWarps + warp] == 0) {
+            // no key of this warp equals tau: the keys above it, in position order
+#pragma unroll 1
+            for (int base = w_lo; base < w_hi; base += 128) {  // warp-uniform steps (ballots below)
+                const int i0 = base + 4 * lane;
+                const uint4 k4 = keys4_at(i0);
+                const uint32_t kv[4] = {k4.x, k4.y, k4.z, k4.w};
+                unsigned sb[4];
+#pragma unroll
+                for (int u = 0; u < 4; ++u) sb[u] = __ballot_sync(0xffffffffu, i0 + u < w_hi && kv[u] > tau);
+                if ((sb[0] | sb[1] | sb[2] | sb[3]) == 0u) continue;
+                int o = out_run + __popc(sb[0] & lt) + __popc(sb[1] & lt) + __popc(sb[2] & lt) + __popc(sb[3] & lt);
+#pragma unroll
+                for (int u = 0; u < 4; ++u) {
+                    if ((sb[u] >> lane) & 1u) {
+                        if (o < a.k) out[o] = lo + i0 + u;
+                        ++o;
+                    }
+                }
+                out_run += __popc(sb[0]) + __popc(sb[1]) + __popc(sb[2]) + __popc(sb[3]);
+            }
+        } else
 #pragma unroll 1
         for (int base = w_lo; base < w_hi; base += 128) {  // warp-uniform steps (ballots below)
             const int i0 = base + 4 * lane;
