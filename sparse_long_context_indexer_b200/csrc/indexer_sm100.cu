@@ -27,22 +27,25 @@
 // in registers) rather than by a second commit.
 //
 // The epilogue is ALU bound in prefill: per (token, head) one ReLU (FMNMX, on
-// the half-rate ALU pipe) and half a packed fp32 FMA, with the weights
-// broadcast from shared memory.  Sixteen epilogue warps, four per TMEM
-// sub-partition, each own one 64-column block of every accumulator, and give
-// the accumulator back as soon as their loads have landed, so the tensor pipe
-// never waits for the arithmetic.
+// the half-rate ALU pipe) and half a packed fp32 FMA.  Sixteen epilogue warps,
+// four per TMEM sub-partition, give an accumulator back as soon as their loads
+// have landed, so the tensor pipe never waits for the arithmetic.  Decode: each
+// warp owns one 64-column block of every accumulator.  Prefill: two groups of
+// eight warps take alternate stages (accumulators), each warp two blocks, so
+// one group's arithmetic overlaps the other's TMEM loads and waits.
 //
 // Roles (one persistent CTA per SM, each owning a contiguous range of the
 // flat list of (unit, stage) pairs; a unit is one query row in decode, four
 // in prefill):
-//   warp 0       producer: lane 0 issues the TMA copies of each key stage and
-//                of its fp32 scales into a stage ring; at a new unit the warp
-//                writes the folded weights w*q_scale to shared memory and lane
-//                0 fetches the unit's q8 block by TMA
-//   warp 1       TMEM allocator and single-thread tcgen05.mma issuer
-//   warps 2..    epilogue, quad q (one warp per TMEM sub-partition) reading
-//                block q of every accumulator
+//   producer     decode: warps 0-1 copy each key stage and its fp32 scales with
+//                16-byte cp.async into the swizzled stage ring; prefill: warp 0,
+//                lane 0 issuing TMA boxes.  At a new unit warp 0 has lane 0
+//                fetch the unit's q8 block by TMA and writes the folded weights
+//                w*q_scale to shared memory
+//   next warp    TMEM allocator and single-thread tcgen05.mma issuer
+//   the rest     epilogue quads (one warp per TMEM sub-partition), each reading
+//                one block of every accumulator (decode) or two blocks of every
+//                other accumulator (prefill)
 // Every wait is bounded; a timeout records DSA_ERR_TIMEOUT and the CTA drains
 // and exits instead of hanging.
 #include <cuda.h>
@@ -83,7 +86,10 @@ struct IdxCfg {
     // epilogue quad (four warps, one per TMEM sub-partition) reads one block; a group of NB
     // quads covers an accumulator, and with QP groups group g takes the stages it % QP == g.
     static constexpr int NB = SUB * R;
-    static constexpr int QP = R == 2 ? 2 : 1;
+    // Prefill splits its epilogue into QP = 2 groups on alternating stages (accumulators),
+    // each warp reading BPQ = 2 blocks; decode keeps one group of one block per warp.
+    static constexpr int QP = R == 1 ? 1 : 2;
+    static constexpr int BPQ = R == 4 ? 2 : 1;
     // Decode streams its keys with 16-byte cp.async copies from two producer warps, which write
     // the swizzled tile themselves (measured on B200: the long decode's 142.7 MB of keys and
     // scales stream in 27.6 us with plain 16-byte loads against 33.6 us with 64-byte TMA box
@@ -97,7 +103,11 @@ struct IdxCfg {
     static constexpr int SCHUNKS = STOK / 4;         // 16-byte pieces of its scales
     static_assert(!CPASYNC || (KCHUNKS % PROD_THREADS == 0 && SCHUNKS % PROD_THREADS == 0),
                   "every producer thread copies the same number of pieces per stage");
-    static constexpr int EPI_WARPS = 4 * NB * QP;
+    static constexpr int EPI_QUADS = NB * QP / BPQ;  // epilogue quads
+    static constexpr int GQ = EPI_QUADS / QP;          // quads per group
+    static_assert(EPI_QUADS * BPQ == NB * QP && GQ * QP == EPI_QUADS && GQ * BPQ == NB,
+                  "every block of an accumulator is read by one quad of its group");
+    static constexpr int EPI_WARPS = 4 * EPI_QUADS;
     static constexpr int THREADS = (EPI_WARP0 + EPI_WARPS) * 32;
     static constexpr int K_STEPS = D_I / 32;      // kind::f8f6f4 consumes 32 bytes of K per MMA
     // shared memory map (offsets from a 1024-byte aligned base)
@@ -527,44 +537,54 @@ __global__ void __launch_bounds__(IdxCfg<D_I, R>::THREADS, 1)
                 mbar_wait(bar_tfull(last_acc), (last_it / C::ACC) & 1, nullptr, nullptr, 50000000ull);
         }
     } else {
-        // ---------------- epilogue: one 64-column block of its group's accumulators per warp
-        // A warp reads its block (32 token lanes x 64 heads) in the 16x256b shape: thread t
-        // holds tokens g, g+8, g+16, g+24 (g = t/4) at the 16 heads 8k + 2(t%4) + {0, 1}, so
-        // its 16 folded weights stay in registers for the whole unit; four threads then
-        // combine their partial sums by shuffles.
+        // ---------------- epilogue: BPQ 64-column blocks of its group's accumulators per warp
+        // A warp reads a block (32 token lanes x 64 heads) in the 16x256b shape: thread t holds
+        // tokens g, g+8, g+16, g+24 (g = t/4) at the 16 heads 8k + 2(t%4) + {0, 1}, so its 16
+        // folded weights per block stay in registers for the whole unit; four threads then
+        // combine their partial sums by shuffles.  With two groups (prefill) each group takes
+        // every other stage, so one group's arithmetic overlaps the other's loads and waits;
+        // its warps then read two blocks each, half a block (16 token lanes) at a time.
         const int q = (warp - C::EPI_WARP0) >> 2;  // quad
-        const int grp = q / C::NB;                 // group: stages it % QP == grp
-        const int blk = q % C::NB;                 // block of the group's accumulators
+        const int grp = q / C::GQ;                 // group: stages it % QP == grp
+        const int qq = q % C::GQ;                  // quad within the group: blocks qq + b GQ
         const int sub = warp & 3;                  // TMEM sub-partition this warp may access
-        const int h = R == 1 ? blk : 0;            // the block's tile within the stage
-        const int r = R == 1 ? 0 : blk;            // the block's query row within the unit
         const int g = lane >> 2;
         const int i4 = lane & 3;
         // after the shuffles thread t owns token slot u = 2 (t%2) + (t%4)/2: token g + 8u of the
-        // warp's 32 lanes, i.e. token `tok` of every stage
-        const int tok = h * C::TILE + sub * 32 + g + 8 * (2 * (i4 & 1) + (i4 >> 1));
+        // warp's 32 lanes, i.e. token `tok` of every stage (R = 1: of the block's tile)
+        const int tok = (R == 1 ? qq : 0) * C::TILE + sub * 32 + g + 8 * (2 * (i4 & 1) + (i4 >> 1));
         TileCursor<C::STOK, R> cur;
         if (count > 0) cur.start(sh->row0, sh->j0, sh->n0, sh->b0, sh->nt0);
         int qi = -1;
-        int nrow = 0;               // this thread's scores exist for s < nrow (s = stage base + tok)
-        float* srow = nullptr;      // score row of the block's query row, offset by tok
+        int nrow[C::BPQ];           // this thread's scores of block b exist for s < nrow[b] (s = stage base + tok)
+        float* srow[C::BPQ];        // score row of block b's query row, offset by tok
         int acc = 0, accph = 0;     // accumulator of stage `it` and its phase parity
-        uint64_t w2[8];             // folded weights of heads 8k + 2(t%4) + {0, 1}, packed in pairs
+        uint64_t w2[C::BPQ][8];     // folded weights of heads 8k + 2(t%4) + {0, 1}, packed in pairs
 #pragma unroll
-        for (int k = 0; k < 8; ++k) w2[k] = 0;
+        for (int b = 0; b < C::BPQ; ++b) {
+            nrow[b] = 0;
+            srow[b] = nullptr;
+#pragma unroll
+            for (int k = 0; k < 8; ++k) w2[b][k] = 0;
+        }
         for (int it = 0; it < count; ++it) {
             if (it == 0 || cur.j == 0) {
                 ++qi;
                 const int qb = qi & 1;
-                const int64_t row = (int64_t)cur.row * R + r;
-                nrow = (R == 1 ? cur.n : (row < a.Nq ? max(0, min(a.q_len[row], cur.n)) : 0)) - tok;
-                srow = a.scores + row * a.ld + tok;
                 // folded weights of the unit: published by the producer with the q8 block
                 const bool okq = mbar_wait(bar_qfull(qb), (qi >> 1) & 1, abort_flag, a.status);
                 if (!__all_sync(0xffffffffu, okq)) break;
-                const float* wsrc = wq_smem + qb * C::NCOL + r * C::HEADS + 2 * i4;
 #pragma unroll
-                for (int k = 0; k < 8; ++k) w2[k] = pack_f32x2(wsrc[8 * k], wsrc[8 * k + 1]);
+                for (int b = 0; b < C::BPQ; ++b) {
+                    const int blk = qq + b * C::GQ;
+                    const int r = R == 1 ? 0 : blk;  // the block's query row within the unit
+                    const int64_t row = (int64_t)cur.row * R + r;
+                    nrow[b] = (R == 1 ? cur.n : (row < a.Nq ? max(0, min(a.q_len[row], cur.n)) : 0)) - tok;
+                    srow[b] = a.scores + row * a.ld + tok;
+                    const float* wsrc = wq_smem + qb * C::NCOL + r * C::HEADS + 2 * i4;
+#pragma unroll
+                    for (int k = 0; k < 8; ++k) w2[b][k] = pack_f32x2(wsrc[8 * k], wsrc[8 * k + 1]);
+                }
                 // the weights are in registers: the producer may reuse the buffer
                 __syncwarp();
                 if (lane == 0) mbar_arrive(bar_qempty(qb));
@@ -575,55 +595,77 @@ __global__ void __launch_bounds__(IdxCfg<D_I, R>::THREADS, 1)
                 ok = ok && mbar_wait(bar_full(st), (it / C::STAGES) & 1, abort_flag, a.status);
                 if (!__all_sync(0xffffffffu, ok)) break;
                 tc_fence_after();
-                uint32_t v[2][32];
-                {
+                const int sb = cur.j * C::STOK;
+#pragma unroll
+                for (int b = 0; b < C::BPQ; ++b) {
+                    const int blk = qq + b * C::GQ;
                     const uint32_t taddr =
                         tmem + ((uint32_t)(sub * 32) << 16) + acc * (C::SUB * C::NCOL) + blk * C::HEADS;
-                    tmem_ld16x256b_x8(taddr, v[0]);
-                    tmem_ld16x256b_x8(taddr + (16u << 16), v[1]);
-                    tmem_wait_ld_regs(v[0]);
-                    tmem_wait_ld_regs(v[1]);
-                }
-                const int sb = cur.j * C::STOK;
-                const float ks = scale_smem[st * C::STOK + tok];
-                // the accumulator is free (the values are in registers) and so is the key stage (the
-                // MMA that read it has completed; the scale is in a register)
-                tc_fence_before();
-                __syncwarp();
-                if (lane == 0) {
-                    mbar_arrive(bar_tempty(acc));
-                    mbar_arrive(bar_empty(st));
-                }
-                // p2[u]: this thread's 16 heads of token slot u (tokens g, g+8 from the first load,
-                // g+16, g+24 from the second), two heads per packed FMA
-                uint64_t p2[4] = {0, 0, 0, 0};
+                    // p2[u]: this thread's 16 heads of token slot u (tokens g, g+8 from the first
+                    // 16 lanes, g+16, g+24 from the second), two heads per packed FMA
+                    uint64_t p2[4] = {0, 0, 0, 0};
+                    auto accumulate = [&](const uint32_t (&v)[32], int u0) {
 #pragma unroll
-                for (int k = 0; k < 8; ++k) {
+                        for (int k = 0; k < 8; ++k) {
 #pragma unroll
-                    for (int u = 0; u < 4; ++u) {
-                        const uint32_t* x = &v[u >> 1][4 * k + 2 * (u & 1)];
-                        p2[u] = fma_f32x2(w2[k],
-                                          pack_f32x2(fmaxf(__uint_as_float(x[0]), 0.f),
-                                                     fmaxf(__uint_as_float(x[1]), 0.f)),
-                                          p2[u]);
+                            for (int uu = 0; uu < 2; ++uu) {
+                                const uint32_t* x = &v[4 * k + 2 * uu];
+                                p2[u0 + uu] = fma_f32x2(w2[b][k],
+                                                        pack_f32x2(fmaxf(__uint_as_float(x[0]), 0.f),
+                                                                   fmaxf(__uint_as_float(x[1]), 0.f)),
+                                                        p2[u0 + uu]);
+                            }
+                        }
+                    };
+                    // the key scale (from the stage's shared copy); then the accumulator block and the
+                    // key stage are released (the MMA that read the keys has completed)
+                    auto release = [&]() {
+                        tc_fence_before();
+                        __syncwarp();
+                        if (lane == 0) {
+                            mbar_arrive(bar_tempty(acc));
+                            mbar_arrive(bar_empty(st));
+                        }
+                    };
+                    float ks;
+                    if constexpr (C::BPQ == 1) {
+                        uint32_t v[2][32];
+                        tmem_ld16x256b_x8(taddr, v[0]);
+                        tmem_ld16x256b_x8(taddr + (16u << 16), v[1]);
+                        tmem_wait_ld_regs(v[0]);
+                        tmem_wait_ld_regs(v[1]);
+                        ks = scale_smem[st * C::STOK + tok];
+                        release();
+                        accumulate(v[0], 0);
+                        accumulate(v[1], 2);
+                    } else {
+                        uint32_t v[32];
+                        tmem_ld16x256b_x8(taddr, v);
+                        tmem_wait_ld_regs(v);
+                        accumulate(v, 0);
+                        tmem_ld16x256b_x8(taddr + (16u << 16), v);
+                        tmem_wait_ld_regs(v);
+                        ks = scale_smem[st * C::STOK + tok];
+                        release();
+                        accumulate(v, 2);
                     }
+                    float s0, s1, s2, s3, t0, t1, t2, t3;
+                    unpack_f32x2(p2[0], s0, t0);
+                    unpack_f32x2(p2[1], s1, t1);
+                    unpack_f32x2(p2[2], s2, t2);
+                    unpack_f32x2(p2[3], s3, t3);
+                    s0 += t0;
+                    s1 += t1;
+                    s2 += t2;
+                    s3 += t3;
+                    // sum over the four threads of a token group, leaving slot 2 (t%2) + (t%4)/2 here
+                    const bool odd = i4 & 1;
+                    const float qa = (odd ? s2 : s0) + __shfl_xor_sync(0xffffffffu, odd ? s0 : s2, 1);
+                    const float qc = (odd ? s3 : s1) + __shfl_xor_sync(0xffffffffu, odd ? s1 : s3, 1);
+                    const bool hi = i4 & 2;
+                    const float sum = (hi ? qc : qa) + __shfl_xor_sync(0xffffffffu, hi ? qa : qc, 2);
+                    if (sb < nrow[b]) srow[b][sb] = ks * sum;
                 }
-                float s0, s1, s2, s3, t0, t1, t2, t3;
-                unpack_f32x2(p2[0], s0, t0);
-                unpack_f32x2(p2[1], s1, t1);
-                unpack_f32x2(p2[2], s2, t2);
-                unpack_f32x2(p2[3], s3, t3);
-                s0 += t0;
-                s1 += t1;
-                s2 += t2;
-                s3 += t3;
-                // sum over the four threads of a token group, leaving slot 2 (t%2) + (t%4)/2 here
-                const bool odd = i4 & 1;
-                const float qa = (odd ? s2 : s0) + __shfl_xor_sync(0xffffffffu, odd ? s0 : s2, 1);
-                const float qc = (odd ? s3 : s1) + __shfl_xor_sync(0xffffffffu, odd ? s1 : s3, 1);
-                const bool hi = i4 & 2;
-                const float sum = (hi ? qc : qa) + __shfl_xor_sync(0xffffffffu, hi ? qa : qc, 2);
-                if (sb < nrow) srow[sb] = ks * sum;
             }
             if (++acc == C::ACC) {
                 acc = 0;
