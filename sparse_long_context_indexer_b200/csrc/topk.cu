@@ -113,9 +113,13 @@ __device__ __forceinline__ int block_scan1(int v, int* scratch, int* total) {
     return r;
 }
 
-template <int T>
-__global__ void __launch_bounds__(T, T == 512 ? 2 : 1) topk_radix_kernel(const TopkArgs a, int cached_cap) {
+// BATCH: some rows' slices exceed the shared-memory cache, so their passes read the scores
+// from global memory (L2); those reads go out 16 bytes and U steps at a time per thread (one
+// CTA per SM then, for the registers).  Launches whose slices all fit compile without it.
+template <int T, bool BATCH>
+__global__ void __launch_bounds__(T, (T == 512 && !BATCH) ? 2 : 1) topk_radix_kernel(const TopkArgs a, int cached_cap) {
     using L = TopkLayout<T>;
+    constexpr int U = BATCH ? 4 : 1;  // steps of every pass loaded before any is used
     constexpr int kThreads = T;
     constexpr int kWarps = L::kWarps;
     constexpr int kOffPriv = L::kOffPriv, kOffHist = L::kOffHist, kOffTot = L::kOffTot, kOffMisc = L::kOffMisc;
@@ -194,6 +198,32 @@ __global__ void __launch_bounds__(T, T == 512 ? 2 : 1) topk_radix_kernel(const T
             kmn = min(kmn, kk);
             kmx = max(kmx, kk);
         }
+    } else if constexpr (BATCH) {
+        // the same 16-byte loads, eight in flight per thread, keys not kept
+        const int nv = len >> 2;
+        const float4* r4 = reinterpret_cast<const float4*>(row + lo);
+        for (int i0 = 0; i0 < nv; i0 += kLoadBatch * kThreads) {
+            float4 f[kLoadBatch];
+#pragma unroll
+            for (int u = 0; u < kLoadBatch; ++u) {
+                const int i = i0 + u * kThreads + tid;
+                f[u] = i < nv ? __ldg(r4 + i) : make_float4(0.f, 0.f, 0.f, 0.f);
+            }
+#pragma unroll
+            for (int u = 0; u < kLoadBatch; ++u) {
+                if (i0 + u * kThreads + tid < nv) {
+                    const uint32_t k0 = score_key(f[u].x), k1 = score_key(f[u].y), k2 = score_key(f[u].z),
+                                   k3 = score_key(f[u].w);
+                    kmn = min(kmn, min(min(k0, k1), min(k2, k3)));
+                    kmx = max(kmx, max(max(k0, k1), max(k2, k3)));
+                }
+            }
+        }
+        for (int i = 4 * nv + tid; i < len; i += kThreads) {
+            const uint32_t kk = score_key(__ldg(row + lo + i));
+            kmn = min(kmn, kk);
+            kmx = max(kmx, kk);
+        }
     } else {
         for (int i = tid; i < len; i += kThreads) {
             const uint32_t kk = score_key(__ldg(row + lo + i));
@@ -216,6 +246,10 @@ __global__ void __launch_bounds__(T, T == 512 ? 2 : 1) topk_radix_kernel(const T
     // the caller checks i < len)
     auto keys4_at = [&](int i) -> uint4 {
         if (cached && i + 3 < len) return reinterpret_cast<const uint4*>(keys)[i >> 2];
+        if (BATCH && i + 3 < len) {
+            const float4 f = __ldg(reinterpret_cast<const float4*>(row + lo + i));
+            return make_uint4(score_key(f.x), score_key(f.y), score_key(f.z), score_key(f.w));
+        }
         uint4 r;
         r.x = i < len ? key_at(i) : 0u;
         r.y = i + 1 < len ? key_at(i + 1) : 0u;
@@ -286,16 +320,39 @@ __global__ void __launch_bounds__(T, T == 512 ? 2 : 1) topk_radix_kernel(const T
         // keys at or below the base (most of a row's keys once the base is raised) are counted
         // in registers: one shared-memory address taking every one of them serialises the atomics
         int below = 0;
-        for (int i0 = 4 * tid; i0 < len; i0 += 4 * kThreads) {
-            const uint4 k4 = keys4_at(i0);
-            const uint32_t kv[4] = {k4.x, k4.y, k4.z, k4.w};
+        if constexpr (U == 1) {
+            for (int i0 = 4 * tid; i0 < len; i0 += 4 * kThreads) {
+                const uint4 k4 = keys4_at(i0);
+                const uint32_t kv[4] = {k4.x, k4.y, k4.z, k4.w};
 #pragma unroll
-            for (int u = 0; u < 4; ++u) {
-                if (i0 + u < len) {
-                    if (kv[u] <= kbase)
-                        ++below;
-                    else
-                        atomicAdd(&fine[bin_of(kv[u])], 1u);
+                for (int u = 0; u < 4; ++u) {
+                    if (i0 + u < len) {
+                        if (kv[u] <= kbase)
+                            ++below;
+                        else
+                            atomicAdd(&fine[bin_of(kv[u])], 1u);
+                    }
+                }
+            }
+        } else {
+#pragma unroll 1
+            for (int i00 = 4 * tid; i00 < len; i00 += 4 * kThreads * U) {
+                uint4 kq[U];
+#pragma unroll
+                for (int uu = 0; uu < U; ++uu) kq[uu] = keys4_at(i00 + uu * 4 * kThreads);
+#pragma unroll
+                for (int uu = 0; uu < U; ++uu) {
+                    const int i0 = i00 + uu * 4 * kThreads;
+                    const uint32_t kv[4] = {kq[uu].x, kq[uu].y, kq[uu].z, kq[uu].w};
+#pragma unroll
+                    for (int u = 0; u < 4; ++u) {
+                        if (i0 + u < len) {
+                            if (kv[u] <= kbase)
+                                ++below;
+                            else
+                                atomicAdd(&fine[bin_of(kv[u])], 1u);
+                        }
+                    }
                 }
             }
         }
@@ -397,20 +454,25 @@ __global__ void __launch_bounds__(T, T == 512 ? 2 : 1) topk_radix_kernel(const T
                 const int w_lo = min(len, warp * seg), w_hi = min(len, w_lo + seg);
                 int above = 0;
 #pragma unroll 1
-                for (int base = w_lo; base < w_hi; base += 128) {
-                    const int i0 = base + 4 * lane;
-                    const uint4 k4 = keys4_at(i0);
-                    const uint32_t kv[4] = {k4.x, k4.y, k4.z, k4.w};
+                for (int base0 = w_lo; base0 < w_hi; base0 += 128 * U) {
+                    uint4 kq[U];
 #pragma unroll
-                    for (int u = 0; u < 4; ++u) {
-                        if (i0 + u < w_hi) {
-                            const int bb = bin_of(kv[u]);
-                            if (bb > bstar) {
-                                ++above;
-                            } else if (bb == bstar) {
-                                const int slot = atomicAdd(misc + 13, 1);
-                                cand[slot] = kv[u];
-                                cand_w[slot] = (uint32_t)warp;
+                    for (int uu = 0; uu < U; ++uu) kq[uu] = keys4_at(base0 + uu * 128 + 4 * lane);
+#pragma unroll
+                    for (int uu = 0; uu < U; ++uu) {
+                        const int i0 = base0 + uu * 128 + 4 * lane;
+                        const uint32_t kv[4] = {kq[uu].x, kq[uu].y, kq[uu].z, kq[uu].w};
+#pragma unroll
+                        for (int u = 0; u < 4; ++u) {
+                            if (i0 + u < w_hi) {
+                                const int bb = bin_of(kv[u]);
+                                if (bb > bstar) {
+                                    ++above;
+                                } else if (bb == bstar) {
+                                    const int slot = atomicAdd(misc + 13, 1);
+                                    cand[slot] = kv[u];
+                                    cand_w[slot] = (uint32_t)warp;
+                                }
                             }
                         }
                     }
@@ -690,15 +752,20 @@ __global__ void __launch_bounds__(T, T == 512 ? 2 : 1) topk_radix_kernel(const T
         if (!warp_counts) {
             int gt = 0, eq = 0;
 #pragma unroll 1
-            for (int base = w_lo; base < w_hi; base += 128) {  // warp-uniform steps
-                const int i0 = base + 4 * lane;
-                const uint4 k4 = keys4_at(i0);
-                const uint32_t kv[4] = {k4.x, k4.y, k4.z, k4.w};
+            for (int base0 = w_lo; base0 < w_hi; base0 += 128 * U) {  // warp-uniform steps
+                uint4 kq[U];
 #pragma unroll
-                for (int u = 0; u < 4; ++u) {
-                    const bool in = i0 + u < w_hi;
-                    gt += in && kv[u] > tau;
-                    eq += in && kv[u] == tau;
+                for (int uu = 0; uu < U; ++uu) kq[uu] = keys4_at(base0 + uu * 128 + 4 * lane);
+#pragma unroll
+                for (int uu = 0; uu < U; ++uu) {
+                    const int i0 = base0 + uu * 128 + 4 * lane;
+                    const uint32_t kv[4] = {kq[uu].x, kq[uu].y, kq[uu].z, kq[uu].w};
+#pragma unroll
+                    for (int u = 0; u < 4; ++u) {
+                        const bool in = i0 + u < w_hi;
+                        gt += in && kv[u] > tau;
+                        eq += in && kv[u] == tau;
+                    }
                 }
             }
             gt = __reduce_add_sync(0xffffffffu, gt);
@@ -739,30 +806,40 @@ __global__ void __launch_bounds__(T, T == 512 ? 2 : 1) topk_radix_kernel(const T
         if (scr[kWarps + warp] == 0) {
             // no key of this warp equals tau: the keys above it, in position order
 #pragma unroll 1
-            for (int base = w_lo; base < w_hi; base += 128) {  // warp-uniform steps (ballots below)
-                const int i0 = base + 4 * lane;
-                const uint4 k4 = keys4_at(i0);
-                const uint32_t kv[4] = {k4.x, k4.y, k4.z, k4.w};
-                unsigned sb[4];
+            for (int base0 = w_lo; base0 < w_hi; base0 += 128 * U) {  // warp-uniform steps (ballots below)
+                uint4 kq[U];
 #pragma unroll
-                for (int u = 0; u < 4; ++u) sb[u] = __ballot_sync(0xffffffffu, i0 + u < w_hi && kv[u] > tau);
-                if ((sb[0] | sb[1] | sb[2] | sb[3]) == 0u) continue;
-                int o = out_run + __popc(sb[0] & lt) + __popc(sb[1] & lt) + __popc(sb[2] & lt) + __popc(sb[3] & lt);
+                for (int uu = 0; uu < U; ++uu) kq[uu] = keys4_at(base0 + uu * 128 + 4 * lane);
 #pragma unroll
-                for (int u = 0; u < 4; ++u) {
-                    if ((sb[u] >> lane) & 1u) {
-                        if (o < a.k) out[o] = lo + i0 + u;
-                        ++o;
+                for (int uu = 0; uu < U; ++uu) {
+                    const int i0 = base0 + uu * 128 + 4 * lane;
+                    const uint32_t kv[4] = {kq[uu].x, kq[uu].y, kq[uu].z, kq[uu].w};
+                    unsigned sb[4];
+#pragma unroll
+                    for (int u = 0; u < 4; ++u) sb[u] = __ballot_sync(0xffffffffu, i0 + u < w_hi && kv[u] > tau);
+                    if ((sb[0] | sb[1] | sb[2] | sb[3]) == 0u) continue;
+                    int o = out_run + __popc(sb[0] & lt) + __popc(sb[1] & lt) + __popc(sb[2] & lt) +
+                            __popc(sb[3] & lt);
+#pragma unroll
+                    for (int u = 0; u < 4; ++u) {
+                        if ((sb[u] >> lane) & 1u) {
+                            if (o < a.k) out[o] = lo + i0 + u;
+                            ++o;
+                        }
                     }
+                    out_run += __popc(sb[0]) + __popc(sb[1]) + __popc(sb[2]) + __popc(sb[3]);
                 }
-                out_run += __popc(sb[0]) + __popc(sb[1]) + __popc(sb[2]) + __popc(sb[3]);
             }
         } else
 #pragma unroll 1
-        for (int base = w_lo; base < w_hi; base += 128) {  // warp-uniform steps (ballots below)
-            const int i0 = base + 4 * lane;
-            const uint4 k4 = keys4_at(i0);
-            const uint32_t kv[4] = {k4.x, k4.y, k4.z, k4.w};
+        for (int base0 = w_lo; base0 < w_hi; base0 += 128 * U) {  // warp-uniform steps (ballots below)
+          uint4 kq[U];
+#pragma unroll
+          for (int uu = 0; uu < U; ++uu) kq[uu] = keys4_at(base0 + uu * 128 + 4 * lane);
+#pragma unroll
+          for (int uu = 0; uu < U; ++uu) {
+            const int i0 = base0 + uu * 128 + 4 * lane;
+            const uint32_t kv[4] = {kq[uu].x, kq[uu].y, kq[uu].z, kq[uu].w};
             unsigned eb[4];
 #pragma unroll
             for (int u = 0; u < 4; ++u) eb[u] = __ballot_sync(0xffffffffu, i0 + u < w_hi && kv[u] == tau);
@@ -789,6 +866,7 @@ __global__ void __launch_bounds__(T, T == 512 ? 2 : 1) topk_radix_kernel(const T
                 }
             }
             out_run += __popc(sb[0]) + __popc(sb[1]) + __popc(sb[2]) + __popc(sb[3]);
+          }
         }
     }
     cluster_wait_acquire();  // keep this CTA's shared memory alive until every peer has read it
@@ -804,13 +882,11 @@ constexpr int smem_keys_cap() {
     return T == 512 ? kTopkSmemKeys : 40960;
 }
 
-template <int T>
-cudaError_t launch_topk_impl(const TopkArgs& a, int cluster, int64_t row_max, cudaStream_t st) {
-    int64_t chunk = (row_max + cluster - 1) / cluster;
-    chunk = (chunk + 3) & ~int64_t(3);
-    const int cap = (int)(chunk < smem_keys_cap<T>() ? chunk : smem_keys_cap<T>());
+template <int T, bool BATCH>
+cudaError_t launch_topk_variant(const TopkArgs& a, int cluster, int cap, cudaStream_t st) {
     const size_t smem = (size_t)(TopkLayout<T>::kBaseWords + cap) * sizeof(uint32_t);
-    cudaError_t e = cudaFuncSetAttribute(topk_radix_kernel<T>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    cudaError_t e =
+        cudaFuncSetAttribute(topk_radix_kernel<T, BATCH>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(cluster, a.Nq, 1);
@@ -826,9 +902,19 @@ cudaError_t launch_topk_impl(const TopkArgs& a, int cluster, int64_t row_max, cu
     attr[1].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = a.pdl ? 2 : 1;
-    e = cudaLaunchKernelEx(&cfg, topk_radix_kernel<T>, a, cap);
+    e = cudaLaunchKernelEx(&cfg, topk_radix_kernel<T, BATCH>, a, cap);
     if (e != cudaSuccess) return e;
     return cudaGetLastError();
+}
+
+// Slices of up to smem_keys_cap keys live in shared memory; a launch whose longest row's
+// slices are longer takes the variant that streams the rest from global memory in batches.
+template <int T>
+cudaError_t launch_topk_impl(const TopkArgs& a, int cluster, int64_t row_max, cudaStream_t st) {
+    int64_t chunk = (row_max + cluster - 1) / cluster;
+    chunk = (chunk + 3) & ~int64_t(3);
+    const int cap = (int)(chunk < smem_keys_cap<T>() ? chunk : smem_keys_cap<T>());
+    return chunk > cap ? launch_topk_variant<T, true>(a, cluster, cap, st) : launch_topk_variant<T, false>(a, cluster, cap, st);
 }
 
 // How many clusters of c 1024-thread CTAs (one per SM) the device holds at once: cluster
@@ -844,7 +930,7 @@ int max_wide_clusters(int c) {
         constexpr int T = 1024;
         const size_t smem = (size_t)(TopkLayout<T>::kBaseWords + smem_keys_cap<T>()) * sizeof(uint32_t);
         int n = -1;
-        if (cudaFuncSetAttribute(topk_radix_kernel<T>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) ==
+        if (cudaFuncSetAttribute(topk_radix_kernel<T, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) ==
             cudaSuccess) {
             cudaLaunchConfig_t cfg = {};
             cfg.gridDim = dim3(c, 1, 1);
@@ -858,7 +944,7 @@ int max_wide_clusters(int c) {
             cfg.attrs = attr;
             cfg.numAttrs = 1;
             int m = 0;
-            if (cudaOccupancyMaxActiveClusters(&m, topk_radix_kernel<T>, &cfg) == cudaSuccess && m > 0) n = m;
+            if (cudaOccupancyMaxActiveClusters(&m, topk_radix_kernel<T, false>, &cfg) == cudaSuccess && m > 0) n = m;
         }
         (void)cudaGetLastError();  // a refused query only means: no wide launch
         slot = n;
