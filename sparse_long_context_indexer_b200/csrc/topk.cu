@@ -46,7 +46,10 @@ namespace cg = cooperative_groups;
 namespace dsa {
 namespace {
 
-constexpr int kMaxCluster = kTopkMaxCluster;
+// Cluster sizes up to 8 are planned for every launch; rows whose slices would not fit shared
+// memory at that size may take up to 16 one-SM CTAs (a non-portable cluster size).
+constexpr int kMaxCluster = 16;
+static_assert(kMaxCluster >= kTopkMaxCluster && 26 + kMaxCluster < 64, "cluster offsets fit the misc words");
 constexpr int kBins = 256;
 constexpr int kLoadBatch = 8;  // 16-byte score loads in flight per thread
 constexpr int kFineBits = 11;
@@ -120,6 +123,7 @@ template <int T, bool BATCH>
 __global__ void __launch_bounds__(T, (T == 512 && !BATCH) ? 2 : 1) topk_radix_kernel(const TopkArgs a, int cached_cap) {
     using L = TopkLayout<T>;
     constexpr int U = BATCH ? 4 : 1;  // steps of every pass loaded before any is used
+    constexpr int kMaxC = BATCH ? kMaxCluster : kTopkMaxCluster;  // cluster size bound of this variant
     constexpr int kThreads = T;
     constexpr int kWarps = L::kWarps;
     constexpr int kOffPriv = L::kOffPriv, kOffHist = L::kOffHist, kOffTot = L::kOffTot, kOffMisc = L::kOffMisc;
@@ -365,7 +369,7 @@ __global__ void __launch_bounds__(T, (T == 512 && !BATCH) ? 2 : 1) topk_radix_ke
         for (int bb = b_lo + tid; bb < b_hi; bb += kThreads) {
             uint32_t tot_b = 0u;
 #pragma unroll
-            for (int r = 0; r < kMaxCluster; ++r) tot_b += r < C ? cluster.map_shared_rank(fine, r)[bb] : 0u;
+            for (int r = 0; r < kMaxC; ++r) tot_b += r < C ? cluster.map_shared_rank(fine, r)[bb] : 0u;
             rng[bb - b_lo] = tot_b;
             part += (int)tot_b;
         }
@@ -493,15 +497,15 @@ __global__ void __launch_bounds__(T, (T == 512 && !BATCH) ? 2 : 1) topk_radix_ke
                     const int u = __shfl_up_sync(0xffffffffu, incl, o);
                     if (lane >= o) incl += u;
                 }
-                if (lane < kMaxCluster) misc[26 + lane] = incl - c;
-                if (lane == 31) misc[26 + kMaxCluster] = incl;
+                if (lane < kMaxC) misc[26 + lane] = incl - c;
+                if (lane == 31) misc[26 + kMaxC] = incl;
             }
             __syncthreads();
-            const int off = misc[26 + kMaxCluster];
+            const int off = misc[26 + kMaxC];
             for (int i = tid; i < off; i += kThreads) {
                 int r = 0, base = 0;
 #pragma unroll
-                for (int q = 1; q < kMaxCluster; ++q) {
+                for (int q = 1; q < kMaxC; ++q) {
                     const int oq = misc[26 + q];
                     if (q < C && i >= oq) {
                         r = q;
@@ -670,7 +674,7 @@ __global__ void __launch_bounds__(T, (T == 512 && !BATCH) ? 2 : 1) topk_radix_ke
                 if (tid < kBins) {
                     uint32_t sum_r = 0u;
 #pragma unroll
-                    for (int r = 0; r < kMaxCluster; ++r) sum_r += r < C ? cluster.map_shared_rank(hist, r)[tid] : 0u;
+                    for (int r = 0; r < kMaxC; ++r) sum_r += r < C ? cluster.map_shared_rank(hist, r)[tid] : 0u;
                     tot[tid] = sum_r;
                 }
                 __syncthreads();
@@ -888,6 +892,10 @@ cudaError_t launch_topk_variant(const TopkArgs& a, int cluster, int cap, cudaStr
     cudaError_t e =
         cudaFuncSetAttribute(topk_radix_kernel<T, BATCH>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
+    if (cluster > 8) {
+        e = cudaFuncSetAttribute(topk_radix_kernel<T, BATCH>, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+        if (e != cudaSuccess) return e;
+    }
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(cluster, a.Nq, 1);
     cfg.blockDim = dim3(T, 1, 1);
@@ -914,13 +922,14 @@ cudaError_t launch_topk_impl(const TopkArgs& a, int cluster, int64_t row_max, cu
     int64_t chunk = (row_max + cluster - 1) / cluster;
     chunk = (chunk + 3) & ~int64_t(3);
     const int cap = (int)(chunk < smem_keys_cap<T>() ? chunk : smem_keys_cap<T>());
-    return chunk > cap ? launch_topk_variant<T, true>(a, cluster, cap, st) : launch_topk_variant<T, false>(a, cluster, cap, st);
+    return chunk > cap || cluster > kTopkMaxCluster ? launch_topk_variant<T, true>(a, cluster, cap, st)
+                                                    : launch_topk_variant<T, false>(a, cluster, cap, st);
 }
 
 // How many clusters of c 1024-thread CTAs (one per SM) the device holds at once: cluster
 // placement is per GPC, so this can be below SMs / c.  Asked once per device and size.
 constexpr int kMaxTopkDevices = 64;
-int g_wide_clusters[kMaxTopkDevices][kTopkMaxCluster + 1];
+int g_wide_clusters[kMaxTopkDevices][kMaxCluster + 1];
 
 int max_wide_clusters(int c) {
     int dev = 0;
@@ -930,8 +939,10 @@ int max_wide_clusters(int c) {
         constexpr int T = 1024;
         const size_t smem = (size_t)(TopkLayout<T>::kBaseWords + smem_keys_cap<T>()) * sizeof(uint32_t);
         int n = -1;
-        if (cudaFuncSetAttribute(topk_radix_kernel<T, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) ==
-            cudaSuccess) {
+        // sizes above 8 exist only in the variant that streams from global memory
+        auto kern = c <= kTopkMaxCluster ? topk_radix_kernel<T, false> : topk_radix_kernel<T, true>;
+        if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) == cudaSuccess &&
+            (c <= 8 || cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) == cudaSuccess)) {
             cudaLaunchConfig_t cfg = {};
             cfg.gridDim = dim3(c, 1, 1);
             cfg.blockDim = dim3(T, 1, 1);
@@ -944,7 +955,7 @@ int max_wide_clusters(int c) {
             cfg.attrs = attr;
             cfg.numAttrs = 1;
             int m = 0;
-            if (cudaOccupancyMaxActiveClusters(&m, topk_radix_kernel<T, false>, &cfg) == cudaSuccess && m > 0) n = m;
+            if (cudaOccupancyMaxActiveClusters(&m, kern, &cfg) == cudaSuccess && m > 0) n = m;
         }
         (void)cudaGetLastError();  // a refused query only means: no wide launch
         slot = n;
@@ -965,6 +976,14 @@ cudaError_t launch_topk(const TopkArgs& a, int cluster, cudaStream_t st) {
     // slices still fit shared memory wherever the planned launch's would.
     int sms = 0, dev = 0;
     if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    // Rows whose slices would not fit shared memory even as 1,024-thread slices of the planned
+    // cluster: more, smaller slices -- up to 16 one-SM CTAs per row, when the device holds
+    // every row's cluster in one wave (the passes over the scores in global memory then take
+    // proportionally less per CTA).
+    if (sms > 0 && (row_max + cluster - 1) / cluster > smem_keys_cap<1024>()) {
+        for (int c = kMaxCluster; c > cluster; --c)
+            if ((int64_t)a.Nq * c <= sms && a.Nq <= max_wide_clusters(c)) return launch_topk_impl<1024>(a, c, row_max, st);
+    }
     if (sms > 0 && (int64_t)a.Nq * cluster <= sms) {
         const bool planned_fits = (row_max + cluster - 1) / cluster <= smem_keys_cap<512>();
         for (int c = cluster; c >= 1; --c) {
