@@ -16,9 +16,10 @@
 //     fixed digits would need several full passes).  base is the row's
 //     minimum key, raised to 2^-8 of its largest score when that is positive
 //     (keys below count in bin 0; if the threshold lands there the histogram
-//     is rebuilt from the minimum).  CTA r of the
-//     cluster sums one range of bins over all CTAs (distributed shared
-//     memory); the owner of the threshold bin b* broadcasts it.
+//     is rebuilt from the minimum).  Every CTA of the cluster then finds the
+//     threshold bin b* itself: the 64 coarse totals (groups of 32 bins) of
+//     all CTAs, read through distributed shared memory, give the group that
+//     holds the k-th largest key, and that group's 32 bins of all CTAs give b*.
 //  2. The keys of bin b* are collected (usually a few dozen); every CTA
 //     gathers all of them from the cluster and finds tau itself, refining with
 //     2048-bin histograms of the bits below the bin's base (at most two
@@ -71,7 +72,7 @@ struct TopkLayout {
     static constexpr int kOffScan = kOffMisc + 64;              // block-scan and compaction scratch
     static constexpr int kScanWords = 4 * kWarps + 16;
     static constexpr int kOffFine = (kOffScan + kScanWords + 3) & ~3;  // kFineBins counts (read remotely)
-    static constexpr int kOffRange = kOffFine + kFineBins;            // this CTA's range of cluster-wide bin totals
+    static constexpr int kOffRange = kOffFine + kFineBins;            // coarse totals (this CTA's, read remotely; the cluster's)
     static constexpr int kOffGather = kOffRange + kFineBins;          // all candidates of the row
     static constexpr int kOffKeys = (kOffGather + kCandMax + 3) & ~3;
     static constexpr int kBaseWords = kOffKeys;
@@ -167,7 +168,6 @@ __global__ void __launch_bounds__(T, (T == 512 && !BATCH) ? 2 : 1) topk_radix_ke
     if (tid == 0) {
         misc[4] = -1;  // key min (as uint32), max
         misc[5] = 0;
-        misc[6] = 0;   // this CTA's range total
         misc[13] = 0;  // local candidate count
     }
     __syncthreads();
@@ -297,8 +297,8 @@ __global__ void __launch_bounds__(T, (T == 512 && !BATCH) ? 2 : 1) topk_radix_ke
         take_eq_total = a.k;
         local_eq = len;
     } else {
-        // ---- 1. adaptive histogram over the row's key range, cluster totals per range of
-        // bins, threshold bin b*.  The bins cover [kbase, kmax]: kbase is the row's minimum,
+        // ---- 1. adaptive histogram over the row's key range, its coarse and fine totals
+        // over the cluster, threshold bin b*.  The bins cover [kbase, kmax]: kbase is the row's minimum,
         // raised to 2^-kFloorOctaves of the largest score when that is positive (the k-th
         // largest score of a row almost always lies within those octaves of the largest, and
         // the narrower range leaves a few keys in b* instead of hundreds); keys below kbase
@@ -312,10 +312,11 @@ __global__ void __launch_bounds__(T, (T == 512 && !BATCH) ? 2 : 1) topk_radix_ke
             return kk <= kbase ? 0 : min(kFineBins - 1, (int)((kk - kbase) >> shift));
         };
         uint32_t* fine = sm + kOffFine;
-        uint32_t* rng = sm + kOffRange;
-        // CTA rank owns bins [b_lo, b_hi): their totals over the cluster
-        const int per = (kFineBins + C - 1) / C;
-        const int b_lo = min(kFineBins, rank * per), b_hi = min(kFineBins, b_lo + per);
+        constexpr int kGroup = kFineBins / 64;  // bins per coarse group (one per lane)
+        static_assert(kGroup == 32, "a coarse group is one warp's worth of bins");
+        uint32_t* coarse = sm + kOffRange;       // this CTA's 64 coarse totals (read by every peer)
+        uint32_t* ctot = coarse + 64;            // the cluster's coarse totals
+        uint32_t* ftot = coarse + 128;           // the cluster's totals of one group's bins
 #pragma unroll 1
         while (true) {
         shift = max(0, 32 - __clz((int)(kmax - kbase)) - kFineBits);
@@ -364,78 +365,76 @@ __global__ void __launch_bounds__(T, (T == 512 && !BATCH) ? 2 : 1) topk_radix_ke
         for (int o = 16; o > 0; o >>= 1) below += __shfl_xor_sync(0xffffffffu, below, o);
         if (lane == 0 && below > 0) atomicAdd(&fine[0], (uint32_t)below);
         __syncthreads();
-        cluster.sync();
-        int part = 0;
-        for (int bb = b_lo + tid; bb < b_hi; bb += kThreads) {
-            uint32_t tot_b = 0u;
-#pragma unroll
-            for (int r = 0; r < kMaxC; ++r) tot_b += r < C ? cluster.map_shared_rank(fine, r)[bb] : 0u;
-            rng[bb - b_lo] = tot_b;
-            part += (int)tot_b;
+        // this CTA's coarse totals: 64 groups of kGroup consecutive bins (read by every peer)
+        for (int g = warp; g < 64; g += kWarps) {
+            const uint32_t v = __reduce_add_sync(0xffffffffu, fine[g * kGroup + lane]);
+            if (lane == 0) coarse[g] = v;
         }
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) part += __shfl_xor_sync(0xffffffffu, part, o);
-        if (lane == 0) atomicAdd(misc + 6, part);
         __syncthreads();
         cluster.sync();
-        // every CTA finds b* itself: the range holding the k-th largest key (ranges of higher
-        // ranks hold larger keys), then that range's bins read from its owner, top down
+        // Every CTA finds b* itself from the same totals: the coarse group holding the k-th
+        // largest key (groups summed over the cluster), then that group's bins, summed over the
+        // cluster the same way.  Peers read this CTA's coarse and fine totals until the next
+        // cluster barrier, so neither is written before it.
+        if (tid < 64) {
+            uint32_t tot = 0u;
+#pragma unroll
+            for (int r = 0; r < kMaxC; ++r) tot += r < C ? cluster.map_shared_rank(coarse, r)[tid] : 0u;
+            ctot[tid] = tot;
+        }
+        __syncthreads();
         if (warp == 0) {
-            // lane r reads CTA r's range total; keys above range r = the totals of the ranges
-            // above it (a suffix sum); the owner's range holds the k-th largest key
-            const int rs = lane < C ? cluster.map_shared_rank(misc, lane)[6] : 0;
-            int suf = rs;  // inclusive suffix sum over lanes >= this one
+            // lane l holds groups 63 - 2l and 62 - 2l: lanes in descending key order
+            const int v_hi = (int)ctot[63 - 2 * lane], v_lo = (int)ctot[62 - 2 * lane];
+            const int v = v_hi + v_lo;
+            int incl = v;
 #pragma unroll
             for (int o = 1; o < 32; o <<= 1) {
-                const int u = __shfl_down_sync(0xffffffffu, suf, o);
-                if (lane + o < 32) suf += u;
+                const int u = __shfl_up_sync(0xffffffffu, incl, o);
+                if (lane >= o) incl += u;
             }
-            const int above = suf - rs;
-            const bool own = lane < C && above < a.k && a.k <= suf;
-            const unsigned m = __ballot_sync(0xffffffffu, own);
-            const int ow = m ? __ffs(m) - 1 : 0;
-            const int above_ow = __shfl_sync(0xffffffffu, above, ow);
-            if (lane == 0) {
-                misc[24] = ow;
-                misc[25] = above_ow;
+            const int excl = incl - v;
+            const unsigned m = __ballot_sync(0xffffffffu, excl < a.k && a.k <= incl);
+            if (m != 0u && lane == __ffs(m) - 1) {
+                const bool upper = a.k <= excl + v_hi;
+                misc[24] = upper ? 63 - 2 * lane : 62 - 2 * lane;
+                misc[25] = upper ? excl : excl + v_hi;
             }
         }
         __syncthreads();
-        const int owner = misc[24], above_r = misc[25];
-        {
-            const int o_lo = min(kFineBins, owner * per), o_hi = min(kFineBins, o_lo + per);
-            const uint32_t* orng = cluster.map_shared_rank(rng, owner);
-            const int need = a.k - above_r;
-            int cb[4], c4 = 0;
+        const int grp = misc[24], above_g = misc[25];
+        if (tid < kGroup) {
+            uint32_t tot = 0u;
 #pragma unroll
-            for (int u = 0; u < 4; ++u) {
-                const int bb = o_hi - 1 - 4 * tid - u;
-                cb[u] = bb >= o_lo ? (int)orng[bb - o_lo] : 0;
-                c4 += cb[u];
-            }
-            int tsum;
-            const int before = block_scan1<T>(c4, scr, &tsum);
-            if (before < need && need <= before + c4) {
-                int run = before;
-#pragma unroll
-                for (int u = 0; u < 4; ++u) {
-                    if (run < need && need <= run + cb[u]) {
-                        misc[8] = o_hi - 1 - 4 * tid - u;
-                        misc[9] = above_r + run;
-                        misc[10] = cb[u];
-                    }
-                    run += cb[u];
-                }
-            }
-            __syncthreads();
+            for (int r = 0; r < kMaxC; ++r) tot += r < C ? cluster.map_shared_rank(fine, r)[grp * kGroup + tid] : 0u;
+            ftot[tid] = tot;
         }
+        __syncthreads();
+        if (warp == 0) {
+            // lane j holds bin grp * kGroup + kGroup - 1 - j: descending again
+            const int v = (int)ftot[kGroup - 1 - lane];
+            int incl = v;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const int u = __shfl_up_sync(0xffffffffu, incl, o);
+                if (lane >= o) incl += u;
+            }
+            const int excl = incl - v;
+            const int need = a.k - above_g;
+            const unsigned m = __ballot_sync(0xffffffffu, excl < need && need <= incl);
+            if (m != 0u && lane == __ffs(m) - 1) {
+                misc[8] = grp * kGroup + kGroup - 1 - lane;
+                misc[9] = above_g + excl;
+                misc[10] = v;
+            }
+        }
+        __syncthreads();
         // the same b* in every CTA of the cluster (read from the same totals): a uniform exit
         if (misc[8] != 0 || kbase == kmin) break;
         // b* fell to the floor bin: rebuild over the full range once every peer has read this
-        // CTA's range totals
+        // CTA's coarse and fine totals
         kbase = kmin;
         cluster.sync();
-        if (tid == 0) misc[6] = 0;
         }
         const int bstar = misc[8];
         const int above_total = misc[9];
