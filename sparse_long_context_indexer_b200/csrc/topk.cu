@@ -58,6 +58,8 @@ constexpr int kFineBins = 1 << kFineBits;  // adaptive histogram bins
 constexpr int kCandMax = 2048;             // threshold-bin keys resolved on chip by every CTA
 constexpr int kRankMax = 64;               // up to this many, tau is found by direct ranking
 constexpr uint32_t kFloorOctaves = 8;      // the first histogram's floor: 2^-8 of the row's largest score
+constexpr int kMiscAbove = 48;             // misc words 48 .. 63: every rank's keys above b* (local copies)
+static_assert(kMiscAbove >= 26 + 16 + 1 && kMiscAbove + 16 <= 64, "the copies fit beside the cluster offsets");
 
 // Shared-memory map (32-bit words) of a CTA of T threads.  512-thread CTAs fit two per SM
 // (launches with more rows than one wave holds); 1024-thread CTAs take a whole SM (launches
@@ -489,7 +491,10 @@ __global__ void __launch_bounds__(T, (T == 512 && !BATCH) ? 2 : 1) topk_radix_ke
             // every CTA's candidate count (lane r of warp 0 reads CTA r's) and their offsets in
             // the gathered list, then all copies at once
             if (warp == 0) {
-                const int c = lane < C ? cluster.map_shared_rank(misc, lane)[13] : 0;
+                const int* rm = cluster.map_shared_rank(misc, lane < C ? lane : 0);
+                const int c = lane < C ? rm[13] : 0;
+                // each rank's keys above b* come along (used for the counts once tau is known)
+                if (lane < C) misc[kMiscAbove + lane] = rm[7];
                 int incl = c;
 #pragma unroll
                 for (int o = 1; o < 32; o <<= 1) {
@@ -591,7 +596,7 @@ __global__ void __launch_bounds__(T, (T == 512 && !BATCH) ? 2 : 1) topk_radix_ke
             if (warp == 0) {
                 int g = 0, e = 0;
                 if (lane < C) {
-                    g = lane == rank ? latot : cluster.map_shared_rank(misc, lane)[7];
+                    g = misc[kMiscAbove + lane];
                     const int b0 = misc[26 + lane], b1 = misc[27 + lane];
                     for (int i = b0; i < b1; ++i) {
                         g += gbuf[i] > tau;
