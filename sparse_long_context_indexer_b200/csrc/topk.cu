@@ -838,43 +838,46 @@ __global__ void __launch_bounds__(T, (T == 512 && !BATCH) ? 2 : 1) topk_radix_ke
                     out_run += __popc(sb[0]) + __popc(sb[1]) + __popc(sb[2]) + __popc(sb[3]);
                 }
             }
-        } else
+        } else {
 #pragma unroll 1
-        for (int base0 = w_lo; base0 < w_hi; base0 += 128 * U) {  // warp-uniform steps (ballots below)
-          uint4 kq[U];
+            for (int base0 = w_lo; base0 < w_hi; base0 += 128 * U) {  // warp-uniform steps (ballots below)
+                uint4 kq[U];
 #pragma unroll
-          for (int uu = 0; uu < U; ++uu) kq[uu] = keys4_at(base0 + uu * 128 + 4 * lane);
+                for (int uu = 0; uu < U; ++uu) kq[uu] = keys4_at(base0 + uu * 128 + 4 * lane);
 #pragma unroll
-          for (int uu = 0; uu < U; ++uu) {
-            const int i0 = base0 + uu * 128 + 4 * lane;
-            const uint32_t kv[4] = {kq[uu].x, kq[uu].y, kq[uu].z, kq[uu].w};
-            unsigned eb[4];
+                for (int uu = 0; uu < U; ++uu) {
+                    const int i0 = base0 + uu * 128 + 4 * lane;
+                    const uint32_t kv[4] = {kq[uu].x, kq[uu].y, kq[uu].z, kq[uu].w};
+                    unsigned eb[4];
 #pragma unroll
-            for (int u = 0; u < 4; ++u) eb[u] = __ballot_sync(0xffffffffu, i0 + u < w_hi && kv[u] == tau);
-            // ties at lower positions in this step: lower lanes (all four keys), then this lane's
-            int eq_before = eq_run + __popc(eb[0] & lt) + __popc(eb[1] & lt) + __popc(eb[2] & lt) + __popc(eb[3] & lt);
-            bool sel[4];
+                    for (int u = 0; u < 4; ++u) eb[u] = __ballot_sync(0xffffffffu, i0 + u < w_hi && kv[u] == tau);
+                    // ties at lower positions in this step: lower lanes (all four keys), then this lane's
+                    int eq_before = eq_run + __popc(eb[0] & lt) + __popc(eb[1] & lt) + __popc(eb[2] & lt) +
+                                    __popc(eb[3] & lt);
+                    bool sel[4];
 #pragma unroll
-            for (int u = 0; u < 4; ++u) {
-                const bool in = i0 + u < w_hi;
-                const bool is_eq = (eb[u] >> lane) & 1u;
-                sel[u] = in && (kv[u] > tau || (is_eq && eq_before < take_eq_local));
-                eq_before += is_eq;
-            }
-            eq_run += __popc(eb[0]) + __popc(eb[1]) + __popc(eb[2]) + __popc(eb[3]);
-            unsigned sb[4];
+                    for (int u = 0; u < 4; ++u) {
+                        const bool in = i0 + u < w_hi;
+                        const bool is_eq = (eb[u] >> lane) & 1u;
+                        sel[u] = in && (kv[u] > tau || (is_eq && eq_before < take_eq_local));
+                        eq_before += is_eq;
+                    }
+                    eq_run += __popc(eb[0]) + __popc(eb[1]) + __popc(eb[2]) + __popc(eb[3]);
+                    unsigned sb[4];
 #pragma unroll
-            for (int u = 0; u < 4; ++u) sb[u] = __ballot_sync(0xffffffffu, sel[u]);
-            int o = out_run + __popc(sb[0] & lt) + __popc(sb[1] & lt) + __popc(sb[2] & lt) + __popc(sb[3] & lt);
+                    for (int u = 0; u < 4; ++u) sb[u] = __ballot_sync(0xffffffffu, sel[u]);
+                    int o = out_run + __popc(sb[0] & lt) + __popc(sb[1] & lt) + __popc(sb[2] & lt) +
+                            __popc(sb[3] & lt);
 #pragma unroll
-            for (int u = 0; u < 4; ++u) {
-                if (sel[u]) {
-                    if (o < a.k) out[o] = lo + i0 + u;
-                    ++o;
+                    for (int u = 0; u < 4; ++u) {
+                        if (sel[u]) {
+                            if (o < a.k) out[o] = lo + i0 + u;
+                            ++o;
+                        }
+                    }
+                    out_run += __popc(sb[0]) + __popc(sb[1]) + __popc(sb[2]) + __popc(sb[3]);
                 }
             }
-            out_run += __popc(sb[0]) + __popc(sb[1]) + __popc(sb[2]) + __popc(sb[3]);
-          }
         }
     }
     cluster_wait_acquire();  // keep this CTA's shared memory alive until every peer has read it
@@ -986,7 +989,8 @@ cudaError_t launch_topk(const TopkArgs& a, int cluster, cudaStream_t st) {
     // proportionally less per CTA).
     if (sms > 0 && (row_max + cluster - 1) / cluster > smem_keys_cap<1024>()) {
         for (int c = kMaxCluster; c > cluster; --c)
-            if ((int64_t)a.Nq * c <= sms && a.Nq <= max_wide_clusters(c)) return launch_topk_impl<1024>(a, c, row_max, st);
+            if ((int64_t)a.Nq * c <= sms && a.Nq <= max_wide_clusters(c))
+                return launch_topk_impl<1024>(a, c, row_max, st);
     }
     if (sms > 0 && (int64_t)a.Nq * cluster <= sms) {
         const bool planned_fits = (row_max + cluster - 1) / cluster <= smem_keys_cap<512>();
