@@ -246,7 +246,6 @@ __global__ void __launch_bounds__(T, (T == 512 && !BATCH) ? 2 : 1) topk_radix_ke
         atomicMin(reinterpret_cast<unsigned*>(misc + 4), kmn);
         atomicMax(reinterpret_cast<unsigned*>(misc + 5), kmx);
     }
-    __syncthreads();
     auto key_at = [&](int i) -> uint32_t { return cached ? keys[i] : score_key(__ldg(row + lo + i)); };
     // the 4 consecutive keys starting at i (a multiple of 4); out-of-range keys read as 0 (never selected:
     // the caller checks i < len)
@@ -263,7 +262,7 @@ __global__ void __launch_bounds__(T, (T == 512 && !BATCH) ? 2 : 1) topk_radix_ke
         r.w = i + 3 < len ? key_at(i + 3) : 0u;
         return r;
     };
-    cluster.sync();
+    cluster.sync();  // (a cluster barrier orders this CTA's own shared memory as well)
     // the row's key range: lane r of warp 0 reads CTA r's min and max (one remote read each,
     // instead of every thread reading every rank), shared through this CTA's memory
     if (warp == 0) {
@@ -372,7 +371,6 @@ __global__ void __launch_bounds__(T, (T == 512 && !BATCH) ? 2 : 1) topk_radix_ke
             const uint32_t v = __reduce_add_sync(0xffffffffu, fine[g * kGroup + lane]);
             if (lane == 0) coarse[g] = v;
         }
-        __syncthreads();
         cluster.sync();
         // Every CTA finds b* itself from the same totals: the coarse group holding the k-th
         // largest key (groups summed over the cluster), then that group's bins, summed over the
@@ -485,7 +483,6 @@ __global__ void __launch_bounds__(T, (T == 512 && !BATCH) ? 2 : 1) topk_radix_ke
                 above = __reduce_add_sync(0xffffffffu, above);
                 if (lane == 0) scr[2 * kWarps + warp] = above;  // block_scan1 uses scr[0 .. kWarps] only
             }
-            __syncthreads();
             cluster.sync();
             uint32_t* gbuf = sm + kOffGather;
             // every CTA's candidate count (lane r of warp 0 reads CTA r's) and their offsets in
