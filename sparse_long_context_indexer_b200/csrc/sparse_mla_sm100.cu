@@ -662,8 +662,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int rank = (int)cluster_ctarank();
         const int hp = (kCtaHeads + S - 1) / S;
         const float* pub = reinterpret_cast<const float*>(smem + kOffP);
-        __syncthreads();
-        cluster_sync_all();
+        cluster_sync_all();  // (also the CTA's own barrier: every warp has left its role)
         tc_fence_after();
         {
             // receive slot of (split s, owned head hl): 1 KB row at sKv + (s * hp + hl) * 1024, its
