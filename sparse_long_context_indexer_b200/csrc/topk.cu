@@ -292,6 +292,31 @@ __global__ void __launch_bounds__(T, (T == 512 && !BATCH) ? 2 : 1) topk_radix_ke
     int eq_before = 0, out_before = 0;  // ties / outputs of the lower ranks
     bool counts_done = false;           // (cluster-uniform) the lower ranks' counts are known
     bool warp_counts = false;           // (block-uniform) scr holds every warp's counts for the compaction
+    bool slots_done = false;            // (block-uniform) scr holds every warp's first tie rank and slot
+    // Warp 0, lane w: from warp w's keys above tau (scr[w]) and equal to it (scr[kWarps + w]),
+    // warp w's first tie rank (scr[2 kWarps + w]) and first output slot (scr[3 kWarps + w]).
+    auto warp_slots = [&](int take_eq_local, int first_out) {
+        const int g = lane < kWarps ? scr[lane] : 0;
+        const int e = lane < kWarps ? scr[kWarps + lane] : 0;
+        int e_incl = e;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int v = __shfl_up_sync(0xffffffffu, e_incl, o);
+            if (lane >= o) e_incl += v;
+        }
+        const int e_excl = e_incl - e;
+        const int taken = g + max(0, min(take_eq_local - e_excl, e));
+        int t_incl = taken;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int v = __shfl_up_sync(0xffffffffu, t_incl, o);
+            if (lane >= o) t_incl += v;
+        }
+        if (lane < kWarps) {
+            scr[2 * kWarps + lane] = e_excl;
+            scr[3 * kWarps + lane] = first_out + t_incl - taken;
+        }
+    };
     if (kmin == kmax) {
         // every key of the row is equal: the first k positions
         tau = kmin;
@@ -517,24 +542,95 @@ __global__ void __launch_bounds__(T, (T == 512 && !BATCH) ? 2 : 1) topk_radix_ke
             }
             __syncthreads();
             if (off <= kRankMax) {
-                // a few candidates: tau is the candidate c with #{> c} < rem <= #{>= c}, found by
-                // ranking every candidate against all others (quadratic, so only for small sets)
-                const int rem = a.k - above_total;
-                if (tid < off) {
-                    const uint32_t c = gbuf[tid];
-                    int gt = 0, ge = 0;
-                    for (int j = 0; j < off; ++j) {
-                        const uint32_t o = gbuf[j];
-                        gt += o > c;
-                        ge += o >= c;
+                // A few candidates, two per lane of warp 0, which alone finds tau, every rank's
+                // counts, this CTA's per-warp counts and the compaction's slots; the other warps
+                // wait at one barrier.  tau is the candidate c with #{> c} < rem <= #{>= c}, found
+                // by ranking every candidate against all others.
+                if (warp == 0) {
+                    const int rem = a.k - above_total;
+                    const bool v0 = lane < off, v1 = lane + 32 < off;
+                    const uint32_t c0 = v0 ? gbuf[lane] : 0u;
+                    const uint32_t c1 = v1 ? gbuf[lane + 32] : 0u;
+                    int gt0 = 0, ge0 = 0, gt1 = 0, ge1 = 0;
+                    const int n0 = min(off, 32);
+#pragma unroll 4
+                    for (int j = 0; j < n0; ++j) {
+                        const uint32_t o = __shfl_sync(0xffffffffu, c0, j);
+                        gt0 += o > c0;
+                        ge0 += o >= c0;
+                        gt1 += o > c1;
+                        ge1 += o >= c1;
                     }
-                    if (gt < rem && rem <= ge) {
-                        // every thread holding a copy of tau writes the same values
-                        misc[11] = (int)c;
-                        misc[12] = rem - gt;  // candidates equal to tau that are taken
+#pragma unroll 4
+                    for (int j = 0; j < off - 32; ++j) {
+                        const uint32_t o = __shfl_sync(0xffffffffu, c1, j);
+                        gt0 += o > c0;
+                        ge0 += o >= c0;
+                        gt1 += o > c1;
+                        ge1 += o >= c1;
+                    }
+                    // every copy of tau has the same counts: take the first
+                    const unsigned h0 = __ballot_sync(0xffffffffu, v0 && gt0 < rem && rem <= ge0);
+                    const unsigned h1 = __ballot_sync(0xffffffffu, v1 && gt1 < rem && rem <= ge1);
+                    const int src = h0 ? __ffs(h0) - 1 : __ffs(h1) - 1;
+                    const uint32_t t = __shfl_sync(0xffffffffu, h0 ? c0 : c1, src);
+                    const int take_eq = rem - __shfl_sync(0xffffffffu, h0 ? gt0 : gt1, src);
+                    // bit i of mgt / meq: candidate gbuf[i] is above / equal to tau; rank r's
+                    // candidates are gbuf[misc[26 + r], misc[27 + r]), lane r counts rank r
+                    const uint64_t mgt = (uint64_t)__ballot_sync(0xffffffffu, v1 && c1 > t) << 32 |
+                                         __ballot_sync(0xffffffffu, v0 && c0 > t);
+                    const uint64_t meq = (uint64_t)__ballot_sync(0xffffffffu, v1 && c1 == t) << 32 |
+                                         __ballot_sync(0xffffffffu, v0 && c0 == t);
+                    int g = 0, e = 0;
+                    if (lane < C) {
+                        const int b0 = misc[26 + lane], b1 = misc[27 + lane];
+                        const uint64_t below0 = b0 >= 64 ? ~0ull : (1ull << b0) - 1ull;
+                        const uint64_t below1 = b1 >= 64 ? ~0ull : (1ull << b1) - 1ull;
+                        g = misc[kMiscAbove + lane] + __popcll(mgt & below1 & ~below0);
+                        e = __popcll(meq & below1 & ~below0);
+                    }
+                    int e_incl = e;
+#pragma unroll
+                    for (int o = 1; o < 32; o <<= 1) {
+                        const int u = __shfl_up_sync(0xffffffffu, e_incl, o);
+                        if (lane >= o) e_incl += u;
+                    }
+                    const int e_excl = e_incl - e;
+                    int ob = lane < rank ? g + max(0, min(take_eq - e_excl, e)) : 0;
+#pragma unroll
+                    for (int o = 16; o > 0; o >>= 1) ob += __shfl_xor_sync(0xffffffffu, ob, o);
+                    const int my_eq = __shfl_sync(0xffffffffu, e, rank);
+                    const int my_eq_before = __shfl_sync(0xffffffffu, e_excl, rank);
+                    // this CTA's per-warp counts: the warp's keys above b* plus its own candidates
+                    // above and equal to tau (local candidate i is cand[i], found by warp cand_w[i])
+                    if (lane < kWarps) {
+                        scr[lane] = scr[2 * kWarps + lane];
+                        scr[kWarps + lane] = 0;
+                    }
+                    __syncwarp();
+                    const int nloc = misc[13];
+#pragma unroll
+                    for (int i = lane; i < 64; i += 32) {
+                        if (i < nloc) {
+                            const uint32_t kk = cand[i];
+                            if (kk > t)
+                                atomicAdd(&scr[cand_w[i]], 1);
+                            else if (kk == t)
+                                atomicAdd(&scr[kWarps + cand_w[i]], 1);
+                        }
+                    }
+                    __syncwarp();
+                    warp_slots(max(0, min(take_eq - my_eq_before, my_eq)), ob);
+                    if (lane == 0) {
+                        misc[11] = (int)t;
+                        misc[12] = take_eq;
+                        misc[17] = my_eq;
+                        misc[20] = ob;
+                        misc[21] = my_eq_before;
                     }
                 }
                 __syncthreads();
+                slots_done = true;
             } else {
                 // tau among the candidates (keys in [base, base + 2^shift)): refine by 2048-bin
                 // histograms of the bits below the bin base, at most two levels for shift <= 22;
@@ -590,7 +686,7 @@ __global__ void __launch_bounds__(T, (T == 512 && !BATCH) ? 2 : 1) topk_radix_ke
             // Every rank's counts come from the gathered list (rank r's candidates are
             // gbuf[misc[26 + r], misc[27 + r])) and from its keys above b* (its misc[7]): lane r
             // of warp 0 counts rank r; ties are taken lowest rank first.  No further exchange.
-            if (warp == 0) {
+            if (!slots_done && warp == 0) {
                 int g = 0, e = 0;
                 if (lane < C) {
                     g = misc[kMiscAbove + lane];
@@ -620,20 +716,22 @@ __global__ void __launch_bounds__(T, (T == 512 && !BATCH) ? 2 : 1) topk_radix_ke
             }
             // every warp's counts for the compaction: its keys above b* plus its own candidates
             // above and equal to tau
-            if (tid < kWarps) {
-                scr[tid] = scr[2 * kWarps + tid];
-                scr[kWarps + tid] = 0;
-            }
-            __syncthreads();
-            for (int i = tid; i < misc[13]; i += kThreads) {
-                const uint32_t kk = cand[i];
-                if (kk > tau)
-                    atomicAdd(&scr[cand_w[i]], 1);
-                else if (kk == tau)
-                    atomicAdd(&scr[kWarps + cand_w[i]], 1);
+            if (!slots_done) {
+                if (tid < kWarps) {
+                    scr[tid] = scr[2 * kWarps + tid];
+                    scr[kWarps + tid] = 0;
+                }
+                __syncthreads();
+                for (int i = tid; i < misc[13]; i += kThreads) {
+                    const uint32_t kk = cand[i];
+                    if (kk > tau)
+                        atomicAdd(&scr[cand_w[i]], 1);
+                    else if (kk == tau)
+                        atomicAdd(&scr[kWarps + cand_w[i]], 1);
+                }
+                local_gt = misc[16];
             }
             warp_counts = true;
-            local_gt = misc[16];
             local_eq = misc[17];
             out_before = misc[20];
             eq_before = misc[21];
@@ -739,9 +837,9 @@ __global__ void __launch_bounds__(T, (T == 512 && !BATCH) ? 2 : 1) topk_radix_ke
         out_before = misc[20];
         eq_before = misc[21];
     }
-    // This CTA reads no peer's shared memory from here on: arrive now, wait before exiting
-    // (peers may still be reading this CTA's candidates and counts until they arrive).
-    __syncthreads();
+    // This thread reads no peer's shared memory from here on: arrive now, wait before exiting
+    // (peers may still be reading this CTA's candidates and counts until they arrive).  The
+    // arrival is per thread, so no block barrier is needed in front of it.
     cluster_arrive_release();
     const int take_eq_local = max(0, min(take_eq_total - eq_before, local_eq));
 
@@ -780,31 +878,11 @@ __global__ void __launch_bounds__(T, (T == 512 && !BATCH) ? 2 : 1) topk_radix_ke
                 scr[kWarps + warp] = eq;
             }
         }
-        __syncthreads();
-        if (warp == 0) {
-            // lane w: warp w's first tie rank and first output slot
-            const int g = lane < kWarps ? scr[lane] : 0;
-            const int e = lane < kWarps ? scr[kWarps + lane] : 0;
-            int e_incl = e;
-#pragma unroll
-            for (int o = 1; o < 32; o <<= 1) {
-                const int v = __shfl_up_sync(0xffffffffu, e_incl, o);
-                if (lane >= o) e_incl += v;
-            }
-            const int e_excl = e_incl - e;
-            const int taken = g + max(0, min(take_eq_local - e_excl, e));
-            int t_incl = taken;
-#pragma unroll
-            for (int o = 1; o < 32; o <<= 1) {
-                const int v = __shfl_up_sync(0xffffffffu, t_incl, o);
-                if (lane >= o) t_incl += v;
-            }
-            if (lane < kWarps) {
-                scr[2 * kWarps + lane] = e_excl;
-                scr[3 * kWarps + lane] = out_before + t_incl - taken;
-            }
+        if (!slots_done) {
+            __syncthreads();
+            if (warp == 0) warp_slots(take_eq_local, out_before);
+            __syncthreads();
         }
-        __syncthreads();
         int eq_run = scr[2 * kWarps + warp];
         int out_run = scr[3 * kWarps + warp];
         const unsigned lt = (1u << lane) - 1u;
