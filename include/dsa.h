@@ -224,7 +224,12 @@ dsa_status_t dsa_sparse_mla_attn_noalloc(const dsa_dims* dims, const void* q, co
  * position (kgptalkie, "How Does the Selector Pick 1,024?": a short prompt is
  * read in full), so when scores_out is NULL the indexer skips such rows and
  * the top-k writes 0 .. q_len[t]-1 without reading scores; the outputs are
- * the same.  events may be NULL. */
+ * the same.  When the whole cache is that short (T_max <= k and
+ * ld_scores >= T_max, a bf16 or FP8 latent cache), the step is attention over
+ * every position s < q_len[t]: it runs the attention kernel's dense form (the
+ * computation of dsa_dense_mla_attn, same output bits), and the indexer and
+ * the top-k run only to fill scores_out / idx_out when those are given.  A
+ * stage with nothing to run still records its events.  events may be NULL. */
 dsa_status_t dsa_decode_step(const dsa_dims* dims,
                              const void* q_I, const float* q_scale, const void* w,
                              const void* k_I, const float* k_scale,

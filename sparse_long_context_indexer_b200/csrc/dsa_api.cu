@@ -134,6 +134,15 @@ dsa_dims dense_dims(const dsa_dims* d) {
     return e;
 }
 
+// A decode over a cache of at most k positions per sequence: every row selects all of its
+// positions (min(k, n) = n), so the step is attention over every position s < q_len[t], which
+// the attention kernel's dense form computes with no indexer and no top-k.  Rows can then exceed
+// neither k nor the scores' row length without exceeding T_max, which the attention checks.
+// The fp32 cache has no dense form.
+bool short_cache_decode(const dsa_dims* d) {
+    return d->T_max <= d->k && d->ld_scores >= d->T_max && d->kv_dtype != DSA_F32;
+}
+
 Layout layout_for(const dsa_dims* d, int op) {
     Layout L;
     if (op == DSA_OP_SPARSE_MLA) {
@@ -147,7 +156,14 @@ Layout layout_for(const dsa_dims* d, int op) {
         L.total = align_up(L.total + (size_t)rows * d->ld_scores * sizeof(float));
         L.idx = L.total;
         L.total = align_up(L.total + (size_t)rows * d->k * sizeof(int32_t));
-        add_mla_partials(L, d, rows, plan_mla(d, rows));
+        MlaPlan p = plan_mla(d, rows);
+        if (op == DSA_OP_DECODE && short_cache_decode(d)) {
+            // the dense form plans its splits over T_max rounded up to whole tiles
+            const dsa_dims e = dense_dims(d);
+            const MlaPlan pe = plan_mla(&e, rows);
+            if (pe.splits > p.splits) p = pe;
+        }
+        add_mla_partials(L, d, rows, p);
     }
     return L;
 }
@@ -441,20 +457,33 @@ dsa_status_t decode_impl(const dsa_dims* dims, const void* q_I, const float* q_s
     int* status = status_word(workspace);
     float* scores = scores_out ? scores_out : reinterpret_cast<float*>(ws + L.scores);
     int32_t* idx = idx_out ? idx_out : reinterpret_cast<int32_t*>(ws + L.idx);
+    // Short-context dispatch.  Rows with at most k positions select all of them: unless the
+    // caller asked for the scores, the indexer skips those rows.  When the whole cache is that
+    // short, the attention runs in dense form and the indexer and top-k run only for the
+    // outputs the caller asked for (the top-k copies such rows' positions through).
+    const bool short_cache = short_cache_decode(dims);
     record_event(events, 0, st);
-    // rows with at most k positions select all of them: unless the caller asked for the
-    // scores, the indexer skips those rows (short-context dispatch, same results)
-    s = run_indexer(dims, dims->Nq, q_I, q_scale, w, k_I, k_scale, q_seq, q_len, scores, status, st, false,
-                    scores_out ? 0 : dims->k, paged);
-    if (s != DSA_OK) return s;
+    if (!short_cache || scores_out) {
+        s = run_indexer(dims, dims->Nq, q_I, q_scale, w, k_I, k_scale, q_seq, q_len, scores, status, st, false,
+                        scores_out ? 0 : dims->k, paged);
+        if (s != DSA_OK) return s;
+    }
     record_event(events, 1, st);
     // top-k and attention follow their producer as programmatic dependents: their setup
     // overlaps the previous kernel's tail and they wait on the device for its output
-    s = run_topk(dims, dims->Nq, scores, q_len, idx, status, st, true);
-    if (s != DSA_OK) return s;
+    if (!short_cache || idx_out) {
+        s = run_topk(dims, dims->Nq, scores, q_len, idx, status, st, true);
+        if (s != DSA_OK) return s;
+    }
     record_event(events, 2, st);
-    s = run_mla(dims, dims->Nq, q, kv, idx, q_seq, q_len, softmax_scale, out, lse, workspace, L, events, st, true,
-                true, paged);
+    if (short_cache) {
+        const dsa_dims e = dense_dims(dims);
+        s = run_mla(&e, dims->Nq, q, kv, nullptr, q_seq, q_len, softmax_scale, out, lse, workspace, L, events, st,
+                    true, true, paged);
+    } else {
+        s = run_mla(dims, dims->Nq, q, kv, idx, q_seq, q_len, softmax_scale, out, lse, workspace, L, events, st,
+                    true, true, paged);
+    }
     if (s != DSA_OK) return s;
     record_event(events, 4, st);
     return DSA_OK;

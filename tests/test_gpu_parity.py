@@ -276,6 +276,72 @@ def test_short_rows_skip_the_indexer_with_the_same_outputs(lib):
     check_attention(out_a.float().cpu().numpy(), out_o, lse_a.cpu().numpy(), lse_o, rows=rows)
 
 
+SHORT_CACHE_CASES = {
+    # name: (row lengths, k, T_max, FP8 latent, paged block size)
+    "partials": ([2048, 1500, 700, 64, 1, 0], 2048, 2048, False, 0),   # 11 splits: partials + merge kernel
+    "cluster": ([(37 * t) % 2048 + 1 for t in range(20)], 2048, 2048, False, 0),  # 3 splits: on-chip merge
+    "fp8_latent": ([2048, 999, 2, 0], 2048, 2048, True, 0),
+    "paged": ([2048, 1300, 65, 1], 2048, 2048, False, 64),
+    "k1000": ([1000, 999, 513, 1], 1000, 1000, False, 0),              # T_max not a whole 64-row tile
+}
+
+
+@pytest.mark.parametrize("case", list(SHORT_CACHE_CASES))
+def test_short_cache_decode_is_dense_attention_and_matches_oracle(lib, case):
+    # A cache of at most k positions: every row selects all of its positions (the smaller of the
+    # budget and the number of tokens, kgptalkie "How Does the Selector Pick 1,024?"), and the
+    # decode step runs the attention's dense form, with the indexer and the top-k only for the
+    # outputs the caller asks for.  The outputs must equal the dense entry's bit for bit and the
+    # oracle's decode within the attention tolerance; the positions asked for are 0..n-1.
+    lens, k, T_max, fp8_latent, block = SHORT_CACHE_CASES[case]
+    inp = inputs.make_decode_inputs(f"short_cache_{case}", lens, k=k, T_max=T_max, anchor_frac=0.01,
+                                    seed=90 + len(case))
+    if fp8_latent:
+        inp = inputs.with_fp8_latent(inp)
+    sc_o, idx_o, out_o, lse_o = oracle.decode(inp)
+    g = inp.to("cuda")
+    dims = api.dims_of(g)
+    ws = api.make_workspace(dims, _lib.DSA_OP_DECODE)
+    if block:
+        k_pool, s_pool, kv_pool, table = inputs.paged_layout(g, block, seed=block)
+        cache = api.PagedCache(k_pool, s_pool, kv_pool, table, block)
+
+    def step(idx_out=None, scores_out=None):
+        if not block:
+            return api.run_decode(g, ws=ws, idx_out=idx_out, scores_out=scores_out, dims=dims)
+        out, lse = api.alloc_outputs(g)
+        api.decode_step_paged(dims, g.q_I, g.q_scale, g.w, cache, g.q, g.q_seq, g.q_len, g.softmax_scale, out, lse,
+                              ws, scores_out=scores_out, idx_out=idx_out)
+        return out, lse
+
+    out_a, lse_a = step()                                                  # attention alone
+    idx_b = torch.full((len(lens), k), 7, dtype=torch.int32, device="cuda")
+    out_b, lse_b = step(idx_out=idx_b)                                     # + the top-k's positions
+    idx_c = torch.full_like(idx_b, 7)
+    sc_c = torch.empty((len(lens), dims.ld_scores), device="cuda")
+    out_c, lse_c = step(idx_out=idx_c, scores_out=sc_c)                    # + the indexer's scores
+    ws_d = api.make_workspace(dims, _lib.DSA_OP_DENSE_MLA)
+    out_d, lse_d = api.alloc_outputs(g)
+    if not block:
+        api.dense_mla_attn(dims, g.q, g.kv, g.q_seq, g.q_len, g.softmax_scale, out_d, lse_d, ws_d)
+    torch.cuda.synchronize()
+    assert api.get_device_status(ws) == 0 and api.get_device_status(ws_d) == 0
+    assert torch.equal(out_a, out_b) and torch.equal(lse_a, lse_b)
+    assert torch.equal(out_a, out_c) and torch.equal(lse_a, lse_c)
+    if not block:
+        assert torch.equal(out_a, out_d) and torch.equal(lse_a, lse_d)
+    want = np.full((len(lens), k), -1, np.int32)
+    for t, n in enumerate(lens):
+        want[t, :n] = np.arange(n)
+    assert np.array_equal(idx_o, want)  # the oracle selects every position too
+    assert np.array_equal(idx_b.cpu().numpy(), want) and np.array_equal(idx_c.cpu().numpy(), want)
+    check_scores(np_scores(sc_c), sc_o, inp.q_len.numpy())
+    check_attention(out_a.float().cpu().numpy(), out_o, lse_a.cpu().numpy(), lse_o)
+    for t, n in enumerate(lens):
+        if n == 0:
+            assert torch.all(out_a[t] == 0) and torch.all(torch.isneginf(lse_a[t]))
+
+
 @pytest.mark.parametrize("block_size", [64, 256])
 def test_paged_decode_matches_oracle_and_contiguous(lib, block_size):
     # the same cache in blocks of a pool, in a random physical order, read through a block
