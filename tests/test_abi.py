@@ -59,6 +59,20 @@ def test_workspace_sizes(lib):
     assert pre <= (64 << 20) + (16 << 20), "prefill works in L2-sized row chunks"
 
 
+def test_short_cache_decode_workspace_holds_the_dense_plan(lib):
+    # a decode over a cache of at most k tokens runs the attention's dense form, whose splits are
+    # planned over T_max rounded up to whole 64-row tiles: the decode workspace must hold those
+    # partials beside its scores and index lists, for every batch size and width
+    for k in (64, 100, 1000, 1100, 2048):
+        for T_max in sorted({x // 4 * 4 for x in (k, k - 37, 64) if 4 <= x <= k}):  # FP8 keys: T_max % 4 == 0
+            for nq in range(1, 41):
+                ld = (T_max + 3) // 4 * 4
+                d = decode_dims(B=nq, Nq=nq, k=k, T_max=T_max, ld_scores=ld)
+                dec = api.workspace_size(d, _lib.DSA_OP_DECODE)
+                dense = api.workspace_size(d, _lib.DSA_OP_DENSE_MLA)
+                assert dec >= dense + nq * ld * 4 + nq * k * 4, (k, T_max, nq)
+
+
 @pytest.mark.parametrize("bad,code", [
     (dict(d_I=96), _lib.DSA_ERR_UNSUPPORTED),
     (dict(H_I=32), _lib.DSA_ERR_UNSUPPORTED),
