@@ -120,8 +120,9 @@ __device__ __forceinline__ int block_scan1(int v, int* scratch, int* total) {
 }
 
 // BATCH: some rows' slices exceed the shared-memory cache, so their passes read the scores
-// from global memory (L2); those reads go out 16 bytes and U steps at a time per thread (one
-// CTA per SM then, for the registers).  Launches whose slices all fit compile without it.
+// past the cached first part of the slice from global memory (L2); those reads go out 16 bytes
+// and U steps at a time per thread (one CTA per SM then, for the registers).  Launches whose
+// slices all fit compile without it.
 template <int T, bool BATCH>
 __global__ void __launch_bounds__(T, (T == 512 && !BATCH) ? 2 : 1) topk_radix_kernel(const TopkArgs a, int cached_cap) {
     using L = TopkLayout<T>;
@@ -167,6 +168,10 @@ __global__ void __launch_bounds__(T, (T == 512 && !BATCH) ? 2 : 1) topk_radix_ke
     const int hi = min(n, lo + chunk);
     const int len = hi - lo;
     const bool cached = len <= cached_cap;
+    // keys kept in shared memory: the whole slice when it fits; otherwise (the variant that
+    // streams from global memory) its first cached_cap keys, so that every later pass reads
+    // only the rest of the slice from L2
+    const int ncache = cached ? len : (BATCH ? (cached_cap & ~3) : 0);
     if (tid == 0) {
         misc[4] = -1;  // key min (as uint32), max
         misc[5] = 0;
@@ -205,9 +210,11 @@ __global__ void __launch_bounds__(T, (T == 512 && !BATCH) ? 2 : 1) topk_radix_ke
             kmx = max(kmx, kk);
         }
     } else if constexpr (BATCH) {
-        // the same 16-byte loads, eight in flight per thread, keys not kept
+        // the same 16-byte loads, eight in flight per thread, the first ncache keys kept
         const int nv = len >> 2;
+        const int nc4 = ncache >> 2;
         const float4* r4 = reinterpret_cast<const float4*>(row + lo);
+        uint4* k4 = reinterpret_cast<uint4*>(keys);
         for (int i0 = 0; i0 < nv; i0 += kLoadBatch * kThreads) {
             float4 f[kLoadBatch];
 #pragma unroll
@@ -217,9 +224,11 @@ __global__ void __launch_bounds__(T, (T == 512 && !BATCH) ? 2 : 1) topk_radix_ke
             }
 #pragma unroll
             for (int u = 0; u < kLoadBatch; ++u) {
-                if (i0 + u * kThreads + tid < nv) {
+                const int i = i0 + u * kThreads + tid;
+                if (i < nv) {
                     const uint32_t k0 = score_key(f[u].x), k1 = score_key(f[u].y), k2 = score_key(f[u].z),
                                    k3 = score_key(f[u].w);
+                    if (i < nc4) k4[i] = make_uint4(k0, k1, k2, k3);
                     kmn = min(kmn, min(min(k0, k1), min(k2, k3)));
                     kmx = max(kmx, max(max(k0, k1), max(k2, k3)));
                 }
@@ -246,11 +255,11 @@ __global__ void __launch_bounds__(T, (T == 512 && !BATCH) ? 2 : 1) topk_radix_ke
         atomicMin(reinterpret_cast<unsigned*>(misc + 4), kmn);
         atomicMax(reinterpret_cast<unsigned*>(misc + 5), kmx);
     }
-    auto key_at = [&](int i) -> uint32_t { return cached ? keys[i] : score_key(__ldg(row + lo + i)); };
+    auto key_at = [&](int i) -> uint32_t { return i < ncache ? keys[i] : score_key(__ldg(row + lo + i)); };
     // the 4 consecutive keys starting at i (a multiple of 4); out-of-range keys read as 0 (never selected:
     // the caller checks i < len)
     auto keys4_at = [&](int i) -> uint4 {
-        if (cached && i + 3 < len) return reinterpret_cast<const uint4*>(keys)[i >> 2];
+        if (i + 3 < ncache) return reinterpret_cast<const uint4*>(keys)[i >> 2];
         if (BATCH && i + 3 < len) {
             const float4 f = __ldg(reinterpret_cast<const float4*>(row + lo + i));
             return make_uint4(score_key(f.x), score_key(f.y), score_key(f.z), score_key(f.w));
