@@ -8,8 +8,11 @@
 //
 // Method: each score becomes an order-preserving 32-bit key; the selection is
 // the k-th largest key tau plus how many keys equal to tau are taken.  A row is
-// split across a thread-block cluster of C CTAs (C <= 8); every CTA keeps its
-// slice of the row in shared memory as keys and tracks their min and max.
+// split across a thread-block cluster of C CTAs (C <= 8, or up to 16 one-SM CTAs
+// for rows too long for shared memory at 8); every CTA keeps its slice of the
+// row in shared memory as keys -- a slice too long for it keeps its first part
+// there and reads the rest from global memory in every pass -- and tracks the
+// keys' min and max.
 //  1. One histogram of 2048 bins over (key - base) >> shift, the shift chosen
 //     so that [base, max] fills the bins (the top digits of a float key --
 //     sign and exponent -- put most scores of a row in a handful of bins, so
@@ -21,9 +24,11 @@
 //     all CTAs, read through distributed shared memory, give the group that
 //     holds the k-th largest key, and that group's 32 bins of all CTAs give b*.
 //  2. The keys of bin b* are collected (usually a few dozen); every CTA
-//     gathers all of them from the cluster and finds tau itself, refining with
-//     2048-bin histograms of the bits below the bin's base (at most two
-//     levels).  If bin b* holds more than kCandMax keys (extremely
+//     gathers all of them from the cluster and finds tau itself: with at most
+//     64 of them warp 0 ranks them directly (and also sets every rank's counts
+//     and the compaction's slots), otherwise it refines with 2048-bin histograms
+//     of the bits below the bin's base (at most two levels).  If bin b* holds
+//     more than kCandMax keys (extremely
 //     concentrated scores) the kernel falls back to a radix select over four
 //     8-bit digits of all keys (warp-private histograms with match_any
 //     aggregation, merged across the cluster).  Rows whose keys are all equal
@@ -33,9 +38,10 @@
 //     positions, with ballots ranking the keys inside each step.  Its counts
 //     come from the candidate pass of step 2, which reads the same segments
 //     (keys above b*, and its own candidates against tau); the rare paths
-//     without that pass (all-equal rows, the radix fallback) count first.  CTA r knows from the gathered threshold-bin keys
-//     how many ties and outputs the lower-ranked CTAs hold, which gives the
-//     lower-index tie rule across the whole row.
+//     without that pass (all-equal rows, the radix fallback) count first.
+//     CTA r knows from the gathered threshold-bin keys how many ties and
+//     outputs the lower-ranked CTAs hold, which gives the lower-index tie rule
+//     across the whole row.
 #include <cooperative_groups.h>
 #include <cuda_runtime.h>
 
