@@ -255,9 +255,10 @@ typedef struct {
     int32_t reserved;            /* must be 0 */
 } dsa_paged_cache;
 
-/* dsa_decode_step over a paged cache: the same stages and outputs, with the
- * indexer's key and scale copies (one TMA box per block piece of a stage) and
- * the attention's row gather translated through the block table.  Only blocks
+/* dsa_decode_step over a paged cache: the same stages, dispatch and outputs,
+ * with the indexer's key and scale copies (16-byte asynchronous copies, each
+ * within one block) and the attention's row gather translated through the
+ * block table.  Only blocks
  * holding positions s < q_len[t] are read; a table entry outside
  * [0, num_blocks) for such a block records DSA_ERR_INDEX_OOB in the status
  * word (its rows are skipped).  FP8 indexer; bf16 or FP8 (656-byte) latent pool
