@@ -5,6 +5,7 @@ import os
 import re
 
 import pytest
+import torch
 
 from sparse_long_context_indexer_b200 import _lib, api, build
 
@@ -189,3 +190,26 @@ def test_dense_and_prefill_host_checks(lib):
     empty = decode_dims(B=1, Nq=0, T_max=4096, ld_scores=4096).c()
     assert lib.dsa_prefill(ctypes.byref(empty), *args, ctypes.c_float(0.07), P, P, None, P, 1 << 30,
                            None) == _lib.DSA_OK
+
+
+def planned_splits(nq, k=2048, sms=148):
+    """The attention's split plan: SMs // (2 nq) clamped to [1, 16], rows per split rounded up to
+    whole 64-row tiles, then the splits those rows need (a CPU without a GPU plans for 148 SMs)."""
+    s = max(1, min(16, sms // (2 * nq)))
+    rows = -(-(-(-k // s)) // 64) * 64
+    return -(-k // rows)
+
+
+@pytest.mark.skipif(torch.cuda.is_available(), reason="host-side refusal only: without a GPU no call can launch")
+def test_noalloc_refuses_exactly_the_plans_beyond_its_scratch(lib):
+    # more than 8 splits go through a static buffer of 64 (split, row) partials; at k = 2048 on
+    # 148 SMs only Nq = 6 (11 splits x 6 rows = 66) exceeds it, which the entry refuses on the
+    # host.  Only refused calls are made here (they return before any CUDA call).
+    refused = [nq for nq in range(1, 80) if planned_splits(nq) > 8 and planned_splits(nq) * nq > 64]
+    assert refused == [6]
+    for nq in refused:
+        d = decode_dims(B=nq, Nq=nq).c()
+        P = ctypes.c_void_p(1 << 20)
+        rc = lib.dsa_sparse_mla_attn_noalloc(ctypes.byref(d), P, P, P, P, P, ctypes.c_float(0.07), P, P,
+                                             ctypes.c_void_p(0))
+        assert rc == _lib.DSA_ERR_UNSUPPORTED
